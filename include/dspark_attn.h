@@ -1,0 +1,155 @@
+/*
+ * dspark_attn.h — C ABI of the B200 (sm_100a) DSpark draft MLA attention.
+ *
+ * The operation (page "GLM 5.2 DSpark speculative-training design"):
+ *   The KV axis is [S context positions | N draft blocks x 5 positions]
+ *   (§2 "QKV construction"). The queries are the 5N draft positions. A query of
+ *   block n, anchor A = anchors[b][n], sees exactly
+ *     - the context window max(0, A-W+1) <= kv < A, shared by the 5 offsets of
+ *       the block and excluding position A (§3 "attention mask"), and
+ *     - the 5 positions of its own block, bidirectionally (§3);
+ *   a block with keep[b][n] = 0 (block_keep_mask, a padding block) sees nothing.
+ *   Per head the query is [q^C ; q^R] and the key [k^C ; k^R], where the rope key
+ *   k^R is one d_r-wide vector per position shared by all heads (§4 "MLA").
+ *   RoPE rotates only the rope slice, interleaved adjacent pairs (2i, 2i+1), by
+ *   angle pos * rope_base^(-2i/d_r); positions are 0..S-1 for context and
+ *   A_n .. A_n+4 for block n (§2, §4 "RoPE").
+ *   O = softmax(Q K^T / sqrt(d_c + d_r) + Lambda(M)) V with Lambda = -inf off the
+ *   mask (appendix "Attention implementation"). Rows of padding blocks give
+ *   O = 0, LSE = -inf and zero gradients.
+ *
+ * Layouts (contiguous, row-major; "dtype" is fp32 or bf16 as given by
+ * dspark_problem.dtype; all tensors on the CUDA device unless stated):
+ *   q   [B, n_h, 5N, d_c + d_r]  dtype   query, rope slice last, NOT rotated
+ *   kc  [B, n_h, S + 5N, d_c]    dtype   per-head key, non-rope part
+ *   kr  [B, S + 5N, d_r]         dtype   rope key shared by heads, NOT rotated
+ *   v   [B, n_h, S + 5N, d_v]    dtype
+ *   anchors [B, N] int32; keep [B, N] uint8 (0 = padding block)
+ *   o   [B, n_h, 5N, d_v]        dtype;  lse [B, n_h, 5N] fp32 (natural log)
+ *   do_ like o; dq like q; dkc like kc; dkr like kr; dv like v
+ *   (gradients are with respect to the un-rotated inputs).
+ * Row r = 5n + j of q / o is offset j of block n. Every element of every output
+ * is written (zeros included).
+ *
+ * Ownership: the caller allocates and owns every buffer, the workspace
+ * included. The library allocates no device memory, launches only on the
+ * given stream (a cudaStream_t passed as void*, NULL = legacy default stream)
+ * and never synchronises, except dspark_get_error.
+ *
+ * Errors: argument checks run on the host before any launch and return a
+ * status without touching device memory. A kept anchor outside [0, S-2] can
+ * only be seen on the device: that block is then treated as a padding block
+ * and a bit is set in the workspace error word, read by dspark_get_error.
+ */
+#ifndef DSPARK_ATTN_H
+#define DSPARK_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSPARK_API __attribute__((visibility("default")))
+#else
+#define DSPARK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSPARK_OK = 0,
+    DSPARK_ERR_NULL = 1,        /* a required pointer is NULL */
+    DSPARK_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+    DSPARK_ERR_DTYPE = 3,       /* unknown dtype */
+    DSPARK_ERR_ANCHOR = 4,      /* (device) a kept anchor outside [0, S-2] */
+    DSPARK_ERR_WORKSPACE = 5,   /* workspace NULL, too small or misaligned */
+    DSPARK_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    DSPARK_ERR_DEVICE = 7,      /* (device) a bounded wait gave up */
+    DSPARK_ERR_ALIGN = 8,       /* a tensor pointer is not 16-byte aligned */
+    DSPARK_ERR_UNSUPPORTED = 9  /* sizes outside what the kernels implement */
+} dspark_status;
+
+typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype;
+
+/* Problem sizes (page notation). Limits checked on the host:
+ *   B >= 0, n_h >= 1, S >= 1, N >= 0, 1 <= W <= 4096, N <= 8192,
+ *   d_c >= 0, d_r >= 0 even, d_v >= 1, d_c + d_r >= 1, d_c + d_r <= 256,
+ *   d_v <= 256, (S + 5N) * n_h * max(d_c, d_v) < 2^31, rope_base > 0. */
+typedef struct {
+    int32_t B;          /* batch */
+    int32_t n_h;        /* heads */
+    int32_t S;          /* context positions */
+    int32_t N;          /* draft blocks (5 positions each) */
+    int32_t W;          /* sliding window: W-1 context positions visible */
+    int32_t d_c;        /* per-head non-rope query/key width */
+    int32_t d_r;        /* rope width (shared rope key) */
+    int32_t d_v;        /* per-head value width */
+    double rope_base;   /* RoPE base, e.g. 10000 */
+    int32_t dtype;      /* dspark_dtype of q, kc, kr, v, o, do, dq, dkc, dkr, dv */
+    int32_t reserved;   /* must be 0 */
+} dspark_problem;
+
+/* Flags of dspark_attn_fwd / dspark_attn_bwd. */
+#define DSPARK_FLAG_REUSE_DESCRIPTOR 1u /* the workspace already holds the
+        descriptor built by dspark_build_descriptor (or by an earlier fwd/bwd)
+        for the same anchors, keep and sizes: skip rebuilding it. The page's
+        mask is built once and shared by the three draft layers (§3, §4). */
+
+/* Bytes of device workspace needed for problem *p (0 if *p is invalid). The
+ * workspace must be 256-byte aligned. */
+DSPARK_API size_t dspark_workspace_size(const dspark_problem *p);
+
+/* Build the mask descriptor into the workspace: kept blocks of each batch row
+ * sorted by anchor (ties by block index), per-row kept counts, and the RoPE
+ * cos/sin table for positions 0 .. S+7. Validates kept anchors on the device
+ * (see dspark_get_error). Clears the workspace error word first, so the word
+ * reports what happened since the last descriptor build.
+ * anchors, keep: device pointers [B, N]. */
+DSPARK_API dspark_status dspark_build_descriptor(const dspark_problem *p, const int32_t *anchors, const uint8_t *keep,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* Forward: o and lse (layouts above). Builds the descriptor first unless
+ * flags has DSPARK_FLAG_REUSE_DESCRIPTOR. */
+DSPARK_API dspark_status dspark_attn_fwd(const dspark_problem *p, const void *q, const void *kc, const void *kr,
+                              const void *v, const int32_t *anchors, const uint8_t *keep, void *o, float *lse,
+                              void *workspace, size_t workspace_bytes, uint32_t flags, void *stream);
+
+/* Backward of the forward for a loss L with dL/dO = do_: writes dq, dkc, dkr,
+ * dv. o and lse are the forward's outputs for the same inputs. Builds the
+ * descriptor first unless flags has DSPARK_FLAG_REUSE_DESCRIPTOR. */
+DSPARK_API dspark_status dspark_attn_bwd(const dspark_problem *p, const void *q, const void *kc, const void *kr,
+                              const void *v, const int32_t *anchors, const uint8_t *keep, const void *o,
+                              const float *lse, const void *do_, void *dq, void *dkc, void *dkr, void *dv,
+                              void *workspace, size_t workspace_bytes, uint32_t flags, void *stream);
+
+/* Synchronises the stream, reads and clears the workspace error word.
+ * Returns DSPARK_OK, DSPARK_ERR_ANCHOR (a kept anchor was out of range) or
+ * DSPARK_ERR_DEVICE (a bounded wait in a kernel gave up). */
+DSPARK_API dspark_status dspark_get_error(void *workspace, void *stream);
+
+/* Static description of a status code. */
+DSPARK_API const char *dspark_status_string(dspark_status s);
+
+/* Number of kernels this library has launched in the calling process since it
+ * was loaded (host-side count, incremented at every launch; monotonic). Lets a
+ * caller count the device work of a timed region. */
+DSPARK_API uint64_t dspark_launch_counter(void);
+
+/* Host helper, page §2 "anchor sampling": for each batch row, the candidates
+ * are A in [0, S-2] with loss_mask[A] = loss_mask[A+1] = 1, where
+ * loss_mask[S-1] is read as 0 (appendix A: the last position is neither an
+ * anchor nor a label). Draws min(N, #candidates) of them uniformly without
+ * replacement (a Fisher-Yates shuffle driven by SplitMix64 seeded with
+ * seed + row), writes them in draw order, and pads the rest with anchor 0,
+ * keep 0 (padding blocks, §3). All pointers are host memory:
+ * loss_mask [B, S] uint8, anchors_out [B, N] int32, keep_out [B, N] uint8.
+ * Returns the total number of kept blocks, or -1 on bad arguments. */
+DSPARK_API int64_t dspark_sample_anchors(const uint8_t *loss_mask, int32_t B, int32_t S, int32_t N, uint64_t seed,
+                              int32_t *anchors_out, uint8_t *keep_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_ATTN_H */

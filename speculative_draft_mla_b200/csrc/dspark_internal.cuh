@@ -1,0 +1,110 @@
+// Internal declarations shared by the translation units of the DSpark
+// attention library: problem view, workspace layout, error bits and the
+// launch functions of each kernel family.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dspark_attn.h"
+
+namespace dspark {
+
+constexpr int kBlock = 5;  // draft block length (block_size = 5)
+
+// Device error word bits (workspace offset 0).
+constexpr uint32_t kErrAnchor = 1u;   // kept anchor outside [0, S-2]
+constexpr uint32_t kErrTimeout = 2u;  // a bounded mbarrier wait gave up
+
+struct Prob {
+    int B, n_h, S, N, W, d_c, d_r, d_v;
+    int dqk;   // d_c + d_r
+    int R;     // 5N query rows per (b, h)
+    int L;     // S + 5N kv positions
+    int P;     // rope table positions (S + 8)
+    double base;
+    int dtype;
+    float scale_log2;  // (d_c + d_r)^(-1/2) * log2(e)
+    float scale;       // (d_c + d_r)^(-1/2)
+};
+
+// Workspace layout (byte offsets, each 256-aligned).
+struct WsLayout {
+    size_t err;       // uint32 error word (+ pad)
+    size_t cnt;       // int32 [B]     kept blocks per batch row
+    size_t sorted_n;  // int32 [B, N]  block index of the i-th smallest anchor
+    size_t sorted_a;  // int32 [B, N]  its anchor
+    size_t rope;      // float2 [P, d_r/2] (cos, sin) of pos * base^(-2i/d_r)
+    size_t kr_rot;    // dtype [B, L, d_r] rotated rope keys
+    size_t dvec;      // float [B, n_h, 5N] D = rowsum(dO * O)
+    size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(const Prob &p) {
+    WsLayout w;
+    size_t off = 0;
+    size_t esz = p.dtype == DSPARK_BF16 ? 2 : 4;
+    w.err = off;       off = align256(off + 256);
+    w.cnt = off;       off = align256(off + sizeof(int32_t) * (size_t)p.B);
+    w.sorted_n = off;  off = align256(off + sizeof(int32_t) * (size_t)p.B * p.N);
+    w.sorted_a = off;  off = align256(off + sizeof(int32_t) * (size_t)p.B * p.N);
+    w.rope = off;      off = align256(off + sizeof(float2) * (size_t)p.P * (p.d_r / 2));
+    w.kr_rot = off;    off = align256(off + esz * (size_t)p.B * p.L * p.d_r);
+    w.dvec = off;      off = align256(off + sizeof(float) * (size_t)p.B * p.n_h * p.R);
+    w.total = off;
+    return w;
+}
+
+// Typed views of the workspace.
+struct Ws {
+    uint32_t *err;
+    int32_t *cnt, *sorted_n, *sorted_a;
+    float2 *rope;
+    void *kr_rot;
+    float *dvec;
+};
+
+inline Ws ws_view(const Prob &p, void *base) {
+    WsLayout l = ws_layout(p);
+    char *c = (char *)base;
+    Ws w;
+    w.err = (uint32_t *)(c + l.err);
+    w.cnt = (int32_t *)(c + l.cnt);
+    w.sorted_n = (int32_t *)(c + l.sorted_n);
+    w.sorted_a = (int32_t *)(c + l.sorted_a);
+    w.rope = (float2 *)(c + l.rope);
+    w.kr_rot = (void *)(c + l.kr_rot);
+    w.dvec = (float *)(c + l.dvec);
+    return w;
+}
+
+// ---- element conversions -------------------------------------------------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---- launch accounting -----------------------------------------------------
+// Every kernel launch goes through count_launch() so that the launch counter of
+// the C ABI reports the device work a caller issued.
+void count_launch(unsigned n = 1);
+
+// ---- launch functions ------------------------------------------------------
+// descriptor: sort kept blocks by anchor, validate anchors, rope table
+cudaError_t launch_build_descriptor(const Prob &p, const int32_t *anchors, const uint8_t *keep, const Ws &ws,
+                                    cudaStream_t st);
+// rotated rope keys for all kv positions
+cudaError_t launch_rotate_kr(const Prob &p, const void *kr, const int32_t *anchors, const Ws &ws, cudaStream_t st);
+
+// SIMT (CUDA-core) forward / backward, any supported dims, fp32 or bf16
+cudaError_t launch_fwd_simt(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
+                            const uint8_t *keep, void *o, float *lse, const Ws &ws, cudaStream_t st);
+cudaError_t launch_bwd_simt(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
+                            const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,
+                            void *dkc, void *dkr, void *dv, const Ws &ws, cudaStream_t st);
+
+}  // namespace dspark

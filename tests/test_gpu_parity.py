@@ -1,0 +1,168 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small workloads are compared element by element on every output; the tiny
+fp32 workload and the 2048-context bf16 workload are compared in full. The
+three large workloads run at full size in the launch configuration the
+benchmark times and are checked on sampled rows and keys that the oracle
+computes one by one, plus properties that hold at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity import assert_close, compare_full, oracle_full, run_gpu, to_dev
+from speculative_draft_mla_b200 import build as dbuild
+from speculative_draft_mla_b200 import capi, synth
+
+pytestmark = pytest.mark.gpu
+BASE = 10000.0
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dbuild.build()
+    return capi.load()
+
+
+def test_tiny_f32_workload_full(oracle_mod):
+    wl = synth.WORKLOADS[1]
+    c = synth.make_inputs(wl)
+    gpu = run_gpu(c, wl.S, wl.W)
+    compare_full(gpu, oracle_full(oracle_mod, c, wl.S, wl.W), torch.float32)
+
+
+# (name, seed, B, S, N, W, n_h, d_c, d_r, d_v, keep_frac, dup)
+EDGE = [
+    ("window_wider_than_context", 31, 2, 12, 3, 16, 2, 16, 8, 16, 1.0, False),
+    ("window_one", 32, 1, 50, 6, 1, 2, 16, 8, 16, 1.0, False),
+    ("ragged_tiles", 33, 2, 77, 9, 20, 3, 24, 16, 40, 1.0, False),
+    ("duplicate_anchors", 34, 1, 40, 12, 8, 2, 16, 8, 16, 1.0, True),
+    ("padding_blocks", 35, 2, 64, 10, 16, 2, 16, 8, 16, 0.5, False),
+    ("all_padding", 36, 1, 30, 4, 8, 2, 16, 8, 16, 0.0, False),
+    ("no_rope", 37, 1, 40, 5, 9, 2, 32, 0, 16, 1.0, False),
+    ("rope_only", 38, 1, 40, 5, 9, 2, 0, 16, 24, 1.0, False),
+    ("minimal_context", 39, 1, 2, 2, 4, 1, 8, 8, 8, 1.0, True),
+    ("page_dims_small", 40, 1, 300, 20, 128, 2, 192, 64, 256, 1.0, False),
+    ("page_dims_dense", 41, 1, 200, 60, 128, 2, 192, 64, 256, 0.9, True),
+    ("page_dims_ragged", 42, 2, 133, 7, 128, 1, 192, 64, 256, 1.0, False),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_cases_full(oracle_mod, case, dtype):
+    name, seed, B, S, N, W, n_h, d_c, d_r, d_v, kf, dup = case
+    c = synth.random_case(seed, B, S, N, W, n_h, d_c, d_r, d_v, dtype, keep_frac=kf, allow_dup=dup)
+    if S >= 3:
+        c["anchors"][0, 0] = 0          # empty context window
+        c["anchors"][-1, -1] = S - 2    # last valid anchor
+    gpu = run_gpu(c, S, W)
+    compare_full(gpu, oracle_full(oracle_mod, c, S, W), synth.torch_dtype(dtype))
+
+
+def test_no_blocks():
+    """N = 0: nothing to attend; the backward still writes zero key gradients."""
+    c = synth.random_case(50, 2, 40, 0, 8, 2, 16, 8, 16, "bf16")
+    gpu = run_gpu(c, 40, 8)
+    assert gpu["o"].numel() == 0 and gpu["dq"].numel() == 0
+    for k in ("dkc", "dkr", "dv"):
+        assert torch.count_nonzero(gpu[k]) == 0
+
+
+def test_out_of_range_anchor_is_reported():
+    """A kept anchor outside [0, S-2] is reported and its block treated as padding."""
+    c = synth.random_case(51, 1, 32, 4, 8, 2, 16, 8, 16, "f32")
+    c["anchors"][0, 1] = 31  # S - 1: not a valid anchor
+    d = to_dev(c)
+    o, lse, ws = capi.attn_fwd(d["q"], d["kc"], d["kr"], d["v"], d["anchors"], d["keep"], 32, 8, BASE)
+    with pytest.raises(capi.DsparkError) as e:
+        capi.get_error(ws)
+    assert e.value.status == 4
+    assert torch.count_nonzero(o[0, :, 5:10]) == 0 and torch.isneginf(lse[0, :, 5:10]).all()
+    capi.get_error(ws)  # the word was cleared
+
+
+def test_s2048_workload_full(oracle_mod):
+    wl = synth.WORKLOADS[2]
+    c = synth.make_inputs(wl)
+    gpu = run_gpu(c, wl.S, wl.W)
+    compare_full(gpu, oracle_full(oracle_mod, c, wl.S, wl.W), torch.bfloat16)
+
+
+def test_deterministic():
+    wl = synth.WORKLOADS[2]
+    c = synth.make_inputs(wl)
+    a = run_gpu(c, wl.S, wl.W)
+    b = run_gpu(c, wl.S, wl.W)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def _slice(c, b, h):
+    return dict(q=c["q"][b:b + 1, h:h + 1], kc=c["kc"][b:b + 1, h:h + 1], kr=c["kr"][b:b + 1],
+                v=c["v"][b:b + 1, h:h + 1], dout=c["dout"][b:b + 1, h:h + 1],
+                anchors=c["anchors"][b:b + 1], keep=c["keep"][b:b + 1])
+
+
+def _np(s):
+    return [s[k].double().numpy() for k in ("q", "kc", "kr", "v")]
+
+
+@pytest.mark.parametrize("wid", [3, 4, 5])
+def test_full_size_sampled(oracle_mod, wid):
+    wl = synth.WORKLOADS[wid]
+    c = synth.make_inputs(wl)
+    gpu = run_gpu(c, wl.S, wl.W)
+    rng = np.random.default_rng(wid)
+    an, kp = c["anchors"].numpy(), c["keep"].numpy()
+    S, W = wl.S, wl.W
+    # properties at full size: padding rows are zero / -inf, all finite elsewhere
+    pad = np.repeat(kp == 0, 5, axis=1)
+    for b in range(wl.B):
+        rows = np.nonzero(pad[b])[0]
+        if rows.size:
+            assert torch.count_nonzero(gpu["o"][b][:, rows]) == 0
+            assert torch.isneginf(gpu["lse"][b][:, rows]).all()
+            assert torch.count_nonzero(gpu["dq"][b][:, rows]) == 0
+    for k in ("o", "dq", "dkc", "dkr", "dv"):
+        assert torch.isfinite(gpu[k].float()).all(), k
+    # sampled rows: random ones plus the block with the smallest anchor
+    picks = []
+    for _ in range(24):
+        b, h = int(rng.integers(wl.B)), int(rng.integers(wl.n_h))
+        picks.append((b, h, int(rng.integers(5 * wl.N))))
+    b0 = 0
+    n_small = int(np.argmin(np.where(kp[b0] == 1, an[b0], 1 << 30)))
+    picks += [(b0, 0, 5 * n_small + j) for j in range(5)]
+    for b, h, r in picks:
+        s = _slice(c, b, h)
+        o_ref, lse_ref = oracle_mod.attn_fwd_rows(*_np(s), s["anchors"].numpy(), s["keep"].numpy(), S, W, BASE,
+                                                  np.array([[0, 0, r]]))
+        assert_close(gpu["o"][b, h, r][None], o_ref, torch.bfloat16, "o[%d,%d,%d]" % (b, h, r))
+        assert_close(gpu["lse"][b, h, r][None], lse_ref, torch.bfloat16, "lse")
+        dq_ref = oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
+                                           s["dout"].double().numpy(), S, W, BASE, "dq", np.array([[0, 0, r]]))
+        assert_close(gpu["dq"][b, h, r][None], dq_ref, torch.bfloat16, "dq[%d,%d,%d]" % (b, h, r))
+    # sampled keys: context (covered, edge and possibly uncovered) and draft keys
+    keys = [0, S - 1, int(an[0][n_small]) - 1 if an[0][n_small] > 0 else 1]
+    keys += [int(x) for x in rng.integers(0, S, 8)]
+    keys += [S + 5 * int(rng.integers(wl.N)) + int(rng.integers(5)) for _ in range(4)]
+    pads = np.nonzero(kp[0] == 0)[0]
+    if pads.size:
+        keys.append(S + 5 * int(pads[0]))
+    for key in keys:
+        b, h = 0, int(rng.integers(wl.n_h))
+        s = _slice(c, b, h)
+        ref = oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
+                                        s["dout"].double().numpy(), S, W, BASE, "dkv", np.array([[0, 0, key]]))
+        assert_close(gpu["dkc"][b, h, key][None], ref[:, :wl.d_c], torch.bfloat16, "dkc[%d]" % key)
+        assert_close(gpu["dv"][b, h, key][None], ref[:, wl.d_c:], torch.bfloat16, "dv[%d]" % key)
+    # rope-key gradient: sum over heads of per-head oracle contributions
+    dkr_keys = np.array([[0, k] for k in keys[:4]])
+    tot = np.zeros((len(dkr_keys), wl.d_r))
+    for h in range(wl.n_h):
+        s = _slice(c, 0, h)
+        tot += oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
+                                         s["dout"].double().numpy(), S, W, BASE, "dkr", dkr_keys)
+    assert_close(gpu["dkr"][0, dkr_keys[:, 1]], tot, torch.bfloat16, "dkr")
