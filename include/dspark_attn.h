@@ -115,6 +115,34 @@ DSPARK_API dspark_status dspark_attn_fwd(const dspark_problem *p, const void *q,
                               const void *v, const int32_t *anchors, const uint8_t *keep, void *o, float *lse,
                               void *workspace, size_t workspace_bytes, uint32_t flags, void *stream);
 
+/* Forward without a caller workspace. The page has no counterpart to this
+ * entry point: it exists for callers that get only their input and output
+ * buffers and may not allocate device memory (a plugin inside another
+ * framework's execution hook, whose device memory that framework already owns;
+ * a latency-bound loop that cannot afford the device synchronisation of
+ * cudaMalloc/cudaFree). It runs the dspark_attn_fwd sequence with the
+ * workspace in a device array compiled into the library, so it allocates
+ * nothing at run time; every GPU that loads the library keeps that array,
+ * DSPARK_NOALLOC_SCRATCH_BYTES (16 MiB), until the process exits.
+ *   - Arguments and layouts as dspark_attn_fwd. error_word (device pointer,
+ *     may be NULL) receives, in stream order, the error word of this call
+ *     (bit 0: a kept anchor was out of range and its block treated as padding;
+ *     bit 1: a bounded device-side wait gave up).
+ *   - Returns DSPARK_ERR_UNSUPPORTED when the problem needs more scratch than
+ *     the array holds (dspark_workspace_size(p) > DSPARK_NOALLOC_SCRATCH_BYTES);
+ *     other statuses as dspark_attn_fwd.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents: two
+ *     calls whose work overlaps on the GPU (different streams, or different
+ *     host threads on the same device) race on it. Serialise them. */
+#define DSPARK_NOALLOC_SCRATCH_BYTES (16u << 20)
+DSPARK_API dspark_status dspark_attn_fwd_noalloc(const dspark_problem *p, const void *q, const void *kc,
+                                                 const void *kr, const void *v, const int32_t *anchors,
+                                                 const uint8_t *keep, void *o, float *lse, uint32_t *error_word,
+                                                 void *stream);
+
 /* Backward of the forward for a loss L with dL/dO = do_: writes dq, dkc, dkr,
  * dv. o and lse are the forward's outputs for the same inputs. Builds the
  * descriptor first unless flags has DSPARK_FLAG_REUSE_DESCRIPTOR. */

@@ -57,6 +57,8 @@ def load():
     lib.dspark_status_string.restype = ctypes.c_char_p
     lib.dspark_sample_anchors.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_uint64, vp, vp]
     lib.dspark_sample_anchors.restype = ctypes.c_int64
+    lib.dspark_attn_fwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.dspark_attn_fwd_noalloc.restype = ctypes.c_int
     lib.dspark_launch_counter.argtypes = []
     lib.dspark_launch_counter.restype = ctypes.c_uint64
     for f in ("dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd", "dspark_get_error"):
@@ -161,6 +163,25 @@ def attn_bwd(q, kc, kr, v, anchors, keep, o, lse, dout, S, W, rope_base=10000.0,
                                   _ptr(keep), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dkc), _ptr(dkr),
                                   _ptr(dv), _ptr(workspace), workspace.numel(), flags, st), "dspark_attn_bwd")
     return dq, dkc, dkr, dv
+
+
+def attn_fwd_noalloc(q, kc, kr, v, anchors, keep, S, W, rope_base=10000.0, out=None, error_word=None,
+                     stream=None):
+    """Forward through dspark_attn_fwd_noalloc (no workspace argument: the
+    library's built-in scratch array is used). Returns (o, lse)."""
+    _cuda(q, kc, kr, v, anchors, keep, error_word)
+    prob = problem_of(q, kc, kr, v, anchors, S, W, rope_base)
+    if out is None:
+        o = torch.empty(q.shape[:3] + (v.shape[-1],), dtype=q.dtype, device=q.device)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _cuda(o, lse)
+    st = _stream(stream, q.device)
+    _check(load().dspark_attn_fwd_noalloc(ctypes.byref(prob), _ptr(q), _ptr(kc), _ptr(kr), _ptr(v), _ptr(anchors),
+                                          _ptr(keep), _ptr(o), _ptr(lse), _ptr(error_word), st),
+           "dspark_attn_fwd_noalloc")
+    return o, lse
 
 
 def get_error(workspace, stream=None):
