@@ -144,7 +144,10 @@ dspark_status dspark_attn_fwd(const dspark_problem *pp, const void *q, const voi
     const Ws w = ws_view(p, workspace);
     if (!(flags & DSPARK_FLAG_REUSE_DESCRIPTOR)) DSPARK_TRY(build(p, anchors, keep, w, st));
     DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, w, st));
-    DSPARK_CUDA(launch_fwd_simt(p, q, kc, v, anchors, keep, o, lse, w, st));
+    if (fwd_tc_supported(p))
+        DSPARK_CUDA(launch_fwd_tc(p, q, kc, v, anchors, keep, o, lse, w, st));
+    else
+        DSPARK_CUDA(launch_fwd_simt(p, q, kc, v, anchors, keep, o, lse, w, st));
     return DSPARK_OK;
 }
 

@@ -107,4 +107,9 @@ cudaError_t launch_bwd_simt(const Prob &p, const void *q, const void *kc, const 
                             const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,
                             void *dkc, void *dkr, void *dv, const Ws &ws, cudaStream_t st);
 
+// tcgen05 forward for bf16 at the page's head widths (192 + 64 / 256)
+bool fwd_tc_supported(const Prob &p);
+cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
+                          const uint8_t *keep, void *o, float *lse, const Ws &ws, cudaStream_t st);
+
 }  // namespace dspark

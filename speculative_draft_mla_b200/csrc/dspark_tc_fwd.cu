@@ -1,0 +1,527 @@
+// Tensor-core (tcgen05 / TMEM / TMA) forward of the DSpark draft attention for
+// the page's head widths (d_c = 192, d_r = 64, d_v = 256), bf16.
+//
+// Work unit: one CTA per (batch b, head h, group of up to 25 kept blocks that
+// are consecutive in anchor order) = up to 125 query rows, the M = 128 of one
+// MMA. The group's key set is the union of its blocks' context windows,
+// [max(0, A_first - W + 1), A_last), walked in 64-key tiles, followed by the
+// group's own draft keys (5 per block) gathered into one or two more tiles.
+// Each row masks every key that is not in its own key set (page "GLM 5.2
+// DSpark speculative-training design", §3: window [A-W+1, A) shared by the 5
+// offsets, own block bidirectional, other blocks invisible). Because blocks
+// are sorted by anchor, neighbouring groups (adjacent blockIdx.x) read
+// overlapping windows close together in time, so the overlap is served by L2.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread t owns query row t = TMEM lane t. Loads and
+//              RoPE-rotates Q at the start, turns each S tile into P (bf16, in
+//              shared memory) with an online softmax, rescales its O row when
+//              the running max grows by more than 2^8, and writes O and LSE.
+//   warp 4     producer: TMA loads of context K (K^C 3 x 64 columns plus the
+//              pre-rotated shared K^R) and V tiles, cp.async gathers of the
+//              draft-key tiles; two stages each for K and V.
+//   warp 5     TMEM owner and MMA issuer (one thread): S = Q K^T into two
+//              alternating 64-column TMEM buffers, O += P V into 256 columns.
+// Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
+// all roles leave their loops, in-flight copies and MMAs are drained with a
+// bounded wait, TMEM is freed and the workspace error word gets kErrTimeout.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "dspark_tc_common.cuh"
+
+namespace dspark {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kG = 25;    // blocks per CTA
+constexpr int kM = 128;   // query rows per CTA (MMA M)
+constexpr int kBN = 64;   // keys per tile
+constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
+
+constexpr int kQChunk = kM * 128;   // one 64-column slice of the Q tile
+constexpr int kKChunk = kBN * 128;  // one 64-column slice of a K or V tile
+constexpr int kQBytes = 4 * kQChunk;
+constexpr int kKBytes = 4 * kKChunk;
+constexpr int kVBytes = 4 * kKChunk;
+constexpr int kPBytes = kM * 128;
+
+constexpr int oQ = 0;
+constexpr int oK0 = oQ + kQBytes;
+constexpr int oK1 = oK0 + kKBytes;
+constexpr int oV0 = oK1 + kKBytes;
+constexpr int oV1 = oV0 + kVBytes;
+constexpr int oP0 = oV1 + kVBytes;
+constexpr int oP1 = oP0 + kPBytes;
+constexpr int oBar = oP1 + kPBytes;
+constexpr int kSmemBytes = oBar + 256 + 1024;  // barriers + alignment slack
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0;
+constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct FwdArgs {
+    int n_h, S, N, W, L, R;
+    float scale_log2;
+    const __nv_bfloat16 *q, *kc, *krr, *v;
+    const int32_t *cnt, *sorted_n, *sorted_a;
+    const float2 *tab;
+    __nv_bfloat16 *o;
+    float *lse;
+    uint32_t *err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&t);
+}
+
+__device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
+             const __grid_constant__ CUtensorMap tm_v, const FwdArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
+    uint64_t *kfull = bars + 0, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
+    uint64_t *sfull = bars + 8, *pready = bars + 10, *pvdone = bars + 12, *qready = bars + 14;
+    uint64_t *drain = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+    // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed
+    int *counters = reinterpret_cast<int *>(bars + 18);
+
+    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int cnt = p.cnt[b];
+    const int i0 = g * kG;
+    if (i0 >= cnt) return;  // uniform: this batch row has fewer groups
+    const int gcnt = min(kG, cnt - i0);
+    const int nrows = kBlock * gcnt;
+    const int32_t *sa = p.sorted_a + (size_t)b * p.N + i0;
+    const int32_t *sn = p.sorted_n + (size_t)b * p.N + i0;
+    const int ctx_lo = max(0, sa[0] - p.W + 1);
+    const int ctx_hi = sa[gcnt - 1];
+    const int n_ctx = ctx_hi > ctx_lo ? (ctx_hi - ctx_lo + kBN - 1) / kBN : 0;
+    const int n_draft = (nrows + kBN - 1) / kBN;
+    const int T = n_ctx + n_draft;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t bh = (size_t)b * p.n_h + h;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
+            mbar_init(&sfull[s], 1);
+            mbar_init(&pready[s], 4);
+            mbar_init(&pvdone[s], 1);
+        }
+        mbar_init(qready, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        for (int c = 0; c < 4; c++) counters[c] = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_kc);
+            tma_prefetch_desc(&tm_kr);
+            tma_prefetch_desc(&tm_v);
+        }
+        for (int t = 0; t < T; ++t) {
+            const int s = t & 1;
+            uint8_t *kt = sm + (s ? oK1 : oK0);
+            uint8_t *vt = sm + (s ? oV1 : oV0);
+            if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+            if (t < n_ctx) {
+                const int pos0 = ctx_lo + t * kBN;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&kfull[s], kKBytes);
+                    for (int c = 0; c < 3; c++)
+                        tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[s], c * 64, (int)(bh * p.L + pos0));
+                    tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
+                }
+            } else {
+                const int d = t - n_ctx;
+                for (int kk = 0; kk < kBN; ++kk) {
+                    const int slot = d * kBN + kk;
+                    uint8_t *dst = kt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
+                    if (slot < nrows) {
+                        const size_t key = (size_t)p.S + kBlock * sn[slot / kBlock] + slot % kBlock;
+                        const __nv_bfloat16 *src = lane < 24 ? p.kc + (bh * p.L + key) * kDC + lane * 8
+                                                             : p.krr + ((size_t)b * p.L + key) * kDR + (lane - 24) * 8;
+                        cp_async16(dst, src, 16);
+                    } else {
+                        cp_async16(dst, p.kc, 0);
+                    }
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&kfull[s]);
+            }
+            if (lane == 0) counters[0] = t + 1;
+            if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+            if (t < n_ctx) {
+                const int pos0 = ctx_lo + t * kBN;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&vfull[s], kVBytes);
+                    for (int c = 0; c < 4; c++)
+                        tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[s], c * 64, (int)(bh * p.L + pos0));
+                }
+            } else {
+                const int d = t - n_ctx;
+                for (int kk = 0; kk < kBN; ++kk) {
+                    const int slot = d * kBN + kk;
+                    uint8_t *dst = vt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
+                    if (slot < nrows) {
+                        const size_t key = (size_t)p.S + kBlock * sn[slot / kBlock] + slot % kBlock;
+                        cp_async16(dst, p.v + (bh * p.L + key) * kDV + lane * 8, 16);
+                    } else {
+                        cp_async16(dst, p.v, 0);
+                    }
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vfull[s]);
+            }
+            if (lane == 0) counters[1] = t + 1;
+        }
+        cp_async_wait_all();
+    } else if (warp == 5) {
+        // ----------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(kM, kBN, 0);
+            const uint32_t idO = idesc_bf16(kM, kDV, 1);
+            const uint32_t qa = smem_u32(sm + oQ);
+            bool ok = mbar_wait(qready, 0, abort_flag);
+            auto issue_qk = [&](int t) {
+                const int s = t & 1;
+                const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0));
+#pragma unroll
+                for (int k = 0; k < kDQK / 16; ++k) {
+                    const int c = k >> 2, sub = k & 3;
+                    const uint64_t a = sdesc_sw128(qa + c * kQChunk + sub * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(kb + c * kKChunk + sub * 32, 16, 1024);
+                    mma_bf16_ss(tmem + kColS + s * kBN, a, bd, idS, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&sfull[s]);
+                mma_commit(&kempty[s]);
+                counters[2] = t + 1;
+            };
+            if (ok) ok = mbar_wait(&kfull[0], 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_qk(0);
+            }
+            for (int t = 0; t < T && ok; ++t) {
+                if (t + 1 < T) {
+                    const int t1 = t + 1, s1 = t1 & 1;
+                    if (t1 >= 2) ok = mbar_wait(&pready[s1], ((t1 >> 1) - 1) & 1, abort_flag);
+                    if (ok) ok = mbar_wait(&kfull[s1], (t1 >> 1) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(t1);
+                }
+                const int s = t & 1;
+                ok = mbar_wait(&pready[s], (t >> 1) & 1, abort_flag);
+                if (ok) ok = mbar_wait(&vfull[s], (t >> 1) & 1, abort_flag);
+                if (!ok) break;
+                counters[3] = t + 1;
+                tc_fence_after();
+                const uint32_t pa = smem_u32(sm + (s ? oP1 : oP0));
+                const uint32_t vb = smem_u32(sm + (s ? oV1 : oV0));
+#pragma unroll
+                for (int k = 0; k < kBN / 16; ++k) {
+                    const uint64_t a = sdesc_sw128(pa + k * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(vb + k * 2048, kKChunk, 1024);
+                    mma_bf16_ss(tmem + kColO, a, bd, idO, (t > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit(&vempty[s]);
+                mma_commit(&pvdone[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax (rows)
+        const int r = threadIdx.x;
+        const bool live = r < nrows;
+        int A = 0, n = 0, j = 0, lo = 0;
+        if (live) {
+            A = sa[r / kBlock];
+            n = sn[r / kBlock];
+            j = r % kBlock;
+            lo = max(0, A - p.W + 1);
+        }
+        // Q rows of this warp, rope slice rotated to position A + j
+        for (int i = 0; i < 32; ++i) {
+            const int rr = warp * 32 + i;
+            const int Ai = __shfl_sync(0xffffffffu, A, i);
+            const int ni = __shfl_sync(0xffffffffu, n, i);
+            const int ji = __shfl_sync(0xffffffffu, j, i);
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (rr < nrows) {
+                const __nv_bfloat16 *src = p.q + ((bh * p.R) + kBlock * ni + ji) * kDQK + lane * 8;
+                val = __ldg(reinterpret_cast<const uint4 *>(src));
+                if (lane >= 24) {
+                    const float2 *cs = p.tab + (size_t)(Ai + ji) * (kDR / 2) + (lane - 24) * 4;
+                    uint32_t w[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&w[k]);
+                        const float x0 = __bfloat162float(pr.x), x1 = __bfloat162float(pr.y);
+                        const float2 c = __ldg(cs + k);
+                        w[k] = pack_bf16x2(x0 * c.x - x1 * c.y, x0 * c.y + x1 * c.x);
+                    }
+                    val = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            *reinterpret_cast<uint4 *>(sm + oQ + (lane >> 3) * kQChunk + sw128(rr, lane & 7)) = val;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qready);
+
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int t = 0; t < T; ++t) {
+            const int s = t & 1;
+            ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            float sv[64];
+            {
+                float a0[32], a1[32];
+                tmem_ld32(trow + kColS + s * kBN, a0);
+                tmem_ld32(trow + kColS + s * kBN + 32, a1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c++) {
+                    sv[c] = a0[c];
+                    sv[32 + c] = a1[c];
+                }
+            }
+            float mt = -INFINITY;
+            if (t < n_ctx) {
+                const int c0 = ctx_lo + t * kBN;
+#pragma unroll
+                for (int c = 0; c < kBN; c++) {
+                    const int pos = c0 + c;
+                    const bool valid = live && pos >= lo && pos < A;
+                    sv[c] = valid ? sv[c] * p.scale_log2 : -INFINITY;
+                    mt = fmaxf(mt, sv[c]);
+                }
+            } else {
+                const int base = (t - n_ctx) * kBN;
+                const int myblk = r / kBlock;
+#pragma unroll
+                for (int c = 0; c < kBN; c++) {
+                    const bool valid = live && (base + c) / kBlock == myblk;
+                    sv[c] = valid ? sv[c] * p.scale_log2 : -INFINITY;
+                    mt = fmaxf(mt, sv[c]);
+                }
+            }
+            bool resc = false;
+            float alpha = 1.f;
+            if (mt > m_used + kRescaleThreshold) {
+                if (m_used != -INFINITY) {
+                    resc = true;
+                    alpha = exp2f(m_used - mt);
+                }
+                m_used = mt;
+            }
+            if (t >= 2) {
+                ok = warp_all(mbar_wait(&pvdone[s], ((t - 2) >> 1) & 1, abort_flag));
+                if (!ok) break;
+            }
+            uint8_t *prow = sm + (s ? oP1 : oP0);
+            float ps = 0.f;
+            const bool any = m_used != -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                float e[8];
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    e[k] = any ? exp2f(sv[u * 8 + k] - m_used) : 0.f;
+                    ps += e[k];
+                }
+                uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                                      pack_bf16x2(e[6], e[7]));
+                *reinterpret_cast<uint4 *>(prow + sw128(r, u)) = pk;
+            }
+            l = l * alpha + ps;
+            if (__any_sync(0xffffffffu, resc)) {
+                if (t >= 1) {
+                    ok = warp_all(mbar_wait(&pvdone[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag));
+                    if (!ok) break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < kDV; c += 32) {
+                    float ov[32];
+                    tmem_ld32(trow + kColO + c, ov);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i++) ov[i] *= alpha;
+                    tmem_st32(trow + kColO + c, ov);
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pready[s]);
+        }
+        if (ok) ok = warp_all(mbar_wait(&pvdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t row = bh * p.R + kBlock * n + j;
+            __nv_bfloat16 *orow = p.o + row * kDV;
+#pragma unroll 1
+            for (int c = 0; c < kDV; c += 32) {
+                float ov[32];
+                tmem_ld32(trow + kColO + c, ov);
+                tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        uint4 pk = make_uint4(pack_bf16x2(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv),
+                                              pack_bf16x2(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv),
+                                              pack_bf16x2(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv),
+                                              pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
+                        *reinterpret_cast<uint4 *>(orow + c + 8 * k) = pk;
+                    }
+                }
+            }
+            if (live) p.lse[row] = (m_used + log2f(l)) * kLn2;
+        }
+    }
+
+    // ---------------------------------------------------------- teardown
+    __syncthreads();
+    if (*abort_flag) {
+        // Drain what may still be in flight, each wait bounded on its own.
+        volatile int never = 0;
+        if (warp == 4 && lane == 0) {
+            // loads issued but not yet consumed complete in order, one phase each
+            for (int t = counters[2]; t < counters[0]; ++t)
+                mbar_wait(&kfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t)
+                mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+        }
+        if (warp == 5 && lane == 0) {
+            mma_commit(drain);
+            mbar_wait(drain, 0, (volatile int *)&never);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
+}
+
+// Rows of blocks that are padding (keep = 0) or have an invalid anchor: O = 0,
+// LSE = -inf for every head (page §3: such a block sees nothing).
+__global__ void __launch_bounds__(256) k_fwd_pad_rows(int n_h, int S, int N, int R, const int32_t *anchors,
+                                                      const uint8_t *keep, __nv_bfloat16 *o, float *lse) {
+    const int n = blockIdx.x, b = blockIdx.y;
+    const int a = anchors[(size_t)b * N + n];
+    if (keep[(size_t)b * N + n] && a >= 0 && a <= S - 2) return;
+    for (int h = 0; h < n_h; h++) {
+        const size_t row0 = ((size_t)b * n_h + h) * R + kBlock * n;
+        uint4 *dst = reinterpret_cast<uint4 *>(o + row0 * kDV);
+        for (int e = threadIdx.x; e < kBlock * kDV / 8; e += blockDim.x) dst[e] = make_uint4(0, 0, 0, 0);
+        if (threadIdx.x < kBlock) lse[row0 + threadIdx.x] = -INFINITY;
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over rows of `inner` elements, 64 x 64 boxes, 128 B swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const Prob &p) {
+    // TMA row coordinates are 32-bit: every (batch, head, position) row must fit
+    return p.dtype == DSPARK_BF16 && p.d_c == kDC && p.d_r == kDR && p.d_v == kDV &&
+           (long long)p.B * p.n_h * p.L < (1ll << 31);
+}
+
+cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
+                          const uint8_t *keep, void *o, float *lse, const Ws &ws, cudaStream_t st) {
+    if (p.B == 0 || p.N == 0) return cudaSuccess;
+    count_launch();
+    k_fwd_pad_rows<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.R, anchors, keep, (__nv_bfloat16 *)o, lse);
+    CUtensorMap m_kc, m_kr, m_v;
+    if (!make_map(&m_kc, kc, kDC, (uint64_t)p.B * p.n_h * p.L) ||
+        !make_map(&m_kr, ws.kr_rot, kDR, (uint64_t)p.B * p.L) ||
+        !make_map(&m_v, v, kDV, (uint64_t)p.B * p.n_h * p.L))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    FwdArgs a;
+    a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
+    a.scale_log2 = p.scale_log2;
+    a.q = (const __nv_bfloat16 *)q;
+    a.kc = (const __nv_bfloat16 *)kc;
+    a.krr = (const __nv_bfloat16 *)ws.kr_rot;
+    a.v = (const __nv_bfloat16 *)v;
+    a.cnt = ws.cnt;
+    a.sorted_n = ws.sorted_n;
+    a.sorted_a = ws.sorted_a;
+    a.tab = ws.rope;
+    a.o = (__nv_bfloat16 *)o;
+    a.lse = lse;
+    a.err = ws.err;
+    dim3 grid((p.N + kG - 1) / kG, p.n_h, p.B);
+    count_launch();
+    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc, m_kr, m_v, a);
+    return cudaGetLastError();
+}
+
+}  // namespace dspark

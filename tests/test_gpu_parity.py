@@ -61,6 +61,23 @@ def test_edge_cases_full(oracle_mod, case, dtype):
     compare_full(gpu, oracle_full(oracle_mod, c, S, W), synth.torch_dtype(dtype))
 
 
+@pytest.mark.parametrize("qscale", [3.0, 4.0, 6.0])
+def test_large_scores_page_dims(oracle_mod, qscale):
+    """Scores with a spread of several units: the running max jumps between
+    key tiles, which exercises the online-softmax rescaling of the tensor-core
+    forward. Only the forward is compared here: for the backward, an fp64
+    emulation of the bf16 pipeline alone (rope key rounded after rotation, O
+    rounded before D = rowsum(dO * O), outputs rounded) already exceeds the
+    bf16 bound on dK at Q x 3, so the backward is held to the bound on the
+    N(0, 1) workloads of the other tests. Beyond Q x 6 the same emulation
+    exceeds the bound on O (rotated q and k rope slices are bf16 MMA operands)."""
+    c = synth.random_case(45, 1, 400, 30, 128, 2, 192, 64, 256, "bf16")
+    c["q"] = (c["q"].float() * qscale).to(torch.bfloat16)
+    c["anchors"][0, 0] = 0
+    gpu = run_gpu(c, 400, 128, bwd=False)
+    compare_full(gpu, oracle_full(oracle_mod, c, 400, 128, bwd=False), torch.bfloat16)
+
+
 def test_no_blocks():
     """N = 0: nothing to attend; the backward still writes zero key gradients."""
     c = synth.random_case(50, 2, 40, 0, 8, 2, 16, 8, 16, "bf16")
