@@ -96,8 +96,10 @@ typedef struct {
         for the same anchors, keep and sizes: skip rebuilding it. The page's
         mask is built once and shared by the three draft layers (§3, §4). */
 
-/* Bytes of device workspace needed for problem *p (0 if *p is invalid). The
- * workspace must be 256-byte aligned. */
+/* Bytes of device workspace needed for problem *p (0 if *p is invalid): the
+ * size dspark_attn_bwd requires. dspark_build_descriptor and dspark_attn_fwd
+ * use only a leading part of it, so a workspace of this size serves every
+ * entry point. The workspace must be 256-byte aligned. */
 DSPARK_API size_t dspark_workspace_size(const dspark_problem *p);
 
 /* Build the mask descriptor into the workspace: kept blocks of each batch row
@@ -128,9 +130,8 @@ DSPARK_API dspark_status dspark_attn_fwd(const dspark_problem *p, const void *q,
  *     may be NULL) receives, in stream order, the error word of this call
  *     (bit 0: a kept anchor was out of range and its block treated as padding;
  *     bit 1: a bounded device-side wait gave up).
- *   - Returns DSPARK_ERR_UNSUPPORTED when the problem needs more scratch than
- *     the array holds (dspark_workspace_size(p) > DSPARK_NOALLOC_SCRATCH_BYTES);
- *     other statuses as dspark_attn_fwd.
+ *   - Returns DSPARK_ERR_UNSUPPORTED when the forward needs more scratch than
+ *     the array holds; other statuses as dspark_attn_fwd.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make that
  *     first call before any stream capture.

@@ -48,10 +48,13 @@ bool make_prob(const dspark_problem *pp, Prob *out, dspark_status *why) {
 
 bool aligned16(const void *x) { return ((uintptr_t)x & 15u) == 0; }
 
-dspark_status check_ws(const Prob &p, void *ws, size_t bytes) {
+// need_bwd: the backward uses the whole layout, the forward and the
+// descriptor only its leading sections.
+dspark_status check_ws(const Prob &p, void *ws, size_t bytes, bool need_bwd) {
     if (!ws) return DSPARK_ERR_WORKSPACE;
     if (((uintptr_t)ws & 255u) != 0) return DSPARK_ERR_WORKSPACE;
-    if (bytes < ws_layout(p).total) return DSPARK_ERR_WORKSPACE;
+    const WsLayout l = ws_layout(p);
+    if (bytes < (need_bwd ? l.total : l.fwd_total)) return DSPARK_ERR_WORKSPACE;
     return DSPARK_OK;
 }
 
@@ -109,6 +112,17 @@ dspark_status build(const Prob &p, const int32_t *anchors, const uint8_t *keep, 
 
 }  // namespace
 
+namespace dspark {
+// Workspace bytes the forward alone needs (a prefix of the full layout); 0 if
+// the problem is invalid.
+size_t fwd_workspace_size(const dspark_problem *pp) {
+    Prob p;
+    dspark_status why;
+    if (!make_prob(pp, &p, &why)) return 0;
+    return ws_layout(p).fwd_total;
+}
+}  // namespace dspark
+
 extern "C" {
 
 size_t dspark_workspace_size(const dspark_problem *pp) {
@@ -123,7 +137,7 @@ dspark_status dspark_build_descriptor(const dspark_problem *pp, const int32_t *a
     Prob p;
     dspark_status why;
     if (!make_prob(pp, &p, &why)) return why;
-    DSPARK_TRY(check_ws(p, workspace, workspace_bytes));
+    DSPARK_TRY(check_ws(p, workspace, workspace_bytes, false));
     if ((size_t)p.B * p.N && (!anchors || !keep)) return DSPARK_ERR_NULL;
     cudaStream_t st = (cudaStream_t)stream;
     return build(p, anchors, keep, ws_view(p, workspace), st);
@@ -135,7 +149,7 @@ dspark_status dspark_attn_fwd(const dspark_problem *pp, const void *q, const voi
     Prob p;
     dspark_status why;
     if (!make_prob(pp, &p, &why)) return why;
-    DSPARK_TRY(check_ws(p, workspace, workspace_bytes));
+    DSPARK_TRY(check_ws(p, workspace, workspace_bytes, false));
     DSPARK_TRY(check_inputs(p, q, kc, kr, v, anchors, keep));
     const Sizes s = sizes(p);
     DSPARK_TRY(check_tensor(o, s.o));
@@ -158,7 +172,7 @@ dspark_status dspark_attn_bwd(const dspark_problem *pp, const void *q, const voi
     Prob p;
     dspark_status why;
     if (!make_prob(pp, &p, &why)) return why;
-    DSPARK_TRY(check_ws(p, workspace, workspace_bytes));
+    DSPARK_TRY(check_ws(p, workspace, workspace_bytes, true));
     DSPARK_TRY(check_inputs(p, q, kc, kr, v, anchors, keep));
     const Sizes s = sizes(p);
     DSPARK_TRY(check_tensor(o, s.o));
@@ -172,7 +186,10 @@ dspark_status dspark_attn_bwd(const dspark_problem *pp, const void *q, const voi
     const Ws w = ws_view(p, workspace);
     if (!(flags & DSPARK_FLAG_REUSE_DESCRIPTOR)) DSPARK_TRY(build(p, anchors, keep, w, st));
     DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, w, st));
-    DSPARK_CUDA(launch_bwd_simt(p, q, kc, v, anchors, keep, o, lse, do_, dq, dkc, dkr, dv, w, st));
+    if (bwd_tc_supported(p))
+        DSPARK_CUDA(launch_bwd_tc(p, q, kc, v, anchors, keep, o, lse, do_, dq, dkc, dkr, dv, w, st));
+    else
+        DSPARK_CUDA(launch_bwd_simt(p, q, kc, v, anchors, keep, o, lse, do_, dq, dkc, dkr, dv, w, st));
     return DSPARK_OK;
 }
 

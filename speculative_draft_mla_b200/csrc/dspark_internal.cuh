@@ -37,9 +37,19 @@ struct WsLayout {
     size_t sorted_a;  // int32 [B, N]  its anchor
     size_t rope;      // float2 [P, d_r/2] (cos, sin) of pos * base^(-2i/d_r)
     size_t kr_rot;    // dtype [B, L, d_r] rotated rope keys
+    size_t fwd_total; // the forward needs only the sections above
     size_t dvec;      // float [B, n_h, 5N] D = rowsum(dO * O)
+    // tensor-core backward only (empty otherwise)
+    size_t lses;      // float [B, n_h, 5N] LSE * log2(e), anchor-sorted rows
+    size_t qs;        // bf16 [B, n_h, 5N, 256] rotated Q, anchor-sorted rows
+    size_t dos;       // bf16 [B, n_h, 5N, 256] dO, anchor-sorted rows
+    size_t dkr_part;  // float [HG, B, L, d_r] rope-key gradient per head group
     size_t total;
 };
+
+bool bwd_tc_supported(const Prob &p);
+int bwd_head_groups(const Prob &p);
+size_t fwd_workspace_size(const dspark_problem *p);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -53,7 +63,15 @@ inline WsLayout ws_layout(const Prob &p) {
     w.sorted_a = off;  off = align256(off + sizeof(int32_t) * (size_t)p.B * p.N);
     w.rope = off;      off = align256(off + sizeof(float2) * (size_t)p.P * (p.d_r / 2));
     w.kr_rot = off;    off = align256(off + esz * (size_t)p.B * p.L * p.d_r);
+    w.fwd_total = off;
     w.dvec = off;      off = align256(off + sizeof(float) * (size_t)p.B * p.n_h * p.R);
+    const bool tc = bwd_tc_supported(p);
+    const size_t rows = tc ? (size_t)p.B * p.n_h * p.R : 0;
+    w.lses = off;      off = align256(off + sizeof(float) * rows);
+    w.qs = off;        off = align256(off + 2 * rows * p.dqk);
+    w.dos = off;       off = align256(off + 2 * rows * p.d_v);
+    w.dkr_part = off;
+    off = align256(off + (tc ? sizeof(float) * (size_t)bwd_head_groups(p) * p.B * p.L * p.d_r : 0));
     w.total = off;
     return w;
 }
@@ -65,6 +83,9 @@ struct Ws {
     float2 *rope;
     void *kr_rot;
     float *dvec;
+    float *lses;
+    void *qs, *dos;
+    float *dkr_part;
 };
 
 inline Ws ws_view(const Prob &p, void *base) {
@@ -78,6 +99,10 @@ inline Ws ws_view(const Prob &p, void *base) {
     w.rope = (float2 *)(c + l.rope);
     w.kr_rot = (void *)(c + l.kr_rot);
     w.dvec = (float *)(c + l.dvec);
+    w.lses = (float *)(c + l.lses);
+    w.qs = (void *)(c + l.qs);
+    w.dos = (void *)(c + l.dos);
+    w.dkr_part = (float *)(c + l.dkr_part);
     return w;
 }
 
@@ -106,6 +131,11 @@ cudaError_t launch_fwd_simt(const Prob &p, const void *q, const void *kc, const 
 cudaError_t launch_bwd_simt(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
                             const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,
                             void *dkc, void *dkr, void *dv, const Ws &ws, cudaStream_t st);
+
+// tcgen05 backward for bf16 at the page's head widths
+cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
+                          const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,
+                          void *dkc, void *dkr, void *dv, const Ws &ws, cudaStream_t st);
 
 // tcgen05 forward for bf16 at the page's head widths (192 + 64 / 256)
 bool fwd_tc_supported(const Prob &p);

@@ -51,7 +51,7 @@ extern "C" dspark_status dspark_attn_fwd_noalloc(const dspark_problem *p, const 
                                                  const void *kr, const void *v, const int32_t *anchors,
                                                  const uint8_t *keep, void *o, float *lse, uint32_t *error_word,
                                                  void *stream) {
-    const size_t need = dspark_workspace_size(p);
+    const size_t need = dspark::fwd_workspace_size(p);  // the forward's part of the layout
     if (need == 0) {
         // invalid problem: the regular entry point reports the precise status
         // from its host-side checks, before any device work

@@ -1,0 +1,977 @@
+// Tensor-core (tcgen05 / TMEM / TMA) backward of the DSpark draft attention for
+// the page's head widths (d_c = 192, d_r = 64, d_v = 256), bf16.
+//
+// The gradient of softmax(Q K^T s + Lambda(M)) V (appendix "Attention
+// implementation" of the "GLM 5.2 DSpark speculative-training design" page,
+// with the §3 mask) for the loss with dL/dO = dO:
+//   P = exp(S - LSE), dP = dO V^T, D = rowsum(dO * O), dS = P * (dP - D) * s,
+//   dQ = dS K, dK = dS^T Q, dV = P^T dO,
+// on rotated q and k rope slices; the rope parts of dQ and dK are rotated back,
+// and dK^R, shared by every head (§4), is the sum over heads.
+//
+// Launch sequence (one stream, no atomics, every output element written once):
+//   1. k_bwd_prep      per kept block and head: rotated Q and dO copied into
+//                      anchor-sorted row order, D, LSE*log2(e); padding rows 0.
+//   2. k_bwd_pad       zeros for padding blocks' rows and draft keys.
+//   3. k_bwd_dq_tc     query-major, one CTA per (b, h, 25 sorted blocks):
+//                      32-key tiles of the group's key set; S and dP in TMEM,
+//                      dS through shared memory, dQ += dS K in TMEM.
+//   4. k_bwd_kv_tc<V>  key-major, one CTA per (b, 128-key tile, head group):
+//      k_bwd_kv_tc<K>  rows of the blocks whose key sets meet the tile, in
+//                      chunks of 64: S^T = K Q^T (and dP^T = V dO^T) in TMEM,
+//                      P^T (dS^T) through shared memory, dV += P^T dO
+//                      (dK += dS^T Q) accumulated in TMEM over the rows. A
+//                      128-key tile's dV and dK accumulators would need all
+//                      512 TMEM columns together, so they are produced by two
+//                      CTA roles that each recompute S^T.
+//   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
+//                      them back and writes dK^R.
+// Key tiles are either context tiles [t0, t0+128) or the draft keys of one
+// group of 25 blocks; the blocks whose windows meet a context tile are a
+// contiguous run of the anchor-sorted list (t0 < A <= t0 + 127 + W - 1).
+#include <algorithm>
+
+#include "dspark_tc_common.cuh"
+
+namespace dspark {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
+constexpr int kG = 25;  // blocks per query group
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ prep
+// One warp per row of a kept block (5 warps): rotated q -> qs, do -> dos,
+// D = rowsum(dO * O), LSE * log2(e); rows past the kept blocks are zeroed so
+// tiles that overhang them multiply finite values.
+__global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfloat16 *__restrict__ q,
+                                                  const __nv_bfloat16 *__restrict__ o,
+                                                  const __nv_bfloat16 *__restrict__ dout,
+                                                  const float *__restrict__ lse, const int32_t *__restrict__ cnt,
+                                                  const int32_t *__restrict__ sorted_n,
+                                                  const int32_t *__restrict__ sorted_a,
+                                                  const float2 *__restrict__ tab, __nv_bfloat16 *__restrict__ qs,
+                                                  __nv_bfloat16 *__restrict__ dos, float *__restrict__ ds_,
+                                                  float *__restrict__ lses) {
+    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int R = kBlock * N;
+    const size_t bh = (size_t)b * n_h + h;
+    const size_t srow = bh * R + kBlock * i + j;
+    uint4 *qd = reinterpret_cast<uint4 *>(qs + srow * kDQK) + lane;
+    uint4 *dd = reinterpret_cast<uint4 *>(dos + srow * kDV) + lane;
+    if (i >= cnt[b]) {
+        *qd = make_uint4(0, 0, 0, 0);
+        *dd = make_uint4(0, 0, 0, 0);
+        if (lane == 0) {
+            ds_[srow] = 0.f;
+            lses[srow] = 0.f;
+        }
+        return;
+    }
+    const int n = sorted_n[(size_t)b * N + i], a = sorted_a[(size_t)b * N + i];
+    const size_t orow = bh * R + kBlock * n + j;
+    uint4 qv = __ldg(reinterpret_cast<const uint4 *>(q + orow * kDQK) + lane);
+    if (lane >= 24) {
+        const float2 *cs = tab + (size_t)(a + j) * (kDR / 2) + (lane - 24) * 4;
+        uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&w[k]);
+            const float x0 = __bfloat162float(pr.x), x1 = __bfloat162float(pr.y);
+            const float2 c = __ldg(cs + k);
+            w[k] = pack_bf16x2(x0 * c.x - x1 * c.y, x0 * c.y + x1 * c.x);
+        }
+        qv = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *qd = qv;
+    const uint4 dv = __ldg(reinterpret_cast<const uint4 *>(dout + orow * kDV) + lane);
+    const uint4 ov = __ldg(reinterpret_cast<const uint4 *>(o + orow * kDV) + lane);
+    *dd = dv;
+    const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&dw[k]);
+        const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162 *>(&ow[k]);
+        acc = fmaf(__bfloat162float(x.x), __bfloat162float(y.x), acc);
+        acc = fmaf(__bfloat162float(x.y), __bfloat162float(y.y), acc);
+    }
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        ds_[srow] = acc;
+        lses[srow] = lse[orow] * kLog2e;
+    }
+}
+
+// -------------------------------------------------------------- padding
+// Padding blocks (keep = 0 or invalid anchor): dq rows and the block's own
+// draft keys' dkc / dv get zeros (their dkr is zeroed by the reduction).
+__global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, const int32_t *anchors,
+                                                 const uint8_t *keep, __nv_bfloat16 *dq, __nv_bfloat16 *dkc,
+                                                 __nv_bfloat16 *dv) {
+    const int n = blockIdx.x, b = blockIdx.y;
+    const int a = anchors[(size_t)b * N + n];
+    if (keep[(size_t)b * N + n] && a >= 0 && a <= S - 2) return;
+    const int R = kBlock * N;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int h = 0; h < n_h; h++) {
+        const size_t bh = (size_t)b * n_h + h;
+        uint4 *q4 = reinterpret_cast<uint4 *>(dq + (bh * R + kBlock * n) * kDQK);
+        uint4 *k4 = reinterpret_cast<uint4 *>(dkc + (bh * L + S + kBlock * n) * kDC);
+        uint4 *v4 = reinterpret_cast<uint4 *>(dv + (bh * L + S + kBlock * n) * kDV);
+        for (int e = threadIdx.x; e < kBlock * kDQK / 8; e += blockDim.x) q4[e] = z;
+        for (int e = threadIdx.x; e < kBlock * kDC / 8; e += blockDim.x) k4[e] = z;
+        for (int e = threadIdx.x; e < kBlock * kDV / 8; e += blockDim.x) v4[e] = z;
+    }
+}
+
+// ================================================================ dQ
+// CTA = (group g of 25 sorted blocks, head h, batch b); warps 0-3 rows
+// (thread t = row t = TMEM lane t), warp 4 producer, warp 5 MMA.
+namespace dq {
+constexpr int kM = 128, kBN = 32;
+constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
+constexpr int kKChunk = kBN * 128;     // 4 KB: 32 keys x 64 columns
+constexpr int kTile = 4 * kKChunk;     // 16 KB
+constexpr int oQ = 0, oDO = oQ + 4 * kQChunk, oK0 = oDO + 4 * kQChunk, oK1 = oK0 + kTile, oV0 = oK1 + kTile,
+              oV1 = oV0 + kTile, oS0 = oV1 + kTile, oS1 = oS0 + kQChunk, oBar = oS1 + kQChunk;
+constexpr int kSmem = oBar + 256 + 1024;
+constexpr int kThreads = 192;
+constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320;  // S: 256/288, dP: 320/352
+}  // namespace dq
+
+struct BwdArgs {
+    int n_h, S, N, W, L, R;
+    float scale_log2, scale;
+    const __nv_bfloat16 *kc, *krr, *v;
+    const __nv_bfloat16 *qs, *dos;
+    const float *ds_, *lses;
+    const int32_t *cnt, *sorted_n, *sorted_a;
+    const float2 *tab;
+    __nv_bfloat16 *dq, *dkc, *dv;
+    float *dkr_part;
+    int hpg;  // heads per head group (key-major kernel)
+    int n_ctx_items;
+    uint32_t *err;
+};
+
+__global__ void __launch_bounds__(dq::kThreads, 1)
+    k_bwd_dq_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
+                const __grid_constant__ CUtensorMap tm_dos, const BwdArgs p) {
+    using namespace dq;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
+    uint64_t *kfull = bars + 0, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
+    uint64_t *sfull = bars + 8, *dsready = bars + 10, *dqdone = bars + 12, *qfull = bars + 14, *drain = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+    int *counters = reinterpret_cast<int *>(bars + 18);  // K issued, V issued, K consumed, V consumed, q issued
+
+    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int cnt = p.cnt[b];
+    const int i0 = g * kG;
+    if (i0 >= cnt) return;
+    const int gcnt = min(kG, cnt - i0);
+    const int nrows = kBlock * gcnt;
+    const int32_t *sa = p.sorted_a + (size_t)b * p.N + i0;
+    const int32_t *sn = p.sorted_n + (size_t)b * p.N + i0;
+    const int ctx_lo = max(0, sa[0] - p.W + 1);
+    const int ctx_hi = sa[gcnt - 1];
+    const int n_ctx = ctx_hi > ctx_lo ? (ctx_hi - ctx_lo + kBN - 1) / kBN : 0;
+    const int n_draft = (nrows + kBN - 1) / kBN;
+    const int T = n_ctx + n_draft;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t bh = (size_t)b * p.n_h + h;
+    const size_t srow0 = bh * p.R + (size_t)kBlock * i0;  // first sorted row of the group
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
+            mbar_init(&sfull[s], 1);
+            mbar_init(&dsready[s], 4);
+            mbar_init(&dqdone[s], 1);
+        }
+        mbar_init(qfull, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        for (int c = 0; c < 5; c++) counters[c] = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(qfull, 8 * kQChunk);
+            for (int c = 0; c < 4; c++) {
+                tma_load_2d(sm + oQ + c * kQChunk, &tm_qs, qfull, c * 64, (int)srow0);
+                tma_load_2d(sm + oDO + c * kQChunk, &tm_dos, qfull, c * 64, (int)srow0);
+            }
+            counters[4] = 1;
+        }
+        // lane l holds the block index of group block l (l < gcnt)
+        const int my_n = lane < gcnt ? sn[lane] : 0;
+        for (int t = 0; t < T; ++t) {
+            const int s = t & 1;
+            uint8_t *kt = sm + (s ? oK1 : oK0);
+            uint8_t *vt = sm + (s ? oV1 : oV0);
+            if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+            if (t < n_ctx) {
+                const int pos0 = ctx_lo + t * kBN;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&kfull[s], kTile);
+                    for (int c = 0; c < 3; c++)
+                        tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[s], c * 64, (int)(bh * p.L + pos0));
+                    tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
+                }
+            } else {
+                const int d = t - n_ctx;
+                for (int kk = 0; kk < kBN; ++kk) {
+                    const int slot = d * kBN + kk;
+                    const int nb = __shfl_sync(0xffffffffu, my_n, min(slot / kBlock, kG - 1));
+                    uint8_t *dst = kt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
+                    if (slot < nrows) {
+                        const size_t key = (size_t)p.S + kBlock * nb + slot % kBlock;
+                        const __nv_bfloat16 *src = lane < 24 ? p.kc + (bh * p.L + key) * kDC + lane * 8
+                                                             : p.krr + ((size_t)b * p.L + key) * kDR + (lane - 24) * 8;
+                        cp_async16(dst, src, 16);
+                    } else {
+                        cp_async16(dst, p.kc, 0);
+                    }
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&kfull[s]);
+            }
+            if (lane == 0) counters[0] = t + 1;
+            if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+            if (t < n_ctx) {
+                const int pos0 = ctx_lo + t * kBN;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&vfull[s], kTile);
+                    for (int c = 0; c < 4; c++)
+                        tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[s], c * 64, (int)(bh * p.L + pos0));
+                }
+            } else {
+                const int d = t - n_ctx;
+                for (int kk = 0; kk < kBN; ++kk) {
+                    const int slot = d * kBN + kk;
+                    const int nb = __shfl_sync(0xffffffffu, my_n, min(slot / kBlock, kG - 1));
+                    uint8_t *dst = vt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
+                    if (slot < nrows) {
+                        const size_t key = (size_t)p.S + kBlock * nb + slot % kBlock;
+                        cp_async16(dst, p.v + (bh * p.L + key) * kDV + lane * 8, 16);
+                    } else {
+                        cp_async16(dst, p.v, 0);
+                    }
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vfull[s]);
+            }
+            if (lane == 0) counters[1] = t + 1;
+        }
+        cp_async_wait_all();
+    } else if (warp == 5) {
+        // ----------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(kM, kBN, 0);    // S, dP: B = K / V tile, K-major
+            const uint32_t idQ = idesc_bf16(kM, kDQK, 1);   // dQ: B = K tile, MN-major
+            const uint32_t qa = smem_u32(sm + oQ), da = smem_u32(sm + oDO);
+            bool ok = mbar_wait(qfull, 0, abort_flag);
+            auto issue_sdp = [&](int t) {
+                const int s = t & 1;
+                const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0)), vb = smem_u32(sm + (s ? oV1 : oV0));
+#pragma unroll
+                for (int k = 0; k < kDQK / 16; ++k) {
+                    const int c = k >> 2, sub = k & 3;
+                    mma_bf16_ss(tmem + kColS + s * kBN, sdesc_sw128(qa + c * kQChunk + sub * 32, 16, 1024),
+                                sdesc_sw128(kb + c * kKChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int k = 0; k < kDV / 16; ++k) {
+                    const int c = k >> 2, sub = k & 3;
+                    mma_bf16_ss(tmem + kColP + s * kBN, sdesc_sw128(da + c * kQChunk + sub * 32, 16, 1024),
+                                sdesc_sw128(vb + c * kKChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&sfull[s]);
+                mma_commit(&vempty[s]);
+            };
+            auto wait_kv = [&](int t) {
+                const int s = t & 1;
+                bool r = mbar_wait(&kfull[s], (t >> 1) & 1, abort_flag);
+                if (r) r = mbar_wait(&vfull[s], (t >> 1) & 1, abort_flag);
+                if (r) {
+                    counters[2] = t + 1;
+                    counters[3] = t + 1;
+                }
+                return r;
+            };
+            if (ok) ok = wait_kv(0);
+            if (ok) {
+                tc_fence_after();
+                issue_sdp(0);
+            }
+            for (int t = 0; t < T && ok; ++t) {
+                if (t + 1 < T) {
+                    const int t1 = t + 1, s1 = t1 & 1;
+                    if (t1 >= 2) ok = mbar_wait(&dsready[s1], ((t1 >> 1) - 1) & 1, abort_flag);
+                    if (ok) ok = wait_kv(t1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_sdp(t1);
+                }
+                const int s = t & 1;
+                ok = mbar_wait(&dsready[s], (t >> 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t dsa = smem_u32(sm + (s ? oS1 : oS0));
+                const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0));
+#pragma unroll
+                for (int k = 0; k < kBN / 16; ++k)
+                    mma_bf16_ss(tmem + kColDQ, sdesc_sw128(dsa + k * 32, 16, 1024),
+                                sdesc_sw128(kb + k * 2048, kKChunk, 1024), idQ, (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&kempty[s]);
+                mma_commit(&dqdone[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------ rows (warps 0-3)
+        const int r = threadIdx.x;
+        const bool live = r < nrows;
+        int A = 0, n = 0, j = 0, lo = 0;
+        float lse2 = 0.f, Dr = 0.f;
+        if (live) {
+            A = sa[r / kBlock];
+            n = sn[r / kBlock];
+            j = r % kBlock;
+            lo = max(0, A - p.W + 1);
+            lse2 = p.lses[srow0 + r];
+            Dr = p.ds_[srow0 + r];
+        }
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        bool ok = true;
+        for (int t = 0; t < T; ++t) {
+            const int s = t & 1;
+            ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            float sv[32], pv[32];
+            tmem_ld32(trow + kColS + s * kBN, sv);
+            tmem_ld32(trow + kColP + s * kBN, pv);
+            tmem_wait_ld();
+            if (t >= 2) {
+                ok = warp_all(mbar_wait(&dqdone[s], ((t - 2) >> 1) & 1, abort_flag));
+                if (!ok) break;
+            }
+            uint8_t *drow = sm + (s ? oS1 : oS0);
+            const bool ctx = t < n_ctx;
+            const int c0 = ctx ? ctx_lo + t * kBN : (t - n_ctx) * kBN;
+            const int myblk = r / kBlock;
+#pragma unroll
+            for (int u = 0; u < kBN / 8; u++) {
+                float e[8];
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    const int c = u * 8 + k;
+                    const bool valid = live && (ctx ? (c0 + c >= lo && c0 + c < A) : ((c0 + c) / kBlock == myblk));
+                    const float pp = valid ? exp2f(sv[c] * p.scale_log2 - lse2) : 0.f;
+                    e[k] = pp * (pv[c] - Dr) * p.scale;
+                }
+                *reinterpret_cast<uint4 *>(drow + sw128(r, u)) =
+                    make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                               pack_bf16x2(e[6], e[7]));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dsready[s]);
+        }
+        if (ok) ok = warp_all(mbar_wait(&dqdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            __nv_bfloat16 *orow = p.dq + (bh * p.R + kBlock * n + j) * kDQK;
+#pragma unroll 1
+            for (int c = 0; c < kDQK; c += 32) {
+                float v[32];
+                tmem_ld32(trow + kColDQ + c, v);
+                tmem_wait_ld();
+                if (c >= kDC) {  // rope slice: rotate back by the query position A + j
+                    const float2 *cs = p.tab + (size_t)(A + j) * (kDR / 2) + (c - kDC) / 2;
+#pragma unroll
+                    for (int k = 0; k < 16; k++) {
+                        const float2 t2 = live ? __ldg(cs + k) : make_float2(1.f, 0.f);
+                        const float x0 = v[2 * k], x1 = v[2 * k + 1];
+                        v[2 * k] = x0 * t2.x + x1 * t2.y;
+                        v[2 * k + 1] = x1 * t2.x - x0 * t2.y;
+                    }
+                }
+                if (live) {
+#pragma unroll
+                    for (int k = 0; k < 4; k++)
+                        *reinterpret_cast<uint4 *>(orow + c + 8 * k) = make_uint4(
+                            pack_bf16x2(v[8 * k + 0], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                            pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        volatile int never = 0;
+        if (warp == 4 && lane == 0) {
+            if (counters[4]) mbar_wait(qfull, 0, (volatile int *)&never);
+            for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(&kfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+        }
+        if (warp == 5 && lane == 0) {
+            mma_commit(drain);
+            mbar_wait(drain, 0, (volatile int *)&never);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
+}
+
+// ============================================================== dK / dV
+namespace kv {
+constexpr int kMK = 128;                 // keys per tile (MMA M)
+constexpr int kRC = 64;                  // rows per chunk (MMA N of S^T)
+constexpr int kKChunk = kMK * 128;       // 16 KB: 128 keys x 64 columns
+constexpr int kRChunk = kRC * 128;       // 8 KB: 64 rows x 64 columns
+constexpr int oK = 0, oV = oK + 4 * kKChunk, oQ = oV + 4 * kKChunk, oDO = oQ + 4 * kRChunk,
+              oPT = oDO + 4 * kRChunk, oMeta = oPT + kKChunk, oBar = oMeta + 3 * kRC * 4;
+constexpr int kSmem = oBar + 256 + 1024;
+constexpr int kThreads = 192;
+constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320;
+}  // namespace kv
+
+template <bool ROLE_K>
+__global__ void __launch_bounds__(kv::kThreads, 1)
+    k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
+                const __grid_constant__ CUtensorMap tm_dos, const BwdArgs p) {
+    using namespace kv;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
+    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *chfull = bars + 2, *chfree = bars + 3, *sfull = bars + 4;
+    uint64_t *dsready = bars + 5, *accdone = bars + 6, *epidone = bars + 7, *drain = bars + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 10);
+    int *counters = reinterpret_cast<int *>(bars + 11);  // kv issued, ch issued, kv consumed, ch consumed
+    int *band = reinterpret_cast<int *>(bars + 14);      // first sorted row, row count
+    float *mlse = reinterpret_cast<float *>(sm + oMeta);
+    float *mD = mlse + kRC;
+    int *mA = reinterpret_cast<int *>(mD + kRC);
+
+    const int item = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cnt = p.cnt[b];
+    const bool is_ctx = item < p.n_ctx_items;
+    int t0 = 0, gcnt = 0, i0 = 0;
+    if (is_ctx) {
+        t0 = item * kMK;
+    } else {
+        i0 = (item - p.n_ctx_items) * kG;
+        if (i0 >= cnt) return;  // uniform: fewer groups in this batch row
+        gcnt = min(kG, cnt - i0);
+    }
+    const int32_t *sa = p.sorted_a + (size_t)b * p.N;
+    const int32_t *sn = p.sorted_n + (size_t)b * p.N;
+    if (threadIdx.x == 0) {
+        int r0, nr;
+        if (is_ctx) {
+            // blocks with t0 < A <= t0 + kMK - 1 + W - 1
+            int lo = 0, hi = cnt;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (sa[mid] > t0) hi = mid; else lo = mid + 1;
+            }
+            const long long lim = (long long)t0 + kMK - 1 + p.W - 1;
+            int lo2 = lo, hi2 = cnt;
+            while (lo2 < hi2) {
+                const int mid = (lo2 + hi2) >> 1;
+                if ((long long)sa[mid] > lim) hi2 = mid; else lo2 = mid + 1;
+            }
+            r0 = kBlock * lo;
+            nr = kBlock * (lo2 - lo);
+        } else {
+            r0 = kBlock * i0;
+            nr = kBlock * gcnt;
+        }
+        band[0] = r0;
+        band[1] = nr;
+    }
+    __syncthreads();
+    const int row0 = band[0], nrows = band[1];
+    const int nchunks = (nrows + kRC - 1) / kRC;
+    const int h0 = hg * p.hpg;
+    // the tile's keys that this CTA writes: context keys below S, or the
+    // draft keys of the group's blocks
+    const int key_local = threadIdx.x;  // for warps 0-3
+    bool key_valid = false;
+    size_t key_pos = 0;
+    if (warp < 4) {
+        if (is_ctx) {
+            key_valid = t0 + key_local < p.S;
+            key_pos = (size_t)t0 + key_local;
+        } else {
+            key_valid = key_local < kBlock * gcnt;
+            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + key_local / kBlock] + key_local % kBlock;
+        }
+    }
+
+    if (nrows == 0) {
+        // no row sees these keys: zero gradients for every head of the group
+        if (warp < 4 && key_valid) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            for (int hh = 0; hh < p.hpg; hh++) {
+                const size_t bh = (size_t)b * p.n_h + h0 + hh;
+                if (ROLE_K) {
+                    uint4 *d = reinterpret_cast<uint4 *>(p.dkc + (bh * p.L + key_pos) * kDC);
+                    for (int e = 0; e < kDC / 8; e++) d[e] = z;
+                } else {
+                    uint4 *d = reinterpret_cast<uint4 *>(p.dv + (bh * p.L + key_pos) * kDV);
+                    for (int e = 0; e < kDV / 8; e++) d[e] = z;
+                }
+            }
+            if (ROLE_K) {
+                float4 *d = reinterpret_cast<float4 *>(p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR);
+                for (int e = 0; e < kDR / 4; e++) d[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        return;
+    }
+
+    if (threadIdx.x == 0) {
+        mbar_init(kvfull, 1);
+        mbar_init(kvfree, 1);
+        mbar_init(chfull, 1);
+        mbar_init(chfree, 1);
+        mbar_init(sfull, 1);
+        mbar_init(dsready, 4);
+        mbar_init(accdone, 1);
+        mbar_init(epidone, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        for (int c = 0; c < 4; c++) counters[c] = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int H = p.hpg;
+
+    if (warp == 4) {
+        // ------------------------------------------------------- producer
+        const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
+        int q = 0;  // chunk counter over all heads
+        bool ok = true;
+        for (int hh = 0; hh < H && ok; ++hh) {
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+            if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
+            // K tile (and V tile for dK)
+            if (is_ctx) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(kvfull, (ROLE_K ? 8 : 4) * kKChunk);
+                    for (int c = 0; c < 3; c++)
+                        tma_load_2d(sm + oK + c * kKChunk, &tm_kc, kvfull, c * 64, (int)(bh * p.L + t0));
+                    tma_load_2d(sm + oK + 3 * kKChunk, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
+                    if (ROLE_K)
+                        for (int c = 0; c < 4; c++)
+                            tma_load_2d(sm + oV + c * kKChunk, &tm_v, kvfull, c * 64, (int)(bh * p.L + t0));
+                }
+            } else {
+                for (int kk = 0; kk < kMK; ++kk) {
+                    const int nb = __shfl_sync(0xffffffffu, my_n, min(kk / kBlock, kG - 1));
+                    const bool in = kk < kBlock * gcnt;
+                    const size_t key = (size_t)p.S + kBlock * nb + kk % kBlock;
+                    const __nv_bfloat16 *src = lane < 24 ? p.kc + (bh * p.L + key) * kDC + lane * 8
+                                                         : p.krr + ((size_t)b * p.L + key) * kDR + (lane - 24) * 8;
+                    cp_async16(sm + oK + (lane >> 3) * kKChunk + sw128(kk, lane & 7), in ? src : (const void *)p.kc,
+                               in ? 16u : 0u);
+                    if (ROLE_K)
+                        cp_async16(sm + oV + (lane >> 3) * kKChunk + sw128(kk, lane & 7),
+                                   in ? (const void *)(p.v + (bh * p.L + key) * kDV + lane * 8) : (const void *)p.v,
+                                   in ? 16u : 0u);
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(kvfull);
+            }
+            if (lane == 0) counters[0] = hh + 1;
+            for (int c = 0; c < nchunks; ++c, ++q) {
+                if (q >= 1 && !warp_all(mbar_wait(chfree, (q - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                const int r0 = row0 + c * kRC;
+                // per-row metadata of the chunk
+                for (int rr = lane; rr < kRC; rr += 32) {
+                    const int rowi = r0 + rr;
+                    const bool in = rowi < row0 + nrows;
+                    mA[rr] = in ? sa[rowi / kBlock] : -1;
+                    mlse[rr] = in ? p.lses[bh * p.R + rowi] : 0.f;
+                    mD[rr] = in ? p.ds_[bh * p.R + rowi] : 0.f;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(chfull, 8 * kRChunk);
+                    for (int cc = 0; cc < 4; cc++) {
+                        tma_load_2d(sm + oQ + cc * kRChunk, &tm_qs, chfull, cc * 64, (int)(bh * p.R + r0));
+                        tma_load_2d(sm + oDO + cc * kRChunk, &tm_dos, chfull, cc * 64, (int)(bh * p.R + r0));
+                    }
+                    counters[1] = q + 1;
+                }
+            }
+        }
+        cp_async_wait_all();
+    } else if (warp == 5) {
+        // ----------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(kMK, kRC, 0);    // S^T, dP^T: B = Q / dO chunk, K-major
+            const uint32_t idA = idesc_bf16(kMK, 256, 1);    // acc: B = dO / Q chunk, MN-major
+            const uint32_t ka = smem_u32(sm + oK), va = smem_u32(sm + oV);
+            const uint32_t qb = smem_u32(sm + oQ), db = smem_u32(sm + oDO), pa = smem_u32(sm + oPT);
+            int q = 0;
+            bool ok = true;
+            for (int hh = 0; hh < H && ok; ++hh) {
+                ok = mbar_wait(kvfull, hh & 1, abort_flag);
+                if (!ok) break;
+                counters[2] = hh + 1;
+                for (int c = 0; c < nchunks; ++c, ++q) {
+                    ok = mbar_wait(chfull, q & 1, abort_flag);
+                    if (!ok) break;
+                    counters[3] = q + 1;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kDQK / 16; ++k) {
+                        const int cc = k >> 2, sub = k & 3;
+                        mma_bf16_ss(tmem + kColS, sdesc_sw128(ka + cc * kKChunk + sub * 32, 16, 1024),
+                                    sdesc_sw128(qb + cc * kRChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+                    }
+                    if (ROLE_K) {
+#pragma unroll
+                        for (int k = 0; k < kDV / 16; ++k) {
+                            const int cc = k >> 2, sub = k & 3;
+                            mma_bf16_ss(tmem + kColP, sdesc_sw128(va + cc * kKChunk + sub * 32, 16, 1024),
+                                        sdesc_sw128(db + cc * kRChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(sfull);
+                    if (c == nchunks - 1) mma_commit(kvfree);
+                    ok = mbar_wait(dsready, q & 1, abort_flag);
+                    if (ok && c == 0 && hh >= 1) ok = mbar_wait(epidone, (hh - 1) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t bsrc = ROLE_K ? qb : db;
+#pragma unroll
+                    for (int k = 0; k < kRC / 16; ++k)
+                        mma_bf16_ss(tmem + kColAcc, sdesc_sw128(pa + k * 32, 16, 1024),
+                                    sdesc_sw128(bsrc + k * 2048, kRChunk, 1024), idA, (c > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(chfree);
+                    if (c == nchunks - 1) mma_commit(accdone);
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ keys (warps 0-3)
+        const int k = threadIdx.x;  // key slot = TMEM lane
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        float racc[kDR];
+#pragma unroll
+        for (int i = 0; i < kDR; i++) racc[i] = 0.f;
+        int q = 0;
+        bool ok = true;
+        const int kpos = t0 + k;                     // context position of this key (context tiles)
+        const int kblk = is_ctx ? 0 : k / kBlock;    // draft tiles: the key's block within the group
+        for (int hh = 0; hh < H && ok; ++hh) {
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+            for (int c = 0; c < nchunks; ++c, ++q) {
+                // chunk q's row metadata (written by the producer) and its S^T
+                ok = warp_all(mbar_wait(chfull, q & 1, abort_flag));
+                if (ok) ok = warp_all(mbar_wait(sfull, q & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                float sv[64];
+                float pv[ROLE_K ? 64 : 1];
+                {
+                    float a0[32], a1[32];
+                    tmem_ld32(trow + kColS, a0);
+                    tmem_ld32(trow + kColS + 32, a1);
+                    if (ROLE_K) {
+                        float b0[32], b1[32];
+                        tmem_ld32(trow + kColP, b0);
+                        tmem_ld32(trow + kColP + 32, b1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; i++) {
+                            pv[i] = b0[i];
+                            pv[32 + i] = b1[i];
+                        }
+                    } else {
+                        tmem_wait_ld();
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; i++) {
+                        sv[i] = a0[i];
+                        sv[32 + i] = a1[i];
+                    }
+                }
+                if (q >= 1) {
+                    ok = warp_all(mbar_wait(chfree, (q - 1) & 1, abort_flag));
+                    if (!ok) break;
+                }
+                const int crow0 = row0 + c * kRC;  // sorted row of column 0
+                uint8_t *prow = sm + oPT;
+#pragma unroll
+                for (int u = 0; u < kRC / 8; u++) {
+                    float e[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        const int col = u * 8 + i;
+                        const int A = mA[col];
+                        bool valid;
+                        if (is_ctx)
+                            valid = A >= 0 && kpos < A && kpos >= A - p.W + 1;
+                        else
+                            valid = A >= 0 && key_valid && (crow0 + col - row0) / kBlock == kblk;
+                        const float pp = valid ? exp2f(sv[col] * p.scale_log2 - mlse[col]) : 0.f;
+                        if (ROLE_K)
+                            e[i] = pp * (pv[col] - mD[col]) * p.scale;
+                        else
+                            e[i] = pp;
+                    }
+                    *reinterpret_cast<uint4 *>(prow + sw128(k, u)) =
+                        make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                                   pack_bf16x2(e[6], e[7]));
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dsready);
+            }
+            if (!ok) break;
+            // head epilogue: the accumulator holds dV (dK) of this head's keys
+            ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int out_cols = ROLE_K ? kDC : kDV;
+#pragma unroll 1
+            for (int c = 0; c < out_cols; c += 32) {
+                float v[32];
+                tmem_ld32(trow + kColAcc + c, v);
+                tmem_wait_ld();
+                if (key_valid) {
+                    __nv_bfloat16 *dst = ROLE_K ? p.dkc + (bh * p.L + key_pos) * kDC + c
+                                                : p.dv + (bh * p.L + key_pos) * kDV + c;
+#pragma unroll
+                    for (int i = 0; i < 4; i++)
+                        *reinterpret_cast<uint4 *>(dst + 8 * i) = make_uint4(
+                            pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                            pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                }
+            }
+            if (ROLE_K) {  // rope slice of dK: summed over the group's heads
+                float v0[32], v1[32];
+                tmem_ld32(trow + kColAcc + kDC, v0);
+                tmem_ld32(trow + kColAcc + kDC + 32, v1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    racc[i] += v0[i];
+                    racc[32 + i] += v1[i];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epidone);
+        }
+        if (ok && ROLE_K && key_valid) {
+            float4 *d = reinterpret_cast<float4 *>(p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR);
+#pragma unroll
+            for (int i = 0; i < kDR / 4; i++) d[i] = make_float4(racc[4 * i], racc[4 * i + 1], racc[4 * i + 2], racc[4 * i + 3]);
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        volatile int never = 0;
+        if (warp == 4 && lane == 0) {
+            for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(kvfull, t & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(chfull, t & 1, (volatile int *)&never);
+        }
+        if (warp == 5 && lane == 0) {
+            mma_commit(drain);
+            mbar_wait(drain, 0, (volatile int *)&never);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
+}
+
+// ------------------------------------------------------------ dK^R reduce
+// One warp per (b, key): sum the head-group partials (rotated frame), rotate
+// back by the key's position, write dkr. Draft keys of padding blocks: 0.
+__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int L, int HG,
+                                                        const int32_t *anchors, const uint8_t *keep,
+                                                        const float2 *tab, const float *part,
+                                                        __nv_bfloat16 *dkr) {
+    const size_t wid = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (wid >= (size_t)B * L) return;
+    const int b = (int)(wid / L), key = (int)(wid % L);
+    int pos = key;
+    bool live = true;
+    if (key >= S) {
+        const int n = (key - S) / kBlock, i = (key - S) % kBlock;
+        const int a = anchors[(size_t)b * N + n];
+        live = keep[(size_t)b * N + n] && a >= 0 && a <= S - 2;
+        pos = a + i;
+    }
+    float x0 = 0.f, x1 = 0.f;
+    if (live) {
+        for (int g = 0; g < HG; g++) {
+            const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
+            x0 += v.x;
+            x1 += v.y;
+        }
+        const float2 cs = tab[(size_t)pos * (kDR / 2) + lane];
+        const float y0 = x0 * cs.x + x1 * cs.y, y1 = x1 * cs.x - x0 * cs.y;
+        x0 = y0;
+        x1 = y1;
+    }
+    *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const Prob &p) {
+    return p.dtype == DSPARK_BF16 && p.d_c == kDC && p.d_r == kDR && p.d_v == kDV &&
+           (long long)p.B * p.n_h * p.L < (1ll << 31) && (long long)p.B * p.n_h * p.R < (1ll << 31);
+}
+
+int bwd_head_groups(const Prob &p) {
+    const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kG - 1) / kG) * p.B;
+    int hg = 1;
+    while (hg < p.n_h && items * hg < 2 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
+    return hg;
+}
+
+cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
+                          const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,
+                          void *dkc, void *dkr, void *dv, const Ws &ws, cudaStream_t st) {
+    if (p.B == 0) return cudaSuccess;
+    const int HG = bwd_head_groups(p);
+    if (p.N > 0) {
+        count_launch();
+        k_bwd_prep<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(
+            p.n_h, p.N, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dout, lse, ws.cnt,
+            ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs, (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses);
+        count_launch();
+        k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
+                                                   (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
+    }
+    CUtensorMap m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs64, m_dos64;
+    const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
+    const void *qs = ws.qs, *dos = ws.dos;
+    if (p.N > 0 && q_rows > 0) {
+        if (!make_map_bf16(&m_kc32, kc, kDC, kv_rows, 32) || !make_map_bf16(&m_kr32, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 32) ||
+            !make_map_bf16(&m_v32, v, kDV, kv_rows, 32) || !make_map_bf16(&m_qs128, qs, kDQK, q_rows, 128) ||
+            !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map_bf16(&m_qs64, qs, kDQK, q_rows, 64) ||
+            !make_map_bf16(&m_dos64, dos, kDV, q_rows, 64))
+            return cudaErrorInvalidValue;
+    }
+    if (!make_map_bf16(&m_kc128, kc, kDC, kv_rows, 128) ||
+        !make_map_bf16(&m_kr128, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 128) ||
+        !make_map_bf16(&m_v128, v, kDV, kv_rows, 128))
+        return cudaErrorInvalidValue;
+    if (p.N == 0 || q_rows == 0) {  // maps over Q rows are never read: any valid map will do
+        m_qs64 = m_kc128;
+        m_dos64 = m_kc128;
+    }
+    BwdArgs a;
+    a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
+    a.scale_log2 = p.scale_log2;
+    a.scale = p.scale;
+    a.kc = (const __nv_bfloat16 *)kc;
+    a.krr = (const __nv_bfloat16 *)ws.kr_rot;
+    a.v = (const __nv_bfloat16 *)v;
+    a.qs = (const __nv_bfloat16 *)ws.qs;
+    a.dos = (const __nv_bfloat16 *)ws.dos;
+    a.ds_ = ws.dvec;
+    a.lses = ws.lses;
+    a.cnt = ws.cnt;
+    a.sorted_n = ws.sorted_n;
+    a.sorted_a = ws.sorted_a;
+    a.tab = ws.rope;
+    a.dq = (__nv_bfloat16 *)dq;
+    a.dkc = (__nv_bfloat16 *)dkc;
+    a.dv = (__nv_bfloat16 *)dv;
+    a.dkr_part = ws.dkr_part;
+    a.hpg = p.n_h / HG;
+    a.n_ctx_items = (p.S + kv::kMK - 1) / kv::kMK;
+    a.err = ws.err;
+    cudaError_t e;
+    if (p.N > 0) {
+        e = cudaFuncSetAttribute(k_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::kSmem);
+        if (e != cudaSuccess) return e;
+        count_launch();
+        k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
+            m_kc32, m_kr32, m_v32, m_qs128, m_dos128, a);
+    }
+    const dim3 kv_grid(a.n_ctx_items + (p.N + kG - 1) / kG, HG, p.B);
+    e = cudaFuncSetAttribute(k_bwd_kv_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_bwd_kv_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    k_bwd_kv_tc<false><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, a);
+    count_launch();
+    k_bwd_kv_tc<true><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, a);
+    const size_t warps = (size_t)p.B * p.L;
+    count_launch();
+    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
+                                                                   ws.dkr_part, (__nv_bfloat16 *)dkr);
+    return cudaGetLastError();
+}
+
+}  // namespace dspark

@@ -25,8 +25,6 @@
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait, TMEM is freed and the workspace error word gets kErrTimeout.
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 
 #include "dspark_tc_common.cuh"
@@ -76,13 +74,6 @@ struct FwdArgs {
     float *lse;
     uint32_t *err;
 };
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-    __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&t);
-}
-
-__device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
@@ -459,31 +450,6 @@ __global__ void __launch_bounds__(256) k_fwd_pad_rows(int n_h, int S, int N, int
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 2-D bf16 tensor map over rows of `inner` elements, 64 x 64 boxes, 128 B swizzle.
-bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool fwd_tc_supported(const Prob &p) {
@@ -498,9 +464,9 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     count_launch();
     k_fwd_pad_rows<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.R, anchors, keep, (__nv_bfloat16 *)o, lse);
     CUtensorMap m_kc, m_kr, m_v;
-    if (!make_map(&m_kc, kc, kDC, (uint64_t)p.B * p.n_h * p.L) ||
-        !make_map(&m_kr, ws.kr_rot, kDR, (uint64_t)p.B * p.L) ||
-        !make_map(&m_v, v, kDV, (uint64_t)p.B * p.n_h * p.L))
+    if (!make_map_bf16(&m_kc, kc, kDC, (uint64_t)p.B * p.n_h * p.L, 64) ||
+        !make_map_bf16(&m_kr, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
+        !make_map_bf16(&m_v, v, kDV, (uint64_t)p.B * p.n_h * p.L, 64))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
