@@ -40,7 +40,8 @@ namespace {
 using namespace tc;
 
 constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
-constexpr int kG = 25;  // blocks per query group
+constexpr int kG = 25;   // blocks per query group (query-major kernel)
+constexpr int kGD = 16;  // blocks per draft-key tile of the key-major kernel (8 slots each)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
@@ -162,7 +163,8 @@ struct BwdArgs {
 __global__ void __launch_bounds__(dq::kThreads, 1)
     k_bwd_dq_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-                const __grid_constant__ CUtensorMap tm_dos, const BwdArgs p) {
+                const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
+                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
     using namespace dq;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -184,11 +186,17 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     const int ctx_lo = max(0, sa[0] - p.W + 1);
     const int ctx_hi = sa[gcnt - 1];
     const int n_ctx = ctx_hi > ctx_lo ? (ctx_hi - ctx_lo + kBN - 1) / kBN : 0;
-    const int n_draft = (nrows + kBN - 1) / kBN;
+    constexpr int kDraftBlocks = kBN / 8;  // draft tiles: 8 key slots per block
+    const int n_draft = (gcnt + kDraftBlocks - 1) / kDraftBlocks;
     const int T = n_ctx + n_draft;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t bh = (size_t)b * p.n_h + h;
     const size_t srow0 = bh * p.R + (size_t)kBlock * i0;  // first sorted row of the group
+
+    // K/V stages start zeroed (masked key slots must hold finite values)
+    for (int e = threadIdx.x; e < (oS0 - oK0) / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + oK0)[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; s++) {
@@ -228,10 +236,19 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         }
         // lane l holds the block index of group block l (l < gcnt)
         const int my_n = lane < gcnt ? sn[lane] : 0;
+        int pf_next = 2;
         for (int t = 0; t < T; ++t) {
             const int s = t & 1;
             uint8_t *kt = sm + (s ? oK1 : oK0);
             uint8_t *vt = sm + (s ? oV1 : oV0);
+            if (lane == 0) {
+                for (; pf_next <= t + 5 && pf_next < n_ctx; ++pf_next) {
+                    const int pos = ctx_lo + pf_next * kBN;
+                    for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
+                    tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
+                    for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
+                }
+            }
             if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
@@ -242,24 +259,19 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
                 }
             } else {
+                // draft tile: 8 key slots per block (its 5 keys, then 3 masked rows)
                 const int d = t - n_ctx;
-                for (int kk = 0; kk < kBN; ++kk) {
-                    const int slot = d * kBN + kk;
-                    const int nb = __shfl_sync(0xffffffffu, my_n, min(slot / kBlock, kG - 1));
-                    uint8_t *dst = kt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
-                    if (slot < nrows) {
-                        const size_t key = (size_t)p.S + kBlock * nb + slot % kBlock;
-                        const __nv_bfloat16 *src = lane < 24 ? p.kc + (bh * p.L + key) * kDC + lane * 8
-                                                             : p.krr + ((size_t)b * p.L + key) * kDR + (lane - 24) * 8;
-                        cp_async16(dst, src, 16);
-                    } else {
-                        cp_async16(dst, p.kc, 0);
+                const int nb = min(kDraftBlocks, gcnt - d * kDraftBlocks);
+                if (lane == 0) mbar_arrive_expect_tx(&kfull[s], nb * 8 * kDQK * 2);
+                for (int bb = 0; bb < nb; ++bb) {
+                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
+                    if (lane == 0) {
+                        const int row = p.S + kBlock * n;
+                        for (int c = 0; c < 3; c++)
+                            tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[s], c * 64, (int)(bh * p.L + row));
+                        tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
                     }
                 }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&kfull[s]);
             }
             if (lane == 0) counters[0] = t + 1;
             if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
@@ -272,21 +284,16 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 }
             } else {
                 const int d = t - n_ctx;
-                for (int kk = 0; kk < kBN; ++kk) {
-                    const int slot = d * kBN + kk;
-                    const int nb = __shfl_sync(0xffffffffu, my_n, min(slot / kBlock, kG - 1));
-                    uint8_t *dst = vt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
-                    if (slot < nrows) {
-                        const size_t key = (size_t)p.S + kBlock * nb + slot % kBlock;
-                        cp_async16(dst, p.v + (bh * p.L + key) * kDV + lane * 8, 16);
-                    } else {
-                        cp_async16(dst, p.v, 0);
+                const int nb = min(kDraftBlocks, gcnt - d * kDraftBlocks);
+                if (lane == 0) mbar_arrive_expect_tx(&vfull[s], nb * 8 * kDV * 2);
+                for (int bb = 0; bb < nb; ++bb) {
+                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
+                    if (lane == 0) {
+                        const int row = p.S + kBlock * n;
+                        for (int c = 0; c < 4; c++)
+                            tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[s], c * 64, (int)(bh * p.L + row));
                     }
                 }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&vfull[s]);
             }
             if (lane == 0) counters[1] = t + 1;
         }
@@ -331,27 +338,50 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 tc_fence_after();
                 issue_sdp(0);
             }
-            for (int t = 0; t < T && ok; ++t) {
-                if (t + 1 < T) {
-                    const int t1 = t + 1, s1 = t1 & 1;
-                    if (t1 >= 2) ok = mbar_wait(&dsready[s1], ((t1 >> 1) - 1) & 1, abort_flag);
-                    if (ok) ok = wait_kv(t1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_sdp(t1);
+            // Issue whichever is ready first: S/dP of tile ns (its K and V
+            // landed; it runs at most one tile ahead, so its S/dP buffer was
+            // released by the dQ of tile ns - 2) or dQ of tile nq (its dS is
+            // written). Neither waits for the other's inputs.
+            int ns = 1, nq = 0;
+            uint64_t t_idle = 0;
+            while (ok && nq < T) {
+                bool issued = false;
+                if (ns < T && ns <= nq + 1) {
+                    const int s1 = ns & 1;
+                    if (mbar_try_wait(&kfull[s1], (ns >> 1) & 1) && mbar_try_wait(&vfull[s1], (ns >> 1) & 1)) {
+                        counters[2] = ns + 1;
+                        counters[3] = ns + 1;
+                        tc_fence_after();
+                        issue_sdp(ns);
+                        ++ns;
+                        issued = true;
+                    }
                 }
-                const int s = t & 1;
-                ok = mbar_wait(&dsready[s], (t >> 1) & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t dsa = smem_u32(sm + (s ? oS1 : oS0));
-                const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0));
+                if (!issued && mbar_try_wait(&dsready[nq & 1], (nq >> 1) & 1)) {
+                    const int s = nq & 1;
+                    tc_fence_after();
+                    const uint32_t dsa = smem_u32(sm + (s ? oS1 : oS0));
+                    const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0));
 #pragma unroll
-                for (int k = 0; k < kBN / 16; ++k)
-                    mma_bf16_ss(tmem + kColDQ, sdesc_sw128(dsa + k * 32, 16, 1024),
-                                sdesc_sw128(kb + k * 2048, kKChunk, 1024), idQ, (t > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&kempty[s]);
-                mma_commit(&dqdone[s]);
+                    for (int k = 0; k < kBN / 16; ++k)
+                        mma_bf16_ss(tmem + kColDQ, sdesc_sw128(dsa + k * 32, 16, 1024),
+                                    sdesc_sw128(kb + k * 2048, kKChunk, 1024), idQ, (nq > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(&kempty[s]);
+                    mma_commit(&dqdone[s]);
+                    ++nq;
+                    issued = true;
+                }
+                if (issued) {
+                    t_idle = 0;
+                } else {
+                    const uint64_t now = globaltimer();
+                    if (t_idle == 0) t_idle = now;
+                    if (*abort_flag) ok = false;
+                    else if (now - t_idle > kWaitTimeoutNs) {
+                        *abort_flag = 1;
+                        ok = false;
+                    }
+                }
             }
         }
     } else {
@@ -384,17 +414,24 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 if (!ok) break;
             }
             uint8_t *drow = sm + (s ? oS1 : oS0);
-            const bool ctx = t < n_ctx;
-            const int c0 = ctx ? ctx_lo + t * kBN : (t - n_ctx) * kBN;
-            const int myblk = r / kBlock;
+            // the row's keys in this tile: one contiguous column range [clo, chi)
+            int clo, chi;
+            if (t < n_ctx) {
+                const int c0 = ctx_lo + t * kBN;
+                clo = lo - c0;
+                chi = A - c0;
+            } else {
+                clo = 8 * (r / kBlock) - (t - n_ctx) * kBN;
+                chi = clo + kBlock;
+            }
+            if (!live) chi = clo;
 #pragma unroll
             for (int u = 0; u < kBN / 8; u++) {
                 float e[8];
 #pragma unroll
                 for (int k = 0; k < 8; k++) {
                     const int c = u * 8 + k;
-                    const bool valid = live && (ctx ? (c0 + c >= lo && c0 + c < A) : ((c0 + c) / kBlock == myblk));
-                    const float pp = valid ? exp2f(sv[c] * p.scale_log2 - lse2) : 0.f;
+                    const float pp = (c >= clo && c < chi) ? ex2(fmaf(sv[c], p.scale_log2, -lse2)) : 0.f;
                     e[k] = pp * (pv[c] - Dr) * p.scale;
                 }
                 *reinterpret_cast<uint4 *>(drow + sw128(r, u)) =
@@ -475,7 +512,8 @@ template <bool ROLE_K>
 __global__ void __launch_bounds__(kv::kThreads, 1)
     k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-                const __grid_constant__ CUtensorMap tm_dos, const BwdArgs p) {
+                const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
+                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
     using namespace kv;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -498,9 +536,9 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     if (is_ctx) {
         t0 = item * kMK;
     } else {
-        i0 = (item - p.n_ctx_items) * kG;
+        i0 = (item - p.n_ctx_items) * kGD;
         if (i0 >= cnt) return;  // uniform: fewer groups in this batch row
-        gcnt = min(kG, cnt - i0);
+        gcnt = min(kGD, cnt - i0);
     }
     const int32_t *sa = p.sorted_a + (size_t)b * p.N;
     const int32_t *sn = p.sorted_n + (size_t)b * p.N;
@@ -541,9 +579,9 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         if (is_ctx) {
             key_valid = t0 + key_local < p.S;
             key_pos = (size_t)t0 + key_local;
-        } else {
-            key_valid = key_local < kBlock * gcnt;
-            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + key_local / kBlock] + key_local % kBlock;
+        } else {  // 8 key slots per block: its 5 keys, then 3 masked rows
+            key_valid = key_local / 8 < gcnt && key_local % 8 < kBlock;
+            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + key_local / 8] + key_local % 8;
         }
     }
 
@@ -569,6 +607,10 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         return;
     }
 
+    // K/V tiles start zeroed (masked key slots must hold finite values)
+    for (int e = threadIdx.x; e < (oQ - oK) / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + oK)[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         mbar_init(kvfull, 1);
         mbar_init(kvfree, 1);
@@ -614,25 +656,37 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                             tma_load_2d(sm + oV + c * kKChunk, &tm_v, kvfull, c * 64, (int)(bh * p.L + t0));
                 }
             } else {
-                for (int kk = 0; kk < kMK; ++kk) {
-                    const int nb = __shfl_sync(0xffffffffu, my_n, min(kk / kBlock, kG - 1));
-                    const bool in = kk < kBlock * gcnt;
-                    const size_t key = (size_t)p.S + kBlock * nb + kk % kBlock;
-                    const __nv_bfloat16 *src = lane < 24 ? p.kc + (bh * p.L + key) * kDC + lane * 8
-                                                         : p.krr + ((size_t)b * p.L + key) * kDR + (lane - 24) * 8;
-                    cp_async16(sm + oK + (lane >> 3) * kKChunk + sw128(kk, lane & 7), in ? src : (const void *)p.kc,
-                               in ? 16u : 0u);
-                    if (ROLE_K)
-                        cp_async16(sm + oV + (lane >> 3) * kKChunk + sw128(kk, lane & 7),
-                                   in ? (const void *)(p.v + (bh * p.L + key) * kDV + lane * 8) : (const void *)p.v,
-                                   in ? 16u : 0u);
+                if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * (ROLE_K ? 2 : 1) * kDQK * 2);
+                for (int bb = 0; bb < gcnt; ++bb) {
+                    const int nb = __shfl_sync(0xffffffffu, my_n, bb);
+                    if (lane == 0) {
+                        const int row = p.S + kBlock * nb;
+                        for (int c = 0; c < 3; c++)
+                            tma_load_2d(sm + oK + c * kKChunk + bb * 1024, &tm_kc8, kvfull, c * 64, (int)(bh * p.L + row));
+                        tma_load_2d(sm + oK + 3 * kKChunk + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
+                        if (ROLE_K)
+                            for (int c = 0; c < 4; c++)
+                                tma_load_2d(sm + oV + c * kKChunk + bb * 1024, &tm_v8, kvfull, c * 64, (int)(bh * p.L + row));
+                    }
                 }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(kvfull);
             }
             if (lane == 0) counters[0] = hh + 1;
+            // the next head's K (and V) tile into L2 while this head runs
+            if (hh + 1 < H) {
+                const size_t bh1 = bh + 1;
+                if (is_ctx) {
+                    if (lane == 0) {
+                        for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh1 * p.L + t0));
+                        if (ROLE_K)
+                            for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh1 * p.L + t0));
+                    }
+                } else if (lane < gcnt) {
+                    const int row = p.S + kBlock * my_n;
+                    for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc8, c * 64, (int)(bh1 * p.L + row));
+                    if (ROLE_K)
+                        for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v8, c * 64, (int)(bh1 * p.L + row));
+                }
+            }
             for (int c = 0; c < nchunks; ++c, ++q) {
                 if (q >= 1 && !warp_all(mbar_wait(chfree, (q - 1) & 1, abort_flag))) {
                     ok = false;
@@ -655,6 +709,15 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                         tma_load_2d(sm + oDO + cc * kRChunk, &tm_dos, chfull, cc * 64, (int)(bh * p.R + r0));
                     }
                     counters[1] = q + 1;
+                    // the following chunk (this head's next, or the next head's first) into L2
+                    const bool last = c + 1 == nchunks;
+                    if (!last || hh + 1 < H) {
+                        const size_t nrow = (last ? bh + 1 : bh) * p.R + (last ? row0 : r0 + kRC);
+                        for (int cc = 0; cc < 4; cc++) {
+                            tma_prefetch_2d(&tm_qs, cc * 64, (int)nrow);
+                            tma_prefetch_2d(&tm_dos, cc * 64, (int)nrow);
+                        }
+                    }
                 }
             }
         }
@@ -717,7 +780,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         int q = 0;
         bool ok = true;
         const int kpos = t0 + k;                     // context position of this key (context tiles)
-        const int kblk = is_ctx ? 0 : k / kBlock;    // draft tiles: the key's block within the group
+        const int kblk = is_ctx ? 0 : k / 8;         // draft tiles: the key's block within the group
         for (int hh = 0; hh < H && ok; ++hh) {
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
             for (int c = 0; c < nchunks; ++c, ++q) {
@@ -768,8 +831,8 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                         if (is_ctx)
                             valid = A >= 0 && kpos < A && kpos >= A - p.W + 1;
                         else
-                            valid = A >= 0 && key_valid && (crow0 + col - row0) / kBlock == kblk;
-                        const float pp = valid ? exp2f(sv[col] * p.scale_log2 - mlse[col]) : 0.f;
+                            valid = A >= 0 && key_valid && (crow0 + col - row0) / kBlock == kblk;  // own block
+                        const float pp = valid ? ex2(fmaf(sv[col], p.scale_log2, -mlse[col])) : 0.f;
                         if (ROLE_K)
                             e[i] = pp * (pv[col] - mD[col]) * p.scale;
                         else
@@ -890,7 +953,7 @@ bool bwd_tc_supported(const Prob &p) {
 }
 
 int bwd_head_groups(const Prob &p) {
-    const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kG - 1) / kG) * p.B;
+    const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kGD - 1) / kGD) * p.B;
     int hg = 1;
     while (hg < p.n_h && items * hg < 2 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
     return hg;
@@ -910,7 +973,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs64, m_dos64;
+    CUtensorMap m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs64, m_dos64, m_kc8, m_kr8, m_v8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
     if (p.N > 0 && q_rows > 0) {
@@ -920,7 +983,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
             !make_map_bf16(&m_dos64, dos, kDV, q_rows, 64))
             return cudaErrorInvalidValue;
     }
-    if (!make_map_bf16(&m_kc128, kc, kDC, kv_rows, 128) ||
+    if (!make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) || !make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
+        !make_map_bf16(&m_v8, v, kDV, kv_rows, 8) || !make_map_bf16(&m_kc128, kc, kDC, kv_rows, 128) ||
         !make_map_bf16(&m_kr128, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 128) ||
         !make_map_bf16(&m_v128, v, kDV, kv_rows, 128))
         return cudaErrorInvalidValue;
@@ -956,17 +1020,19 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         if (e != cudaSuccess) return e;
         count_launch();
         k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
-            m_kc32, m_kr32, m_v32, m_qs128, m_dos128, a);
+            m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc8, m_kr8, m_v8, a);
     }
-    const dim3 kv_grid(a.n_ctx_items + (p.N + kG - 1) / kG, HG, p.B);
+    const dim3 kv_grid(a.n_ctx_items + (p.N + kGD - 1) / kGD, HG, p.B);
     e = cudaFuncSetAttribute(k_bwd_kv_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k_bwd_kv_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_kv_tc<false><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, a);
+    k_bwd_kv_tc<false><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, m_kc8,
+                                                                  m_kr8, m_v8, a);
     count_launch();
-    k_bwd_kv_tc<true><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, a);
+    k_bwd_kv_tc<true><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, m_kc8,
+                                                                 m_kr8, m_v8, a);
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
     k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,

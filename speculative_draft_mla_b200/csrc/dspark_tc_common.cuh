@@ -88,6 +88,22 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
         "l"((uint64_t)m), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// 1-D bulk copy of `bytes` contiguous bytes (16-byte aligned addresses, size a
+// multiple of 16) completing on bar's transaction count.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Prefetch a 2-D tile of a tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *m, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"((uint64_t)m), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
 // 16-byte cp.async; src_bytes = 0 writes 16 zero bytes without reading src.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
@@ -188,6 +204,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&t);
 }
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
+// 2^x with the hardware approximation (MUFU.EX2; results below 2^-126 flush
+// to 0, which only drops softmax weights far below bf16 resolution).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // ---- host: tensor maps ----------------------------------------------------
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

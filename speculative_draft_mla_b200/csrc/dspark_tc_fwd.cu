@@ -55,6 +55,11 @@ constexpr int oV1 = oV0 + kVBytes;
 constexpr int oP0 = oV1 + kVBytes;
 constexpr int oP1 = oP0 + kPBytes;
 constexpr int oBar = oP1 + kPBytes;
+// Q staging area (raw rows) before the swizzled Q tile is built: the second V
+// stage and both P buffers, contiguous and idle at that point
+constexpr int oStage = oV1;
+static_assert(oP1 + kPBytes - oStage >= kM * kDQK * 2, "staging area too small");
+constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 constexpr int kSmemBytes = oBar + 256 + 1024;  // barriers + alignment slack
 
 constexpr int kThreads = 192;
@@ -77,17 +82,19 @@ struct FwdArgs {
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
-             const __grid_constant__ CUtensorMap tm_v, const FwdArgs p) {
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc8,
+             const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const FwdArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint64_t *kfull = bars + 0, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
     uint64_t *sfull = bars + 8, *pready = bars + 10, *pvdone = bars + 12, *qready = bars + 14;
-    uint64_t *drain = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
-    // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed
-    int *counters = reinterpret_cast<int *>(bars + 18);
+    uint64_t *drain = bars + 15, *qraw = bars + 16, *qstaged = bars + 17;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
+    // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
+    // [4] raw Q issued
+    int *counters = reinterpret_cast<int *>(bars + 20);
 
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int cnt = p.cnt[b];
@@ -100,11 +107,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ctx_lo = max(0, sa[0] - p.W + 1);
     const int ctx_hi = sa[gcnt - 1];
     const int n_ctx = ctx_hi > ctx_lo ? (ctx_hi - ctx_lo + kBN - 1) / kBN : 0;
-    const int n_draft = (nrows + kBN - 1) / kBN;
+    const int n_draft = (gcnt + kDraftBlocksPerTile - 1) / kDraftBlocksPerTile;
     const int T = n_ctx + n_draft;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t bh = (size_t)b * p.n_h + h;
 
+    // K/V stages start zeroed: masked key slots of a tile are multiplied by a
+    // zero weight, and must not hold stale non-finite bits.
+    for (int e = threadIdx.x; e < (oP0 - oK0) / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + oK0)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; s++) {
             mbar_init(&kfull[s], 1);
@@ -117,15 +128,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(qready, 4);
         mbar_init(drain, 1);
+        mbar_init(qraw, 1);
+        mbar_init(qstaged, 4);
         *abort_flag = 0;
-        for (int c = 0; c < 4; c++) counters[c] = 0;
+        for (int c = 0; c < 5; c++) counters[c] = 0;
         fence_barrier_init();
-        fence_proxy_async_smem();
     }
     if (warp == 5) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    fence_proxy_async_smem();  // the zeroed stages are read by TMA-fed MMAs
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -133,15 +146,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 4) {
         // ------------------------------------------------------- producer
+        // lane l holds the block index of group block l
+        const int my_n = lane < gcnt ? sn[lane] : 0;
         if (lane == 0) {
             tma_prefetch_desc(&tm_kc);
             tma_prefetch_desc(&tm_kr);
             tma_prefetch_desc(&tm_v);
+            // raw Q rows of the group: each block's 5 rows are one contiguous
+            // 2560-byte run; they land row-major in the staging area
+            mbar_arrive_expect_tx(qraw, nrows * kDQK * 2);
+            counters[4] = 1;
         }
+        __syncwarp();
+        if (lane < gcnt)
+            bulk_load(sm + oStage + lane * (kBlock * kDQK * 2),
+                      p.q + (bh * p.R + (size_t)kBlock * my_n) * kDQK, kBlock * kDQK * 2, qraw);
+        int pf_next = 2;  // next context tile to prefetch into L2
         for (int t = 0; t < T; ++t) {
             const int s = t & 1;
             uint8_t *kt = sm + (s ? oK1 : oK0);
             uint8_t *vt = sm + (s ? oV1 : oV0);
+            if (lane == 0) {
+                for (; pf_next <= t + 3 && pf_next < n_ctx; ++pf_next) {
+                    const int pos = ctx_lo + pf_next * kBN;
+                    for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
+                    tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
+                    for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
+                }
+            }
             if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
@@ -152,25 +184,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
                 }
             } else {
+                // draft tile: 8 key slots per block, its 5 keys first (the 3
+                // rows after them are other keys, masked out)
                 const int d = t - n_ctx;
-                for (int kk = 0; kk < kBN; ++kk) {
-                    const int slot = d * kBN + kk;
-                    uint8_t *dst = kt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
-                    if (slot < nrows) {
-                        const size_t key = (size_t)p.S + kBlock * sn[slot / kBlock] + slot % kBlock;
-                        const __nv_bfloat16 *src = lane < 24 ? p.kc + (bh * p.L + key) * kDC + lane * 8
-                                                             : p.krr + ((size_t)b * p.L + key) * kDR + (lane - 24) * 8;
-                        cp_async16(dst, src, 16);
-                    } else {
-                        cp_async16(dst, p.kc, 0);
+                const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
+                if (lane == 0) mbar_arrive_expect_tx(&kfull[s], nb * 8 * kDQK * 2);
+                __syncwarp();
+                for (int bb = 0; bb < nb; ++bb) {
+                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
+                    if (lane == 0) {
+                        const int row = p.S + kBlock * n;
+                        for (int c = 0; c < 3; c++)
+                            tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[s], c * 64, (int)(bh * p.L + row));
+                        tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
                     }
                 }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&kfull[s]);
             }
             if (lane == 0) counters[0] = t + 1;
+            // V: the second V stage doubles as the Q staging area until the
+            // softmax warps have moved Q into place
+            if (t == 1 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
             if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
@@ -181,24 +214,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
                 const int d = t - n_ctx;
-                for (int kk = 0; kk < kBN; ++kk) {
-                    const int slot = d * kBN + kk;
-                    uint8_t *dst = vt + (lane >> 3) * kKChunk + sw128(kk, lane & 7);
-                    if (slot < nrows) {
-                        const size_t key = (size_t)p.S + kBlock * sn[slot / kBlock] + slot % kBlock;
-                        cp_async16(dst, p.v + (bh * p.L + key) * kDV + lane * 8, 16);
-                    } else {
-                        cp_async16(dst, p.v, 0);
+                const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
+                if (lane == 0) mbar_arrive_expect_tx(&vfull[s], nb * 8 * kDV * 2);
+                __syncwarp();
+                for (int bb = 0; bb < nb; ++bb) {
+                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
+                    if (lane == 0) {
+                        const int row = p.S + kBlock * n;
+                        for (int c = 0; c < 4; c++)
+                            tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[s], c * 64, (int)(bh * p.L + row));
                     }
                 }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&vfull[s]);
             }
             if (lane == 0) counters[1] = t + 1;
         }
-        cp_async_wait_all();
     } else if (warp == 5) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
@@ -263,39 +292,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             j = r % kBlock;
             lo = max(0, A - p.W + 1);
         }
-        // Q rows of this warp, rope slice rotated to position A + j
-        for (int i = 0; i < 32; ++i) {
-            const int rr = warp * 32 + i;
-            const int Ai = __shfl_sync(0xffffffffu, A, i);
-            const int ni = __shfl_sync(0xffffffffu, n, i);
-            const int ji = __shfl_sync(0xffffffffu, j, i);
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (rr < nrows) {
-                const __nv_bfloat16 *src = p.q + ((bh * p.R) + kBlock * ni + ji) * kDQK + lane * 8;
-                val = __ldg(reinterpret_cast<const uint4 *>(src));
-                if (lane >= 24) {
-                    const float2 *cs = p.tab + (size_t)(Ai + ji) * (kDR / 2) + (lane - 24) * 4;
-                    uint32_t w[4] = {val.x, val.y, val.z, val.w};
+        bool ok = true;
+        {
+            // Q: row r of the staging area (raw) -> row r of the swizzled Q
+            // tile, rope slice rotated to position A + j; rows past the group 0
+            float4 cs[kDR / 4];  // (cos, sin) of the 32 rope frequencies at A + j
+            const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2));
 #pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&w[k]);
-                        const float x0 = __bfloat162float(pr.x), x1 = __bfloat162float(pr.y);
-                        const float2 c = __ldg(cs + k);
-                        w[k] = pack_bf16x2(x0 * c.x - x1 * c.y, x0 * c.y + x1 * c.x);
-                    }
-                    val = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int k = 0; k < kDR / 4; k++) cs[k] = __ldg(tp + k);
+            ok = warp_all(mbar_wait(qraw, 0, abort_flag));
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + r * (kDQK * 2));
+            const bool have = live && ok;
+#pragma unroll 4
+            for (int u = 0; u < kDC / 8; u++)
+                *reinterpret_cast<uint4 *>(sm + oQ + (u >> 3) * kQChunk + sw128(r, u & 7)) =
+                    have ? src[u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < kDR / 8; u++) {  // rope slice: 4 pairs per unit
+                const uint4 val = have ? src[kDC / 8 + u] : make_uint4(0, 0, 0, 0);
+                uint32_t w[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    const __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&w[k]);
+                    const float x0 = __bfloat162float(pr.x), x1 = __bfloat162float(pr.y);
+                    const float4 c2 = cs[(4 * u + k) >> 1];
+                    const float c = (k & 1) ? c2.z : c2.x, sn_ = (k & 1) ? c2.w : c2.y;
+                    w[k] = pack_bf16x2(x0 * c - x1 * sn_, x0 * sn_ + x1 * c);
                 }
+                *reinterpret_cast<uint4 *>(sm + oQ + 3 * kQChunk + sw128(r, u)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            *reinterpret_cast<uint4 *>(sm + oQ + (lane >> 3) * kQChunk + sw128(rr, lane & 7)) = val;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(qstaged);  // staging area free for V tiles and P
+                mbar_arrive(qready);
+            }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(qready);
 
         float m_used = -INFINITY, l = 0.f;
-        bool ok = true;
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        for (int t = 0; t < T; ++t) {
+        for (int t = 0; t < T && ok; ++t) {
             const int s = t & 1;
             ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
             if (!ok) break;
@@ -312,32 +348,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sv[32 + c] = a1[c];
                 }
             }
-            float mt = -INFINITY;
+            // every row's keys in a tile form one contiguous column range
+            // [clo, chi): the window [lo, A) for context tiles, its block's 5
+            // key slots for draft tiles
+            int clo, chi;
             if (t < n_ctx) {
                 const int c0 = ctx_lo + t * kBN;
-#pragma unroll
-                for (int c = 0; c < kBN; c++) {
-                    const int pos = c0 + c;
-                    const bool valid = live && pos >= lo && pos < A;
-                    sv[c] = valid ? sv[c] * p.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, sv[c]);
-                }
+                clo = lo - c0;
+                chi = A - c0;
             } else {
-                const int base = (t - n_ctx) * kBN;
-                const int myblk = r / kBlock;
-#pragma unroll
-                for (int c = 0; c < kBN; c++) {
-                    const bool valid = live && (base + c) / kBlock == myblk;
-                    sv[c] = valid ? sv[c] * p.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, sv[c]);
-                }
+                clo = 8 * (r / kBlock) - (t - n_ctx) * kBN;
+                chi = clo + kBlock;
             }
+            if (!live) chi = clo;
+            float mx[8];
+#pragma unroll
+            for (int k = 0; k < 8; k++) mx[k] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kBN; c++) {
+                sv[c] = (c >= clo && c < chi) ? sv[c] : -INFINITY;
+                mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+            }
+            const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float mt = mraw * p.scale_log2;
             bool resc = false;
             float alpha = 1.f;
             if (mt > m_used + kRescaleThreshold) {
                 if (m_used != -INFINITY) {
                     resc = true;
-                    alpha = exp2f(m_used - mt);
+                    alpha = ex2(m_used - mt);
                 }
                 m_used = mt;
             }
@@ -346,20 +386,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
             }
             uint8_t *prow = sm + (s ? oP1 : oP0);
-            float ps = 0.f;
+            float psum[8];
+#pragma unroll
+            for (int k = 0; k < 8; k++) psum[k] = 0.f;
             const bool any = m_used != -INFINITY;
+            const float mneg = any ? -m_used : 0.f;
 #pragma unroll
             for (int u = 0; u < 8; u++) {
                 float e[8];
 #pragma unroll
                 for (int k = 0; k < 8; k++) {
-                    e[k] = any ? exp2f(sv[u * 8 + k] - m_used) : 0.f;
-                    ps += e[k];
+                    e[k] = any ? ex2(fmaf(sv[u * 8 + k], p.scale_log2, mneg)) : 0.f;
+                    psum[k] += e[k];
                 }
                 uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
                                       pack_bf16x2(e[6], e[7]));
                 *reinterpret_cast<uint4 *>(prow + sw128(r, u)) = pk;
             }
+            const float ps = ((psum[0] + psum[1]) + (psum[2] + psum[3])) + ((psum[4] + psum[5]) + (psum[6] + psum[7]));
             l = l * alpha + ps;
             if (__any_sync(0xffffffffu, resc)) {
                 if (t >= 1) {
@@ -415,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Drain what may still be in flight, each wait bounded on its own.
         volatile int never = 0;
         if (warp == 4 && lane == 0) {
+            if (counters[4]) mbar_wait(qraw, 0, (volatile int *)&never);
             // loads issued but not yet consumed complete in order, one phase each
             for (int t = counters[2]; t < counters[0]; ++t)
                 mbar_wait(&kfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
@@ -463,10 +508,11 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     if (p.B == 0 || p.N == 0) return cudaSuccess;
     count_launch();
     k_fwd_pad_rows<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.R, anchors, keep, (__nv_bfloat16 *)o, lse);
-    CUtensorMap m_kc, m_kr, m_v;
-    if (!make_map_bf16(&m_kc, kc, kDC, (uint64_t)p.B * p.n_h * p.L, 64) ||
-        !make_map_bf16(&m_kr, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
-        !make_map_bf16(&m_v, v, kDV, (uint64_t)p.B * p.n_h * p.L, 64))
+    CUtensorMap m_kc, m_kr, m_v, m_kc8, m_kr8, m_v8;
+    const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, kr_rows = (uint64_t)p.B * p.L;
+    if (!make_map_bf16(&m_kc, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr, ws.kr_rot, kDR, kr_rows, 64) ||
+        !make_map_bf16(&m_v, v, kDV, kv_rows, 64) || !make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) ||
+        !make_map_bf16(&m_kr8, ws.kr_rot, kDR, kr_rows, 8) || !make_map_bf16(&m_v8, v, kDV, kv_rows, 8))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -486,7 +532,7 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.err = ws.err;
     dim3 grid((p.N + kG - 1) / kG, p.n_h, p.B);
     count_launch();
-    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc, m_kr, m_v, a);
+    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc, m_kr, m_v, m_kc8, m_kr8, m_v8, a);
     return cudaGetLastError();
 }
 
