@@ -16,14 +16,15 @@
 //   3. k_bwd_dq_tc     query-major, one CTA per (b, h, 25 sorted blocks):
 //                      32-key tiles of the group's key set; S and dP in TMEM,
 //                      dS through shared memory, dQ += dS K in TMEM.
-//   4. k_bwd_kv_tc<V>  key-major, one CTA per (b, 128-key tile, head group):
-//      k_bwd_kv_tc<K>  rows of the blocks whose key sets meet the tile, in
-//                      chunks of 64: S^T = K Q^T (and dP^T = V dO^T) in TMEM,
-//                      P^T (dS^T) through shared memory, dV += P^T dO
+//   4. k_bwd_kv_tc     key-major, one CTA per (b, 128-key tile, role, head
+//                      group): rows of the blocks whose key sets meet the tile,
+//                      in chunks of 32: S^T = K Q^T (and dP^T = V dO^T) in
+//                      TMEM, P^T (dS^T) through shared memory, dV += P^T dO
 //                      (dK += dS^T Q) accumulated in TMEM over the rows. A
 //                      128-key tile's dV and dK accumulators would need all
 //                      512 TMEM columns together, so they are produced by two
-//                      CTA roles that each recompute S^T.
+//                      CTA roles that each recompute S^T; the two are adjacent
+//                      in launch order so one of them reads K from L2.
 //   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
 //                      them back and writes dK^R.
 // Key tiles are either context tiles [t0, t0+128) or the draft keys of one
@@ -498,17 +499,22 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
 // ============================================================== dK / dV
 namespace kv {
 constexpr int kMK = 128;                 // keys per tile (MMA M)
-constexpr int kRC = 64;                  // rows per chunk (MMA N of S^T)
+constexpr int kRC = 32;                  // rows per chunk (MMA N of S^T)
 constexpr int kKChunk = kMK * 128;       // 16 KB: 128 keys x 64 columns
-constexpr int kRChunk = kRC * 128;       // 8 KB: 64 rows x 64 columns
-constexpr int oK = 0, oV = oK + 4 * kKChunk, oQ = oV + 4 * kKChunk, oDO = oQ + 4 * kRChunk,
-              oPT = oDO + 4 * kRChunk, oMeta = oPT + kKChunk, oBar = oMeta + 3 * kRC * 4;
+constexpr int kRChunk = kRC * 128;       // 4 KB: 32 rows x 64 columns
+constexpr int kPT = kMK * 128;           // 16 KB: [128 keys][64-column swizzled rows], 32 used
+constexpr int oK = 0, oV = oK + 4 * kKChunk, oQ0 = oV + 4 * kKChunk, oQ1 = oQ0 + 4 * kRChunk,
+              oD0 = oQ1 + 4 * kRChunk, oD1 = oD0 + 4 * kRChunk, oP0 = oD1 + 4 * kRChunk, oP1 = oP0 + kPT,
+              oMeta = oP1 + kPT, oBar = oMeta + 2 * kRC * 12;
 constexpr int kSmem = oBar + 256 + 1024;
-constexpr int kThreads = 192;
-constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320;
+constexpr int kKeyWarps = 8;             // two per TMEM sub-partition, each half of a chunk's rows
+constexpr int kThreads = (kKeyWarps + 2) * 32;
+constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320;  // S^T: 256 / 288, dP^T: 320 / 352
 }  // namespace kv
 
-template <bool ROLE_K>
+// One CTA per (key tile, role, head group, batch). Role 0 accumulates dV =
+// P^T dO, role 1 dK = dS^T Q; the two roles of a tile are adjacent in launch
+// order so the second reads K and the row chunks from L2.
 __global__ void __launch_bounds__(kv::kThreads, 1)
     k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
@@ -518,17 +524,15 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *chfull = bars + 2, *chfree = bars + 3, *sfull = bars + 4;
-    uint64_t *dsready = bars + 5, *accdone = bars + 6, *epidone = bars + 7, *drain = bars + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 10);
-    int *counters = reinterpret_cast<int *>(bars + 11);  // kv issued, ch issued, kv consumed, ch consumed
-    int *band = reinterpret_cast<int *>(bars + 14);      // first sorted row, row count
-    float *mlse = reinterpret_cast<float *>(sm + oMeta);
-    float *mD = mlse + kRC;
-    int *mA = reinterpret_cast<int *>(mD + kRC);
+    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *chfull = bars + 2, *chfree = bars + 4, *sfull = bars + 6;
+    uint64_t *dsready = bars + 8, *accdone = bars + 10, *epidone = bars + 11, *drain = bars + 12;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 14);
+    int *counters = reinterpret_cast<int *>(bars + 15);  // kv issued, ch issued, kv consumed, ch consumed
+    int *band = reinterpret_cast<int *>(bars + 17);      // first sorted row, row count
 
-    const int item = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    const int item = blockIdx.x >> 1, role_k = blockIdx.x & 1;
+    const int hg = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cnt = p.cnt[b];
     const bool is_ctx = item < p.n_ctx_items;
@@ -537,7 +541,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         t0 = item * kMK;
     } else {
         i0 = (item - p.n_ctx_items) * kGD;
-        if (i0 >= cnt) return;  // uniform: fewer groups in this batch row
+        if (i0 >= cnt) return;  // uniform: fewer draft tiles in this batch row
         gcnt = min(kGD, cnt - i0);
     }
     const int32_t *sa = p.sorted_a + (size_t)b * p.N;
@@ -570,321 +574,314 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     const int row0 = band[0], nrows = band[1];
     const int nchunks = (nrows + kRC - 1) / kRC;
     const int h0 = hg * p.hpg;
-    // the tile's keys that this CTA writes: context keys below S, or the
-    // draft keys of the group's blocks
-    const int key_local = threadIdx.x;  // for warps 0-3
+    const int H = p.hpg;
+    // the key this thread stands for (key warps): TMEM lane = key slot
+    const int k = (threadIdx.x & 127);
+    const int half = warp >> 2;  // which half of a chunk's rows / of the accumulator columns
     bool key_valid = false;
     size_t key_pos = 0;
-    if (warp < 4) {
+    if (warp < kKeyWarps) {
         if (is_ctx) {
-            key_valid = t0 + key_local < p.S;
-            key_pos = (size_t)t0 + key_local;
+            key_valid = t0 + k < p.S;
+            key_pos = (size_t)t0 + k;
         } else {  // 8 key slots per block: its 5 keys, then 3 masked rows
-            key_valid = key_local / 8 < gcnt && key_local % 8 < kBlock;
-            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + key_local / 8] + key_local % 8;
+            key_valid = k / 8 < gcnt && k % 8 < kBlock;
+            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + k / 8] + k % 8;
         }
     }
+    float *dkr_part_row = p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR;
 
     if (nrows == 0) {
         // no row sees these keys: zero gradients for every head of the group
-        if (warp < 4 && key_valid) {
+        if (warp < kKeyWarps && key_valid) {
             const uint4 z = make_uint4(0, 0, 0, 0);
-            for (int hh = 0; hh < p.hpg; hh++) {
+            for (int hh = 0; hh < H; hh++) {
                 const size_t bh = (size_t)b * p.n_h + h0 + hh;
-                if (ROLE_K) {
+                if (role_k) {
                     uint4 *d = reinterpret_cast<uint4 *>(p.dkc + (bh * p.L + key_pos) * kDC);
-                    for (int e = 0; e < kDC / 8; e++) d[e] = z;
+                    for (int e = half; e < kDC / 8; e += 2) d[e] = z;
                 } else {
                     uint4 *d = reinterpret_cast<uint4 *>(p.dv + (bh * p.L + key_pos) * kDV);
-                    for (int e = 0; e < kDV / 8; e++) d[e] = z;
+                    for (int e = half; e < kDV / 8; e += 2) d[e] = z;
                 }
             }
-            if (ROLE_K) {
-                float4 *d = reinterpret_cast<float4 *>(p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR);
-                for (int e = 0; e < kDR / 4; e++) d[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            if (role_k && half == 0)
+                for (int e = 0; e < kDR / 4; e++)
+                    reinterpret_cast<float4 *>(dkr_part_row)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
 
     // K/V tiles start zeroed (masked key slots must hold finite values)
-    for (int e = threadIdx.x; e < (oQ - oK) / 16; e += blockDim.x)
+    for (int e = threadIdx.x; e < (oQ0 - oK) / 16; e += blockDim.x)
         reinterpret_cast<uint4 *>(sm + oK)[e] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         mbar_init(kvfull, 1);
         mbar_init(kvfree, 1);
-        mbar_init(chfull, 1);
-        mbar_init(chfree, 1);
-        mbar_init(sfull, 1);
-        mbar_init(dsready, 4);
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&chfull[s], 1);
+            mbar_init(&chfree[s], 1);
+            mbar_init(&sfull[s], 1);
+            mbar_init(&dsready[s], kKeyWarps);
+        }
         mbar_init(accdone, 1);
-        mbar_init(epidone, 4);
+        mbar_init(epidone, kKeyWarps);
         mbar_init(drain, 1);
         *abort_flag = 0;
         for (int c = 0; c < 4; c++) counters[c] = 0;
         fence_barrier_init();
-        fence_proxy_async_smem();
     }
-    if (warp == 5) {
+    if (warp == kKeyWarps + 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int H = p.hpg;
+    const int QT = H * nchunks;  // chunks over all heads of the group
 
-    if (warp == 4) {
+    if (warp == kKeyWarps) {
         // ------------------------------------------------------- producer
         const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
-        int q = 0;  // chunk counter over all heads
         bool ok = true;
-        for (int hh = 0; hh < H && ok; ++hh) {
+        for (int q = 0; q < QT && ok; ++q) {
+            const int hh = q / nchunks, c = q % nchunks, s = q & 1;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
-            // K tile (and V tile for dK)
-            if (is_ctx) {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(kvfull, (ROLE_K ? 8 : 4) * kKChunk);
-                    for (int c = 0; c < 3; c++)
-                        tma_load_2d(sm + oK + c * kKChunk, &tm_kc, kvfull, c * 64, (int)(bh * p.L + t0));
-                    tma_load_2d(sm + oK + 3 * kKChunk, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
-                    if (ROLE_K)
-                        for (int c = 0; c < 4; c++)
-                            tma_load_2d(sm + oV + c * kKChunk, &tm_v, kvfull, c * 64, (int)(bh * p.L + t0));
-                }
-            } else {
-                if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * (ROLE_K ? 2 : 1) * kDQK * 2);
-                for (int bb = 0; bb < gcnt; ++bb) {
-                    const int nb = __shfl_sync(0xffffffffu, my_n, bb);
-                    if (lane == 0) {
-                        const int row = p.S + kBlock * nb;
-                        for (int c = 0; c < 3; c++)
-                            tma_load_2d(sm + oK + c * kKChunk + bb * 1024, &tm_kc8, kvfull, c * 64, (int)(bh * p.L + row));
-                        tma_load_2d(sm + oK + 3 * kKChunk + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
-                        if (ROLE_K)
-                            for (int c = 0; c < 4; c++)
-                                tma_load_2d(sm + oV + c * kKChunk + bb * 1024, &tm_v8, kvfull, c * 64, (int)(bh * p.L + row));
-                    }
-                }
-            }
-            if (lane == 0) counters[0] = hh + 1;
-            // the next head's K (and V) tile into L2 while this head runs
-            if (hh + 1 < H) {
-                const size_t bh1 = bh + 1;
+            if (c == 0) {
+                if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
                 if (is_ctx) {
                     if (lane == 0) {
-                        for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh1 * p.L + t0));
-                        if (ROLE_K)
-                            for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh1 * p.L + t0));
-                    }
-                } else if (lane < gcnt) {
-                    const int row = p.S + kBlock * my_n;
-                    for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc8, c * 64, (int)(bh1 * p.L + row));
-                    if (ROLE_K)
-                        for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v8, c * 64, (int)(bh1 * p.L + row));
-                }
-            }
-            for (int c = 0; c < nchunks; ++c, ++q) {
-                if (q >= 1 && !warp_all(mbar_wait(chfree, (q - 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                const int r0 = row0 + c * kRC;
-                // per-row metadata of the chunk
-                for (int rr = lane; rr < kRC; rr += 32) {
-                    const int rowi = r0 + rr;
-                    const bool in = rowi < row0 + nrows;
-                    mA[rr] = in ? sa[rowi / kBlock] : -1;
-                    mlse[rr] = in ? p.lses[bh * p.R + rowi] : 0.f;
-                    mD[rr] = in ? p.ds_[bh * p.R + rowi] : 0.f;
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(chfull, 8 * kRChunk);
-                    for (int cc = 0; cc < 4; cc++) {
-                        tma_load_2d(sm + oQ + cc * kRChunk, &tm_qs, chfull, cc * 64, (int)(bh * p.R + r0));
-                        tma_load_2d(sm + oDO + cc * kRChunk, &tm_dos, chfull, cc * 64, (int)(bh * p.R + r0));
-                    }
-                    counters[1] = q + 1;
-                    // the following chunk (this head's next, or the next head's first) into L2
-                    const bool last = c + 1 == nchunks;
-                    if (!last || hh + 1 < H) {
-                        const size_t nrow = (last ? bh + 1 : bh) * p.R + (last ? row0 : r0 + kRC);
-                        for (int cc = 0; cc < 4; cc++) {
-                            tma_prefetch_2d(&tm_qs, cc * 64, (int)nrow);
-                            tma_prefetch_2d(&tm_dos, cc * 64, (int)nrow);
+                        mbar_arrive_expect_tx(kvfull, (role_k ? 8 : 4) * kKChunk);
+                        for (int cc = 0; cc < 3; cc++)
+                            tma_load_2d(sm + oK + cc * kKChunk, &tm_kc, kvfull, cc * 64, (int)(bh * p.L + t0));
+                        tma_load_2d(sm + oK + 3 * kKChunk, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
+                        if (role_k)
+                            for (int cc = 0; cc < 4; cc++)
+                                tma_load_2d(sm + oV + cc * kKChunk, &tm_v, kvfull, cc * 64, (int)(bh * p.L + t0));
+                        if (hh + 1 < H) {  // the next head's tiles into L2
+                            for (int cc = 0; cc < 3; cc++) tma_prefetch_2d(&tm_kc, cc * 64, (int)((bh + 1) * p.L + t0));
+                            if (role_k)
+                                for (int cc = 0; cc < 4; cc++) tma_prefetch_2d(&tm_v, cc * 64, (int)((bh + 1) * p.L + t0));
                         }
+                    }
+                } else {
+                    if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * (role_k ? 2 : 1) * kDQK * 2);
+                    for (int bb = 0; bb < gcnt; ++bb) {
+                        const int nb = __shfl_sync(0xffffffffu, my_n, bb);
+                        if (lane == 0) {
+                            const int row = p.S + kBlock * nb;
+                            for (int cc = 0; cc < 3; cc++)
+                                tma_load_2d(sm + oK + cc * kKChunk + bb * 1024, &tm_kc8, kvfull, cc * 64,
+                                            (int)(bh * p.L + row));
+                            tma_load_2d(sm + oK + 3 * kKChunk + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
+                            if (role_k)
+                                for (int cc = 0; cc < 4; cc++)
+                                    tma_load_2d(sm + oV + cc * kKChunk + bb * 1024, &tm_v8, kvfull, cc * 64,
+                                                (int)(bh * p.L + row));
+                        }
+                    }
+                }
+                if (lane == 0) counters[0] = hh + 1;
+            }
+            if (q >= 2 && !warp_all(mbar_wait(&chfree[s], ((q >> 1) - 1) & 1, abort_flag))) break;
+            const int r0 = row0 + c * kRC;
+            // chunk metadata: anchor (INT_MAX past the band), LSE*log2(e), D
+            int *mA = reinterpret_cast<int *>(sm + oMeta + s * kRC * 12);
+            float2 *mLD = reinterpret_cast<float2 *>(mA + kRC);
+            {
+                const int rowi = r0 + lane;
+                const bool in = rowi < row0 + nrows;
+                mA[lane] = in ? sa[rowi / kBlock] : 0x7fffffff;
+                mLD[lane] = in ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi]) : make_float2(0.f, 0.f);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&chfull[s], 8 * kRChunk);
+                for (int cc = 0; cc < 4; cc++) {
+                    tma_load_2d(sm + (s ? oQ1 : oQ0) + cc * kRChunk, &tm_qs, &chfull[s], cc * 64, (int)(bh * p.R + r0));
+                    tma_load_2d(sm + (s ? oD1 : oD0) + cc * kRChunk, &tm_dos, &chfull[s], cc * 64, (int)(bh * p.R + r0));
+                }
+                counters[1] = q + 1;
+                if (q + 2 < QT) {  // two chunks ahead into L2
+                    const int q2 = q + 2, h2 = q2 / nchunks, c2 = q2 % nchunks;
+                    const size_t nrow = ((size_t)b * p.n_h + h0 + h2) * p.R + row0 + c2 * kRC;
+                    for (int cc = 0; cc < 4; cc++) {
+                        tma_prefetch_2d(&tm_qs, cc * 64, (int)nrow);
+                        tma_prefetch_2d(&tm_dos, cc * 64, (int)nrow);
                     }
                 }
             }
         }
-        cp_async_wait_all();
-    } else if (warp == 5) {
+    } else if (warp == kKeyWarps + 1) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idS = idesc_bf16(kMK, kRC, 0);    // S^T, dP^T: B = Q / dO chunk, K-major
-            const uint32_t idA = idesc_bf16(kMK, 256, 1);    // acc: B = dO / Q chunk, MN-major
+            const uint32_t idS = idesc_bf16(kMK, kRC, 0);   // S^T, dP^T: B = Q / dO chunk, K-major
+            const uint32_t idA = idesc_bf16(kMK, 256, 1);   // acc: B = dO / Q chunk, MN-major
             const uint32_t ka = smem_u32(sm + oK), va = smem_u32(sm + oV);
-            const uint32_t qb = smem_u32(sm + oQ), db = smem_u32(sm + oDO), pa = smem_u32(sm + oPT);
-            int q = 0;
             bool ok = true;
-            for (int hh = 0; hh < H && ok; ++hh) {
-                ok = mbar_wait(kvfull, hh & 1, abort_flag);
-                if (!ok) break;
-                counters[2] = hh + 1;
-                for (int c = 0; c < nchunks; ++c, ++q) {
-                    ok = mbar_wait(chfull, q & 1, abort_flag);
+            auto do_acc = [&](int q) {
+                const int hh = q / nchunks, c = q % nchunks, s = q & 1;
+                bool r = mbar_wait(&dsready[s], (q >> 1) & 1, abort_flag);
+                if (r && c == 0 && hh >= 1) r = mbar_wait(epidone, (hh - 1) & 1, abort_flag);
+                if (!r) return false;
+                tc_fence_after();
+                const uint32_t pa = smem_u32(sm + (s ? oP1 : oP0));
+                const uint32_t bsrc = smem_u32(sm + (role_k ? (s ? oQ1 : oQ0) : (s ? oD1 : oD0)));
+#pragma unroll
+                for (int kk = 0; kk < kRC / 16; ++kk)
+                    mma_bf16_ss(tmem + kColAcc, sdesc_sw128(pa + kk * 32, 16, 1024),
+                                sdesc_sw128(bsrc + kk * 2048, kRChunk, 1024), idA, (c > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&chfree[s]);
+                if (c == nchunks - 1) mma_commit(accdone);
+                return true;
+            };
+            for (int q = 0; q < QT && ok; ++q) {
+                const int hh = q / nchunks, c = q % nchunks, s = q & 1;
+                if (c == 0) {
+                    ok = mbar_wait(kvfull, hh & 1, abort_flag);
                     if (!ok) break;
-                    counters[3] = q + 1;
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < kDQK / 16; ++k) {
-                        const int cc = k >> 2, sub = k & 3;
-                        mma_bf16_ss(tmem + kColS, sdesc_sw128(ka + cc * kKChunk + sub * 32, 16, 1024),
-                                    sdesc_sw128(qb + cc * kRChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
-                    }
-                    if (ROLE_K) {
-#pragma unroll
-                        for (int k = 0; k < kDV / 16; ++k) {
-                            const int cc = k >> 2, sub = k & 3;
-                            mma_bf16_ss(tmem + kColP, sdesc_sw128(va + cc * kKChunk + sub * 32, 16, 1024),
-                                        sdesc_sw128(db + cc * kRChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
-                        }
-                    }
-                    mma_commit(sfull);
-                    if (c == nchunks - 1) mma_commit(kvfree);
-                    ok = mbar_wait(dsready, q & 1, abort_flag);
-                    if (ok && c == 0 && hh >= 1) ok = mbar_wait(epidone, (hh - 1) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t bsrc = ROLE_K ? qb : db;
-#pragma unroll
-                    for (int k = 0; k < kRC / 16; ++k)
-                        mma_bf16_ss(tmem + kColAcc, sdesc_sw128(pa + k * 32, 16, 1024),
-                                    sdesc_sw128(bsrc + k * 2048, kRChunk, 1024), idA, (c > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(chfree);
-                    if (c == nchunks - 1) mma_commit(accdone);
+                    counters[2] = hh + 1;
                 }
+                ok = mbar_wait(&chfull[s], (q >> 1) & 1, abort_flag);
+                if (!ok) break;
+                counters[3] = q + 1;
+                tc_fence_after();
+                const uint32_t qb = smem_u32(sm + (s ? oQ1 : oQ0)), db = smem_u32(sm + (s ? oD1 : oD0));
+#pragma unroll
+                for (int kk = 0; kk < kDQK / 16; ++kk) {
+                    const int cc = kk >> 2, sub = kk & 3;
+                    mma_bf16_ss(tmem + kColS + s * kRC, sdesc_sw128(ka + cc * kKChunk + sub * 32, 16, 1024),
+                                sdesc_sw128(qb + cc * kRChunk + sub * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                }
+                if (role_k) {
+#pragma unroll
+                    for (int kk = 0; kk < kDV / 16; ++kk) {
+                        const int cc = kk >> 2, sub = kk & 3;
+                        mma_bf16_ss(tmem + kColP + s * kRC, sdesc_sw128(va + cc * kKChunk + sub * 32, 16, 1024),
+                                    sdesc_sw128(db + cc * kRChunk + sub * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(&sfull[s]);
+                if (c == nchunks - 1) mma_commit(kvfree);
+                if (q >= 1 && !(ok = do_acc(q - 1))) break;
             }
+            if (ok && QT > 0) do_acc(QT - 1);
         }
     } else {
-        // ------------------------------------------------ keys (warps 0-3)
-        const int k = threadIdx.x;  // key slot = TMEM lane
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        float racc[kDR];
+        // ------------------------------------------ key warps (0..7)
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const int kpos = t0 + k;               // context position of this key (context tiles)
+        const int kblk = k / 8;                // draft tiles: the key's block within the group
+        const int col0 = half * (kRC / 2);     // this warp's rows within a chunk
+        float racc[kDR];                       // rope slice of dK summed over heads (half-1 warps)
 #pragma unroll
         for (int i = 0; i < kDR; i++) racc[i] = 0.f;
-        int q = 0;
         bool ok = true;
-        const int kpos = t0 + k;                     // context position of this key (context tiles)
-        const int kblk = is_ctx ? 0 : k / 8;         // draft tiles: the key's block within the group
-        for (int hh = 0; hh < H && ok; ++hh) {
-            const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            for (int c = 0; c < nchunks; ++c, ++q) {
-                // chunk q's row metadata (written by the producer) and its S^T
-                ok = warp_all(mbar_wait(chfull, q & 1, abort_flag));
-                if (ok) ok = warp_all(mbar_wait(sfull, q & 1, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-                float sv[64];
-                float pv[ROLE_K ? 64 : 1];
-                {
-                    float a0[32], a1[32];
-                    tmem_ld32(trow + kColS, a0);
-                    tmem_ld32(trow + kColS + 32, a1);
-                    if (ROLE_K) {
-                        float b0[32], b1[32];
-                        tmem_ld32(trow + kColP, b0);
-                        tmem_ld32(trow + kColP + 32, b1);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; i++) {
-                            pv[i] = b0[i];
-                            pv[32 + i] = b1[i];
-                        }
-                    } else {
-                        tmem_wait_ld();
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        sv[i] = a0[i];
-                        sv[32 + i] = a1[i];
-                    }
-                }
-                if (q >= 1) {
-                    ok = warp_all(mbar_wait(chfree, (q - 1) & 1, abort_flag));
-                    if (!ok) break;
-                }
-                const int crow0 = row0 + c * kRC;  // sorted row of column 0
-                uint8_t *prow = sm + oPT;
-#pragma unroll
-                for (int u = 0; u < kRC / 8; u++) {
-                    float e[8];
-#pragma unroll
-                    for (int i = 0; i < 8; i++) {
-                        const int col = u * 8 + i;
-                        const int A = mA[col];
-                        bool valid;
-                        if (is_ctx)
-                            valid = A >= 0 && kpos < A && kpos >= A - p.W + 1;
-                        else
-                            valid = A >= 0 && key_valid && (crow0 + col - row0) / kBlock == kblk;  // own block
-                        const float pp = valid ? ex2(fmaf(sv[col], p.scale_log2, -mlse[col])) : 0.f;
-                        if (ROLE_K)
-                            e[i] = pp * (pv[col] - mD[col]) * p.scale;
-                        else
-                            e[i] = pp;
-                    }
-                    *reinterpret_cast<uint4 *>(prow + sw128(k, u)) =
-                        make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
-                                   pack_bf16x2(e[6], e[7]));
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(dsready);
-            }
+        for (int q = 0; q < QT && ok; ++q) {
+            const int hh = q / nchunks, c = q % nchunks, s = q & 1;
+            ok = warp_all(mbar_wait(&chfull[s], (q >> 1) & 1, abort_flag));
+            if (ok) ok = warp_all(mbar_wait(&sfull[s], (q >> 1) & 1, abort_flag));
             if (!ok) break;
-            // head epilogue: the accumulator holds dV (dK) of this head's keys
+            tc_fence_after();
+            float sv[16], pv[16];
+            {
+                float a[32];
+                tmem_ld32(trow + kColS + s * kRC, a);  // all 32 rows; this warp uses its half
+                if (role_k) {
+                    float bq[32];
+                    tmem_ld32(trow + kColP + s * kRC, bq);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; i++) pv[i] = half ? bq[16 + i] : bq[i];
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; i++) pv[i] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; i++) sv[i] = half ? a[16 + i] : a[i];
+            }
+            // rows of the chunk that see this key: one contiguous range [jlo, jhi)
+            const int *mA = reinterpret_cast<const int *>(sm + oMeta + s * kRC * 12);
+            const float2 *mLD = reinterpret_cast<const float2 *>(mA + kRC);
+            int jlo, jhi;
+            if (is_ctx) {
+                // rows are anchor-sorted: visible iff kpos < A <= kpos + W - 1
+                int lo = 0, hi = kRC;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (mA[mid] > kpos) hi = mid; else lo = mid + 1;
+                }
+                jlo = lo;
+                const long long lim = (long long)kpos + p.W - 1;
+                hi = kRC;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if ((long long)mA[mid] > lim) hi = mid; else lo = mid + 1;
+                }
+                jhi = lo;
+            } else {
+                jlo = kBlock * kblk - c * kRC;  // the key's own block rows
+                jhi = jlo + kBlock;
+            }
+            if (!key_valid) jhi = jlo;
+            if (q >= 2) {
+                ok = warp_all(mbar_wait(&chfree[s], ((q >> 1) - 1) & 1, abort_flag));
+                if (!ok) break;
+            }
+            float e[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int j = col0 + i;
+                const float2 ld = mLD[j];
+                const float pp = (j >= jlo && j < jhi) ? ex2(fmaf(sv[i], p.scale_log2, -ld.x)) : 0.f;
+                e[i] = role_k ? pp * (pv[i] - ld.y) * p.scale : pp;
+            }
+            uint8_t *prow = sm + (s ? oP1 : oP0);
+#pragma unroll
+            for (int u = 0; u < 2; u++)
+                *reinterpret_cast<uint4 *>(prow + sw128(k, 2 * half + u)) =
+                    make_uint4(pack_bf16x2(e[8 * u + 0], e[8 * u + 1]), pack_bf16x2(e[8 * u + 2], e[8 * u + 3]),
+                               pack_bf16x2(e[8 * u + 4], e[8 * u + 5]), pack_bf16x2(e[8 * u + 6], e[8 * u + 7]));
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dsready[s]);
+            if (c != nchunks - 1) continue;
+            // head epilogue: accumulator columns [128 * half, 128 * half + 128)
             ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const int out_cols = ROLE_K ? kDC : kDV;
-#pragma unroll 1
-            for (int c = 0; c < out_cols; c += 32) {
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int col = half * 128 + cc * 32;
                 float v[32];
-                tmem_ld32(trow + kColAcc + c, v);
+                tmem_ld32(trow + kColAcc + col, v);
                 tmem_wait_ld();
-                if (key_valid) {
-                    __nv_bfloat16 *dst = ROLE_K ? p.dkc + (bh * p.L + key_pos) * kDC + c
-                                                : p.dv + (bh * p.L + key_pos) * kDV + c;
+                if (role_k && half == 1 && cc >= 2) {  // rope slice of dK (columns 192..255)
 #pragma unroll
-                    for (int i = 0; i < 4; i++)
-                        *reinterpret_cast<uint4 *>(dst + 8 * i) = make_uint4(
-                            pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                            pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                    for (int i = 0; i < 32; i++) racc[(cc - 2) * 32 + i] += v[i];
+                    continue;
                 }
-            }
-            if (ROLE_K) {  // rope slice of dK: summed over the group's heads
-                float v0[32], v1[32];
-                tmem_ld32(trow + kColAcc + kDC, v0);
-                tmem_ld32(trow + kColAcc + kDC + 32, v1);
-                tmem_wait_ld();
+                if (!key_valid) continue;
+                __nv_bfloat16 *dst = role_k ? p.dkc + (bh * p.L + key_pos) * kDC + col
+                                            : p.dv + (bh * p.L + key_pos) * kDV + col;
 #pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    racc[i] += v0[i];
-                    racc[32 + i] += v1[i];
-                }
+                for (int i = 0; i < 4; i++)
+                    *reinterpret_cast<uint4 *>(dst + 8 * i) = make_uint4(
+                        pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                        pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(epidone);
         }
-        if (ok && ROLE_K && key_valid) {
-            float4 *d = reinterpret_cast<float4 *>(p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR);
+        if (ok && role_k && key_valid && half == 1) {
+            // this warp held accumulator columns 128..255: dK^C 128..191 and the rope slice 192..255
+            float4 *d = reinterpret_cast<float4 *>(dkr_part_row);
 #pragma unroll
             for (int i = 0; i < kDR / 4; i++) d[i] = make_float4(racc[4 * i], racc[4 * i + 1], racc[4 * i + 2], racc[4 * i + 3]);
         }
@@ -893,18 +890,18 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     __syncthreads();
     if (*abort_flag) {
         volatile int never = 0;
-        if (warp == 4 && lane == 0) {
+        if (warp == kKeyWarps && lane == 0) {
             for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(kvfull, t & 1, (volatile int *)&never);
-            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(chfull, t & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(&chfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
         }
-        if (warp == 5 && lane == 0) {
+        if (warp == kKeyWarps + 1 && lane == 0) {
             mma_commit(drain);
             mbar_wait(drain, 0, (volatile int *)&never);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kKeyWarps + 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -954,8 +951,9 @@ bool bwd_tc_supported(const Prob &p) {
 
 int bwd_head_groups(const Prob &p) {
     const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kGD - 1) / kGD) * p.B;
+    // two CTA roles per key tile; aim for about four waves on 148 SMs
     int hg = 1;
-    while (hg < p.n_h && items * hg < 2 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
+    while (hg < p.n_h && 2 * items * hg < 4 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
     return hg;
 }
 
@@ -973,14 +971,14 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs64, m_dos64, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs32, m_dos32, m_kc8, m_kr8, m_v8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
     if (p.N > 0 && q_rows > 0) {
         if (!make_map_bf16(&m_kc32, kc, kDC, kv_rows, 32) || !make_map_bf16(&m_kr32, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 32) ||
             !make_map_bf16(&m_v32, v, kDV, kv_rows, 32) || !make_map_bf16(&m_qs128, qs, kDQK, q_rows, 128) ||
-            !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map_bf16(&m_qs64, qs, kDQK, q_rows, 64) ||
-            !make_map_bf16(&m_dos64, dos, kDV, q_rows, 64))
+            !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map_bf16(&m_qs32, qs, kDQK, q_rows, 32) ||
+            !make_map_bf16(&m_dos32, dos, kDV, q_rows, 32))
             return cudaErrorInvalidValue;
     }
     if (!make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) || !make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
@@ -989,8 +987,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         !make_map_bf16(&m_v128, v, kDV, kv_rows, 128))
         return cudaErrorInvalidValue;
     if (p.N == 0 || q_rows == 0) {  // maps over Q rows are never read: any valid map will do
-        m_qs64 = m_kc128;
-        m_dos64 = m_kc128;
+        m_qs32 = m_kc128;
+        m_dos32 = m_kc128;
     }
     BwdArgs a;
     a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
@@ -1022,17 +1020,12 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
             m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc8, m_kr8, m_v8, a);
     }
-    const dim3 kv_grid(a.n_ctx_items + (p.N + kGD - 1) / kGD, HG, p.B);
-    e = cudaFuncSetAttribute(k_bwd_kv_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_bwd_kv_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
+    const dim3 kv_grid(2 * (a.n_ctx_items + (p.N + kGD - 1) / kGD), HG, p.B);
+    e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_kv_tc<false><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, m_kc8,
-                                                                  m_kr8, m_v8, a);
-    count_launch();
-    k_bwd_kv_tc<true><<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs64, m_dos64, m_kc8,
-                                                                 m_kr8, m_v8, a);
+    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs32, m_dos32, m_kc8, m_kr8,
+                                                        m_v8, a);
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
     k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
