@@ -2,6 +2,8 @@
 // workspace layout, and the launch sequence of each entry point.
 #include <atomic>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "dspark_internal.cuh"
@@ -72,9 +74,20 @@ dspark_status check_tensor(const void *ptr, size_t elems) {
         if (_s != DSPARK_OK) return _s;        \
     } while (0)
 
-#define DSPARK_CUDA(x)                                  \
-    do {                                                \
-        if ((x) != cudaSuccess) return DSPARK_ERR_CUDA; \
+// With DSPARK_VERBOSE set in the environment, failing CUDA calls are printed
+// to stderr with the call that failed.
+bool verbose() {
+    static const bool v = getenv("DSPARK_VERBOSE") != nullptr;
+    return v;
+}
+
+#define DSPARK_CUDA(x)                                                                           \
+    do {                                                                                         \
+        const cudaError_t _e = (x);                                                              \
+        if (_e != cudaSuccess) {                                                                 \
+            if (verbose()) fprintf(stderr, "dspark: %s failed: %s\n", #x, cudaGetErrorString(_e)); \
+            return DSPARK_ERR_CUDA;                                                              \
+        }                                                                                        \
     } while (0)
 
 struct Sizes {

@@ -142,6 +142,7 @@ constexpr int kTile = 4 * kKChunk;     // 16 KB
 constexpr int oQ = 0, oDO = oQ + 4 * kQChunk, oK0 = oDO + 4 * kQChunk, oK1 = oK0 + kTile, oV0 = oK1 + kTile,
               oV1 = oV0 + kTile, oS0 = oV1 + kTile, oS1 = oS0 + kQChunk, oBar = oS1 + kQChunk;
 constexpr int kSmem = oBar + 256 + 1024;
+static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 constexpr int kThreads = 192;
 constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320;  // S: 256/288, dP: 320/352
 }  // namespace dq
@@ -447,7 +448,10 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         if (ok) ok = warp_all(mbar_wait(&dqdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
         if (ok) {
             tc_fence_after();
-            __nv_bfloat16 *orow = p.dq + (bh * p.R + kBlock * n + j) * kDQK;
+            // dQ row (rope slice rotated back by A + j) -> staging in the idle
+            // K/V stages (unit u of row r at u ^ (r & 31)) -> one 512-byte row
+            // per warp instruction
+            uint8_t *stage = sm + oK0 + warp * (32 * kDQK * 2);
 #pragma unroll 1
             for (int c = 0; c < kDQK; c += 32) {
                 float v[32];
@@ -463,13 +467,21 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                         v[2 * k + 1] = x1 * t2.x - x0 * t2.y;
                     }
                 }
-                if (live) {
 #pragma unroll
-                    for (int k = 0; k < 4; k++)
-                        *reinterpret_cast<uint4 *>(orow + c + 8 * k) = make_uint4(
-                            pack_bf16x2(v[8 * k + 0], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
-                            pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+                for (int k = 0; k < 4; k++) {
+                    const int u = c / 8 + k;
+                    *reinterpret_cast<uint4 *>(stage + lane * 512 + ((u ^ lane) << 4)) = make_uint4(
+                        pack_bf16x2(v[8 * k + 0], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                        pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
                 }
+            }
+            __syncwarp();
+            for (int i = 0; i < 32; i++) {
+                const int rr = warp * 32 + i;
+                if (rr >= nrows) break;  // uniform
+                const int ni = __shfl_sync(0xffffffffu, n, i), ji = __shfl_sync(0xffffffffu, j, i);
+                const uint4 val = *reinterpret_cast<const uint4 *>(stage + i * 512 + ((lane ^ i) << 4));
+                *reinterpret_cast<uint4 *>(p.dq + (bh * p.R + kBlock * ni + ji) * kDQK + 8 * lane) = val;
             }
         }
     }
@@ -507,6 +519,12 @@ constexpr int oK = 0, oV = oK + 4 * kKChunk, oQ0 = oV + 4 * kKChunk, oQ1 = oQ0 +
               oD0 = oQ1 + 4 * kRChunk, oD1 = oD0 + 4 * kRChunk, oP0 = oD1 + 4 * kRChunk, oP1 = oP0 + kPT,
               oMeta = oP1 + kPT, oBar = oMeta + 2 * kRC * 12;
 constexpr int kSmem = oBar + 256 + 1024;
+static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+// The head epilogue stages through both P^T / dS^T buffers: by then the MMAs
+// that read them have completed, and the key warps write them again only
+// after the epilogue.
+constexpr int oStage = oP0;
+static_assert(2 * kPT >= 8 * 32 * 128, "epilogue staging does not fit");
 constexpr int kKeyWarps = 8;             // two per TMEM sub-partition, each half of a chunk's rows
 constexpr int kThreads = (kKeyWarps + 2) * 32;
 constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320;  // S^T: 256 / 288, dP^T: 320 / 352
@@ -775,6 +793,31 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         const int kpos = t0 + k;               // context position of this key (context tiles)
         const int kblk = k / 8;                // draft tiles: the key's block within the group
         const int col0 = half * (kRC / 2);     // this warp's rows within a chunk
+        // The rows that see this key, in sorted-row order relative to the band:
+        // one range [rlo, rhi), the same for every head. Context key: blocks
+        // with kpos < A <= kpos + W - 1; draft key slot: its own block.
+        int rlo = 0, rhi = 0;
+        if (key_valid) {
+            if (is_ctx) {
+                int lo = row0 / kBlock, hi = (row0 + nrows) / kBlock;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (sa[mid] > kpos) hi = mid; else lo = mid + 1;
+                }
+                rlo = kBlock * lo - row0;
+                const long long lim = (long long)kpos + p.W - 1;
+                hi = (row0 + nrows) / kBlock;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if ((long long)sa[mid] > lim) hi = mid; else lo = mid + 1;
+                }
+                rhi = kBlock * lo - row0;
+            } else {
+                rlo = kBlock * kblk;
+                rhi = rlo + kBlock;
+            }
+        }
+        uint8_t *stage = sm + oStage + warp * (32 * 128);
         float racc[kDR];                       // rope slice of dK summed over heads (half-1 warps)
 #pragma unroll
         for (int i = 0; i < kDR; i++) racc[i] = 0.f;
@@ -803,30 +846,9 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; i++) sv[i] = half ? a[16 + i] : a[i];
             }
-            // rows of the chunk that see this key: one contiguous range [jlo, jhi)
-            const int *mA = reinterpret_cast<const int *>(sm + oMeta + s * kRC * 12);
-            const float2 *mLD = reinterpret_cast<const float2 *>(mA + kRC);
-            int jlo, jhi;
-            if (is_ctx) {
-                // rows are anchor-sorted: visible iff kpos < A <= kpos + W - 1
-                int lo = 0, hi = kRC;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (mA[mid] > kpos) hi = mid; else lo = mid + 1;
-                }
-                jlo = lo;
-                const long long lim = (long long)kpos + p.W - 1;
-                hi = kRC;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if ((long long)mA[mid] > lim) hi = mid; else lo = mid + 1;
-                }
-                jhi = lo;
-            } else {
-                jlo = kBlock * kblk - c * kRC;  // the key's own block rows
-                jhi = jlo + kBlock;
-            }
-            if (!key_valid) jhi = jlo;
+            // rows of the chunk that see this key: [jlo, jhi)
+            const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + s * kRC * 12 + kRC * 4);
+            const int jlo = rlo - c * kRC, jhi = rhi - c * kRC;
             if (q >= 2) {
                 ok = warp_all(mbar_wait(&chfree[s], ((q >> 1) - 1) & 1, abort_flag));
                 if (!ok) break;
@@ -855,28 +877,48 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
+            // Accumulator columns [128 * half, +128) of the warp's 32 keys, in
+            // two rounds of 64: each thread stages its key's 64 values (bf16,
+            // 16-byte unit u at u ^ (key & 7)), then the warp writes 4 keys'
+            // 128-byte row segments per instruction.
 #pragma unroll
-            for (int cc = 0; cc < 4; cc++) {
-                const int col = half * 128 + cc * 32;
-                float v[32];
-                tmem_ld32(trow + kColAcc + col, v);
+            for (int rd = 0; rd < 2; rd++) {
+                const int col = half * 128 + rd * 64;
+                float v[64];
+                tmem_ld32(trow + kColAcc + col, *reinterpret_cast<float(*)[32]>(&v[0]));
+                tmem_ld32(trow + kColAcc + col + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
                 tmem_wait_ld();
-                if (role_k && half == 1 && cc >= 2) {  // rope slice of dK (columns 192..255)
+                if (role_k && col >= kDC) {  // rope slice of dK (columns 192..255): summed over heads
 #pragma unroll
-                    for (int i = 0; i < 32; i++) racc[(cc - 2) * 32 + i] += v[i];
+                    for (int i = 0; i < 64; i++) racc[i] += v[i];
                     continue;
                 }
-                if (!key_valid) continue;
-                __nv_bfloat16 *dst = role_k ? p.dkc + (bh * p.L + key_pos) * kDC + col
-                                            : p.dv + (bh * p.L + key_pos) * kDV + col;
 #pragma unroll
-                for (int i = 0; i < 4; i++)
-                    *reinterpret_cast<uint4 *>(dst + 8 * i) = make_uint4(
-                        pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                        pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                for (int u = 0; u < 8; u++)
+                    *reinterpret_cast<uint4 *>(stage + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                        make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                   pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+                __syncwarp();
+                const int rowstride = role_k ? kDC : kDV;
+                __nv_bfloat16 *base = role_k ? p.dkc : p.dv;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int kl = 4 * i + (lane >> 3), u = lane & 7;   // key within the warp, unit
+                    const int kk = (warp & 3) * 32 + kl;
+                    const int kkv = __shfl_sync(0xffffffffu, (int)key_valid, kl);
+                    const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
+                    if (kkv) {
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 128 + ((u ^ (kl & 7)) << 4));
+                        *reinterpret_cast<uint4 *>(base + (bh * p.L + (size_t)kposl) * rowstride + col + 8 * u) = val;
+                    }
+                    (void)kk;
+                }
+                __syncwarp();
             }
             tc_fence_before();
-            __syncwarp();
+            // every key warp is done with the staging (both P buffers) before
+            // any of them writes the next chunk's P^T / dS^T there
+            asm volatile("bar.sync 1, %0;" ::"r"(kKeyWarps * 32) : "memory");
             if (lane == 0) mbar_arrive(epidone);
         }
         if (ok && role_k && key_valid && half == 1) {

@@ -61,6 +61,7 @@ constexpr int oStage = oV1;
 static_assert(oP1 + kPBytes - oStage >= kM * kDQK * 2, "staging area too small");
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 constexpr int kSmemBytes = oBar + 256 + 1024;  // barriers + alignment slack
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
@@ -431,25 +432,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t row = bh * p.R + kBlock * n + j;
-            __nv_bfloat16 *orow = p.o + row * kDV;
+            // O row -> staging (the idle K stages; unit u of row r at u ^ (r & 31))
+            // -> one 512-byte row per warp instruction
+            uint8_t *stage = sm + oK0 + warp * (32 * kDV * 2);
 #pragma unroll 1
             for (int c = 0; c < kDV; c += 32) {
                 float ov[32];
                 tmem_ld32(trow + kColO + c, ov);
                 tmem_wait_ld();
-                if (live) {
 #pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        uint4 pk = make_uint4(pack_bf16x2(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv),
-                                              pack_bf16x2(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv),
-                                              pack_bf16x2(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv),
-                                              pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
-                        *reinterpret_cast<uint4 *>(orow + c + 8 * k) = pk;
-                    }
+                for (int k = 0; k < 4; k++) {
+                    const int u = c / 8 + k;
+                    *reinterpret_cast<uint4 *>(stage + lane * 512 + ((u ^ lane) << 4)) =
+                        make_uint4(pack_bf16x2(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv),
+                                   pack_bf16x2(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv),
+                                   pack_bf16x2(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv),
+                                   pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
                 }
             }
-            if (live) p.lse[row] = (m_used + log2f(l)) * kLn2;
+            __syncwarp();
+            for (int i = 0; i < 32; i++) {
+                const int rr = warp * 32 + i;
+                if (rr >= nrows) break;  // uniform
+                const int ni = __shfl_sync(0xffffffffu, n, i), ji = __shfl_sync(0xffffffffu, j, i);
+                const uint4 val = *reinterpret_cast<const uint4 *>(stage + i * 512 + ((lane ^ i) << 4));
+                *reinterpret_cast<uint4 *>(p.o + (bh * p.R + kBlock * ni + ji) * kDV + 8 * lane) = val;
+            }
+            if (live) p.lse[bh * p.R + kBlock * n + j] = (m_used + log2f(l)) * kLn2;
         }
     }
 
