@@ -739,32 +739,8 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             const uint32_t idA = idesc_bf16(kMK, 256, 1);   // acc: B = dO / Q chunk, MN-major
             const uint32_t ka = smem_u32(sm + oK), va = smem_u32(sm + oV);
             bool ok = true;
-            auto do_acc = [&](int q) {
-                const int hh = q / nchunks, c = q % nchunks, s = q & 1;
-                bool r = mbar_wait(&dsready[s], (q >> 1) & 1, abort_flag);
-                if (r && c == 0 && hh >= 1) r = mbar_wait(epidone, (hh - 1) & 1, abort_flag);
-                if (!r) return false;
-                tc_fence_after();
-                const uint32_t pa = smem_u32(sm + (s ? oP1 : oP0));
-                const uint32_t bsrc = smem_u32(sm + (role_k ? (s ? oQ1 : oQ0) : (s ? oD1 : oD0)));
-#pragma unroll
-                for (int kk = 0; kk < kRC / 16; ++kk)
-                    mma_bf16_ss(tmem + kColAcc, sdesc_sw128(pa + kk * 32, 16, 1024),
-                                sdesc_sw128(bsrc + kk * 2048, kRChunk, 1024), idA, (c > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&chfree[s]);
-                if (c == nchunks - 1) mma_commit(accdone);
-                return true;
-            };
-            for (int q = 0; q < QT && ok; ++q) {
-                const int hh = q / nchunks, c = q % nchunks, s = q & 1;
-                if (c == 0) {
-                    ok = mbar_wait(kvfull, hh & 1, abort_flag);
-                    if (!ok) break;
-                    counters[2] = hh + 1;
-                }
-                ok = mbar_wait(&chfull[s], (q >> 1) & 1, abort_flag);
-                if (!ok) break;
-                counters[3] = q + 1;
+            auto issue_s = [&](int q) {
+                const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
                 const uint32_t qb = smem_u32(sm + (s ? oQ1 : oQ0)), db = smem_u32(sm + (s ? oD1 : oD0));
 #pragma unroll
@@ -783,9 +759,60 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 }
                 mma_commit(&sfull[s]);
                 if (c == nchunks - 1) mma_commit(kvfree);
-                if (q >= 1 && !(ok = do_acc(q - 1))) break;
+            };
+            auto issue_acc = [&](int q) {
+                const int c = q % nchunks, s = q & 1;
+                tc_fence_after();
+                const uint32_t pa = smem_u32(sm + (s ? oP1 : oP0));
+                const uint32_t bsrc = smem_u32(sm + (role_k ? (s ? oQ1 : oQ0) : (s ? oD1 : oD0)));
+#pragma unroll
+                for (int kk = 0; kk < kRC / 16; ++kk)
+                    mma_bf16_ss(tmem + kColAcc, sdesc_sw128(pa + kk * 32, 16, 1024),
+                                sdesc_sw128(bsrc + kk * 2048, kRChunk, 1024), idA, (c > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&chfree[s]);
+                if (c == nchunks - 1) mma_commit(accdone);
+            };
+            // Issue whichever is ready: S^T of chunk ns (its K/V tile and row
+            // chunk landed; at most one chunk ahead, so its S buffer was
+            // released by the accumulation of chunk ns - 2) or the
+            // accumulation of chunk na (its P^T / dS^T is written and, at a
+            // head's first chunk, the previous head's epilogue has read the
+            // accumulator).
+            int ns = 0, na = 0;
+            uint64_t t_idle = 0;
+            while (ok && na < QT) {
+                bool issued = false;
+                if (ns < QT && ns <= na + 1) {
+                    const int hh = ns / nchunks, c = ns % nchunks, s = ns & 1;
+                    if ((c != 0 || mbar_try_wait(kvfull, hh & 1)) && mbar_try_wait(&chfull[s], (ns >> 1) & 1)) {
+                        if (c == 0) counters[2] = hh + 1;
+                        counters[3] = ns + 1;
+                        issue_s(ns);
+                        ++ns;
+                        issued = true;
+                    }
+                }
+                if (!issued && na < ns) {
+                    const int hh = na / nchunks, c = na % nchunks, s = na & 1;
+                    if (mbar_try_wait(&dsready[s], (na >> 1) & 1) &&
+                        (c != 0 || hh == 0 || mbar_try_wait(epidone, (hh - 1) & 1))) {
+                        issue_acc(na);
+                        ++na;
+                        issued = true;
+                    }
+                }
+                if (issued) {
+                    t_idle = 0;
+                } else {
+                    const uint64_t now = globaltimer();
+                    if (t_idle == 0) t_idle = now;
+                    if (*abort_flag) ok = false;
+                    else if (now - t_idle > kWaitTimeoutNs) {
+                        *abort_flag = 1;
+                        ok = false;
+                    }
+                }
             }
-            if (ok && QT > 0) do_acc(QT - 1);
         }
     } else {
         // ------------------------------------------ key warps (0..7)
