@@ -134,13 +134,19 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
 // ================================================================ dQ
 // CTA = (group g of 25 sorted blocks, head h, batch b); warps 0-3 rows
 // (thread t = row t = TMEM lane t), warp 4 producer, warp 5 MMA.
+// A K tile is read twice (S, then dQ after the rows' dS is ready), a V tile
+// once (dP), so K gets three stages and V two.
 namespace dq {
 constexpr int kM = 128, kBN = 32;
 constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
 constexpr int kKChunk = kBN * 128;     // 4 KB: 32 keys x 64 columns
 constexpr int kTile = 4 * kKChunk;     // 16 KB
-constexpr int oQ = 0, oDO = oQ + 4 * kQChunk, oK0 = oDO + 4 * kQChunk, oK1 = oK0 + kTile, oV0 = oK1 + kTile,
-              oV1 = oV0 + kTile, oS0 = oV1 + kTile, oS1 = oS0 + kQChunk, oBar = oS1 + kQChunk;
+constexpr int kKStages = 3;
+// dS tile [128 rows][32 keys] bf16 without swizzle: 8 x 8 core matrices of
+// 8 rows x 16 bytes, K-adjacent ones 128 B apart, 8-row groups 512 B apart
+constexpr int kDS = kM * kBN * 2;      // 8 KB
+constexpr int oQ = 0, oDO = oQ + 4 * kQChunk, oK0 = oDO + 4 * kQChunk, oV0 = oK0 + kKStages * kTile,
+              oV1 = oV0 + kTile, oS0 = oV1 + kTile, oS1 = oS0 + kDS, oBar = oS1 + kDS;
 constexpr int kSmem = oBar + 256 + 1024;
 static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 constexpr int kThreads = 192;
@@ -171,11 +177,11 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kfull = bars + 0, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
-    uint64_t *sfull = bars + 8, *dsready = bars + 10, *dqdone = bars + 12, *qfull = bars + 14, *drain = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
-    int *counters = reinterpret_cast<int *>(bars + 18);  // K issued, V issued, K consumed, V consumed, q issued
+    uint64_t *kfull = bars + 0, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 8;
+    uint64_t *sfull = bars + 10, *dsready = bars + 12, *dqdone = bars + 14, *qfull = bars + 16, *drain = bars + 17;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
+    int *counters = reinterpret_cast<int *>(bars + 20);  // K issued, V issued, K consumed, V consumed, q issued
 
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int cnt = p.cnt[b];
@@ -201,9 +207,11 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < kKStages; s++) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < 2; s++) {
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
             mbar_init(&sfull[s], 1);
@@ -240,8 +248,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         const int my_n = lane < gcnt ? sn[lane] : 0;
         int pf_next = 2;
         for (int t = 0; t < T; ++t) {
-            const int s = t & 1;
-            uint8_t *kt = sm + (s ? oK1 : oK0);
+            const int s = t & 1, ks = t % kKStages;
+            uint8_t *kt = sm + oK0 + ks * kTile;
             uint8_t *vt = sm + (s ? oV1 : oV0);
             if (lane == 0) {
                 for (; pf_next <= t + 5 && pf_next < n_ctx; ++pf_next) {
@@ -251,27 +259,29 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
                 }
             }
-            if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+            if (t >= kKStages &&
+                !warp_all(mbar_wait(&kempty[ks], ((t / kKStages) - 1) & 1, abort_flag)))
+                break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&kfull[s], kTile);
+                    mbar_arrive_expect_tx(&kfull[ks], kTile);
                     for (int c = 0; c < 3; c++)
-                        tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[s], c * 64, (int)(bh * p.L + pos0));
-                    tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
+                        tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[ks], c * 64, (int)(bh * p.L + pos0));
+                    tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[ks], 0, (int)((size_t)b * p.L + pos0));
                 }
             } else {
                 // draft tile: 8 key slots per block (its 5 keys, then 3 masked rows)
                 const int d = t - n_ctx;
                 const int nb = min(kDraftBlocks, gcnt - d * kDraftBlocks);
-                if (lane == 0) mbar_arrive_expect_tx(&kfull[s], nb * 8 * kDQK * 2);
+                if (lane == 0) mbar_arrive_expect_tx(&kfull[ks], nb * 8 * kDQK * 2);
                 for (int bb = 0; bb < nb; ++bb) {
                     const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
                     if (lane == 0) {
                         const int row = p.S + kBlock * n;
                         for (int c = 0; c < 3; c++)
-                            tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[s], c * 64, (int)(bh * p.L + row));
-                        tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
+                            tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[ks], c * 64, (int)(bh * p.L + row));
+                        tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[ks], 0, (int)((size_t)b * p.L + row));
                     }
                 }
             }
@@ -309,7 +319,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             bool ok = mbar_wait(qfull, 0, abort_flag);
             auto issue_sdp = [&](int t) {
                 const int s = t & 1;
-                const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0)), vb = smem_u32(sm + (s ? oV1 : oV0));
+                const uint32_t kb = smem_u32(sm + oK0 + (t % kKStages) * kTile), vb = smem_u32(sm + (s ? oV1 : oV0));
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
                     const int c = k >> 2, sub = k & 3;
@@ -327,7 +337,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             };
             auto wait_kv = [&](int t) {
                 const int s = t & 1;
-                bool r = mbar_wait(&kfull[s], (t >> 1) & 1, abort_flag);
+                bool r = mbar_wait(&kfull[t % kKStages], (t / kKStages) & 1, abort_flag);
                 if (r) r = mbar_wait(&vfull[s], (t >> 1) & 1, abort_flag);
                 if (r) {
                     counters[2] = t + 1;
@@ -350,7 +360,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 bool issued = false;
                 if (ns < T && ns <= nq + 1) {
                     const int s1 = ns & 1;
-                    if (mbar_try_wait(&kfull[s1], (ns >> 1) & 1) && mbar_try_wait(&vfull[s1], (ns >> 1) & 1)) {
+                    if (mbar_try_wait(&kfull[ns % kKStages], (ns / kKStages) & 1) &&
+                        mbar_try_wait(&vfull[s1], (ns >> 1) & 1)) {
                         counters[2] = ns + 1;
                         counters[3] = ns + 1;
                         tc_fence_after();
@@ -363,12 +374,12 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     const int s = nq & 1;
                     tc_fence_after();
                     const uint32_t dsa = smem_u32(sm + (s ? oS1 : oS0));
-                    const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0));
+                    const uint32_t kb = smem_u32(sm + oK0 + (nq % kKStages) * kTile);
 #pragma unroll
                     for (int k = 0; k < kBN / 16; ++k)
-                        mma_bf16_ss(tmem + kColDQ, sdesc_sw128(dsa + k * 32, 16, 1024),
+                        mma_bf16_ss(tmem + kColDQ, sdesc_noswz(dsa + k * 256, 128, 512),
                                     sdesc_sw128(kb + k * 2048, kKChunk, 1024), idQ, (nq > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&kempty[s]);
+                    mma_commit(&kempty[nq % kKStages]);
                     mma_commit(&dqdone[s]);
                     ++nq;
                     issued = true;
@@ -436,7 +447,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     const float pp = (c >= clo && c < chi) ? ex2(fmaf(sv[c], p.scale_log2, -lse2)) : 0.f;
                     e[k] = pp * (pv[c] - Dr) * p.scale;
                 }
-                *reinterpret_cast<uint4 *>(drow + sw128(r, u)) =
+                *reinterpret_cast<uint4 *>(drow + (r >> 3) * 512 + u * 128 + (r & 7) * 16) =
                     make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
                                pack_bf16x2(e[6], e[7]));
             }
@@ -491,7 +502,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         volatile int never = 0;
         if (warp == 4 && lane == 0) {
             if (counters[4]) mbar_wait(qfull, 0, (volatile int *)&never);
-            for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(&kfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+            for (int t = counters[2]; t < counters[0]; ++t)
+                mbar_wait(&kfull[t % kKStages], (t / kKStages) & 1, (volatile int *)&never);
             for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
         }
         if (warp == 5 && lane == 0) {

@@ -192,6 +192,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     d |= (uint64_t)2 << 61;  // SWIZZLE_128B
     return d;
 }
+// Shared-memory matrix descriptor, no swizzle (8-row x 16-byte core matrices).
+// For a K-major operand: lbo = byte distance between core matrices adjacent
+// along K, sbo = between core matrices adjacent along M / N.
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100; layout bits 61-63 = 0: no swizzle
+    return d;
+}
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, A K-major,
 // B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {

@@ -12,16 +12,20 @@
 // are sorted by anchor, neighbouring groups (adjacent blockIdx.x) read
 // overlapping windows close together in time, so the overlap is served by L2.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t = TMEM lane t. Loads and
-//              RoPE-rotates Q at the start, turns each S tile into P (bf16, in
-//              shared memory) with an online softmax, rescales its O row when
-//              the running max grows by more than 2^8, and writes O and LSE.
-//   warp 4     producer: TMA loads of context K (K^C 3 x 64 columns plus the
-//              pre-rotated shared K^R) and V tiles, cp.async gathers of the
-//              draft-key tiles; two stages each for K and V.
+// Warp roles (224 threads):
+//   warps 0-3  softmax: thread t owns query row t = TMEM lane t. Lay Q out
+//              for the MMA and RoPE-rotate it at the start, turn each S tile
+//              into P (bf16, in shared memory) with an online softmax, rescale
+//              the O row when the running max grows by more than 2^8, and
+//              write O and LSE.
+//   warp 4     K producer: the group's raw Q rows (one bulk copy per block),
+//              TMA loads of context K tiles (K^C 3 x 64 columns plus the
+//              pre-rotated shared K^R) and of draft-key tiles (8-row boxes per
+//              block), L2 prefetch of the K and V tiles three tiles ahead.
 //   warp 5     TMEM owner and MMA issuer (one thread): S = Q K^T into two
 //              alternating 64-column TMEM buffers, O += P V into 256 columns.
+//   warp 6     V producer: the V tiles, so a K load never queues behind a V
+//              stage that is still being read.
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait, TMEM is freed and the workspace error word gets kErrTimeout.
@@ -63,7 +67,7 @@ constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 constexpr int kSmemBytes = oBar + 256 + 1024;  // barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383
@@ -145,89 +149,112 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
-        // ------------------------------------------------------- producer
+    if (warp == 4 || warp == 6) {
+        // ------------------------------------------------------ producers
         // lane l holds the block index of group block l
         const int my_n = lane < gcnt ? sn[lane] : 0;
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_kc);
-            tma_prefetch_desc(&tm_kr);
-            tma_prefetch_desc(&tm_v);
-            // raw Q rows of the group: each block's 5 rows are one contiguous
-            // 2560-byte run; they land row-major in the staging area
-            mbar_arrive_expect_tx(qraw, nrows * kDQK * 2);
-            counters[4] = 1;
-        }
-        __syncwarp();
-        if (lane < gcnt)
-            bulk_load(sm + oStage + lane * (kBlock * kDQK * 2),
-                      p.q + (bh * p.R + (size_t)kBlock * my_n) * kDQK, kBlock * kDQK * 2, qraw);
-        int pf_next = 2;  // next context tile to prefetch into L2
-        for (int t = 0; t < T; ++t) {
-            const int s = t & 1;
-            uint8_t *kt = sm + (s ? oK1 : oK0);
-            uint8_t *vt = sm + (s ? oV1 : oV0);
+        if (warp == 4) {
             if (lane == 0) {
-                for (; pf_next <= t + 3 && pf_next < n_ctx; ++pf_next) {
-                    const int pos = ctx_lo + pf_next * kBN;
-                    for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
-                    tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
-                    for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
-                }
+                tma_prefetch_desc(&tm_kc);
+                tma_prefetch_desc(&tm_kr);
+                tma_prefetch_desc(&tm_v);
+                // raw Q rows of the group: each block's 5 rows are one contiguous
+                // 2560-byte run; they land row-major in the staging area
+                mbar_arrive_expect_tx(qraw, nrows * kDQK * 2);
+                counters[4] = 1;
             }
-            if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
-            if (t < n_ctx) {
-                const int pos0 = ctx_lo + t * kBN;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&kfull[s], kKBytes);
-                    for (int c = 0; c < 3; c++)
-                        tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[s], c * 64, (int)(bh * p.L + pos0));
-                    tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
-                }
-            } else {
-                // draft tile: 8 key slots per block, its 5 keys first (the 3
-                // rows after them are other keys, masked out)
-                const int d = t - n_ctx;
-                const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
-                if (lane == 0) mbar_arrive_expect_tx(&kfull[s], nb * 8 * kDQK * 2);
-                __syncwarp();
-                for (int bb = 0; bb < nb; ++bb) {
-                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
+            __syncwarp();
+            if (lane < gcnt)
+                bulk_load(sm + oStage + lane * (kBlock * kDQK * 2),
+                          p.q + (bh * p.R + (size_t)kBlock * my_n) * kDQK, kBlock * kDQK * 2, qraw);
+            // L2 prefetch of tile tt's K and V (context rows, or the 8-row
+            // boxes of the draft tile's blocks, one block per lane)
+            auto prefetch_tile = [&](int tt) {
+                if (tt < n_ctx) {
                     if (lane == 0) {
+                        const int pos = ctx_lo + tt * kBN;
+                        for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
+                        tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
+                        for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
+                    }
+                } else {
+                    const int d = tt - n_ctx;
+                    const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
+                    const int n = __shfl_sync(0xffffffffu, my_n, (d * kDraftBlocksPerTile + lane) & 31);
+                    if (lane < nb) {
                         const int row = p.S + kBlock * n;
+                        for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc8, c * 64, (int)(bh * p.L + row));
+                        tma_prefetch_2d(&tm_kr8, 0, (int)((size_t)b * p.L + row));
+                        for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v8, c * 64, (int)(bh * p.L + row));
+                    }
+                }
+            };
+            int pf_next = 2;  // next tile to prefetch into L2
+            for (int t = 0; t < T; ++t) {
+                const int s = t & 1;
+                uint8_t *kt = sm + (s ? oK1 : oK0);
+                for (; pf_next <= t + 3 && pf_next < T; ++pf_next) prefetch_tile(pf_next);
+                if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+                if (t < n_ctx) {
+                    const int pos0 = ctx_lo + t * kBN;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&kfull[s], kKBytes);
                         for (int c = 0; c < 3; c++)
-                            tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[s], c * 64, (int)(bh * p.L + row));
-                        tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
+                            tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[s], c * 64, (int)(bh * p.L + pos0));
+                        tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
+                    }
+                } else {
+                    // draft tile: 8 key slots per block, its 5 keys first (the 3
+                    // rows after them are other keys, masked out)
+                    const int d = t - n_ctx;
+                    const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
+                    if (lane == 0) mbar_arrive_expect_tx(&kfull[s], nb * 8 * kDQK * 2);
+                    __syncwarp();
+                    for (int bb = 0; bb < nb; ++bb) {
+                        const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
+                        if (lane == 0) {
+                            const int row = p.S + kBlock * n;
+                            for (int c = 0; c < 3; c++)
+                                tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[s], c * 64,
+                                            (int)(bh * p.L + row));
+                            tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
+                        }
                     }
                 }
+                if (lane == 0) counters[0] = t + 1;
             }
-            if (lane == 0) counters[0] = t + 1;
-            // V: the second V stage doubles as the Q staging area until the
-            // softmax warps have moved Q into place
-            if (t == 1 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
-            if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
-            if (t < n_ctx) {
-                const int pos0 = ctx_lo + t * kBN;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&vfull[s], kVBytes);
-                    for (int c = 0; c < 4; c++)
-                        tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[s], c * 64, (int)(bh * p.L + pos0));
-                }
-            } else {
-                const int d = t - n_ctx;
-                const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
-                if (lane == 0) mbar_arrive_expect_tx(&vfull[s], nb * 8 * kDV * 2);
-                __syncwarp();
-                for (int bb = 0; bb < nb; ++bb) {
-                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
+        } else {
+            for (int t = 0; t < T; ++t) {
+                const int s = t & 1;
+                uint8_t *vt = sm + (s ? oV1 : oV0);
+                // the second V stage doubles as the Q staging area until the
+                // softmax warps have moved Q into place
+                if (t == 1 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
+                if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+                if (t < n_ctx) {
+                    const int pos0 = ctx_lo + t * kBN;
                     if (lane == 0) {
-                        const int row = p.S + kBlock * n;
+                        mbar_arrive_expect_tx(&vfull[s], kVBytes);
                         for (int c = 0; c < 4; c++)
-                            tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[s], c * 64, (int)(bh * p.L + row));
+                            tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[s], c * 64, (int)(bh * p.L + pos0));
+                    }
+                } else {
+                    const int d = t - n_ctx;
+                    const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
+                    if (lane == 0) mbar_arrive_expect_tx(&vfull[s], nb * 8 * kDV * 2);
+                    __syncwarp();
+                    for (int bb = 0; bb < nb; ++bb) {
+                        const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
+                        if (lane == 0) {
+                            const int row = p.S + kBlock * n;
+                            for (int c = 0; c < 4; c++)
+                                tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[s], c * 64,
+                                            (int)(bh * p.L + row));
+                        }
                     }
                 }
+                if (lane == 0) counters[1] = t + 1;
             }
-            if (lane == 0) counters[1] = t + 1;
         }
     } else if (warp == 5) {
         // ----------------------------------------------------- MMA issuer
@@ -295,32 +322,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         bool ok = true;
         {
-            // Q: row r of the staging area (raw) -> row r of the swizzled Q
-            // tile, rope slice rotated to position A + j; rows past the group 0
+            // Q: raw rows of the staging area -> the swizzled Q tile; rows
+            // past the group are zero. The content slice (16-byte units 0..23
+            // of a row) moves one row per warp instruction, lane l taking unit
+            // l; the rope slice (units 24..31) is rotated to position A + j by
+            // the row's own thread, with cos/sin fetched before Q lands.
             float4 cs[kDR / 4];  // (cos, sin) of the 32 rope frequencies at A + j
             const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2));
 #pragma unroll
             for (int k = 0; k < kDR / 4; k++) cs[k] = __ldg(tp + k);
             ok = warp_all(mbar_wait(qraw, 0, abort_flag));
+            if (lane < kDC / 8) {
+#pragma unroll 8
+                for (int i = 0; i < 32; i++) {
+                    const int row = warp * 32 + i;
+                    const bool have = ok && row < nrows;
+                    *reinterpret_cast<uint4 *>(sm + oQ + (lane >> 3) * kQChunk + sw128(row, lane & 7)) =
+                        have ? *reinterpret_cast<const uint4 *>(sm + oStage + row * (kDQK * 2) + lane * 16)
+                             : make_uint4(0, 0, 0, 0);
+                }
+            }
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + r * (kDQK * 2));
             const bool have = live && ok;
-#pragma unroll 4
-            for (int u = 0; u < kDC / 8; u++)
-                *reinterpret_cast<uint4 *>(sm + oQ + (u >> 3) * kQChunk + sw128(r, u & 7)) =
-                    have ? src[u] : make_uint4(0, 0, 0, 0);
+            // a bf16 pair (x0 low, x1 high) rotated by (c, s)
+            auto rot = [](uint32_t w, float c, float s_) {
+                const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
+                return pack_bf16x2(x0 * c - x1 * s_, x0 * s_ + x1 * c);
+            };
 #pragma unroll
-            for (int u = 0; u < kDR / 8; u++) {  // rope slice: 4 pairs per unit
+            for (int u = 0; u < kDR / 8; u++) {  // 4 pairs per unit: frequencies 4u .. 4u+3
                 const uint4 val = have ? src[kDC / 8 + u] : make_uint4(0, 0, 0, 0);
-                uint32_t w[4] = {val.x, val.y, val.z, val.w};
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&w[k]);
-                    const float x0 = __bfloat162float(pr.x), x1 = __bfloat162float(pr.y);
-                    const float4 c2 = cs[(4 * u + k) >> 1];
-                    const float c = (k & 1) ? c2.z : c2.x, sn_ = (k & 1) ? c2.w : c2.y;
-                    w[k] = pack_bf16x2(x0 * c - x1 * sn_, x0 * sn_ + x1 * c);
-                }
-                *reinterpret_cast<uint4 *>(sm + oQ + 3 * kQChunk + sw128(r, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+                const float4 c01 = cs[2 * u], c23 = cs[2 * u + 1];
+                *reinterpret_cast<uint4 *>(sm + oQ + 3 * kQChunk + sw128(r, u)) =
+                    make_uint4(rot(val.x, c01.x, c01.y), rot(val.y, c01.z, c01.w), rot(val.z, c23.x, c23.y),
+                               rot(val.w, c23.z, c23.w));
             }
             fence_proxy_async_smem();
             __syncwarp();
