@@ -134,23 +134,28 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
 // ================================================================ dQ
 // CTA = (group g of 25 sorted blocks, head h, batch b); warps 0-3 rows
 // (thread t = row t = TMEM lane t), warp 4 producer, warp 5 MMA.
-// A K tile is read twice (S, then dQ after the rows' dS is ready), a V tile
-// once (dP), so K gets three stages and V two.
+// Q stays in shared memory (A operand of S = Q K^T); dO is moved into tensor
+// memory once at the start (A operand of dP = dO V^T read from TMEM), so a
+// key tile's MMAs re-read only Q from shared memory. The 64 KB where dO first
+// lands then holds V stages. A K tile is read twice (S, then dQ once the rows'
+// dS is ready), a V tile once (dP): five K stages, four V stages.
 namespace dq {
 constexpr int kM = 128, kBN = 32;
 constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
 constexpr int kKChunk = kBN * 128;     // 4 KB: 32 keys x 64 columns
 constexpr int kTile = 4 * kKChunk;     // 16 KB
-constexpr int kKStages = 3;
+constexpr int kKS = 5, kVS = 4;        // K and V stages
 // dS tile [128 rows][32 keys] bf16 without swizzle: 8 x 8 core matrices of
 // 8 rows x 16 bytes, K-adjacent ones 128 B apart, 8-row groups 512 B apart
 constexpr int kDS = kM * kBN * 2;      // 8 KB
-constexpr int oQ = 0, oDO = oQ + 4 * kQChunk, oK0 = oDO + 4 * kQChunk, oV0 = oK0 + kKStages * kTile,
-              oV1 = oV0 + kTile, oS0 = oV1 + kTile, oS1 = oS0 + kDS, oBar = oS1 + kDS;
-constexpr int kSmem = oBar + 256 + 1024;
+constexpr int oQ = 0, oK = oQ + 4 * kQChunk, oV = oK + kKS * kTile, oS0 = oV + kVS * kTile, oS1 = oS0 + kDS,
+              oBar = oS1 + kDS;
+constexpr int oDOStage = oV;           // dO lands here first
+static_assert(kVS * kTile >= 4 * kQChunk, "dO staging area too small");
+constexpr int kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 constexpr int kThreads = 192;
-constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320;  // S: 256/288, dP: 320/352
+constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320, kColDO = 384;  // S: 256/288, dP: 320/352, dO: 384..511
 }  // namespace dq
 
 struct BwdArgs {
@@ -177,11 +182,12 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kfull = bars + 0, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 8;
-    uint64_t *sfull = bars + 10, *dsready = bars + 12, *dqdone = bars + 14, *qfull = bars + 16, *drain = bars + 17;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
-    int *counters = reinterpret_cast<int *>(bars + 20);  // K issued, V issued, K consumed, V consumed, q issued
+    uint64_t *kfull = bars + 0, *kempty = bars + kKS, *vfull = bars + 2 * kKS, *vempty = bars + 2 * kKS + kVS;
+    uint64_t *sfull = bars + 2 * (kKS + kVS), *dsready = sfull + 2, *dqdone = sfull + 4, *qfull = sfull + 6,
+             *drain = sfull + 7, *dotmem = sfull + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + 9);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 10);
+    int *counters = reinterpret_cast<int *>(sfull + 11);  // K issued, V issued, K consumed, V consumed, q issued
 
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int cnt = p.cnt[b];
@@ -201,25 +207,28 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     const size_t bh = (size_t)b * p.n_h + h;
     const size_t srow0 = bh * p.R + (size_t)kBlock * i0;  // first sorted row of the group
 
-    // K/V stages start zeroed (masked key slots must hold finite values)
-    for (int e = threadIdx.x; e < (oS0 - oK0) / 16; e += blockDim.x)
-        reinterpret_cast<uint4 *>(sm + oK0)[e] = make_uint4(0, 0, 0, 0);
+    // K stages start zeroed (masked key slots must hold finite values)
+    for (int e = threadIdx.x; e < (oV - oK) / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + oK)[e] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kKStages; s++) {
+        for (int s = 0; s < kKS; s++) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 1);
         }
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < kVS; s++) {
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
+        }
+        for (int s = 0; s < 2; s++) {
             mbar_init(&sfull[s], 1);
             mbar_init(&dsready[s], 4);
             mbar_init(&dqdone[s], 1);
         }
         mbar_init(qfull, 1);
         mbar_init(drain, 1);
+        mbar_init(dotmem, 4);
         *abort_flag = 0;
         for (int c = 0; c < 5; c++) counters[c] = 0;
         fence_barrier_init();
@@ -240,7 +249,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             mbar_arrive_expect_tx(qfull, 8 * kQChunk);
             for (int c = 0; c < 4; c++) {
                 tma_load_2d(sm + oQ + c * kQChunk, &tm_qs, qfull, c * 64, (int)srow0);
-                tma_load_2d(sm + oDO + c * kQChunk, &tm_dos, qfull, c * 64, (int)srow0);
+                tma_load_2d(sm + oDOStage + c * kQChunk, &tm_dos, qfull, c * 64, (int)srow0);
             }
             counters[4] = 1;
         }
@@ -248,20 +257,18 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         const int my_n = lane < gcnt ? sn[lane] : 0;
         int pf_next = 2;
         for (int t = 0; t < T; ++t) {
-            const int s = t & 1, ks = t % kKStages;
-            uint8_t *kt = sm + oK0 + ks * kTile;
-            uint8_t *vt = sm + (s ? oV1 : oV0);
+            const int ks = t % kKS, vs = t % kVS;
+            uint8_t *kt = sm + oK + ks * kTile;
+            uint8_t *vt = sm + oV + vs * kTile;
             if (lane == 0) {
-                for (; pf_next <= t + 5 && pf_next < n_ctx; ++pf_next) {
+                for (; pf_next <= t + 7 && pf_next < n_ctx; ++pf_next) {
                     const int pos = ctx_lo + pf_next * kBN;
                     for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
                     tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
                     for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
                 }
             }
-            if (t >= kKStages &&
-                !warp_all(mbar_wait(&kempty[ks], ((t / kKStages) - 1) & 1, abort_flag)))
-                break;
+            if (t >= kKS && !warp_all(mbar_wait(&kempty[ks], ((t / kKS) - 1) & 1, abort_flag))) break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
                 if (lane == 0) {
@@ -286,82 +293,66 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 }
             }
             if (lane == 0) counters[0] = t + 1;
-            if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+            // the V stages hold dO until the row warps have moved it to TMEM
+            if (t == 0 && !warp_all(mbar_wait(dotmem, 0, abort_flag))) break;
+            if (t >= kVS && !warp_all(mbar_wait(&vempty[vs], ((t / kVS) - 1) & 1, abort_flag))) break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&vfull[s], kTile);
+                    mbar_arrive_expect_tx(&vfull[vs], kTile);
                     for (int c = 0; c < 4; c++)
-                        tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[s], c * 64, (int)(bh * p.L + pos0));
+                        tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[vs], c * 64, (int)(bh * p.L + pos0));
                 }
             } else {
                 const int d = t - n_ctx;
                 const int nb = min(kDraftBlocks, gcnt - d * kDraftBlocks);
-                if (lane == 0) mbar_arrive_expect_tx(&vfull[s], nb * 8 * kDV * 2);
+                if (lane == 0) mbar_arrive_expect_tx(&vfull[vs], nb * 8 * kDV * 2);
                 for (int bb = 0; bb < nb; ++bb) {
                     const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
                     if (lane == 0) {
                         const int row = p.S + kBlock * n;
                         for (int c = 0; c < 4; c++)
-                            tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[s], c * 64, (int)(bh * p.L + row));
+                            tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[vs], c * 64, (int)(bh * p.L + row));
                     }
                 }
             }
             if (lane == 0) counters[1] = t + 1;
         }
-        cp_async_wait_all();
     } else if (warp == 5) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kM, kBN, 0);    // S, dP: B = K / V tile, K-major
             const uint32_t idQ = idesc_bf16(kM, kDQK, 1);   // dQ: B = K tile, MN-major
-            const uint32_t qa = smem_u32(sm + oQ), da = smem_u32(sm + oDO);
+            const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + oQ), 16, 1024));
             bool ok = mbar_wait(qfull, 0, abort_flag);
+            if (ok) ok = mbar_wait(dotmem, 0, abort_flag);
             auto issue_sdp = [&](int t) {
                 const int s = t & 1;
-                const uint32_t kb = smem_u32(sm + oK0 + (t % kKStages) * kTile), vb = smem_u32(sm + (s ? oV1 : oV0));
+                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + (t % kKS) * kTile), 16, 1024));
+                const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + oV + (t % kVS) * kTile), 16, 1024));
+                const uint32_t dS = tmem + kColS + s * kBN, dP = tmem + kColP + s * kBN;
+                // S and dP interleaved: two independent accumulation chains
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
-                    const int c = k >> 2, sub = k & 3;
-                    mma_bf16_ss(tmem + kColS + s * kBN, sdesc_sw128(qa + c * kQChunk + sub * 32, 16, 1024),
-                                sdesc_sw128(kb + c * kKChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int k = 0; k < kDV / 16; ++k) {
-                    const int c = k >> 2, sub = k & 3;
-                    mma_bf16_ss(tmem + kColP + s * kBN, sdesc_sw128(da + c * kQChunk + sub * 32, 16, 1024),
-                                sdesc_sw128(vb + c * kKChunk + sub * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+                    const uint32_t qo = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
+                    const uint32_t ko = ((k >> 2) * kKChunk + (k & 3) * 32) >> 4;
+                    mma_bf16_ss(dS, qd.at(qo), kd.at(ko), idS, k > 0 ? 1u : 0u);
+                    mma_bf16_ts(dP, tmem + kColDO + 8 * k, vd.at(ko), idS, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[s]);
-                mma_commit(&vempty[s]);
+                mma_commit(&vempty[t % kVS]);
             };
-            auto wait_kv = [&](int t) {
-                const int s = t & 1;
-                bool r = mbar_wait(&kfull[t % kKStages], (t / kKStages) & 1, abort_flag);
-                if (r) r = mbar_wait(&vfull[s], (t >> 1) & 1, abort_flag);
-                if (r) {
-                    counters[2] = t + 1;
-                    counters[3] = t + 1;
-                }
-                return r;
-            };
-            if (ok) ok = wait_kv(0);
-            if (ok) {
-                tc_fence_after();
-                issue_sdp(0);
-            }
             // Issue whichever is ready first: S/dP of tile ns (its K and V
             // landed; it runs at most one tile ahead, so its S/dP buffer was
             // released by the dQ of tile ns - 2) or dQ of tile nq (its dS is
             // written). Neither waits for the other's inputs.
-            int ns = 1, nq = 0;
+            int ns = 0, nq = 0;
             uint64_t t_idle = 0;
+            if (ok) tc_fence_after();
             while (ok && nq < T) {
                 bool issued = false;
                 if (ns < T && ns <= nq + 1) {
-                    const int s1 = ns & 1;
-                    if (mbar_try_wait(&kfull[ns % kKStages], (ns / kKStages) & 1) &&
-                        mbar_try_wait(&vfull[s1], (ns >> 1) & 1)) {
+                    if (mbar_test(&kfull[ns % kKS], (ns / kKS) & 1) && mbar_test(&vfull[ns % kVS], (ns / kVS) & 1)) {
                         counters[2] = ns + 1;
                         counters[3] = ns + 1;
                         tc_fence_after();
@@ -370,16 +361,14 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                         issued = true;
                     }
                 }
-                if (!issued && mbar_try_wait(&dsready[nq & 1], (nq >> 1) & 1)) {
+                if (!issued && nq < ns && mbar_test(&dsready[nq & 1], (nq >> 1) & 1)) {
                     const int s = nq & 1;
                     tc_fence_after();
-                    const uint32_t dsa = smem_u32(sm + (s ? oS1 : oS0));
-                    const uint32_t kb = smem_u32(sm + oK0 + (nq % kKStages) * kTile);
-#pragma unroll
-                    for (int k = 0; k < kBN / 16; ++k)
-                        mma_bf16_ss(tmem + kColDQ, sdesc_noswz(dsa + k * 256, 128, 512),
-                                    sdesc_sw128(kb + k * 2048, kKChunk, 1024), idQ, (nq > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&kempty[nq % kKStages]);
+                    const SDesc dd = sdesc_split(sdesc_noswz(smem_u32(sm + (s ? oS1 : oS0)), 128, 512));
+                    const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + (nq % kKS) * kTile), kKChunk, 1024));
+                    mma_bf16_ss(tmem + kColDQ, dd.at(0), kd.at(0), idQ, nq > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColDQ, dd.at(16), kd.at(128), idQ, 1u);
+                    mma_commit(&kempty[nq % kKS]);
                     mma_commit(&dqdone[s]);
                     ++nq;
                     issued = true;
@@ -412,8 +401,31 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             Dr = p.ds_[srow0 + r];
         }
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        bool ok = true;
-        for (int t = 0; t < T; ++t) {
+        bool ok = warp_all(mbar_wait(qfull, 0, abort_flag));
+        {
+            // dO row r: shared memory (128-byte swizzled, 64-column chunks) ->
+            // TMEM lane r, columns kColDO.. (bf16 pairs, 8 per 16-byte unit)
+#pragma unroll 1
+            for (int c = 0; c < 4; c++) {
+                uint32_t w[32];
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(sm + oDOStage + c * kQChunk + sw128(r, u));
+                    w[4 * u + 0] = val.x;
+                    w[4 * u + 1] = val.y;
+                    w[4 * u + 2] = val.z;
+                    w[4 * u + 3] = val.w;
+                }
+                tmem_st32u(trow + kColDO + 32 * c, w);
+            }
+            // the V stages now hold dO rows or zero fill: finite, as masked
+            // key slots of draft tiles need
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dotmem);
+        }
+        for (int t = 0; t < T && ok; ++t) {
             const int s = t & 1;
             ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
             if (!ok) break;
@@ -460,9 +472,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         if (ok) {
             tc_fence_after();
             // dQ row (rope slice rotated back by A + j) -> staging in the idle
-            // K/V stages (unit u of row r at u ^ (r & 31)) -> one 512-byte row
+            // K stages (unit u of row r at u ^ (r & 31)) -> one 512-byte row
             // per warp instruction
-            uint8_t *stage = sm + oK0 + warp * (32 * kDQK * 2);
+            uint8_t *stage = sm + oK + warp * (32 * kDQK * 2);
 #pragma unroll 1
             for (int c = 0; c < kDQK; c += 32) {
                 float v[32];
@@ -503,8 +515,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         if (warp == 4 && lane == 0) {
             if (counters[4]) mbar_wait(qfull, 0, (volatile int *)&never);
             for (int t = counters[2]; t < counters[0]; ++t)
-                mbar_wait(&kfull[t % kKStages], (t / kKStages) & 1, (volatile int *)&never);
-            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+                mbar_wait(&kfull[t % kKS], (t / kKS) & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t)
+                mbar_wait(&vfull[t % kVS], (t / kVS) & 1, (volatile int *)&never);
         }
         if (warp == 5 && lane == 0) {
             mma_commit(drain);
@@ -749,24 +762,30 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kMK, kRC, 0);   // S^T, dP^T: B = Q / dO chunk, K-major
             const uint32_t idA = idesc_bf16(kMK, 256, 1);   // acc: B = dO / Q chunk, MN-major
-            const uint32_t ka = smem_u32(sm + oK), va = smem_u32(sm + oV);
+            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + oK), 16, 1024));
+            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + oV), 16, 1024));
             bool ok = true;
             auto issue_s = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
-                const uint32_t qb = smem_u32(sm + (s ? oQ1 : oQ0)), db = smem_u32(sm + (s ? oD1 : oD0));
-#pragma unroll
-                for (int kk = 0; kk < kDQK / 16; ++kk) {
-                    const int cc = kk >> 2, sub = kk & 3;
-                    mma_bf16_ss(tmem + kColS + s * kRC, sdesc_sw128(ka + cc * kKChunk + sub * 32, 16, 1024),
-                                sdesc_sw128(qb + cc * kRChunk + sub * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
-                }
+                const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oQ1 : oQ0)), 16, 1024));
+                const SDesc dd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oD1 : oD0)), 16, 1024));
+                const uint32_t dS = tmem + kColS + s * kRC, dP = tmem + kColP + s * kRC;
                 if (role_k) {
+                    // S^T and dP^T interleaved: two independent accumulation chains
 #pragma unroll
-                    for (int kk = 0; kk < kDV / 16; ++kk) {
-                        const int cc = kk >> 2, sub = kk & 3;
-                        mma_bf16_ss(tmem + kColP + s * kRC, sdesc_sw128(va + cc * kKChunk + sub * 32, 16, 1024),
-                                    sdesc_sw128(db + cc * kRChunk + sub * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kDQK / 16; ++kk) {
+                        const uint32_t ko = ((kk >> 2) * kKChunk + (kk & 3) * 32) >> 4;
+                        const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
+                        mma_bf16_ss(dS, kad.at(ko), qd.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dP, vad.at(ko), dd.at(ro), idS, kk > 0 ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kDQK / 16; ++kk) {
+                        const uint32_t ko = ((kk >> 2) * kKChunk + (kk & 3) * 32) >> 4;
+                        const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
+                        mma_bf16_ss(dS, kad.at(ko), qd.at(ro), idS, kk > 0 ? 1u : 0u);
                     }
                 }
                 mma_commit(&sfull[s]);
@@ -775,12 +794,11 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             auto issue_acc = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
-                const uint32_t pa = smem_u32(sm + (s ? oP1 : oP0));
-                const uint32_t bsrc = smem_u32(sm + (role_k ? (s ? oQ1 : oQ0) : (s ? oD1 : oD0)));
-#pragma unroll
-                for (int kk = 0; kk < kRC / 16; ++kk)
-                    mma_bf16_ss(tmem + kColAcc, sdesc_sw128(pa + kk * 32, 16, 1024),
-                                sdesc_sw128(bsrc + kk * 2048, kRChunk, 1024), idA, (c > 0 || kk > 0) ? 1u : 0u);
+                const SDesc pd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oP1 : oP0)), 16, 1024));
+                const SDesc bd = sdesc_split(
+                    sdesc_sw128(smem_u32(sm + (role_k ? (s ? oQ1 : oQ0) : (s ? oD1 : oD0))), kRChunk, 1024));
+                mma_bf16_ss(tmem + kColAcc, pd.at(0), bd.at(0), idA, c > 0 ? 1u : 0u);
+                mma_bf16_ss(tmem + kColAcc, pd.at(2), bd.at(128), idA, 1u);
                 mma_commit(&chfree[s]);
                 if (c == nchunks - 1) mma_commit(accdone);
             };
@@ -796,7 +814,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 bool issued = false;
                 if (ns < QT && ns <= na + 1) {
                     const int hh = ns / nchunks, c = ns % nchunks, s = ns & 1;
-                    if ((c != 0 || mbar_try_wait(kvfull, hh & 1)) && mbar_try_wait(&chfull[s], (ns >> 1) & 1)) {
+                    if ((c != 0 || mbar_test(kvfull, hh & 1)) && mbar_test(&chfull[s], (ns >> 1) & 1)) {
                         if (c == 0) counters[2] = hh + 1;
                         counters[3] = ns + 1;
                         issue_s(ns);
@@ -806,8 +824,8 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 }
                 if (!issued && na < ns) {
                     const int hh = na / nchunks, c = na % nchunks, s = na & 1;
-                    if (mbar_try_wait(&dsready[s], (na >> 1) & 1) &&
-                        (c != 0 || hh == 0 || mbar_try_wait(epidone, (hh - 1) & 1))) {
+                    if (mbar_test(&dsready[s], (na >> 1) & 1) &&
+                        (c != 0 || hh == 0 || mbar_test(epidone, (hh - 1) & 1))) {
                         issue_acc(na);
                         ++na;
                         issued = true;

@@ -261,17 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kM, kBN, 0);
             const uint32_t idO = idesc_bf16(kM, kDV, 1);
-            const uint32_t qa = smem_u32(sm + oQ);
+            const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + oQ), 16, 1024));
             bool ok = mbar_wait(qready, 0, abort_flag);
             auto issue_qk = [&](int t) {
                 const int s = t & 1;
-                const uint32_t kb = smem_u32(sm + (s ? oK1 : oK0));
+                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oK1 : oK0)), 16, 1024));
+                const uint32_t dS = tmem + kColS + s * kBN;
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
-                    const int c = k >> 2, sub = k & 3;
-                    const uint64_t a = sdesc_sw128(qa + c * kQChunk + sub * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(kb + c * kKChunk + sub * 32, 16, 1024);
-                    mma_bf16_ss(tmem + kColS + s * kBN, a, bd, idS, k > 0 ? 1u : 0u);
+                    const uint32_t qo = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
+                    const uint32_t ko = ((k >> 2) * kKChunk + (k & 3) * 32) >> 4;
+                    mma_bf16_ss(dS, qd.at(qo), kd.at(ko), idS, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[s]);
                 mma_commit(&kempty[s]);
@@ -297,14 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 counters[3] = t + 1;
                 tc_fence_after();
-                const uint32_t pa = smem_u32(sm + (s ? oP1 : oP0));
-                const uint32_t vb = smem_u32(sm + (s ? oV1 : oV0));
+                const SDesc pd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oP1 : oP0)), 16, 1024));
+                const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oV1 : oV0)), kKChunk, 1024));
+                mma_bf16_ss(tmem + kColO, pd.at(0), vd.at(0), idO, t > 0 ? 1u : 0u);
 #pragma unroll
-                for (int k = 0; k < kBN / 16; ++k) {
-                    const uint64_t a = sdesc_sw128(pa + k * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(vb + k * 2048, kKChunk, 1024);
-                    mma_bf16_ss(tmem + kColO, a, bd, idO, (t > 0 || k > 0) ? 1u : 0u);
-                }
+                for (int k = 1; k < kBN / 16; ++k) mma_bf16_ss(tmem + kColO, pd.at(2 * k), vd.at(128 * k), idO, 1u);
                 mma_commit(&vempty[s]);
                 mma_commit(&pvdone[s]);
             }
