@@ -134,20 +134,23 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
 // ================================================================ dQ
 // CTA = (group g of 25 sorted blocks, head h, batch b); warps 0-3 rows
 // (thread t = row t = TMEM lane t), warp 4 producer, warp 5 MMA.
+// Key tiles are 64 keys wide: an M = 128 MMA costs about the same for N = 32
+// and N = 64, so the wider tile halves the MMA count per key.
 // Q stays in shared memory (A operand of S = Q K^T); dO is moved into tensor
-// memory once at the start (A operand of dP = dO V^T read from TMEM), so a
-// key tile's MMAs re-read only Q from shared memory. The 64 KB where dO first
-// lands then holds V stages. A K tile is read twice (S, then dQ once the rows'
-// dS is ready), a V tile once (dP): five K stages, four V stages.
+// memory once at the start (A operand of dP = dO V^T read from TMEM). TMEM:
+// dQ 256 columns, S 64, dP 64, dO 128 - S and dP are single-buffered: the
+// row warps copy them to registers and release them before computing dS, so
+// the next tile's S and dP run while dS is formed. The 64 KB where dO first
+// lands then holds the two V stages.
 namespace dq {
-constexpr int kM = 128, kBN = 32;
+constexpr int kM = 128, kBN = 64;
 constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
-constexpr int kKChunk = kBN * 128;     // 4 KB: 32 keys x 64 columns
-constexpr int kTile = 4 * kKChunk;     // 16 KB
-constexpr int kKS = 5, kVS = 4;        // K and V stages
-// dS tile [128 rows][32 keys] bf16 without swizzle: 8 x 8 core matrices of
-// 8 rows x 16 bytes, K-adjacent ones 128 B apart, 8-row groups 512 B apart
-constexpr int kDS = kM * kBN * 2;      // 8 KB
+constexpr int kKChunk = kBN * 128;     // 8 KB: 64 keys x 64 columns
+constexpr int kTile = 4 * kKChunk;     // 32 KB
+constexpr int kKS = 2, kVS = 2;        // K and V stages
+// dS tile [128 rows][64 keys] bf16 without swizzle: 16 x 8 core matrices of
+// 8 rows x 16 bytes, K-adjacent ones 128 B apart, 8-row groups 1024 B apart
+constexpr int kDS = kM * kBN * 2;      // 16 KB
 constexpr int oQ = 0, oK = oQ + 4 * kQChunk, oV = oK + kKS * kTile, oS0 = oV + kVS * kTile, oS1 = oS0 + kDS,
               oBar = oS1 + kDS;
 constexpr int oDOStage = oV;           // dO lands here first
@@ -155,7 +158,7 @@ static_assert(kVS * kTile >= 4 * kQChunk, "dO staging area too small");
 constexpr int kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 constexpr int kThreads = 192;
-constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320, kColDO = 384;  // S: 256/288, dP: 320/352, dO: 384..511
+constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320, kColDO = 384;  // dO: 384..511
 }  // namespace dq
 
 struct BwdArgs {
@@ -183,8 +186,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint64_t *kfull = bars + 0, *kempty = bars + kKS, *vfull = bars + 2 * kKS, *vempty = bars + 2 * kKS + kVS;
-    uint64_t *sfull = bars + 2 * (kKS + kVS), *dsready = sfull + 2, *dqdone = sfull + 4, *qfull = sfull + 6,
-             *drain = sfull + 7, *dotmem = sfull + 8;
+    uint64_t *sfull = bars + 2 * (kKS + kVS), *sfree = sfull + 1, *dsready = sfull + 2, *dqdone = sfull + 4,
+             *qfull = sfull + 6, *drain = sfull + 7, *dotmem = sfull + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + 9);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 10);
     int *counters = reinterpret_cast<int *>(sfull + 11);  // K issued, V issued, K consumed, V consumed, q issued
@@ -221,8 +224,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
         }
+        mbar_init(sfull, 1);
+        mbar_init(sfree, 4);
         for (int s = 0; s < 2; s++) {
-            mbar_init(&sfull[s], 1);
             mbar_init(&dsready[s], 4);
             mbar_init(&dqdone[s], 1);
         }
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             uint8_t *kt = sm + oK + ks * kTile;
             uint8_t *vt = sm + oV + vs * kTile;
             if (lane == 0) {
-                for (; pf_next <= t + 7 && pf_next < n_ctx; ++pf_next) {
+                for (; pf_next <= t + 4 && pf_next < n_ctx; ++pf_next) {
                     const int pos = ctx_lo + pf_next * kBN;
                     for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
                     tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
@@ -327,10 +331,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             bool ok = mbar_wait(qfull, 0, abort_flag);
             if (ok) ok = mbar_wait(dotmem, 0, abort_flag);
             auto issue_sdp = [&](int t) {
-                const int s = t & 1;
                 const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + (t % kKS) * kTile), 16, 1024));
                 const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + oV + (t % kVS) * kTile), 16, 1024));
-                const uint32_t dS = tmem + kColS + s * kBN, dP = tmem + kColP + s * kBN;
+                const uint32_t dS = tmem + kColS, dP = tmem + kColP;
                 // S and dP interleaved: two independent accumulation chains
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
@@ -339,20 +342,21 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     mma_bf16_ss(dS, qd.at(qo), kd.at(ko), idS, k > 0 ? 1u : 0u);
                     mma_bf16_ts(dP, tmem + kColDO + 8 * k, vd.at(ko), idS, k > 0 ? 1u : 0u);
                 }
-                mma_commit(&sfull[s]);
+                mma_commit(sfull);
                 mma_commit(&vempty[t % kVS]);
             };
             // Issue whichever is ready first: S/dP of tile ns (its K and V
-            // landed; it runs at most one tile ahead, so its S/dP buffer was
-            // released by the dQ of tile ns - 2) or dQ of tile nq (its dS is
-            // written). Neither waits for the other's inputs.
+            // landed and the row warps have copied out S/dP of tile ns - 1) or
+            // dQ of tile nq (its dS is written). Neither waits for the other's
+            // inputs.
             int ns = 0, nq = 0;
             uint64_t t_idle = 0;
             if (ok) tc_fence_after();
             while (ok && nq < T) {
                 bool issued = false;
-                if (ns < T && ns <= nq + 1) {
-                    if (mbar_test(&kfull[ns % kKS], (ns / kKS) & 1) && mbar_test(&vfull[ns % kVS], (ns / kVS) & 1)) {
+                if (ns < T && ns <= nq + 2) {
+                    if ((ns == 0 || mbar_test(sfree, (ns - 1) & 1)) && mbar_test(&kfull[ns % kKS], (ns / kKS) & 1) &&
+                        mbar_test(&vfull[ns % kVS], (ns / kVS) & 1)) {
                         counters[2] = ns + 1;
                         counters[3] = ns + 1;
                         tc_fence_after();
@@ -364,10 +368,11 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 if (!issued && nq < ns && mbar_test(&dsready[nq & 1], (nq >> 1) & 1)) {
                     const int s = nq & 1;
                     tc_fence_after();
-                    const SDesc dd = sdesc_split(sdesc_noswz(smem_u32(sm + (s ? oS1 : oS0)), 128, 512));
+                    const SDesc dd = sdesc_split(sdesc_noswz(smem_u32(sm + (s ? oS1 : oS0)), 128, 1024));
                     const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + (nq % kKS) * kTile), kKChunk, 1024));
                     mma_bf16_ss(tmem + kColDQ, dd.at(0), kd.at(0), idQ, nq > 0 ? 1u : 0u);
-                    mma_bf16_ss(tmem + kColDQ, dd.at(16), kd.at(128), idQ, 1u);
+#pragma unroll
+                    for (int k = 1; k < kBN / 16; ++k) mma_bf16_ss(tmem + kColDQ, dd.at(16 * k), kd.at(128 * k), idQ, 1u);
                     mma_commit(&kempty[nq % kKS]);
                     mma_commit(&dqdone[s]);
                     ++nq;
@@ -427,13 +432,29 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         }
         for (int t = 0; t < T && ok; ++t) {
             const int s = t & 1;
-            ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
+            ok = warp_all(mbar_wait(sfull, t & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float sv[32], pv[32];
-            tmem_ld32(trow + kColS + s * kBN, sv);
-            tmem_ld32(trow + kColP + s * kBN, pv);
-            tmem_wait_ld();
+            float sv[64], pv[64];
+            {
+                float a0[32], a1[32], b0[32], b1[32];
+                tmem_ld32(trow + kColS, a0);
+                tmem_ld32(trow + kColS + 32, a1);
+                tmem_ld32(trow + kColP, b0);
+                tmem_ld32(trow + kColP + 32, b1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c++) {
+                    sv[c] = a0[c];
+                    sv[32 + c] = a1[c];
+                    pv[c] = b0[c];
+                    pv[32 + c] = b1[c];
+                }
+            }
+            // S and dP are in registers: the MMA warp may overwrite them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sfree);
             if (t >= 2) {
                 ok = warp_all(mbar_wait(&dqdone[s], ((t - 2) >> 1) & 1, abort_flag));
                 if (!ok) break;
@@ -459,7 +480,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     const float pp = (c >= clo && c < chi) ? ex2(fmaf(sv[c], p.scale_log2, -lse2)) : 0.f;
                     e[k] = pp * (pv[c] - Dr) * p.scale;
                 }
-                *reinterpret_cast<uint4 *>(drow + (r >> 3) * 512 + u * 128 + (r & 7) * 16) =
+                *reinterpret_cast<uint4 *>(drow + (r >> 3) * 1024 + u * 128 + (r & 7) * 16) =
                     make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
                                pack_bf16x2(e[6], e[7]));
             }
@@ -534,25 +555,28 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
 }
 
 // ============================================================== dK / dV
+// Key tile = 128 keys (MMA M). Rows stream through in chunks of 32 (MMA N of
+// S^T). Each chunk's two row operands have different lifetimes: the one read
+// only by the S^T-stage MMAs (dO for role K, Q for role V) is released as
+// soon as they complete and gets two stages; the one also read by the
+// accumulation (Q for role K, dO for role V) gets three. P^T / dS^T go to
+// tensor memory, where the accumulation MMA reads them as its A operand.
 namespace kv {
 constexpr int kMK = 128;                 // keys per tile (MMA M)
 constexpr int kRC = 32;                  // rows per chunk (MMA N of S^T)
 constexpr int kKChunk = kMK * 128;       // 16 KB: 128 keys x 64 columns
 constexpr int kRChunk = kRC * 128;       // 4 KB: 32 rows x 64 columns
-constexpr int kPT = kMK * 128;           // 16 KB: [128 keys][64-column swizzled rows], 32 used
-constexpr int oK = 0, oV = oK + 4 * kKChunk, oQ0 = oV + 4 * kKChunk, oQ1 = oQ0 + 4 * kRChunk,
-              oD0 = oQ1 + 4 * kRChunk, oD1 = oD0 + 4 * kRChunk, oP0 = oD1 + 4 * kRChunk, oP1 = oP0 + kPT,
-              oMeta = oP1 + kPT, oBar = oMeta + 2 * kRC * 12;
+constexpr int kRBuf = 4 * kRChunk;       // 16 KB: one row operand of a chunk
+constexpr int kES = 2, kLS = 3;          // stages: early-released / late-released row operand
+constexpr int kStageBytes = 8 * 32 * 64; // epilogue staging: 8 warps x 32 keys x 32 columns bf16
+constexpr int oK = 0, oV = oK + 4 * kKChunk, oE = oV + 4 * kKChunk, oL = oE + kES * kRBuf, oStage = oL + kLS * kRBuf,
+              oMeta = oStage + kStageBytes, oBar = oMeta + kLS * kRC * 12;
 constexpr int kSmem = oBar + 256 + 1024;
 static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
-// The head epilogue stages through both P^T / dS^T buffers: by then the MMAs
-// that read them have completed, and the key warps write them again only
-// after the epilogue.
-constexpr int oStage = oP0;
-static_assert(2 * kPT >= 8 * 32 * 128, "epilogue staging does not fit");
 constexpr int kKeyWarps = 8;             // two per TMEM sub-partition, each half of a chunk's rows
 constexpr int kThreads = (kKeyWarps + 2) * 32;
-constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320;  // S^T: 256 / 288, dP^T: 320 / 352
+// TMEM: accumulator 0..255, S^T 256 / 288, dP^T 320 / 352, P^T or dS^T (bf16 pairs) 384 / 400
+constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320, kColPT = 384;
 }  // namespace kv
 
 // One CTA per (key tile, role, head group, batch). Role 0 accumulates dV =
@@ -567,12 +591,14 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *chfull = bars + 2, *chfree = bars + 4, *sfull = bars + 6;
-    uint64_t *dsready = bars + 8, *accdone = bars + 10, *epidone = bars + 11, *drain = bars + 12;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 14);
-    int *counters = reinterpret_cast<int *>(bars + 15);  // kv issued, ch issued, kv consumed, ch consumed
-    int *band = reinterpret_cast<int *>(bars + 17);      // first sorted row, row count
+    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *efull = bars + 2, *efree = efull + kES, *lfull = efree + kES,
+             *lfree = lfull + kLS, *sfull = lfree + kLS, *dsready = sfull + 2, *ptfree = dsready + 2,
+             *accdone = ptfree + 2, *epidone = accdone + 1, *drain = epidone + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(drain + 2);
+    // kv issued, L issued, kv consumed, chunks consumed, E issued
+    int *counters = reinterpret_cast<int *>(drain + 3);
+    int *band = counters + 6;  // first sorted row, row count
 
     const int item = blockIdx.x >> 1, role_k = blockIdx.x & 1;
     const int hg = blockIdx.y, b = blockIdx.z;
@@ -656,22 +682,29 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     }
 
     // K/V tiles start zeroed (masked key slots must hold finite values)
-    for (int e = threadIdx.x; e < (oQ0 - oK) / 16; e += blockDim.x)
+    for (int e = threadIdx.x; e < (oE - oK) / 16; e += blockDim.x)
         reinterpret_cast<uint4 *>(sm + oK)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         mbar_init(kvfull, 1);
         mbar_init(kvfree, 1);
+        for (int s = 0; s < kES; s++) {
+            mbar_init(&efull[s], 1);
+            mbar_init(&efree[s], 1);
+        }
+        for (int s = 0; s < kLS; s++) {
+            mbar_init(&lfull[s], 1);
+            mbar_init(&lfree[s], 1);
+        }
         for (int s = 0; s < 2; s++) {
-            mbar_init(&chfull[s], 1);
-            mbar_init(&chfree[s], 1);
             mbar_init(&sfull[s], 1);
             mbar_init(&dsready[s], kKeyWarps);
+            mbar_init(&ptfree[s], 1);
         }
         mbar_init(accdone, 1);
         mbar_init(epidone, kKeyWarps);
         mbar_init(drain, 1);
         *abort_flag = 0;
-        for (int c = 0; c < 4; c++) counters[c] = 0;
+        for (int c = 0; c < 6; c++) counters[c] = 0;
         fence_barrier_init();
     }
     if (warp == kKeyWarps + 1) {
@@ -684,13 +717,17 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int QT = H * nchunks;  // chunks over all heads of the group
+    // row operands: L = read by the accumulation too (Q for role K, dO for
+    // role V), E = read only by the S^T stage (dO for role K, Q for role V)
+    const CUtensorMap *tm_l = role_k ? &tm_qs : &tm_dos;
+    const CUtensorMap *tm_e = role_k ? &tm_dos : &tm_qs;
 
     if (warp == kKeyWarps) {
         // ------------------------------------------------------- producer
         const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
-        bool ok = true;
-        for (int q = 0; q < QT && ok; ++q) {
-            const int hh = q / nchunks, c = q % nchunks, s = q & 1;
+        for (int q = 0; q < QT; ++q) {
+            const int hh = q / nchunks, c = q % nchunks;
+            const int ls = q % kLS, es = q % kES;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
             if (c == 0) {
                 if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
@@ -703,11 +740,6 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                         if (role_k)
                             for (int cc = 0; cc < 4; cc++)
                                 tma_load_2d(sm + oV + cc * kKChunk, &tm_v, kvfull, cc * 64, (int)(bh * p.L + t0));
-                        if (hh + 1 < H) {  // the next head's tiles into L2
-                            for (int cc = 0; cc < 3; cc++) tma_prefetch_2d(&tm_kc, cc * 64, (int)((bh + 1) * p.L + t0));
-                            if (role_k)
-                                for (int cc = 0; cc < 4; cc++) tma_prefetch_2d(&tm_v, cc * 64, (int)((bh + 1) * p.L + t0));
-                        }
                     }
                 } else {
                     if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * (role_k ? 2 : 1) * kDQK * 2);
@@ -728,12 +760,13 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 }
                 if (lane == 0) counters[0] = hh + 1;
             }
-            if (q >= 2 && !warp_all(mbar_wait(&chfree[s], ((q >> 1) - 1) & 1, abort_flag))) break;
             const int r0 = row0 + c * kRC;
-            // chunk metadata: anchor (INT_MAX past the band), LSE*log2(e), D
-            int *mA = reinterpret_cast<int *>(sm + oMeta + s * kRC * 12);
-            float2 *mLD = reinterpret_cast<float2 *>(mA + kRC);
+            // L operand and the chunk metadata: anchor (INT_MAX past the
+            // band), LSE*log2(e), D
+            if (q >= kLS && !warp_all(mbar_wait(&lfree[ls], ((q / kLS) - 1) & 1, abort_flag))) break;
             {
+                int *mA = reinterpret_cast<int *>(sm + oMeta + ls * kRC * 12);
+                float2 *mLD = reinterpret_cast<float2 *>(mA + kRC);
                 const int rowi = r0 + lane;
                 const bool in = rowi < row0 + nrows;
                 mA[lane] = in ? sa[rowi / kBlock] : 0x7fffffff;
@@ -741,20 +774,17 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(&chfull[s], 8 * kRChunk);
-                for (int cc = 0; cc < 4; cc++) {
-                    tma_load_2d(sm + (s ? oQ1 : oQ0) + cc * kRChunk, &tm_qs, &chfull[s], cc * 64, (int)(bh * p.R + r0));
-                    tma_load_2d(sm + (s ? oD1 : oD0) + cc * kRChunk, &tm_dos, &chfull[s], cc * 64, (int)(bh * p.R + r0));
-                }
+                mbar_arrive_expect_tx(&lfull[ls], kRBuf);
+                for (int cc = 0; cc < 4; cc++)
+                    tma_load_2d(sm + oL + ls * kRBuf + cc * kRChunk, tm_l, &lfull[ls], cc * 64, (int)(bh * p.R + r0));
                 counters[1] = q + 1;
-                if (q + 2 < QT) {  // two chunks ahead into L2
-                    const int q2 = q + 2, h2 = q2 / nchunks, c2 = q2 % nchunks;
-                    const size_t nrow = ((size_t)b * p.n_h + h0 + h2) * p.R + row0 + c2 * kRC;
-                    for (int cc = 0; cc < 4; cc++) {
-                        tma_prefetch_2d(&tm_qs, cc * 64, (int)nrow);
-                        tma_prefetch_2d(&tm_dos, cc * 64, (int)nrow);
-                    }
-                }
+            }
+            if (q >= kES && !warp_all(mbar_wait(&efree[es], ((q / kES) - 1) & 1, abort_flag))) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&efull[es], kRBuf);
+                for (int cc = 0; cc < 4; cc++)
+                    tma_load_2d(sm + oE + es * kRBuf + cc * kRChunk, tm_e, &efull[es], cc * 64, (int)(bh * p.R + r0));
+                counters[4] = q + 1;
             }
         }
     } else if (warp == kKeyWarps + 1) {
@@ -768,44 +798,45 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             auto issue_s = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
-                const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oQ1 : oQ0)), 16, 1024));
-                const SDesc dd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oD1 : oD0)), 16, 1024));
+                const SDesc ld_ = sdesc_split(sdesc_sw128(smem_u32(sm + oL + (q % kLS) * kRBuf), 16, 1024));
+                const SDesc ed = sdesc_split(sdesc_sw128(smem_u32(sm + oE + (q % kES) * kRBuf), 16, 1024));
                 const uint32_t dS = tmem + kColS + s * kRC, dP = tmem + kColP + s * kRC;
                 if (role_k) {
-                    // S^T and dP^T interleaved: two independent accumulation chains
+                    // S^T = K Q^T and dP^T = V dO^T interleaved: two independent chains
 #pragma unroll
                     for (int kk = 0; kk < kDQK / 16; ++kk) {
                         const uint32_t ko = ((kk >> 2) * kKChunk + (kk & 3) * 32) >> 4;
                         const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(dS, kad.at(ko), qd.at(ro), idS, kk > 0 ? 1u : 0u);
-                        mma_bf16_ss(dP, vad.at(ko), dd.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dS, kad.at(ko), ld_.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dP, vad.at(ko), ed.at(ro), idS, kk > 0 ? 1u : 0u);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < kDQK / 16; ++kk) {
                         const uint32_t ko = ((kk >> 2) * kKChunk + (kk & 3) * 32) >> 4;
                         const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(dS, kad.at(ko), qd.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dS, kad.at(ko), ed.at(ro), idS, kk > 0 ? 1u : 0u);
                     }
                 }
                 mma_commit(&sfull[s]);
+                mma_commit(&efree[q % kES]);
                 if (c == nchunks - 1) mma_commit(kvfree);
             };
             auto issue_acc = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
-                const SDesc pd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oP1 : oP0)), 16, 1024));
-                const SDesc bd = sdesc_split(
-                    sdesc_sw128(smem_u32(sm + (role_k ? (s ? oQ1 : oQ0) : (s ? oD1 : oD0))), kRChunk, 1024));
-                mma_bf16_ss(tmem + kColAcc, pd.at(0), bd.at(0), idA, c > 0 ? 1u : 0u);
-                mma_bf16_ss(tmem + kColAcc, pd.at(2), bd.at(128), idA, 1u);
-                mma_commit(&chfree[s]);
+                const SDesc bd = sdesc_split(sdesc_sw128(smem_u32(sm + oL + (q % kLS) * kRBuf), kRChunk, 1024));
+                const uint32_t pa = tmem + kColPT + s * (kRC / 2);
+                mma_bf16_ts(tmem + kColAcc, pa, bd.at(0), idA, c > 0 ? 1u : 0u);
+                mma_bf16_ts(tmem + kColAcc, pa + 8, bd.at(128), idA, 1u);
+                mma_commit(&lfree[q % kLS]);
+                mma_commit(&ptfree[s]);
                 if (c == nchunks - 1) mma_commit(accdone);
             };
-            // Issue whichever is ready: S^T of chunk ns (its K/V tile and row
-            // chunk landed; at most one chunk ahead, so its S buffer was
-            // released by the accumulation of chunk ns - 2) or the
-            // accumulation of chunk na (its P^T / dS^T is written and, at a
+            // Issue whichever is ready: the S^T stage of chunk ns (its K/V tile
+            // and row operands landed; at most one chunk ahead, so its S^T /
+            // dP^T buffer was released by the accumulation of chunk ns - 2) or
+            // the accumulation of chunk na (its P^T / dS^T is in TMEM and, at a
             // head's first chunk, the previous head's epilogue has read the
             // accumulator).
             int ns = 0, na = 0;
@@ -813,8 +844,9 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             while (ok && na < QT) {
                 bool issued = false;
                 if (ns < QT && ns <= na + 1) {
-                    const int hh = ns / nchunks, c = ns % nchunks, s = ns & 1;
-                    if ((c != 0 || mbar_test(kvfull, hh & 1)) && mbar_test(&chfull[s], (ns >> 1) & 1)) {
+                    const int hh = ns / nchunks, c = ns % nchunks;
+                    if ((c != 0 || mbar_test(kvfull, hh & 1)) && mbar_test(&lfull[ns % kLS], (ns / kLS) & 1) &&
+                        mbar_test(&efull[ns % kES], (ns / kES) & 1)) {
                         if (c == 0) counters[2] = hh + 1;
                         counters[3] = ns + 1;
                         issue_s(ns);
@@ -874,14 +906,14 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 rhi = rlo + kBlock;
             }
         }
-        uint8_t *stage = sm + oStage + warp * (32 * 128);
+        uint8_t *stage = sm + oStage + warp * (32 * 64);
         float racc[kDR];                       // rope slice of dK summed over heads (half-1 warps)
 #pragma unroll
         for (int i = 0; i < kDR; i++) racc[i] = 0.f;
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks, s = q & 1;
-            ok = warp_all(mbar_wait(&chfull[s], (q >> 1) & 1, abort_flag));
+            ok = warp_all(mbar_wait(&lfull[q % kLS], (q / kLS) & 1, abort_flag));  // chunk metadata
             if (ok) ok = warp_all(mbar_wait(&sfull[s], (q >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
@@ -904,27 +936,28 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 for (int i = 0; i < 16; i++) sv[i] = half ? a[16 + i] : a[i];
             }
             // rows of the chunk that see this key: [jlo, jhi)
-            const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + s * kRC * 12 + kRC * 4);
+            const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + (q % kLS) * kRC * 12 + kRC * 4);
             const int jlo = rlo - c * kRC, jhi = rhi - c * kRC;
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                float e2[2];
+#pragma unroll
+                for (int d = 0; d < 2; d++) {
+                    const int j = col0 + i + d;
+                    const float2 ldv = mLD[j];
+                    const float pp = (j >= jlo && j < jhi) ? ex2(fmaf(sv[i + d], p.scale_log2, -ldv.x)) : 0.f;
+                    e2[d] = role_k ? pp * (pv[i + d] - ldv.y) * p.scale : pp;
+                }
+                w[i / 2] = pack_bf16x2(e2[0], e2[1]);
+            }
+            // P^T / dS^T buffer s is free once the accumulation of chunk q - 2 completed
             if (q >= 2) {
-                ok = warp_all(mbar_wait(&chfree[s], ((q >> 1) - 1) & 1, abort_flag));
+                ok = warp_all(mbar_wait(&ptfree[s], ((q >> 1) - 1) & 1, abort_flag));
                 if (!ok) break;
             }
-            float e[16];
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int j = col0 + i;
-                const float2 ld = mLD[j];
-                const float pp = (j >= jlo && j < jhi) ? ex2(fmaf(sv[i], p.scale_log2, -ld.x)) : 0.f;
-                e[i] = role_k ? pp * (pv[i] - ld.y) * p.scale : pp;
-            }
-            uint8_t *prow = sm + (s ? oP1 : oP0);
-#pragma unroll
-            for (int u = 0; u < 2; u++)
-                *reinterpret_cast<uint4 *>(prow + sw128(k, 2 * half + u)) =
-                    make_uint4(pack_bf16x2(e[8 * u + 0], e[8 * u + 1]), pack_bf16x2(e[8 * u + 2], e[8 * u + 3]),
-                               pack_bf16x2(e[8 * u + 4], e[8 * u + 5]), pack_bf16x2(e[8 * u + 6], e[8 * u + 7]));
-            fence_proxy_async_smem();
+            tmem_st8u(trow + kColPT + s * (kRC / 2) + half * 8, w);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&dsready[s]);
@@ -934,48 +967,42 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            // Accumulator columns [128 * half, +128) of the warp's 32 keys, in
-            // two rounds of 64: each thread stages its key's 64 values (bf16,
-            // 16-byte unit u at u ^ (key & 7)), then the warp writes 4 keys'
-            // 128-byte row segments per instruction.
+            // Four rounds of 32 columns: each thread stages its key's 32
+            // values (bf16, 16-byte unit u at u ^ (key & 3)), then the warp
+            // writes 8 keys' 64-byte row segments per instruction.
 #pragma unroll
-            for (int rd = 0; rd < 2; rd++) {
-                const int col = half * 128 + rd * 64;
-                float v[64];
-                tmem_ld32(trow + kColAcc + col, *reinterpret_cast<float(*)[32]>(&v[0]));
-                tmem_ld32(trow + kColAcc + col + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            for (int rd = 0; rd < 4; rd++) {
+                const int col = half * 128 + rd * 32;
+                float v[32];
+                tmem_ld32(trow + kColAcc + col, v);
                 tmem_wait_ld();
-                if (role_k && col >= kDC) {  // rope slice of dK (columns 192..255): summed over heads
+                if (role_k && half == 1 && rd >= 2) {  // rope slice of dK (columns 192..255): summed over heads
 #pragma unroll
-                    for (int i = 0; i < 64; i++) racc[i] += v[i];
+                    for (int i = 0; i < 32; i++) racc[(rd - 2) * 32 + i] += v[i];
                     continue;
                 }
 #pragma unroll
-                for (int u = 0; u < 8; u++)
-                    *reinterpret_cast<uint4 *>(stage + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                for (int u = 0; u < 4; u++)
+                    *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
                         make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
                                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
                 __syncwarp();
                 const int rowstride = role_k ? kDC : kDV;
                 __nv_bfloat16 *base = role_k ? p.dkc : p.dv;
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int kl = 4 * i + (lane >> 3), u = lane & 7;   // key within the warp, unit
-                    const int kk = (warp & 3) * 32 + kl;
+                for (int i = 0; i < 4; i++) {
+                    const int kl = 8 * i + (lane >> 2), u = lane & 3;   // key within the warp, unit
                     const int kkv = __shfl_sync(0xffffffffu, (int)key_valid, kl);
                     const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
                     if (kkv) {
-                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 128 + ((u ^ (kl & 7)) << 4));
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
                         *reinterpret_cast<uint4 *>(base + (bh * p.L + (size_t)kposl) * rowstride + col + 8 * u) = val;
                     }
-                    (void)kk;
                 }
                 __syncwarp();
             }
             tc_fence_before();
-            // every key warp is done with the staging (both P buffers) before
-            // any of them writes the next chunk's P^T / dS^T there
-            asm volatile("bar.sync 1, %0;" ::"r"(kKeyWarps * 32) : "memory");
+            __syncwarp();
             if (lane == 0) mbar_arrive(epidone);
         }
         if (ok && role_k && key_valid && half == 1) {
@@ -991,7 +1018,10 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         volatile int never = 0;
         if (warp == kKeyWarps && lane == 0) {
             for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(kvfull, t & 1, (volatile int *)&never);
-            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(&chfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t)
+                mbar_wait(&lfull[t % kLS], (t / kLS) & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[4]; ++t)
+                mbar_wait(&efull[t % kES], (t / kES) & 1, (volatile int *)&never);
         }
         if (warp == kKeyWarps + 1 && lane == 0) {
             mma_commit(drain);
@@ -1070,12 +1100,12 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs32, m_dos32, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc64, m_kr64, m_v64, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs32, m_dos32, m_kc8, m_kr8, m_v8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
     if (p.N > 0 && q_rows > 0) {
-        if (!make_map_bf16(&m_kc32, kc, kDC, kv_rows, 32) || !make_map_bf16(&m_kr32, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 32) ||
-            !make_map_bf16(&m_v32, v, kDV, kv_rows, 32) || !make_map_bf16(&m_qs128, qs, kDQK, q_rows, 128) ||
+        if (!make_map_bf16(&m_kc64, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
+            !make_map_bf16(&m_v64, v, kDV, kv_rows, 64) || !make_map_bf16(&m_qs128, qs, kDQK, q_rows, 128) ||
             !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map_bf16(&m_qs32, qs, kDQK, q_rows, 32) ||
             !make_map_bf16(&m_dos32, dos, kDV, q_rows, 32))
             return cudaErrorInvalidValue;
@@ -1117,7 +1147,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         if (e != cudaSuccess) return e;
         count_launch();
         k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
-            m_kc32, m_kr32, m_v32, m_qs128, m_dos128, m_kc8, m_kr8, m_v8, a);
+            m_kc64, m_kr64, m_v64, m_qs128, m_dos128, m_kc8, m_kr8, m_v8, a);
     }
     const dim3 kv_grid(2 * (a.n_ctx_items + (p.N + kGD - 1) / kGD), HG, p.B);
     e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
