@@ -574,7 +574,8 @@ constexpr int oK = 0, oV = oK + 4 * kKChunk, oE = oV + 4 * kKChunk, oL = oE + kE
 constexpr int kSmem = oBar + 256 + 1024;
 static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 constexpr int kKeyWarps = 8;             // two per TMEM sub-partition, each half of a chunk's rows
-constexpr int kThreads = (kKeyWarps + 2) * 32;
+constexpr int kWarpL = kKeyWarps, kWarpMma = kKeyWarps + 1, kWarpE = kKeyWarps + 2;
+constexpr int kThreads = (kKeyWarps + 3) * 32;
 // TMEM: accumulator 0..255, S^T 256 / 288, dP^T 320 / 352, P^T or dS^T (bf16 pairs) 384 / 400
 constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320, kColPT = 384;
 }  // namespace kv
@@ -707,7 +708,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         for (int c = 0; c < 6; c++) counters[c] = 0;
         fence_barrier_init();
     }
-    if (warp == kKeyWarps + 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -722,12 +723,26 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     const CUtensorMap *tm_l = role_k ? &tm_qs : &tm_dos;
     const CUtensorMap *tm_e = role_k ? &tm_dos : &tm_qs;
 
-    if (warp == kKeyWarps) {
-        // ------------------------------------------------------- producer
+    if (warp == kWarpE) {
+        // ------------------------------------------- producer of E operands
+        for (int q = 0; q < QT; ++q) {
+            const int hh = q / nchunks, c = q % nchunks, es = q % kES;
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+            const int r0 = row0 + c * kRC;
+            if (q >= kES && !warp_all(mbar_wait(&efree[es], ((q / kES) - 1) & 1, abort_flag))) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&efull[es], kRBuf);
+                for (int cc = 0; cc < 4; cc++)
+                    tma_load_2d(sm + oE + es * kRBuf + cc * kRChunk, tm_e, &efull[es], cc * 64, (int)(bh * p.R + r0));
+                counters[4] = q + 1;
+            }
+        }
+    } else if (warp == kWarpL) {
+        // ------------------------- producer of K/V tiles and L operands
         const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
         for (int q = 0; q < QT; ++q) {
             const int hh = q / nchunks, c = q % nchunks;
-            const int ls = q % kLS, es = q % kES;
+            const int ls = q % kLS;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
             if (c == 0) {
                 if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
@@ -779,15 +794,8 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                     tma_load_2d(sm + oL + ls * kRBuf + cc * kRChunk, tm_l, &lfull[ls], cc * 64, (int)(bh * p.R + r0));
                 counters[1] = q + 1;
             }
-            if (q >= kES && !warp_all(mbar_wait(&efree[es], ((q / kES) - 1) & 1, abort_flag))) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&efull[es], kRBuf);
-                for (int cc = 0; cc < 4; cc++)
-                    tma_load_2d(sm + oE + es * kRBuf + cc * kRChunk, tm_e, &efull[es], cc * 64, (int)(bh * p.R + r0));
-                counters[4] = q + 1;
-            }
         }
-    } else if (warp == kKeyWarps + 1) {
+    } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kMK, kRC, 0);   // S^T, dP^T: B = Q / dO chunk, K-major
@@ -1016,21 +1024,21 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     __syncthreads();
     if (*abort_flag) {
         volatile int never = 0;
-        if (warp == kKeyWarps && lane == 0) {
+        if (warp == kWarpL && lane == 0) {
             for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(kvfull, t & 1, (volatile int *)&never);
             for (int t = counters[3]; t < counters[1]; ++t)
                 mbar_wait(&lfull[t % kLS], (t / kLS) & 1, (volatile int *)&never);
             for (int t = counters[3]; t < counters[4]; ++t)
                 mbar_wait(&efull[t % kES], (t / kES) & 1, (volatile int *)&never);
         }
-        if (warp == kKeyWarps + 1 && lane == 0) {
+        if (warp == kWarpMma && lane == 0) {
             mma_commit(drain);
             mbar_wait(drain, 0, (volatile int *)&never);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kKeyWarps + 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
