@@ -12,19 +12,22 @@
 // are sorted by anchor, neighbouring groups (adjacent blockIdx.x) read
 // overlapping windows close together in time, so the overlap is served by L2.
 //
-// Warp roles (224 threads):
-//   warps 0-3  softmax: thread t owns query row t = TMEM lane t. Lay Q out
-//              for the MMA and RoPE-rotate it at the start, turn each S tile
-//              into P (bf16, in shared memory) with an online softmax, rescale
-//              the O row when the running max grows by more than 2^8, and
-//              write O and LSE.
-//   warp 4     K producer: the group's raw Q rows (one bulk copy per block),
+// Warp roles (352 threads):
+//   warps 0-7  softmax: warps w and w + 4 share TMEM sub-partition w % 4, so
+//              query rows 32 (w % 4) .. + 31 (thread = row = TMEM lane), and
+//              split each 64-key tile into two 32-column halves. They lay Q
+//              out for the MMA and RoPE-rotate it at the start, turn each S
+//              tile into P (bf16, in shared memory) with an online softmax
+//              whose row max the pair exchanges through spare TMEM columns,
+//              rescale their half of the O row when the running max grows by
+//              more than 2^8, and write O and LSE.
+//   warp 8     K producer: the group's raw Q rows (one bulk copy per block),
 //              TMA loads of context K tiles (K^C 3 x 64 columns plus the
 //              pre-rotated shared K^R) and of draft-key tiles (8-row boxes per
 //              block), L2 prefetch of the K and V tiles three tiles ahead.
-//   warp 5     TMEM owner and MMA issuer (one thread): S = Q K^T into two
+//   warp 9     TMEM owner and MMA issuer (one thread): S = Q K^T into two
 //              alternating 64-column TMEM buffers, O += P V into 256 columns.
-//   warp 6     V producer: the V tiles, so a K load never queues behind a V
+//   warp 10    V producer: the V tiles, so a K load never queues behind a V
 //              stage that is still being read.
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained with a
@@ -64,13 +67,16 @@ constexpr int oBar = oP1 + kPBytes;
 constexpr int oStage = oV1;
 static_assert(oP1 + kPBytes - oStage >= kM * kDQK * 2, "staging area too small");
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
-constexpr int kSmemBytes = oBar + 256 + 1024;  // barriers + alignment slack
+constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
-constexpr int kThreads = 224;
+constexpr int kSoftWarps = 8;
+constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10;
+constexpr int kThreads = 352;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383
+constexpr uint32_t kColX = 384;  // row-max exchange (2 tiles x 2 halves), then the row-sum exchange
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -100,6 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
     // [4] raw Q issued
     int *counters = reinterpret_cast<int *>(bars + 20);
+    // softmax pair exchange: per TMEM sub-partition and S buffer the tile max,
+    // per sub-partition the row sum (two arrivals each: one per warp)
+    uint64_t *xbar = bars + 24, *lbar = bars + 32;
 
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int cnt = p.cnt[b];
@@ -128,18 +137,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
             mbar_init(&sfull[s], 1);
-            mbar_init(&pready[s], 4);
+            mbar_init(&pready[s], kSoftWarps);
             mbar_init(&pvdone[s], 1);
         }
-        mbar_init(qready, 4);
+        mbar_init(qready, kSoftWarps);
         mbar_init(drain, 1);
         mbar_init(qraw, 1);
-        mbar_init(qstaged, 4);
+        mbar_init(qstaged, kSoftWarps);
+        for (int i = 0; i < 8; i++) mbar_init(&xbar[i], 2);
+        for (int i = 0; i < 4; i++) mbar_init(&lbar[i], 2);
         *abort_flag = 0;
         for (int c = 0; c < 5; c++) counters[c] = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -149,11 +160,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4 || warp == 6) {
+    if (warp == kWarpK || warp == kWarpV) {
         // ------------------------------------------------------ producers
         // lane l holds the block index of group block l
         const int my_n = lane < gcnt ? sn[lane] : 0;
-        if (warp == 4) {
+        if (warp == kWarpK) {
             if (lane == 0) {
                 tma_prefetch_desc(&tm_kc);
                 tma_prefetch_desc(&tm_kr);
@@ -256,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) counters[1] = t + 1;
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kM, kBN, 0);
@@ -308,7 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------ softmax (rows)
-        const int r = threadIdx.x;
+        const int q4 = warp & 3, hf = warp >> 2;  // TMEM sub-partition, column half
+        const int r = q4 * 32 + lane;               // query row = TMEM lane
         const bool live = r < nrows;
         int A = 0, n = 0, j = 0, lo = 0;
         if (live) {
@@ -318,21 +330,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             lo = max(0, A - p.W + 1);
         }
         bool ok = true;
+        const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         {
             // Q: raw rows of the staging area -> the swizzled Q tile; rows
             // past the group are zero. The content slice (16-byte units 0..23
             // of a row) moves one row per warp instruction, lane l taking unit
-            // l; the rope slice (units 24..31) is rotated to position A + j by
-            // the row's own thread, with cos/sin fetched before Q lands.
-            float4 cs[kDR / 4];  // (cos, sin) of the 32 rope frequencies at A + j
-            const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2));
+            // l (warp w: rows 16 w .. 16 w + 15); the rope slice (units 24..31)
+            // is rotated to position A + j by the row's two threads, four
+            // units each, with cos/sin fetched before Q lands.
+            float4 cs[8];  // (cos, sin) of rope frequencies 16 hf .. 16 hf + 15 at A + j
+            const float4 *tp =
+                reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2)) + 8 * hf;
 #pragma unroll
-            for (int k = 0; k < kDR / 4; k++) cs[k] = __ldg(tp + k);
+            for (int k = 0; k < 8; k++) cs[k] = __ldg(tp + k);
             ok = warp_all(mbar_wait(qraw, 0, abort_flag));
             if (lane < kDC / 8) {
 #pragma unroll 8
-                for (int i = 0; i < 32; i++) {
-                    const int row = warp * 32 + i;
+                for (int i = 0; i < 16; i++) {
+                    const int row = warp * 16 + i;
                     const bool have = ok && row < nrows;
                     *reinterpret_cast<uint4 *>(sm + oQ + (lane >> 3) * kQChunk + sw128(row, lane & 7)) =
                         have ? *reinterpret_cast<const uint4 *>(sm + oStage + row * (kDQK * 2) + lane * 16)
@@ -347,9 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return pack_bf16x2(x0 * c - x1 * s_, x0 * s_ + x1 * c);
             };
 #pragma unroll
-            for (int u = 0; u < kDR / 8; u++) {  // 4 pairs per unit: frequencies 4u .. 4u+3
+            for (int uu = 0; uu < 4; uu++) {  // unit u = 4 hf + uu: frequencies 4u .. 4u+3
+                const int u = 4 * hf + uu;
                 const uint4 val = have ? src[kDC / 8 + u] : make_uint4(0, 0, 0, 0);
-                const float4 c01 = cs[2 * u], c23 = cs[2 * u + 1];
+                const float4 c01 = cs[2 * uu], c23 = cs[2 * uu + 1];
                 *reinterpret_cast<uint4 *>(sm + oQ + 3 * kQChunk + sw128(r, u)) =
                     make_uint4(rot(val.x, c01.x, c01.y), rot(val.y, c01.z, c01.w), rot(val.z, c23.x, c23.y),
                                rot(val.w, c23.z, c23.w));
@@ -362,28 +378,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
 
-        float m_used = -INFINITY, l = 0.f;
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
         for (int t = 0; t < T && ok; ++t) {
             const int s = t & 1;
             ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float sv[64];
-            {
-                float a0[32], a1[32];
-                tmem_ld32(trow + kColS + s * kBN, a0);
-                tmem_ld32(trow + kColS + s * kBN + 32, a1);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; c++) {
-                    sv[c] = a0[c];
-                    sv[32 + c] = a1[c];
-                }
-            }
+            float sv[32];
+            tmem_ld32(trow + kColS + s * kBN + 32 * hf, sv);
+            tmem_wait_ld();
             // every row's keys in a tile form one contiguous column range
             // [clo, chi): the window [lo, A) for context tiles, its block's 5
-            // key slots for draft tiles
+            // key slots for draft tiles; this warp holds columns 32 hf .. +31
             int clo, chi;
             if (t < n_ctx) {
                 const int c0 = ctx_lo + t * kBN;
@@ -394,17 +400,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 chi = clo + kBlock;
             }
             if (!live) chi = clo;
-            float mx[8];
+            clo -= 32 * hf;
+            chi -= 32 * hf;
+            float mx[4];
 #pragma unroll
-            for (int k = 0; k < 8; k++) mx[k] = -INFINITY;
+            for (int k = 0; k < 4; k++) mx[k] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kBN; c++) {
+            for (int c = 0; c < 32; c++) {
                 sv[c] = (c >= clo && c < chi) ? sv[c] : -INFINITY;
-                mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+                mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
             }
-            const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            const float mt = mraw * p.scale_log2;
+            // the pair's tile max: each half stores its own in TMEM, both
+            // read the other's after a pair barrier
+            const float mhalf = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            tmem_st1(trow + kColX + 2 * s + hf, mhalf);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xbar[2 * q4 + s]);
+            ok = warp_all(mbar_wait(&xbar[2 * q4 + s], (t >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float mother = tmem_ld1_wait(trow + kColX + 2 * s + (hf ^ 1));
+            const float mt = fmaxf(mhalf, mother) * p.scale_log2;
             bool resc = false;
             float alpha = 1.f;
             if (mt > m_used + kRescaleThreshold) {
@@ -419,25 +437,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
             }
             uint8_t *prow = sm + (s ? oP1 : oP0);
-            float psum[8];
+            float psum[4];
 #pragma unroll
-            for (int k = 0; k < 8; k++) psum[k] = 0.f;
+            for (int k = 0; k < 4; k++) psum[k] = 0.f;
             const bool any = m_used != -INFINITY;
             const float mneg = any ? -m_used : 0.f;
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
+            for (int u = 0; u < 4; u++) {
                 float e[8];
 #pragma unroll
                 for (int k = 0; k < 8; k++) {
                     e[k] = any ? ex2(fmaf(sv[u * 8 + k], p.scale_log2, mneg)) : 0.f;
-                    psum[k] += e[k];
+                    psum[k & 3] += e[k];
                 }
                 uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
                                       pack_bf16x2(e[6], e[7]));
-                *reinterpret_cast<uint4 *>(prow + sw128(r, u)) = pk;
+                *reinterpret_cast<uint4 *>(prow + sw128(r, 4 * hf + u)) = pk;
             }
-            const float ps = ((psum[0] + psum[1]) + (psum[2] + psum[3])) + ((psum[4] + psum[5]) + (psum[6] + psum[7]));
-            l = l * alpha + ps;
+            l = l * alpha + ((psum[0] + psum[1]) + (psum[2] + psum[3]));
             if (__any_sync(0xffffffffu, resc)) {
                 if (t >= 1) {
                     ok = warp_all(mbar_wait(&pvdone[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag));
@@ -445,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < kDV; c += 32) {
+                for (int c = 128 * hf; c < 128 * hf + 128; c += 32) {  // this half's O columns
                     float ov[32];
                     tmem_ld32(trow + kColO + c, ov);
                     tmem_wait_ld();
@@ -463,19 +480,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = warp_all(mbar_wait(&pvdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
         if (ok) {
             tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            // O row -> staging (the idle K stages; unit u of row r at u ^ (r & 31))
-            // -> one 512-byte row per warp instruction
-            uint8_t *stage = sm + oK0 + warp * (32 * kDV * 2);
+            // the row sum: both halves' shares, exchanged like the tile max
+            tmem_st1(trow + kColX + 4 + hf, l);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&lbar[q4]);
+            ok = warp_all(mbar_wait(&lbar[q4], 0, abort_flag));
+        }
+        if (ok) {
+            tc_fence_after();
+            const float ltot = l + tmem_ld1_wait(trow + kColX + 4 + (hf ^ 1));
+            const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+            // this half of the O row (columns 128 hf .. +127) -> staging in the
+            // idle K stages (row i of the warp at 256 i, unit u at u ^ (i & 15))
+            // -> two half rows per warp instruction
+            uint8_t *stage = sm + oK0 + warp * (32 * 256);
 #pragma unroll 1
-            for (int c = 0; c < kDV; c += 32) {
+            for (int c = 0; c < 128; c += 32) {
                 float ov[32];
-                tmem_ld32(trow + kColO + c, ov);
+                tmem_ld32(trow + kColO + 128 * hf + c, ov);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
                     const int u = c / 8 + k;
-                    *reinterpret_cast<uint4 *>(stage + lane * 512 + ((u ^ lane) << 4)) =
+                    *reinterpret_cast<uint4 *>(stage + lane * 256 + ((u ^ (lane & 15)) << 4)) =
                         make_uint4(pack_bf16x2(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv),
                                    pack_bf16x2(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv),
                                    pack_bf16x2(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv),
@@ -483,14 +512,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             __syncwarp();
-            for (int i = 0; i < 32; i++) {
-                const int rr = warp * 32 + i;
-                if (rr >= nrows) break;  // uniform
-                const int ni = __shfl_sync(0xffffffffu, n, i), ji = __shfl_sync(0xffffffffu, j, i);
-                const uint4 val = *reinterpret_cast<const uint4 *>(stage + i * 512 + ((lane ^ i) << 4));
-                *reinterpret_cast<uint4 *>(p.o + (bh * p.R + kBlock * ni + ji) * kDV + 8 * lane) = val;
+            for (int i = 0; i < 16; i++) {
+                const int wr = 2 * i + (lane >> 4), u = lane & 15;  // row within the warp, unit
+                const int rr = q4 * 32 + wr;
+                const int ni = __shfl_sync(0xffffffffu, n, wr), ji = __shfl_sync(0xffffffffu, j, wr);
+                if (rr < nrows) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + wr * 256 + ((u ^ (wr & 15)) << 4));
+                    *reinterpret_cast<uint4 *>(p.o + (bh * p.R + kBlock * ni + ji) * kDV + 128 * hf + 8 * u) = val;
+                }
             }
-            if (live) p.lse[bh * p.R + kBlock * n + j] = (m_used + log2f(l)) * kLn2;
+            if (live && hf == 0) p.lse[bh * p.R + kBlock * n + j] = (m_used + log2f(ltot)) * kLn2;
         }
     }
 
@@ -499,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*abort_flag) {
         // Drain what may still be in flight, each wait bounded on its own.
         volatile int never = 0;
-        if (warp == 4 && lane == 0) {
+        if (warp == kWarpK && lane == 0) {
             if (counters[4]) mbar_wait(qraw, 0, (volatile int *)&never);
             // loads issued but not yet consumed complete in order, one phase each
             for (int t = counters[2]; t < counters[0]; ++t)
@@ -507,14 +538,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = counters[3]; t < counters[1]; ++t)
                 mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
         }
-        if (warp == 5 && lane == 0) {
+        if (warp == kWarpMma && lane == 0) {
             mma_commit(drain);
             mbar_wait(drain, 0, (volatile int *)&never);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
