@@ -17,16 +17,20 @@
 //              query rows 32 (w % 4) .. + 31 (thread = row = TMEM lane), and
 //              split each 64-key tile into two 32-column halves. They lay Q
 //              out for the MMA and RoPE-rotate it at the start, turn each S
-//              tile into P (bf16, in shared memory) with an online softmax
+//              tile into P (bf16, written to TMEM, where the P V MMA reads it
+//              as its A operand) with an online softmax
 //              whose row max the pair exchanges through spare TMEM columns,
 //              rescale their half of the O row when the running max grows by
 //              more than 2^8, and write O and LSE.
 //   warp 8     K producer: the group's raw Q rows (one bulk copy per block),
 //              TMA loads of context K tiles (K^C 3 x 64 columns plus the
 //              pre-rotated shared K^R) and of draft-key tiles (8-row boxes per
-//              block), L2 prefetch of the K and V tiles three tiles ahead.
+//              block), L2 prefetch of the K and V tiles three tiles ahead;
+//              three K stages (a K tile waits on the longest chain: its
+//              stage frees only when the QK MMA two tiles back completes).
 //   warp 9     TMEM owner and MMA issuer (one thread): S = Q K^T into two
-//              alternating 64-column TMEM buffers, O += P V into 256 columns.
+//              alternating 64-column TMEM buffers, O += P V into 256 columns,
+//              each issued as soon as its inputs are ready.
 //   warp 10    V producer: the V tiles, so a K load never queues behind a V
 //              stage that is still being read.
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
@@ -52,20 +56,23 @@ constexpr int kKChunk = kBN * 128;  // one 64-column slice of a K or V tile
 constexpr int kQBytes = 4 * kQChunk;
 constexpr int kKBytes = 4 * kKChunk;
 constexpr int kVBytes = 4 * kKChunk;
-constexpr int kPBytes = kM * 128;
 
 constexpr int oQ = 0;
+constexpr int kKS = 3;  // K stages
 constexpr int oK0 = oQ + kQBytes;
 constexpr int oK1 = oK0 + kKBytes;
 constexpr int oV0 = oK1 + kKBytes;
-constexpr int oV1 = oV0 + kVBytes;
-constexpr int oP0 = oV1 + kVBytes;
-constexpr int oP1 = oP0 + kPBytes;
-constexpr int oBar = oP1 + kPBytes;
-// Q staging area (raw rows) before the swizzled Q tile is built: the second V
-// stage and both P buffers, contiguous and idle at that point
-constexpr int oStage = oV1;
-static_assert(oP1 + kPBytes - oStage >= kM * kDQK * 2, "staging area too small");
+constexpr int oK2 = oV0 + kVBytes;
+constexpr int oV1 = oK2 + kKBytes;
+constexpr int oBar = oV1 + kVBytes;
+// Q staging area (raw rows) before the swizzled Q tile is built: the third K
+// stage and the second V stage, contiguous and idle at that point
+constexpr int oStage = oK2;
+static_assert(oBar - oStage >= kM * kDQK * 2, "staging area too small");
+__device__ __forceinline__ int k_stage_off(int t) {
+    const int s = t % kKS;
+    return s == 0 ? oK0 : (s == 1 ? oK1 : oK2);
+}
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
@@ -76,7 +83,8 @@ constexpr int kThreads = 352;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383
-constexpr uint32_t kColX = 384;  // row-max exchange (2 tiles x 2 halves), then the row-sum exchange
+constexpr uint32_t kColP = 384;  // two P buffers (bf16 pairs): 384..415, 416..447
+constexpr uint32_t kColX = 448;  // row-max exchange (2 tiles x 2 halves), then the row-sum exchange
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -98,17 +106,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kfull = bars + 0, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
-    uint64_t *sfull = bars + 8, *pready = bars + 10, *pvdone = bars + 12, *qready = bars + 14;
-    uint64_t *drain = bars + 15, *qraw = bars + 16, *qstaged = bars + 17;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
+    uint64_t *kfull = bars + 0, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 8;
+    uint64_t *sfull = bars + 10, *pready = bars + 12, *pvdone = bars + 14, *qready = bars + 16;
+    uint64_t *drain = bars + 17, *qraw = bars + 18, *qstaged = bars + 19;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 21);
     // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
     // [4] raw Q issued
-    int *counters = reinterpret_cast<int *>(bars + 20);
+    int *counters = reinterpret_cast<int *>(bars + 22);
     // softmax pair exchange: per TMEM sub-partition and S buffer the tile max,
     // per sub-partition the row sum (two arrivals each: one per warp)
-    uint64_t *xbar = bars + 24, *lbar = bars + 32;
+    uint64_t *xbar = bars + 26, *lbar = bars + 34;
 
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int cnt = p.cnt[b];
@@ -128,12 +136,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // K/V stages start zeroed: masked key slots of a tile are multiplied by a
     // zero weight, and must not hold stale non-finite bits.
-    for (int e = threadIdx.x; e < (oP0 - oK0) / 16; e += blockDim.x)
+    for (int e = threadIdx.x; e < (oBar - oK0) / 16; e += blockDim.x)
         reinterpret_cast<uint4 *>(sm + oK0)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < kKS; s++) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < 2; s++) {
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
             mbar_init(&sfull[s], 1);
@@ -202,10 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             int pf_next = 2;  // next tile to prefetch into L2
             for (int t = 0; t < T; ++t) {
-                const int s = t & 1;
-                uint8_t *kt = sm + (s ? oK1 : oK0);
+                const int s = t % kKS;
+                uint8_t *kt = sm + k_stage_off(t);
                 for (; pf_next <= t + 3 && pf_next < T; ++pf_next) prefetch_tile(pf_next);
-                if (t >= 2 && !warp_all(mbar_wait(&kempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+                // the third K stage doubles as the Q staging area until the
+                // softmax warps have moved Q into place
+                if (t == 2 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
+                if (t >= kKS && !warp_all(mbar_wait(&kempty[s], ((t / kKS) - 1) & 1, abort_flag))) break;
                 if (t < n_ctx) {
                     const int pos0 = ctx_lo + t * kBN;
                     if (lane == 0) {
@@ -276,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = mbar_wait(qready, 0, abort_flag);
             auto issue_qk = [&](int t) {
                 const int s = t & 1;
-                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oK1 : oK0)), 16, 1024));
+                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + k_stage_off(t)), 16, 1024));
                 const uint32_t dS = tmem + kColS + s * kBN;
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
@@ -285,36 +298,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_bf16_ss(dS, qd.at(qo), kd.at(ko), idS, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[s]);
-                mma_commit(&kempty[s]);
+                mma_commit(&kempty[t % kKS]);
                 counters[2] = t + 1;
             };
-            if (ok) ok = mbar_wait(&kfull[0], 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                issue_qk(0);
-            }
-            for (int t = 0; t < T && ok; ++t) {
-                if (t + 1 < T) {
-                    const int t1 = t + 1, s1 = t1 & 1;
-                    if (t1 >= 2) ok = mbar_wait(&pready[s1], ((t1 >> 1) - 1) & 1, abort_flag);
-                    if (ok) ok = mbar_wait(&kfull[s1], (t1 >> 1) & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_qk(t1);
-                }
+            auto issue_pv = [&](int t) {
                 const int s = t & 1;
-                ok = mbar_wait(&pready[s], (t >> 1) & 1, abort_flag);
-                if (ok) ok = mbar_wait(&vfull[s], (t >> 1) & 1, abort_flag);
-                if (!ok) break;
-                counters[3] = t + 1;
-                tc_fence_after();
-                const SDesc pd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oP1 : oP0)), 16, 1024));
                 const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oV1 : oV0)), kKChunk, 1024));
-                mma_bf16_ss(tmem + kColO, pd.at(0), vd.at(0), idO, t > 0 ? 1u : 0u);
+                const uint32_t pa = tmem + kColP + s * (kBN / 2);
+                mma_bf16_ts(tmem + kColO, pa, vd.at(0), idO, t > 0 ? 1u : 0u);
 #pragma unroll
-                for (int k = 1; k < kBN / 16; ++k) mma_bf16_ss(tmem + kColO, pd.at(2 * k), vd.at(128 * k), idO, 1u);
+                for (int k = 1; k < kBN / 16; ++k) mma_bf16_ts(tmem + kColO, pa + 8 * k, vd.at(128 * k), idO, 1u);
                 mma_commit(&vempty[s]);
                 mma_commit(&pvdone[s]);
+            };
+            // Issue whichever is ready: QK of tile nk (its K landed and the
+            // softmax warps have finished tile nk - 2, whose S buffer it
+            // reuses) or P V of tile np (its P is in TMEM and its V landed).
+            int nk = 0, np = 0;
+            uint64_t t_idle = 0;
+            if (ok) tc_fence_after();
+            while (ok && np < T) {
+                bool issued = false;
+                if (nk < T && (nk < 2 || mbar_test(&pready[nk & 1], ((nk >> 1) - 1) & 1)) &&
+                    mbar_test(&kfull[nk % kKS], (nk / kKS) & 1)) {
+                    tc_fence_after();
+                    issue_qk(nk);
+                    ++nk;
+                    issued = true;
+                }
+                if (!issued && np < nk && mbar_test(&pready[np & 1], (np >> 1) & 1) &&
+                    mbar_test(&vfull[np & 1], (np >> 1) & 1)) {
+                    counters[3] = np + 1;
+                    tc_fence_after();
+                    issue_pv(np);
+                    ++np;
+                    issued = true;
+                }
+                if (issued) {
+                    t_idle = 0;
+                } else {
+                    const uint64_t now = globaltimer();
+                    if (t_idle == 0) t_idle = now;
+                    if (*abort_flag) ok = false;
+                    else if (now - t_idle > kWaitTimeoutNs) {
+                        *abort_flag = 1;
+                        ok = false;
+                    }
+                }
             }
         }
     } else {
@@ -384,9 +414,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float sv[32];
-            tmem_ld32(trow + kColS + s * kBN + 32 * hf, sv);
-            tmem_wait_ld();
             // every row's keys in a tile form one contiguous column range
             // [clo, chi): the window [lo, A) for context tiles, its block's 5
             // key slots for draft tiles; this warp holds columns 32 hf .. +31
@@ -402,13 +429,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!live) chi = clo;
             clo -= 32 * hf;
             chi -= 32 * hf;
+            // Rows are anchor-sorted, so for most (warp, half tile) pairs no
+            // row of the warp sees any of the 32 keys: such a half tile only
+            // contributes P = 0 (uniform over the warp, no S read).
+            const bool act = __any_sync(0xffffffffu, clo < chi && clo < 32 && chi > 0);
+            float sv[32];
             float mx[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) mx[k] = -INFINITY;
+            if (act) {
+                tmem_ld32(trow + kColS + s * kBN + 32 * hf, sv);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; c++) {
-                sv[c] = (c >= clo && c < chi) ? sv[c] : -INFINITY;
-                mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+                for (int c = 0; c < 32; c++) {
+                    sv[c] = (c >= clo && c < chi) ? sv[c] : -INFINITY;
+                    mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+                }
             }
             // the pair's tile max: each half stores its own in TMEM, both
             // read the other's after a pair barrier
@@ -436,24 +472,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = warp_all(mbar_wait(&pvdone[s], ((t - 2) >> 1) & 1, abort_flag));
                 if (!ok) break;
             }
-            uint8_t *prow = sm + (s ? oP1 : oP0);
             float psum[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) psum[k] = 0.f;
             const bool any = m_used != -INFINITY;
             const float mneg = any ? -m_used : 0.f;
+            uint32_t pw[16];  // this half's 32 P values as bf16 pairs
+            if (act) {
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                float e[8];
-#pragma unroll
-                for (int k = 0; k < 8; k++) {
-                    e[k] = any ? ex2(fmaf(sv[u * 8 + k], p.scale_log2, mneg)) : 0.f;
-                    psum[k & 3] += e[k];
+                for (int c = 0; c < 32; c += 2) {
+                    const float e0 = any ? ex2(fmaf(sv[c], p.scale_log2, mneg)) : 0.f;
+                    const float e1 = any ? ex2(fmaf(sv[c + 1], p.scale_log2, mneg)) : 0.f;
+                    psum[c & 3] += e0;
+                    psum[(c + 1) & 3] += e1;
+                    pw[c / 2] = pack_bf16x2(e0, e1);
                 }
-                uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
-                                      pack_bf16x2(e[6], e[7]));
-                *reinterpret_cast<uint4 *>(prow + sw128(r, 4 * hf + u)) = pk;
+            } else {
+#pragma unroll
+                for (int c = 0; c < 16; c++) pw[c] = 0u;
             }
+            tmem_st16u(trow + kColP + s * (kBN / 2) + 16 * hf, pw);
             l = l * alpha + ((psum[0] + psum[1]) + (psum[2] + psum[3]));
             if (__any_sync(0xffffffffu, resc)) {
                 if (t >= 1) {
@@ -470,9 +508,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; i++) ov[i] *= alpha;
                     tmem_st32(trow + kColO + c, ov);
                 }
-                tmem_wait_st();
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&pready[s]);
@@ -534,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (counters[4]) mbar_wait(qraw, 0, (volatile int *)&never);
             // loads issued but not yet consumed complete in order, one phase each
             for (int t = counters[2]; t < counters[0]; ++t)
-                mbar_wait(&kfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+                mbar_wait(&kfull[t % kKS], (t / kKS) & 1, (volatile int *)&never);
             for (int t = counters[3]; t < counters[1]; ++t)
                 mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
         }
