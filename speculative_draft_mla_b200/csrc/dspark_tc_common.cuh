@@ -102,6 +102,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
         "l"((uint64_t)m), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// 3-D tiled TMA load (no multicast) completing on bar's transaction count.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+            "r"(smem_u32(dst)),
+        "l"((uint64_t)m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
 // 1-D bulk copy of `bytes` contiguous bytes (16-byte aligned addresses, size a
 // multiple of 16) completing on bar's transaction count.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -113,6 +121,11 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
 // Prefetch a 2-D tile of a tensor map into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *m, int x, int y) {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"((uint64_t)m), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *m, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"((uint64_t)m), "r"(x), "r"(y),
+                 "r"(z)
                  : "memory");
 }
 __device__ __forceinline__ void prefetch_l2(const void *p) {
@@ -323,6 +336,23 @@ inline bool make_map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint
     cuuint32_t box[2] = {64, box_rows};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A row-major [rows][inner] bf16 matrix (inner a multiple of 64) seen as 3-D
+// (64 elements, rows, inner / 64 column chunks): the chunk stride (128 B) is
+// smaller than the row stride, so one box {64, box_rows, inner / 64} lands in
+// shared memory as inner / 64 consecutive [box_rows][128 B] slices, each with
+// the 128-byte swizzle - the K-major operand layout - in a single copy.
+inline bool make_map3_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, rows, inner / 64};
+    cuuint64_t strides[2] = {inner * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, (cuuint32_t)(inner / 64)};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

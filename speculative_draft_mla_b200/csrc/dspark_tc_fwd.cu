@@ -12,27 +12,30 @@
 // are sorted by anchor, neighbouring groups (adjacent blockIdx.x) read
 // overlapping windows close together in time, so the overlap is served by L2.
 //
+// The kernel is bound by how many key/value bytes each SM keeps in flight, so
+// shared memory holds only K and V stages (three each): Q lives in tensor
+// memory (A operand of S = Q K^T read from TMEM), and P is written over its
+// own S columns (A operand of O += P V read from TMEM). TMEM: O 0..255,
+// S 256..319 / 320..383, Q 384..511.
+//
 // Warp roles (352 threads):
 //   warps 0-7  softmax: warps w and w + 4 share TMEM sub-partition w % 4, so
 //              query rows 32 (w % 4) .. + 31 (thread = row = TMEM lane), and
-//              split each 64-key tile into two 32-column halves. They lay Q
-//              out for the MMA and RoPE-rotate it at the start, turn each S
-//              tile into P (bf16, written to TMEM, where the P V MMA reads it
-//              as its A operand) with an online softmax
-//              whose row max the pair exchanges through spare TMEM columns,
+//              split each 64-key tile into two 32-column halves. They move
+//              the row's half of Q into TMEM (RoPE-rotating the rope slice)
+//              at the start, turn each S tile into P with an online softmax
+//              whose row max the pair exchanges through shared memory,
 //              rescale their half of the O row when the running max grows by
 //              more than 2^8, and write O and LSE.
-//   warp 8     K producer: the group's raw Q rows (one bulk copy per block),
-//              TMA loads of context K tiles (K^C 3 x 64 columns plus the
+//   warp 8     K producer: the group's raw Q rows (one bulk copy per row),
+//              TMA loads of context K tiles (K^C as one 3-D box, plus the
 //              pre-rotated shared K^R) and of draft-key tiles (8-row boxes per
-//              block), L2 prefetch of the K and V tiles three tiles ahead;
-//              three K stages (a K tile waits on the longest chain: its
-//              stage frees only when the QK MMA two tiles back completes).
+//              block), L2 prefetch of the K and V tiles three tiles ahead.
 //   warp 9     TMEM owner and MMA issuer (one thread): S = Q K^T into two
-//              alternating 64-column TMEM buffers, O += P V into 256 columns,
-//              each issued as soon as its inputs are ready.
-//   warp 10    V producer: the V tiles, so a K load never queues behind a V
-//              stage that is still being read.
+//              alternating S buffers, O += P V, each issued as soon as its
+//              inputs are ready (an S buffer is reused only after the P V
+//              that reads the P written over it).
+//   warp 10    V producer.
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait, TMEM is freed and the workspace error word gets kErrTimeout.
@@ -51,28 +54,23 @@ constexpr int kM = 128;   // query rows per CTA (MMA M)
 constexpr int kBN = 64;   // keys per tile
 constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
 
-constexpr int kQChunk = kM * 128;   // one 64-column slice of the Q tile
 constexpr int kKChunk = kBN * 128;  // one 64-column slice of a K or V tile
-constexpr int kQBytes = 4 * kQChunk;
 constexpr int kKBytes = 4 * kKChunk;
 constexpr int kVBytes = 4 * kKChunk;
+constexpr int kKS = 3, kVS = 3;     // K and V stages
 
-constexpr int oQ = 0;
-constexpr int kKS = 3;  // K stages
-constexpr int oK0 = oQ + kQBytes;
-constexpr int oK1 = oK0 + kKBytes;
-constexpr int oV0 = oK1 + kKBytes;
-constexpr int oK2 = oV0 + kVBytes;
-constexpr int oV1 = oK2 + kKBytes;
-constexpr int oBar = oV1 + kVBytes;
-// Q staging area (raw rows) before the swizzled Q tile is built: the third K
-// stage and the second V stage, contiguous and idle at that point
-constexpr int oStage = oK2;
-static_assert(oBar - oStage >= kM * kDQK * 2, "staging area too small");
-__device__ __forceinline__ int k_stage_off(int t) {
-    const int s = t % kKS;
-    return s == 0 ? oK0 : (s == 1 ? oK1 : oK2);
-}
+// Stage order K0 K1 V0 K2 V1 V2: the raw Q rows are staged over K2 and V1,
+// so the first two K tiles and the first V tile load while Q is moved.
+constexpr int oStage = 3 * kKBytes;
+constexpr int oX = 6 * kKBytes;  // pair exchange: tile max [2][2][128], row sum [2][128] (floats)
+constexpr int oBar = oX + 3 * 1024;
+__device__ __forceinline__ int k_stage_off(int s) { return s == 0 ? 0 : (s == 1 ? kKBytes : 3 * kKBytes); }
+__device__ __forceinline__ int v_stage_off(int s) { return s == 0 ? 2 * kKBytes : (s == 1 ? 4 * kKBytes : 5 * kKBytes); }
+// Raw Q: one bulk copy per block (5 rows of 512 B), blocks 2576 B apart, so
+// the rows that the threads of a warp read at once fall on at most 5 rows
+// per bank group.
+constexpr int kStageBlockPitch = kBlock * kDQK * 2 + 16;
+static_assert(kG * kStageBlockPitch <= 2 * kKBytes, "staging area too small");
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
@@ -82,9 +80,8 @@ constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10;
 constexpr int kThreads = 352;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
-constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383
-constexpr uint32_t kColP = 384;  // two P buffers (bf16 pairs): 384..415, 416..447
-constexpr uint32_t kColX = 448;  // row-max exchange (2 tiles x 2 halves), then the row-sum exchange
+constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383 (P over the first 16 columns of each half)
+constexpr uint32_t kColQ = 384;  // Q: 256 bf16 per row as 128 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -100,23 +97,25 @@ struct FwdArgs {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
-             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc8,
+    k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc3, const __grid_constant__ CUtensorMap tm_kr,
+             const __grid_constant__ CUtensorMap tm_v3, const __grid_constant__ CUtensorMap tm_kc8,
              const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const FwdArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kfull = bars + 0, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 8;
-    uint64_t *sfull = bars + 10, *pready = bars + 12, *pvdone = bars + 14, *qready = bars + 16;
-    uint64_t *drain = bars + 17, *qraw = bars + 18, *qstaged = bars + 19;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 21);
-    // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
-    // [4] raw Q issued
-    int *counters = reinterpret_cast<int *>(bars + 22);
+    uint64_t *kfull = bars + 0, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 9;
+    uint64_t *sfull = bars + 12, *pready = bars + 14, *pvdone = bars + 16, *qready = bars + 18;
+    uint64_t *drain = bars + 19, *qraw = bars + 20, *qstaged = bars + 21;
     // softmax pair exchange: per TMEM sub-partition and S buffer the tile max,
     // per sub-partition the row sum (two arrivals each: one per warp)
-    uint64_t *xbar = bars + 26, *lbar = bars + 34;
+    uint64_t *xbar = bars + 22, *lbar = bars + 30;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 34);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 35);
+    // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
+    // [4] raw Q issued
+    int *counters = reinterpret_cast<int *>(bars + 36);
+    float *xm = reinterpret_cast<float *>(sm + oX);         // [s][half][row]
+    float *xl = reinterpret_cast<float *>(sm + oX + 2048);  // [half][row]
 
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int cnt = p.cnt[b];
@@ -135,17 +134,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t bh = (size_t)b * p.n_h + h;
 
     // K/V stages start zeroed: masked key slots of a tile are multiplied by a
-    // zero weight, and must not hold stale non-finite bits.
-    for (int e = threadIdx.x; e < (oBar - oK0) / 16; e += blockDim.x)
-        reinterpret_cast<uint4 *>(sm + oK0)[e] = make_uint4(0, 0, 0, 0);
+    // zero weight, and must not hold stale non-finite bits (the V stages then
+    // hold raw Q rows, finite, until V tiles overwrite them).
+    for (int e = threadIdx.x; e < oX / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKS; s++) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 1);
         }
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < kVS; s++) {
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
+        }
+        for (int s = 0; s < 2; s++) {
             mbar_init(&sfull[s], 1);
             mbar_init(&pready[s], kSoftWarps);
             mbar_init(&pvdone[s], 1);
@@ -176,27 +178,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int my_n = lane < gcnt ? sn[lane] : 0;
         if (warp == kWarpK) {
             if (lane == 0) {
-                tma_prefetch_desc(&tm_kc);
+                tma_prefetch_desc(&tm_kc3);
                 tma_prefetch_desc(&tm_kr);
-                tma_prefetch_desc(&tm_v);
-                // raw Q rows of the group: each block's 5 rows are one contiguous
-                // 2560-byte run; they land row-major in the staging area
+                tma_prefetch_desc(&tm_v3);
+                // raw Q rows of the group: each block's 5 rows are one
+                // contiguous 2560-byte run
                 mbar_arrive_expect_tx(qraw, nrows * kDQK * 2);
                 counters[4] = 1;
             }
             __syncwarp();
             if (lane < gcnt)
-                bulk_load(sm + oStage + lane * (kBlock * kDQK * 2),
-                          p.q + (bh * p.R + (size_t)kBlock * my_n) * kDQK, kBlock * kDQK * 2, qraw);
+                bulk_load(sm + oStage + lane * kStageBlockPitch, p.q + (bh * p.R + (size_t)kBlock * my_n) * kDQK,
+                          kBlock * kDQK * 2, qraw);
             // L2 prefetch of tile tt's K and V (context rows, or the 8-row
             // boxes of the draft tile's blocks, one block per lane)
             auto prefetch_tile = [&](int tt) {
                 if (tt < n_ctx) {
                     if (lane == 0) {
                         const int pos = ctx_lo + tt * kBN;
-                        for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
+                        tma_prefetch_3d(&tm_kc3, 0, (int)(bh * p.L + pos), 0);
                         tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
-                        for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
+                        tma_prefetch_3d(&tm_v3, 0, (int)(bh * p.L + pos), 0);
                     }
                 } else {
                     const int d = tt - n_ctx;
@@ -210,21 +212,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             };
-            int pf_next = 2;  // next tile to prefetch into L2
+            int pf_next = kKS;  // next tile to prefetch into L2
             for (int t = 0; t < T; ++t) {
                 const int s = t % kKS;
-                uint8_t *kt = sm + k_stage_off(t);
-                for (; pf_next <= t + 3 && pf_next < T; ++pf_next) prefetch_tile(pf_next);
-                // the third K stage doubles as the Q staging area until the
-                // softmax warps have moved Q into place
+                uint8_t *kt = sm + k_stage_off(s);
+                for (; pf_next <= t + kKS && pf_next < T; ++pf_next) prefetch_tile(pf_next);
+                // the third K stage holds raw Q rows until they are in TMEM
                 if (t == 2 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
                 if (t >= kKS && !warp_all(mbar_wait(&kempty[s], ((t / kKS) - 1) & 1, abort_flag))) break;
                 if (t < n_ctx) {
                     const int pos0 = ctx_lo + t * kBN;
                     if (lane == 0) {
                         mbar_arrive_expect_tx(&kfull[s], kKBytes);
-                        for (int c = 0; c < 3; c++)
-                            tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[s], c * 64, (int)(bh * p.L + pos0));
+                        tma_load_3d(kt, &tm_kc3, &kfull[s], 0, (int)(bh * p.L + pos0), 0);
                         tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
                     }
                 } else {
@@ -249,18 +249,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else {
             for (int t = 0; t < T; ++t) {
-                const int s = t & 1;
-                uint8_t *vt = sm + (s ? oV1 : oV0);
-                // the second V stage doubles as the Q staging area until the
-                // softmax warps have moved Q into place
+                const int s = t % kVS;
+                uint8_t *vt = sm + v_stage_off(s);
+                // the second V stage holds raw Q rows until they are in TMEM
                 if (t == 1 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
-                if (t >= 2 && !warp_all(mbar_wait(&vempty[s], ((t >> 1) - 1) & 1, abort_flag))) break;
+                if (t >= kVS && !warp_all(mbar_wait(&vempty[s], ((t / kVS) - 1) & 1, abort_flag))) break;
                 if (t < n_ctx) {
                     const int pos0 = ctx_lo + t * kBN;
                     if (lane == 0) {
                         mbar_arrive_expect_tx(&vfull[s], kVBytes);
-                        for (int c = 0; c < 4; c++)
-                            tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[s], c * 64, (int)(bh * p.L + pos0));
+                        tma_load_3d(vt, &tm_v3, &vfull[s], 0, (int)(bh * p.L + pos0), 0);
                     }
                 } else {
                     const int d = t - n_ctx;
@@ -285,17 +283,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kM, kBN, 0);
             const uint32_t idO = idesc_bf16(kM, kDV, 1);
-            const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + oQ), 16, 1024));
             bool ok = mbar_wait(qready, 0, abort_flag);
             auto issue_qk = [&](int t) {
                 const int s = t & 1;
-                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + k_stage_off(t)), 16, 1024));
+                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + k_stage_off(t % kKS)), 16, 1024));
                 const uint32_t dS = tmem + kColS + s * kBN;
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
-                    const uint32_t qo = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
                     const uint32_t ko = ((k >> 2) * kKChunk + (k & 3) * 32) >> 4;
-                    mma_bf16_ss(dS, qd.at(qo), kd.at(ko), idS, k > 0 ? 1u : 0u);
+                    mma_bf16_ts(dS, tmem + kColQ + 8 * k, kd.at(ko), idS, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[s]);
                 mma_commit(&kempty[t % kKS]);
@@ -303,31 +299,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_pv = [&](int t) {
                 const int s = t & 1;
-                const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + (s ? oV1 : oV0)), kKChunk, 1024));
-                const uint32_t pa = tmem + kColP + s * (kBN / 2);
+                const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + v_stage_off(t % kVS)), kKChunk, 1024));
+                // P of keys 16 k .. 16 k + 15: half k / 2 of the S buffer, its
+                // columns 8 (k % 2) ..
+                const uint32_t pa = tmem + kColS + s * kBN;
                 mma_bf16_ts(tmem + kColO, pa, vd.at(0), idO, t > 0 ? 1u : 0u);
-#pragma unroll
-                for (int k = 1; k < kBN / 16; ++k) mma_bf16_ts(tmem + kColO, pa + 8 * k, vd.at(128 * k), idO, 1u);
-                mma_commit(&vempty[s]);
+                mma_bf16_ts(tmem + kColO, pa + 8, vd.at(128), idO, 1u);
+                mma_bf16_ts(tmem + kColO, pa + 32, vd.at(256), idO, 1u);
+                mma_bf16_ts(tmem + kColO, pa + 40, vd.at(384), idO, 1u);
+                mma_commit(&vempty[t % kVS]);
                 mma_commit(&pvdone[s]);
             };
-            // Issue whichever is ready: QK of tile nk (its K landed and the
-            // softmax warps have finished tile nk - 2, whose S buffer it
-            // reuses) or P V of tile np (its P is in TMEM and its V landed).
+            // Issue whichever is ready: QK of tile nk (its K landed, and the
+            // P V of tile nk - 2 that reads the P written over its S buffer
+            // is already issued) or P V of tile np (its P is in TMEM and its
+            // V landed).
             int nk = 0, np = 0;
             uint64_t t_idle = 0;
             if (ok) tc_fence_after();
             while (ok && np < T) {
                 bool issued = false;
-                if (nk < T && (nk < 2 || mbar_test(&pready[nk & 1], ((nk >> 1) - 1) & 1)) &&
-                    mbar_test(&kfull[nk % kKS], (nk / kKS) & 1)) {
+                if (nk < T && np >= nk - 1 && mbar_test(&kfull[nk % kKS], (nk / kKS) & 1)) {
                     tc_fence_after();
                     issue_qk(nk);
                     ++nk;
                     issued = true;
                 }
                 if (!issued && np < nk && mbar_test(&pready[np & 1], (np >> 1) & 1) &&
-                    mbar_test(&vfull[np & 1], (np >> 1) & 1)) {
+                    mbar_test(&vfull[np % kVS], (np / kVS) & 1)) {
                     counters[3] = np + 1;
                     tc_fence_after();
                     issue_pv(np);
@@ -362,48 +361,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         {
-            // Q: raw rows of the staging area -> the swizzled Q tile; rows
-            // past the group are zero. The content slice (16-byte units 0..23
-            // of a row) moves one row per warp instruction, lane l taking unit
-            // l (warp w: rows 16 w .. 16 w + 15); the rope slice (units 24..31)
-            // is rotated to position A + j by the row's two threads, four
-            // units each, with cos/sin fetched before Q lands.
-            float4 cs[8];  // (cos, sin) of rope frequencies 16 hf .. 16 hf + 15 at A + j
-            const float4 *tp =
-                reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2)) + 8 * hf;
+            // Q row r, this thread's half (columns 128 hf .. + 127) -> TMEM
+            // lane r, columns kColQ + 64 hf .. + 63; the rope slice (the last
+            // 64 columns, half 1) is rotated to position A + j first. Rows
+            // past the group are zero.
+            float4 cs[16];  // (cos, sin) of the 32 rope frequencies at A + j (half 1)
+            if (hf == 1) {
+                const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2));
 #pragma unroll
-            for (int k = 0; k < 8; k++) cs[k] = __ldg(tp + k);
-            ok = warp_all(mbar_wait(qraw, 0, abort_flag));
-            if (lane < kDC / 8) {
-#pragma unroll 8
-                for (int i = 0; i < 16; i++) {
-                    const int row = warp * 16 + i;
-                    const bool have = ok && row < nrows;
-                    *reinterpret_cast<uint4 *>(sm + oQ + (lane >> 3) * kQChunk + sw128(row, lane & 7)) =
-                        have ? *reinterpret_cast<const uint4 *>(sm + oStage + row * (kDQK * 2) + lane * 16)
-                             : make_uint4(0, 0, 0, 0);
-                }
+                for (int k = 0; k < 16; k++) cs[k] = __ldg(tp + k);
             }
-            const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + r * (kDQK * 2));
+            ok = warp_all(mbar_wait(qraw, 0, abort_flag));
             const bool have = live && ok;
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + (r / kBlock) * kStageBlockPitch +
+                                                               (r % kBlock) * (kDQK * 2) + hf * 256);
             // a bf16 pair (x0 low, x1 high) rotated by (c, s)
             auto rot = [](uint32_t w, float c, float s_) {
                 const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
                 return pack_bf16x2(x0 * c - x1 * s_, x0 * s_ + x1 * c);
             };
 #pragma unroll
-            for (int uu = 0; uu < 4; uu++) {  // unit u = 4 hf + uu: frequencies 4u .. 4u+3
-                const int u = 4 * hf + uu;
-                const uint4 val = have ? src[kDC / 8 + u] : make_uint4(0, 0, 0, 0);
-                const float4 c01 = cs[2 * uu], c23 = cs[2 * uu + 1];
-                *reinterpret_cast<uint4 *>(sm + oQ + 3 * kQChunk + sw128(r, u)) =
-                    make_uint4(rot(val.x, c01.x, c01.y), rot(val.y, c01.z, c01.w), rot(val.z, c23.x, c23.y),
-                               rot(val.w, c23.z, c23.w));
+            for (int part = 0; part < 2; part++) {  // 8 units (64 bf16) per TMEM store
+                uint32_t w[32];
+#pragma unroll
+                for (int uu = 0; uu < 8; uu++) {
+                    uint4 val = have ? src[part * 8 + uu] : make_uint4(0, 0, 0, 0);
+                    if (hf == 1 && part == 1) {  // rope unit uu: frequencies 4 uu .. 4 uu + 3
+                        const float4 c01 = cs[2 * uu], c23 = cs[2 * uu + 1];
+                        val = make_uint4(rot(val.x, c01.x, c01.y), rot(val.y, c01.z, c01.w), rot(val.z, c23.x, c23.y),
+                                         rot(val.w, c23.z, c23.w));
+                    }
+                    w[4 * uu + 0] = val.x;
+                    w[4 * uu + 1] = val.y;
+                    w[4 * uu + 2] = val.z;
+                    w[4 * uu + 3] = val.w;
+                }
+                tmem_st32u(trow + kColQ + 64 * hf + 32 * part, w);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(qstaged);  // staging area free for V tiles and P
+                mbar_arrive(qstaged);  // staging area free for V tiles
                 mbar_arrive(qready);
             }
         }
@@ -446,18 +445,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
                 }
             }
-            // the pair's tile max: each half stores its own in TMEM, both
-            // read the other's after a pair barrier
+            // the pair's tile max, exchanged through shared memory
             const float mhalf = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            tmem_st1(trow + kColX + 2 * s + hf, mhalf);
-            tmem_wait_st();
-            tc_fence_before();
+            xm[(s * 2 + hf) * kM + r] = mhalf;
             __syncwarp();
             if (lane == 0) mbar_arrive(&xbar[2 * q4 + s]);
             ok = warp_all(mbar_wait(&xbar[2 * q4 + s], (t >> 1) & 1, abort_flag));
             if (!ok) break;
-            tc_fence_after();
-            const float mother = tmem_ld1_wait(trow + kColX + 2 * s + (hf ^ 1));
+            const float mother = xm[(s * 2 + (hf ^ 1)) * kM + r];
             const float mt = fmaxf(mhalf, mother) * p.scale_log2;
             bool resc = false;
             float alpha = 1.f;
@@ -467,10 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     alpha = ex2(m_used - mt);
                 }
                 m_used = mt;
-            }
-            if (t >= 2) {
-                ok = warp_all(mbar_wait(&pvdone[s], ((t - 2) >> 1) & 1, abort_flag));
-                if (!ok) break;
             }
             float psum[4];
 #pragma unroll
@@ -491,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 16; c++) pw[c] = 0u;
             }
-            tmem_st16u(trow + kColP + s * (kBN / 2) + 16 * hf, pw);
+            // P over this half's first 16 S columns (the S values are in registers)
+            tmem_st16u(trow + kColS + s * kBN + 32 * hf, pw);
             l = l * alpha + ((psum[0] + psum[1]) + (psum[2] + psum[3]));
             if (__any_sync(0xffffffffu, resc)) {
                 if (t >= 1) {
@@ -516,23 +508,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) ok = warp_all(mbar_wait(&pvdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
         if (ok) {
-            tc_fence_after();
             // the row sum: both halves' shares, exchanged like the tile max
-            tmem_st1(trow + kColX + 4 + hf, l);
-            tmem_wait_st();
-            tc_fence_before();
+            xl[hf * kM + r] = l;
             __syncwarp();
             if (lane == 0) mbar_arrive(&lbar[q4]);
             ok = warp_all(mbar_wait(&lbar[q4], 0, abort_flag));
         }
         if (ok) {
             tc_fence_after();
-            const float ltot = l + tmem_ld1_wait(trow + kColX + 4 + (hf ^ 1));
+            const float ltot = l + xl[(hf ^ 1) * kM + r];
             const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
             // this half of the O row (columns 128 hf .. +127) -> staging in the
-            // idle K stages (row i of the warp at 256 i, unit u at u ^ (i & 15))
-            // -> two half rows per warp instruction
-            uint8_t *stage = sm + oK0 + warp * (32 * 256);
+            // idle K0, K1 stages (row i of the warp at 256 i, unit u at
+            // u ^ (i & 15)) -> two half rows per warp instruction
+            uint8_t *stage = sm + warp * (32 * 256);
 #pragma unroll 1
             for (int c = 0; c < 128; c += 32) {
                 float ov[32];
@@ -573,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = counters[2]; t < counters[0]; ++t)
                 mbar_wait(&kfull[t % kKS], (t / kKS) & 1, (volatile int *)&never);
             for (int t = counters[3]; t < counters[1]; ++t)
-                mbar_wait(&vfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+                mbar_wait(&vfull[t % kVS], (t / kVS) & 1, (volatile int *)&never);
         }
         if (warp == kWarpMma && lane == 0) {
             mma_commit(drain);
@@ -617,10 +606,10 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     if (p.B == 0 || p.N == 0) return cudaSuccess;
     count_launch();
     k_fwd_pad_rows<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.R, anchors, keep, (__nv_bfloat16 *)o, lse);
-    CUtensorMap m_kc, m_kr, m_v, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc3, m_kr, m_v3, m_kc8, m_kr8, m_v8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, kr_rows = (uint64_t)p.B * p.L;
-    if (!make_map_bf16(&m_kc, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr, ws.kr_rot, kDR, kr_rows, 64) ||
-        !make_map_bf16(&m_v, v, kDV, kv_rows, 64) || !make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) ||
+    if (!make_map3_bf16(&m_kc3, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr, ws.kr_rot, kDR, kr_rows, 64) ||
+        !make_map3_bf16(&m_v3, v, kDV, kv_rows, 64) || !make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) ||
         !make_map_bf16(&m_kr8, ws.kr_rot, kDR, kr_rows, 8) || !make_map_bf16(&m_v8, v, kDV, kv_rows, 8))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -641,7 +630,7 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.err = ws.err;
     dim3 grid((p.N + kG - 1) / kG, p.n_h, p.B);
     count_launch();
-    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc, m_kr, m_v, m_kc8, m_kr8, m_v8, a);
+    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc3, m_kr, m_v3, m_kc8, m_kr8, m_v8, a);
     return cudaGetLastError();
 }
 
