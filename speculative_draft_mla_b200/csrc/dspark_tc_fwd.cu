@@ -29,8 +29,9 @@
 //              more than 2^8, and write O and LSE.
 //   warp 8     K producer: the group's raw Q rows (one bulk copy per row),
 //              TMA loads of context K tiles (K^C as one 3-D box, plus the
-//              pre-rotated shared K^R) and of draft-key tiles (8-row boxes per
-//              block), L2 prefetch of the K and V tiles three tiles ahead.
+//              pre-rotated shared K^R) and of draft-key tiles (per block one
+//              3-D box of its 8 K^C rows and one of its K^R rows), L2
+//              prefetch of the K and V tiles three tiles ahead.
 //   warp 9     TMEM owner and MMA issuer (one thread): S = Q K^T into two
 //              alternating S buffers, O += P V, each issued as soon as its
 //              inputs are ready (an S buffer is reused only after the P V
@@ -72,6 +73,11 @@ __device__ __forceinline__ int v_stage_off(int s) { return s == 0 ? 2 * kKBytes 
 constexpr int kStageBlockPitch = kBlock * kDQK * 2 + 16;
 static_assert(kG * kStageBlockPitch <= 2 * kKBytes, "staging area too small");
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
+// Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
+// slices) at bb * 3 KB, its K^R rows at 24 KB + bb * 1 KB; its V rows (4 x 1 KB)
+// at bb * 4 KB. As MMA operands: K^C with 8-row groups 3 KB apart, V with
+// 64-column slices 1 KB apart and 8-key groups 4 KB apart.
+constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
@@ -98,8 +104,8 @@ struct FwdArgs {
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc3, const __grid_constant__ CUtensorMap tm_kr,
-             const __grid_constant__ CUtensorMap tm_v3, const __grid_constant__ CUtensorMap tm_kc8,
-             const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const FwdArgs p) {
+             const __grid_constant__ CUtensorMap tm_v3, const __grid_constant__ CUtensorMap tm_kc38,
+             const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v38, const FwdArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
@@ -206,9 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int n = __shfl_sync(0xffffffffu, my_n, (d * kDraftBlocksPerTile + lane) & 31);
                     if (lane < nb) {
                         const int row = p.S + kBlock * n;
-                        for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc8, c * 64, (int)(bh * p.L + row));
+                        tma_prefetch_3d(&tm_kc38, 0, (int)(bh * p.L + row), 0);
                         tma_prefetch_2d(&tm_kr8, 0, (int)((size_t)b * p.L + row));
-                        for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v8, c * 64, (int)(bh * p.L + row));
+                        tma_prefetch_3d(&tm_v38, 0, (int)(bh * p.L + row), 0);
                     }
                 }
             };
@@ -238,10 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
                         if (lane == 0) {
                             const int row = p.S + kBlock * n;
-                            for (int c = 0; c < 3; c++)
-                                tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[s], c * 64,
-                                            (int)(bh * p.L + row));
-                            tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
+                            tma_load_3d(kt + bb * kDraftKcBlock, &tm_kc38, &kfull[s], 0, (int)(bh * p.L + row), 0);
+                            tma_load_2d(kt + kDraftKr + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
                         }
                     }
                 }
@@ -269,9 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
                         if (lane == 0) {
                             const int row = p.S + kBlock * n;
-                            for (int c = 0; c < 4; c++)
-                                tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[s], c * 64,
-                                            (int)(bh * p.L + row));
+                            tma_load_3d(vt + bb * kDraftVBlock, &tm_v38, &vfull[s], 0, (int)(bh * p.L + row), 0);
                         }
                     }
                 }
@@ -286,12 +288,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = mbar_wait(qready, 0, abort_flag);
             auto issue_qk = [&](int t) {
                 const int s = t & 1;
-                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + k_stage_off(t % kKS)), 16, 1024));
+                const uint32_t kb = smem_u32(sm + k_stage_off(t % kKS));
                 const uint32_t dS = tmem + kColS + s * kBN;
+                if (t < n_ctx) {
+                    const SDesc kd = sdesc_split(sdesc_sw128(kb, 16, 1024));
 #pragma unroll
-                for (int k = 0; k < kDQK / 16; ++k) {
-                    const uint32_t ko = ((k >> 2) * kKChunk + (k & 3) * 32) >> 4;
-                    mma_bf16_ts(dS, tmem + kColQ + 8 * k, kd.at(ko), idS, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < kDQK / 16; ++k) {
+                        const uint32_t ko = ((k >> 2) * kKChunk + (k & 3) * 32) >> 4;
+                        mma_bf16_ts(dS, tmem + kColQ + 8 * k, kd.at(ko), idS, k > 0 ? 1u : 0u);
+                    }
+                } else {
+                    const SDesc kdc = sdesc_split(sdesc_sw128(kb, 16, kDraftKcBlock));
+                    const SDesc kdr = sdesc_split(sdesc_sw128(kb + kDraftKr, 16, 1024));
+#pragma unroll
+                    for (int k = 0; k < kDC / 16; ++k) {
+                        const uint32_t ko = ((k >> 2) * 1024 + (k & 3) * 32) >> 4;
+                        mma_bf16_ts(dS, tmem + kColQ + 8 * k, kdc.at(ko), idS, k > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int k = kDC / 16; k < kDQK / 16; ++k)
+                        mma_bf16_ts(dS, tmem + kColQ + 8 * k, kdr.at(((k & 3) * 32) >> 4), idS, 1u);
                 }
                 mma_commit(&sfull[s]);
                 mma_commit(&kempty[t % kKS]);
@@ -299,14 +315,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_pv = [&](int t) {
                 const int s = t & 1;
-                const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + v_stage_off(t % kVS)), kKChunk, 1024));
+                const uint32_t vb = smem_u32(sm + v_stage_off(t % kVS));
+                const bool ctx = t < n_ctx;
+                // context tile: 64-column slices 8 KB apart, keys 128 B apart;
+                // draft tile: slices 1 KB apart, 8-key groups 4 KB apart
+                const SDesc vd = sdesc_split(ctx ? sdesc_sw128(vb, kKChunk, 1024) : sdesc_sw128(vb, 1024, kDraftVBlock));
+                const uint32_t kstep = ctx ? 128u : 512u;  // 16 keys, in 16-byte units
                 // P of keys 16 k .. 16 k + 15: half k / 2 of the S buffer, its
                 // columns 8 (k % 2) ..
                 const uint32_t pa = tmem + kColS + s * kBN;
                 mma_bf16_ts(tmem + kColO, pa, vd.at(0), idO, t > 0 ? 1u : 0u);
-                mma_bf16_ts(tmem + kColO, pa + 8, vd.at(128), idO, 1u);
-                mma_bf16_ts(tmem + kColO, pa + 32, vd.at(256), idO, 1u);
-                mma_bf16_ts(tmem + kColO, pa + 40, vd.at(384), idO, 1u);
+                mma_bf16_ts(tmem + kColO, pa + 8, vd.at(kstep), idO, 1u);
+                mma_bf16_ts(tmem + kColO, pa + 32, vd.at(2 * kstep), idO, 1u);
+                mma_bf16_ts(tmem + kColO, pa + 40, vd.at(3 * kstep), idO, 1u);
                 mma_commit(&vempty[t % kVS]);
                 mma_commit(&pvdone[s]);
             };
@@ -606,11 +627,11 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     if (p.B == 0 || p.N == 0) return cudaSuccess;
     count_launch();
     k_fwd_pad_rows<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.R, anchors, keep, (__nv_bfloat16 *)o, lse);
-    CUtensorMap m_kc3, m_kr, m_v3, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc3, m_kr, m_v3, m_kc38, m_kr8, m_v38;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, kr_rows = (uint64_t)p.B * p.L;
     if (!make_map3_bf16(&m_kc3, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr, ws.kr_rot, kDR, kr_rows, 64) ||
-        !make_map3_bf16(&m_v3, v, kDV, kv_rows, 64) || !make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) ||
-        !make_map_bf16(&m_kr8, ws.kr_rot, kDR, kr_rows, 8) || !make_map_bf16(&m_v8, v, kDV, kv_rows, 8))
+        !make_map3_bf16(&m_v3, v, kDV, kv_rows, 64) || !make_map3_bf16(&m_kc38, kc, kDC, kv_rows, 8) ||
+        !make_map_bf16(&m_kr8, ws.kr_rot, kDR, kr_rows, 8) || !make_map3_bf16(&m_v38, v, kDV, kv_rows, 8))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -630,7 +651,7 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.err = ws.err;
     dim3 grid((p.N + kG - 1) / kG, p.n_h, p.B);
     count_launch();
-    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc3, m_kr, m_v3, m_kc8, m_kr8, m_v8, a);
+    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc3, m_kr, m_v3, m_kc38, m_kr8, m_v38, a);
     return cudaGetLastError();
 }
 
