@@ -568,6 +568,11 @@ constexpr int kKChunk = kMK * 128;       // 16 KB: 128 keys x 64 columns
 constexpr int kRChunk = kRC * 128;       // 4 KB: 32 rows x 64 columns
 constexpr int kRBuf = 4 * kRChunk;       // 16 KB: one row operand of a chunk
 constexpr int kES = 2, kLS = 3;          // stages: early-released / late-released row operand
+// Draft items are loaded block-major: block bb's 8 K^C rows (3 x 1 KB
+// swizzled slices) at bb * 3 KB, its K^R rows at 48 KB + bb * 1 KB, its V rows
+// (4 x 1 KB) at bb * 4 KB: as MMA A operands, K^C / V with 8-key groups 3 KB /
+// 4 KB apart and 64-column slices 1 KB apart.
+constexpr int kDraftKcBlock = 3 * 1024, kDraftVBlock = 4 * 1024;
 constexpr int kStageBytes = 8 * 32 * 64; // epilogue staging: 8 warps x 32 keys x 32 columns bf16
 constexpr int oK = 0, oV = oK + 4 * kKChunk, oE = oV + 4 * kKChunk, oL = oE + kES * kRBuf, oStage = oL + kLS * kRBuf,
               oMeta = oStage + kStageBytes, oBar = oMeta + kLS * kRC * 12;
@@ -732,8 +737,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             if (q >= kES && !warp_all(mbar_wait(&efree[es], ((q / kES) - 1) & 1, abort_flag))) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&efull[es], kRBuf);
-                for (int cc = 0; cc < 4; cc++)
-                    tma_load_2d(sm + oE + es * kRBuf + cc * kRChunk, tm_e, &efull[es], cc * 64, (int)(bh * p.R + r0));
+                tma_load_3d(sm + oE + es * kRBuf, tm_e, &efull[es], 0, (int)(bh * p.R + r0), 0);
                 counters[4] = q + 1;
             }
         }
@@ -749,12 +753,9 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 if (is_ctx) {
                     if (lane == 0) {
                         mbar_arrive_expect_tx(kvfull, (role_k ? 8 : 4) * kKChunk);
-                        for (int cc = 0; cc < 3; cc++)
-                            tma_load_2d(sm + oK + cc * kKChunk, &tm_kc, kvfull, cc * 64, (int)(bh * p.L + t0));
+                        tma_load_3d(sm + oK, &tm_kc, kvfull, 0, (int)(bh * p.L + t0), 0);
                         tma_load_2d(sm + oK + 3 * kKChunk, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
-                        if (role_k)
-                            for (int cc = 0; cc < 4; cc++)
-                                tma_load_2d(sm + oV + cc * kKChunk, &tm_v, kvfull, cc * 64, (int)(bh * p.L + t0));
+                        if (role_k) tma_load_3d(sm + oV, &tm_v, kvfull, 0, (int)(bh * p.L + t0), 0);
                     }
                 } else {
                     if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * (role_k ? 2 : 1) * kDQK * 2);
@@ -762,14 +763,10 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                         const int nb = __shfl_sync(0xffffffffu, my_n, bb);
                         if (lane == 0) {
                             const int row = p.S + kBlock * nb;
-                            for (int cc = 0; cc < 3; cc++)
-                                tma_load_2d(sm + oK + cc * kKChunk + bb * 1024, &tm_kc8, kvfull, cc * 64,
-                                            (int)(bh * p.L + row));
+                            tma_load_3d(sm + oK + bb * kDraftKcBlock, &tm_kc8, kvfull, 0, (int)(bh * p.L + row), 0);
                             tma_load_2d(sm + oK + 3 * kKChunk + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
                             if (role_k)
-                                for (int cc = 0; cc < 4; cc++)
-                                    tma_load_2d(sm + oV + cc * kKChunk + bb * 1024, &tm_v8, kvfull, cc * 64,
-                                                (int)(bh * p.L + row));
+                                tma_load_3d(sm + oV + bb * kDraftVBlock, &tm_v8, kvfull, 0, (int)(bh * p.L + row), 0);
                         }
                     }
                 }
@@ -790,8 +787,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(&lfull[ls], kRBuf);
-                for (int cc = 0; cc < 4; cc++)
-                    tma_load_2d(sm + oL + ls * kRBuf + cc * kRChunk, tm_l, &lfull[ls], cc * 64, (int)(bh * p.R + r0));
+                tma_load_3d(sm + oL + ls * kRBuf, tm_l, &lfull[ls], 0, (int)(bh * p.R + r0), 0);
                 counters[1] = q + 1;
             }
         }
@@ -800,8 +796,13 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kMK, kRC, 0);   // S^T, dP^T: B = Q / dO chunk, K-major
             const uint32_t idA = idesc_bf16(kMK, 256, 1);   // acc: B = dO / Q chunk, MN-major
-            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + oK), 16, 1024));
-            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + oV), 16, 1024));
+            // A operands: K^C / V slices kcStep / vStep bytes apart (context
+            // tile: 16 KB slices of 128 keys; draft item: block-major); the
+            // K^R slice at 48 KB in both
+            const uint32_t kcStep = is_ctx ? kKChunk : 1024, vStep = is_ctx ? kKChunk : 1024;
+            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + oK), 16, is_ctx ? 1024 : kDraftKcBlock));
+            const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + 3 * kKChunk), 16, 1024));
+            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + oV), 16, is_ctx ? 1024 : kDraftVBlock));
             bool ok = true;
             auto issue_s = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
@@ -813,17 +814,21 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                     // S^T = K Q^T and dP^T = V dO^T interleaved: two independent chains
 #pragma unroll
                     for (int kk = 0; kk < kDQK / 16; ++kk) {
-                        const uint32_t ko = ((kk >> 2) * kKChunk + (kk & 3) * 32) >> 4;
+                        const int cc = kk >> 2;
+                        const uint32_t sub = (kk & 3) * 2;  // 32 bytes, in 16-byte units
+                        const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
                         const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(dS, kad.at(ko), ld_.at(ro), idS, kk > 0 ? 1u : 0u);
-                        mma_bf16_ss(dP, vad.at(ko), ed.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dS, ka, ld_.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dP, vad.at(((cc * vStep) >> 4) + sub), ed.at(ro), idS, kk > 0 ? 1u : 0u);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < kDQK / 16; ++kk) {
-                        const uint32_t ko = ((kk >> 2) * kKChunk + (kk & 3) * 32) >> 4;
+                        const int cc = kk >> 2;
+                        const uint32_t sub = (kk & 3) * 2;
+                        const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
                         const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(dS, kad.at(ko), ed.at(ro), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(dS, ka, ed.at(ro), idS, kk > 0 ? 1u : 0u);
                     }
                 }
                 mma_commit(&sfull[s]);
@@ -1108,24 +1113,26 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc64, m_kr64, m_v64, m_qs128, m_dos128, m_kc128, m_kr128, m_v128, m_qs32, m_dos32, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc64, m_kr64, m_v64, m_qs128, m_dos128, m_kr128, m_qs3_32, m_dos3_32, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc3_128, m_v3_128, m_kc3_8, m_v3_8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
     if (p.N > 0 && q_rows > 0) {
         if (!make_map_bf16(&m_kc64, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
             !make_map_bf16(&m_v64, v, kDV, kv_rows, 64) || !make_map_bf16(&m_qs128, qs, kDQK, q_rows, 128) ||
-            !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map_bf16(&m_qs32, qs, kDQK, q_rows, 32) ||
-            !make_map_bf16(&m_dos32, dos, kDV, q_rows, 32))
+            !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map3_bf16(&m_qs3_32, qs, kDQK, q_rows, 32) ||
+            !make_map3_bf16(&m_dos3_32, dos, kDV, q_rows, 32))
             return cudaErrorInvalidValue;
     }
     if (!make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) || !make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
-        !make_map_bf16(&m_v8, v, kDV, kv_rows, 8) || !make_map_bf16(&m_kc128, kc, kDC, kv_rows, 128) ||
+        !make_map_bf16(&m_v8, v, kDV, kv_rows, 8) || !make_map3_bf16(&m_kc3_128, kc, kDC, kv_rows, 128) ||
         !make_map_bf16(&m_kr128, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 128) ||
-        !make_map_bf16(&m_v128, v, kDV, kv_rows, 128))
+        !make_map3_bf16(&m_v3_128, v, kDV, kv_rows, 128) || !make_map3_bf16(&m_kc3_8, kc, kDC, kv_rows, 8) ||
+        !make_map3_bf16(&m_v3_8, v, kDV, kv_rows, 8))
         return cudaErrorInvalidValue;
     if (p.N == 0 || q_rows == 0) {  // maps over Q rows are never read: any valid map will do
-        m_qs32 = m_kc128;
-        m_dos32 = m_kc128;
+        m_qs3_32 = m_kc3_128;
+        m_dos3_32 = m_kc3_128;
     }
     BwdArgs a;
     a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
@@ -1161,8 +1168,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc128, m_kr128, m_v128, m_qs32, m_dos32, m_kc8, m_kr8,
-                                                        m_v8, a);
+    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc3_128, m_kr128, m_v3_128, m_qs3_32, m_dos3_32, m_kc3_8,
+                                                        m_kr8, m_v3_8, a);
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
     k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
