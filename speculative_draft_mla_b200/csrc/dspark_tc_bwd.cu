@@ -148,6 +148,10 @@ constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
 constexpr int kKChunk = kBN * 128;     // 8 KB: 64 keys x 64 columns
 constexpr int kTile = 4 * kKChunk;     // 32 KB
 constexpr int kKS = 2, kVS = 2;        // K and V stages
+// Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
+// slices) at bb * 3 KB, its K^R rows at 24 KB + bb * 1 KB, its V rows
+// (4 x 1 KB) at bb * 4 KB.
+constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
 // dS tile [128 rows][64 keys] bf16 without swizzle: 16 x 8 core matrices of
 // 8 rows x 16 bytes, K-adjacent ones 128 B apart, 8-row groups 1024 B apart
 constexpr int kDS = kM * kBN * 2;      // 16 KB
@@ -251,10 +255,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         // ------------------------------------------------------- producer
         if (lane == 0) {
             mbar_arrive_expect_tx(qfull, 8 * kQChunk);
-            for (int c = 0; c < 4; c++) {
-                tma_load_2d(sm + oQ + c * kQChunk, &tm_qs, qfull, c * 64, (int)srow0);
-                tma_load_2d(sm + oDOStage + c * kQChunk, &tm_dos, qfull, c * 64, (int)srow0);
-            }
+            tma_load_3d(sm + oQ, &tm_qs, qfull, 0, (int)srow0, 0);
+            tma_load_3d(sm + oDOStage, &tm_dos, qfull, 0, (int)srow0, 0);
             counters[4] = 1;
         }
         // lane l holds the block index of group block l (l < gcnt)
@@ -267,9 +269,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             if (lane == 0) {
                 for (; pf_next <= t + 4 && pf_next < n_ctx; ++pf_next) {
                     const int pos = ctx_lo + pf_next * kBN;
-                    for (int c = 0; c < 3; c++) tma_prefetch_2d(&tm_kc, c * 64, (int)(bh * p.L + pos));
+                    tma_prefetch_3d(&tm_kc, 0, (int)(bh * p.L + pos), 0);
                     tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
-                    for (int c = 0; c < 4; c++) tma_prefetch_2d(&tm_v, c * 64, (int)(bh * p.L + pos));
+                    tma_prefetch_3d(&tm_v, 0, (int)(bh * p.L + pos), 0);
                 }
             }
             if (t >= kKS && !warp_all(mbar_wait(&kempty[ks], ((t / kKS) - 1) & 1, abort_flag))) break;
@@ -277,8 +279,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 const int pos0 = ctx_lo + t * kBN;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&kfull[ks], kTile);
-                    for (int c = 0; c < 3; c++)
-                        tma_load_2d(kt + c * kKChunk, &tm_kc, &kfull[ks], c * 64, (int)(bh * p.L + pos0));
+                    tma_load_3d(kt, &tm_kc, &kfull[ks], 0, (int)(bh * p.L + pos0), 0);
                     tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[ks], 0, (int)((size_t)b * p.L + pos0));
                 }
             } else {
@@ -290,9 +291,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
                     if (lane == 0) {
                         const int row = p.S + kBlock * n;
-                        for (int c = 0; c < 3; c++)
-                            tma_load_2d(kt + c * kKChunk + bb * 1024, &tm_kc8, &kfull[ks], c * 64, (int)(bh * p.L + row));
-                        tma_load_2d(kt + 3 * kKChunk + bb * 1024, &tm_kr8, &kfull[ks], 0, (int)((size_t)b * p.L + row));
+                        tma_load_3d(kt + bb * kDraftKcBlock, &tm_kc8, &kfull[ks], 0, (int)(bh * p.L + row), 0);
+                        tma_load_2d(kt + kDraftKr + bb * 1024, &tm_kr8, &kfull[ks], 0, (int)((size_t)b * p.L + row));
                     }
                 }
             }
@@ -304,8 +304,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 const int pos0 = ctx_lo + t * kBN;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&vfull[vs], kTile);
-                    for (int c = 0; c < 4; c++)
-                        tma_load_2d(vt + c * kKChunk, &tm_v, &vfull[vs], c * 64, (int)(bh * p.L + pos0));
+                    tma_load_3d(vt, &tm_v, &vfull[vs], 0, (int)(bh * p.L + pos0), 0);
                 }
             } else {
                 const int d = t - n_ctx;
@@ -315,8 +314,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
                     if (lane == 0) {
                         const int row = p.S + kBlock * n;
-                        for (int c = 0; c < 4; c++)
-                            tma_load_2d(vt + c * kKChunk + bb * 1024, &tm_v8, &vfull[vs], c * 64, (int)(bh * p.L + row));
+                        tma_load_3d(vt + bb * kDraftVBlock, &tm_v8, &vfull[vs], 0, (int)(bh * p.L + row), 0);
                     }
                 }
             }
@@ -330,17 +328,28 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + oQ), 16, 1024));
             bool ok = mbar_wait(qfull, 0, abort_flag);
             if (ok) ok = mbar_wait(dotmem, 0, abort_flag);
+            const uint32_t idQc = idesc_bf16(kM, kDC, 1);   // draft tiles: dQ^C and dQ^R separately
+            const uint32_t idQr = idesc_bf16(kM, kDR, 1);
             auto issue_sdp = [&](int t) {
-                const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + (t % kKS) * kTile), 16, 1024));
-                const SDesc vd = sdesc_split(sdesc_sw128(smem_u32(sm + oV + (t % kVS) * kTile), 16, 1024));
+                const bool ctx = t < n_ctx;
+                const uint32_t kb = smem_u32(sm + oK + (t % kKS) * kTile), vb = smem_u32(sm + oV + (t % kVS) * kTile);
+                // B operands: context tile slices 8 KB apart with keys 128 B
+                // apart; draft tile block-major (K^C / V 8-key groups 3 KB / 4 KB
+                // apart, slices 1 KB apart; K^R at 24 KB)
+                const uint32_t step = ctx ? kKChunk : 1024;
+                const SDesc kd = sdesc_split(sdesc_sw128(kb, 16, ctx ? 1024 : kDraftKcBlock));
+                const SDesc krd = sdesc_split(sdesc_sw128(kb + kDraftKr, 16, 1024));
+                const SDesc vd = sdesc_split(sdesc_sw128(vb, 16, ctx ? 1024 : kDraftVBlock));
                 const uint32_t dS = tmem + kColS, dP = tmem + kColP;
                 // S and dP interleaved: two independent accumulation chains
 #pragma unroll
                 for (int k = 0; k < kDQK / 16; ++k) {
+                    const int c = k >> 2;
+                    const uint32_t sub = (k & 3) * 2;
                     const uint32_t qo = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
-                    const uint32_t ko = ((k >> 2) * kKChunk + (k & 3) * 32) >> 4;
-                    mma_bf16_ss(dS, qd.at(qo), kd.at(ko), idS, k > 0 ? 1u : 0u);
-                    mma_bf16_ts(dP, tmem + kColDO + 8 * k, vd.at(ko), idS, k > 0 ? 1u : 0u);
+                    const uint64_t kbd = c < 3 ? kd.at(((c * step) >> 4) + sub) : krd.at(sub);
+                    mma_bf16_ss(dS, qd.at(qo), kbd, idS, k > 0 ? 1u : 0u);
+                    mma_bf16_ts(dP, tmem + kColDO + 8 * k, vd.at(((c * step) >> 4) + sub), idS, k > 0 ? 1u : 0u);
                 }
                 mma_commit(sfull);
                 mma_commit(&vempty[t % kVS]);
@@ -369,10 +378,22 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     const int s = nq & 1;
                     tc_fence_after();
                     const SDesc dd = sdesc_split(sdesc_noswz(smem_u32(sm + (s ? oS1 : oS0)), 128, 1024));
-                    const SDesc kd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + (nq % kKS) * kTile), kKChunk, 1024));
-                    mma_bf16_ss(tmem + kColDQ, dd.at(0), kd.at(0), idQ, nq > 0 ? 1u : 0u);
+                    const uint32_t kb = smem_u32(sm + oK + (nq % kKS) * kTile);
+                    if (nq < n_ctx) {  // B: all 256 columns, slices 8 KB apart, 16 keys = 2 KB
+                        const SDesc kd = sdesc_split(sdesc_sw128(kb, kKChunk, 1024));
+                        mma_bf16_ss(tmem + kColDQ, dd.at(0), kd.at(0), idQ, nq > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int k = 1; k < kBN / 16; ++k) mma_bf16_ss(tmem + kColDQ, dd.at(16 * k), kd.at(128 * k), idQ, 1u);
+                        for (int k = 1; k < kBN / 16; ++k) mma_bf16_ss(tmem + kColDQ, dd.at(16 * k), kd.at(128 * k), idQ, 1u);
+                    } else {  // block-major: K^C (slices 1 KB apart, 2 blocks = 6 KB) and K^R (2 KB)
+                        const SDesc kdc = sdesc_split(sdesc_sw128(kb, 1024, kDraftKcBlock));
+                        const SDesc kdr = sdesc_split(sdesc_sw128(kb + kDraftKr, 1024, 1024));
+#pragma unroll
+                        for (int k = 0; k < kBN / 16; ++k) {
+                            const uint32_t acc = (nq > 0 || k > 0) ? 1u : 0u;
+                            mma_bf16_ss(tmem + kColDQ, dd.at(16 * k), kdc.at(((2 * kDraftKcBlock) >> 4) * k), idQc, acc);
+                            mma_bf16_ss(tmem + kColDQ + kDC, dd.at(16 * k), kdr.at(128 * k), idQr, acc);
+                        }
+                    }
                     mma_commit(&kempty[nq % kKS]);
                     mma_commit(&dqdone[s]);
                     ++nq;
@@ -1113,19 +1134,20 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc64, m_kr64, m_v64, m_qs128, m_dos128, m_kr128, m_qs3_32, m_dos3_32, m_kc8, m_kr8, m_v8;
+    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_kr128, m_qs3_32, m_dos3_32, m_kr8;
     CUtensorMap m_kc3_128, m_v3_128, m_kc3_8, m_v3_8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
     if (p.N > 0 && q_rows > 0) {
-        if (!make_map_bf16(&m_kc64, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
-            !make_map_bf16(&m_v64, v, kDV, kv_rows, 64) || !make_map_bf16(&m_qs128, qs, kDQK, q_rows, 128) ||
-            !make_map_bf16(&m_dos128, dos, kDV, q_rows, 128) || !make_map3_bf16(&m_qs3_32, qs, kDQK, q_rows, 32) ||
+        if (!make_map3_bf16(&m_kc3_64, kc, kDC, kv_rows, 64) ||
+            !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
+            !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64) || !make_map3_bf16(&m_qs3_128, qs, kDQK, q_rows, 128) ||
+            !make_map3_bf16(&m_dos3_128, dos, kDV, q_rows, 128) || !make_map3_bf16(&m_qs3_32, qs, kDQK, q_rows, 32) ||
             !make_map3_bf16(&m_dos3_32, dos, kDV, q_rows, 32))
             return cudaErrorInvalidValue;
     }
-    if (!make_map_bf16(&m_kc8, kc, kDC, kv_rows, 8) || !make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
-        !make_map_bf16(&m_v8, v, kDV, kv_rows, 8) || !make_map3_bf16(&m_kc3_128, kc, kDC, kv_rows, 128) ||
+    if (!make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
+        !make_map3_bf16(&m_kc3_128, kc, kDC, kv_rows, 128) ||
         !make_map_bf16(&m_kr128, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 128) ||
         !make_map3_bf16(&m_v3_128, v, kDV, kv_rows, 128) || !make_map3_bf16(&m_kc3_8, kc, kDC, kv_rows, 8) ||
         !make_map3_bf16(&m_v3_8, v, kDV, kv_rows, 8))
@@ -1162,7 +1184,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         if (e != cudaSuccess) return e;
         count_launch();
         k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
-            m_kc64, m_kr64, m_v64, m_qs128, m_dos128, m_kc8, m_kr8, m_v8, a);
+            m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_kc3_8, m_kr8, m_v3_8, a);
     }
     const dim3 kv_grid(2 * (a.n_ctx_items + (p.N + kGD - 1) / kGD), HG, p.B);
     e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
