@@ -576,45 +576,55 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
 }
 
 // ============================================================== dK / dV
-// Key tile = 128 keys (MMA M). Rows stream through in chunks of 32 (MMA N of
-// S^T). Each chunk's two row operands have different lifetimes: the one read
-// only by the S^T-stage MMAs (dO for role K, Q for role V) is released as
-// soon as they complete and gets two stages; the one also read by the
-// accumulation (Q for role K, dO for role V) gets three. P^T / dS^T go to
-// tensor memory, where the accumulation MMA reads them as its A operand.
+// Key tile = 128 keys (MMA M); the rows that see it stream through in chunks
+// (MMA N of S^T). Each chunk's two row operands have different lifetimes: the
+// one read only by the S^T-stage MMAs (dO for role K, Q for role V) is
+// released as soon as they complete; the one also read by the accumulation
+// (Q for role K, dO for role V) is held until it. P^T / dS^T go to tensor
+// memory, where the accumulation MMA reads them as its A operand.
+// Role K (dK = dS^T Q) needs K and V tiles and S^T, dP^T, dS^T: 32-row chunks,
+// 2 + 3 stages. Role V (dV = P^T dO) needs only K and S^T, P^T written over
+// its own S^T columns: 64-row chunks (half the chunks, the per-chunk latency
+// being what bounds a CTA), 2 + 2 stages.
 namespace kv {
 constexpr int kMK = 128;                 // keys per tile (MMA M)
-constexpr int kRC = 32;                  // rows per chunk (MMA N of S^T)
 constexpr int kKChunk = kMK * 128;       // 16 KB: 128 keys x 64 columns
-constexpr int kRChunk = kRC * 128;       // 4 KB: 32 rows x 64 columns
-constexpr int kRBuf = 4 * kRChunk;       // 16 KB: one row operand of a chunk
-constexpr int kES = 2, kLS = 3;          // stages: early-released / late-released row operand
 // Draft items are loaded block-major: block bb's 8 K^C rows (3 x 1 KB
 // swizzled slices) at bb * 3 KB, its K^R rows at 48 KB + bb * 1 KB, its V rows
 // (4 x 1 KB) at bb * 4 KB: as MMA A operands, K^C / V with 8-key groups 3 KB /
 // 4 KB apart and 64-column slices 1 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftVBlock = 4 * 1024;
 constexpr int kStageBytes = 8 * 32 * 64; // epilogue staging: 8 warps x 32 keys x 32 columns bf16
-constexpr int oK = 0, oV = oK + 4 * kKChunk, oE = oV + 4 * kKChunk, oL = oE + kES * kRBuf, oStage = oL + kLS * kRBuf,
-              oMeta = oStage + kStageBytes, oBar = oMeta + kLS * kRC * 12;
-constexpr int kSmem = oBar + 256 + 1024;
-static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+constexpr int oK = 0, oV = oK + 4 * kKChunk;
+template <bool RK> struct KvCfg {
+    static constexpr int kRC = RK ? 32 : 64;  // rows per chunk
+    static constexpr int kES = 2, kLS = RK ? 3 : 2;
+    static constexpr int kRBuf = 4 * kRC * 128;
+    static constexpr int oE = RK ? oV + 4 * kKChunk : oV;  // role V has no V tile
+    static constexpr int oL = oE + kES * kRBuf, oStage = oL + kLS * kRBuf;
+    static constexpr int oMeta = oStage + kStageBytes, oBar = oMeta + kLS * kRC * 12;
+    static constexpr int kSmem = oBar + 256 + 1024;
+    static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+};
+constexpr int kSmem = KvCfg<true>::kSmem > KvCfg<false>::kSmem ? KvCfg<true>::kSmem : KvCfg<false>::kSmem;
 constexpr int kKeyWarps = 8;             // two per TMEM sub-partition, each half of a chunk's rows
 constexpr int kWarpL = kKeyWarps, kWarpMma = kKeyWarps + 1, kWarpE = kKeyWarps + 2;
 constexpr int kThreads = (kKeyWarps + 3) * 32;
-// TMEM: accumulator 0..255, S^T 256 / 288, dP^T 320 / 352, P^T or dS^T (bf16 pairs) 384 / 400
-constexpr uint32_t kColAcc = 0, kColS = 256, kColP = 320, kColPT = 384;
+constexpr uint32_t kColAcc = 0;
 }  // namespace kv
 
 // One CTA per (key tile, role, head group, batch). Role 0 accumulates dV =
 // P^T dO, role 1 dK = dS^T Q; the two roles of a tile are adjacent in launch
 // order so the second reads K and the row chunks from L2.
-__global__ void __launch_bounds__(kv::kThreads, 1)
-    k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-                const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
-                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
+template <bool RK>
+__device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensorMap &tm_kr, const CUtensorMap &tm_v,
+                                        const CUtensorMap &tm_qs, const CUtensorMap &tm_dos, const CUtensorMap &tm_kc8,
+                                        const CUtensorMap &tm_kr8, const CUtensorMap &tm_v8, const BwdArgs &p) {
     using namespace kv;
+    using C = KvCfg<RK>;
+    constexpr int kRC = C::kRC, kRChunk = kRC * 128, kRBuf = 4 * kRChunk, kES = C::kES, kLS = C::kLS;
+    constexpr int oE = C::oE, oL = C::oL, oStage = C::oStage, oMeta = C::oMeta, oBar = C::oBar;
+    constexpr uint32_t kColS = 256, kColP = 320, kColPT = 384;  // dP^T and a separate P^T buffer: role K only
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
@@ -627,7 +637,8 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     int *counters = reinterpret_cast<int *>(drain + 3);
     int *band = counters + 6;  // first sorted row, row count
 
-    const int item = blockIdx.x >> 1, role_k = blockIdx.x & 1;
+    const int item = blockIdx.x >> 1;
+    constexpr bool role_k = RK;
     const int hg = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cnt = p.cnt[b];
@@ -800,10 +811,14 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             {
                 int *mA = reinterpret_cast<int *>(sm + oMeta + ls * kRC * 12);
                 float2 *mLD = reinterpret_cast<float2 *>(mA + kRC);
-                const int rowi = r0 + lane;
-                const bool in = rowi < row0 + nrows;
-                mA[lane] = in ? sa[rowi / kBlock] : 0x7fffffff;
-                mLD[lane] = in ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi]) : make_float2(0.f, 0.f);
+#pragma unroll
+                for (int jj = 0; jj < kRC; jj += 32) {
+                    const int rowi = r0 + jj + lane;
+                    const bool in = rowi < row0 + nrows;
+                    mA[jj + lane] = in ? sa[rowi / kBlock] : 0x7fffffff;
+                    mLD[jj + lane] =
+                        in ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi]) : make_float2(0.f, 0.f);
+                }
             }
             __syncwarp();
             if (lane == 0) {
@@ -860,9 +875,17 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
                 const SDesc bd = sdesc_split(sdesc_sw128(smem_u32(sm + oL + (q % kLS) * kRBuf), kRChunk, 1024));
-                const uint32_t pa = tmem + kColPT + s * (kRC / 2);
-                mma_bf16_ts(tmem + kColAcc, pa, bd.at(0), idA, c > 0 ? 1u : 0u);
-                mma_bf16_ts(tmem + kColAcc, pa + 8, bd.at(128), idA, 1u);
+                if constexpr (RK) {  // dS^T in its own buffer: rows 0..15, 16..31
+                    const uint32_t pa = tmem + kColPT + s * (kRC / 2);
+                    mma_bf16_ts(tmem + kColAcc, pa, bd.at(0), idA, c > 0 ? 1u : 0u);
+                    mma_bf16_ts(tmem + kColAcc, pa + 8, bd.at(128), idA, 1u);
+                } else {  // P^T over the first 16 columns of each 32-row half of the S^T buffer
+                    const uint32_t pa = tmem + kColS + s * kRC;
+                    mma_bf16_ts(tmem + kColAcc, pa, bd.at(0), idA, c > 0 ? 1u : 0u);
+                    mma_bf16_ts(tmem + kColAcc, pa + 8, bd.at(128), idA, 1u);
+                    mma_bf16_ts(tmem + kColAcc, pa + 32, bd.at(256), idA, 1u);
+                    mma_bf16_ts(tmem + kColAcc, pa + 40, bd.at(384), idA, 1u);
+                }
                 mma_commit(&lfree[q % kLS]);
                 mma_commit(&ptfree[s]);
                 if (c == nchunks - 1) mma_commit(accdone);
@@ -951,30 +974,30 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             if (ok) ok = warp_all(mbar_wait(&sfull[s], (q >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float sv[16], pv[16];
-            {
-                float a[32];
+            constexpr int RH = kRC / 2;  // rows of the chunk per warp
+            float sv[RH], pv[RH];
+            if constexpr (RK) {
+                float a[32], bq[32];
                 tmem_ld32(trow + kColS + s * kRC, a);  // all 32 rows; this warp uses its half
-                if (role_k) {
-                    float bq[32];
-                    tmem_ld32(trow + kColP + s * kRC, bq);
-                    tmem_wait_ld();
+                tmem_ld32(trow + kColP + s * kRC, bq);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; i++) pv[i] = half ? bq[16 + i] : bq[i];
-                } else {
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; i++) pv[i] = 0.f;
+                for (int i = 0; i < RH; i++) {
+                    sv[i] = half ? a[RH + i] : a[i];
+                    pv[i] = half ? bq[RH + i] : bq[i];
                 }
+            } else {
+                tmem_ld32(trow + kColS + s * kRC + 32 * half, *reinterpret_cast<float(*)[32]>(&sv[0]));
+                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; i++) sv[i] = half ? a[16 + i] : a[i];
+                for (int i = 0; i < RH; i++) pv[i] = 0.f;
             }
             // rows of the chunk that see this key: [jlo, jhi)
             const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + (q % kLS) * kRC * 12 + kRC * 4);
             const int jlo = rlo - c * kRC, jhi = rhi - c * kRC;
-            uint32_t w[8];
+            uint32_t w[RH / 2];
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
+            for (int i = 0; i < RH; i += 2) {
                 float e2[2];
 #pragma unroll
                 for (int d = 0; d < 2; d++) {
@@ -985,12 +1008,18 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 }
                 w[i / 2] = pack_bf16x2(e2[0], e2[1]);
             }
-            // P^T / dS^T buffer s is free once the accumulation of chunk q - 2 completed
-            if (q >= 2) {
-                ok = warp_all(mbar_wait(&ptfree[s], ((q >> 1) - 1) & 1, abort_flag));
-                if (!ok) break;
+            if constexpr (RK) {
+                // the dS^T buffer s is free once the accumulation of chunk q - 2 completed
+                if (q >= 2) {
+                    ok = warp_all(mbar_wait(&ptfree[s], ((q >> 1) - 1) & 1, abort_flag));
+                    if (!ok) break;
+                }
+                tmem_st8u(trow + kColPT + s * (kRC / 2) + half * 8, *reinterpret_cast<uint32_t(*)[8]>(&w[0]));
+            } else {
+                // over this half's S^T columns (already read; the S^T buffer
+                // is rewritten only after the accumulation that reads P^T)
+                tmem_st16u(trow + kColS + s * kRC + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
             }
-            tmem_st8u(trow + kColPT + s * (kRC / 2) + half * 8, w);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -1071,6 +1100,19 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
 }
 
+__global__ void __launch_bounds__(kv::kThreads, 1)
+    k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs32,
+                const __grid_constant__ CUtensorMap tm_dos32, const __grid_constant__ CUtensorMap tm_qs64,
+                const __grid_constant__ CUtensorMap tm_dos64, const __grid_constant__ CUtensorMap tm_kc8,
+                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
+    if (blockIdx.x & 1)
+        kv_role<true>(tm_kc, tm_kr, tm_v, tm_qs32, tm_dos32, tm_kc8, tm_kr8, tm_v8, p);
+    else
+        kv_role<false>(tm_kc, tm_kr, tm_v, tm_qs64, tm_dos64, tm_kc8, tm_kr8, tm_v8, p);
+}
+
+// ------------------------------------------------------------ dK^R reduce
 // ------------------------------------------------------------ dK^R reduce
 // One warp per (b, key): sum the head-group partials (rotated frame), rotate
 // back by the key's position, write dkr. Draft keys of padding blocks: 0.
@@ -1114,9 +1156,11 @@ bool bwd_tc_supported(const Prob &p) {
 
 int bwd_head_groups(const Prob &p) {
     const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kGD - 1) / kGD) * p.B;
-    // two CTA roles per key tile; aim for about four waves on 148 SMs
+    // two CTA roles per key tile; aim for about eight waves on 148 SMs (shorter
+    // CTAs, smaller tail; measured better than four or sixteen at the
+    // 8192-context workload)
     int hg = 1;
-    while (hg < p.n_h && 2 * items * hg < 4 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
+    while (hg < p.n_h && 2 * items * hg < 8 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
     return hg;
 }
 
@@ -1135,7 +1179,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
     CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_kr128, m_qs3_32, m_dos3_32, m_kr8;
-    CUtensorMap m_kc3_128, m_v3_128, m_kc3_8, m_v3_8;
+    CUtensorMap m_kc3_128, m_v3_128, m_kc3_8, m_v3_8, m_qs3_64, m_dos3_64;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
     if (p.N > 0 && q_rows > 0) {
@@ -1143,7 +1187,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
             !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
             !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64) || !make_map3_bf16(&m_qs3_128, qs, kDQK, q_rows, 128) ||
             !make_map3_bf16(&m_dos3_128, dos, kDV, q_rows, 128) || !make_map3_bf16(&m_qs3_32, qs, kDQK, q_rows, 32) ||
-            !make_map3_bf16(&m_dos3_32, dos, kDV, q_rows, 32))
+            !make_map3_bf16(&m_dos3_32, dos, kDV, q_rows, 32) || !make_map3_bf16(&m_qs3_64, qs, kDQK, q_rows, 64) ||
+            !make_map3_bf16(&m_dos3_64, dos, kDV, q_rows, 64))
             return cudaErrorInvalidValue;
     }
     if (!make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
@@ -1155,6 +1200,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     if (p.N == 0 || q_rows == 0) {  // maps over Q rows are never read: any valid map will do
         m_qs3_32 = m_kc3_128;
         m_dos3_32 = m_kc3_128;
+        m_qs3_64 = m_kc3_128;
+        m_dos3_64 = m_kc3_128;
     }
     BwdArgs a;
     a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
@@ -1190,8 +1237,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc3_128, m_kr128, m_v3_128, m_qs3_32, m_dos3_32, m_kc3_8,
-                                                        m_kr8, m_v3_8, a);
+    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc3_128, m_kr128, m_v3_128, m_qs3_32, m_dos3_32,
+                                                        m_qs3_64, m_dos3_64, m_kc3_8, m_kr8, m_v3_8, a);
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
     k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
