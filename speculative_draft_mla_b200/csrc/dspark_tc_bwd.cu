@@ -138,25 +138,23 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
 // and N = 64, so the wider tile halves the MMA count per key.
 // Q stays in shared memory (A operand of S = Q K^T); dO is moved into tensor
 // memory once at the start (A operand of dP = dO V^T read from TMEM). TMEM:
-// dQ 256 columns, S 64, dP 64, dO 128 - S and dP are single-buffered: the
-// row warps copy them to registers and release them before computing dS, so
-// the next tile's S and dP run while dS is formed. The 64 KB where dO first
-// lands then holds the two V stages.
+// dQ 256 columns, S 64, dP 64, dO 128. The row warps write dS (bf16) over the
+// S columns they have read, where dQ += dS K reads it as its A operand; the
+// next tile's S and dP are issued after that MMA. Shared memory then holds
+// only Q and the K / V stages: a K tile is held from its load until the dQ of
+// its tile, so it gets three stages, V two. The 64 KB where dO first lands
+// then holds the two V stages.
 namespace dq {
 constexpr int kM = 128, kBN = 64;
 constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
 constexpr int kKChunk = kBN * 128;     // 8 KB: 64 keys x 64 columns
 constexpr int kTile = 4 * kKChunk;     // 32 KB
-constexpr int kKS = 2, kVS = 2;        // K and V stages
+constexpr int kKS = 3, kVS = 2;        // K and V stages
 // Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
 // slices) at bb * 3 KB, its K^R rows at 24 KB + bb * 1 KB, its V rows
 // (4 x 1 KB) at bb * 4 KB.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
-// dS tile [128 rows][64 keys] bf16 without swizzle: 16 x 8 core matrices of
-// 8 rows x 16 bytes, K-adjacent ones 128 B apart, 8-row groups 1024 B apart
-constexpr int kDS = kM * kBN * 2;      // 16 KB
-constexpr int oQ = 0, oK = oQ + 4 * kQChunk, oV = oK + kKS * kTile, oS0 = oV + kVS * kTile, oS1 = oS0 + kDS,
-              oBar = oS1 + kDS;
+constexpr int oQ = 0, oK = oQ + 4 * kQChunk, oV = oK + kKS * kTile, oBar = oV + kVS * kTile;
 constexpr int oDOStage = oV;           // dO lands here first
 static_assert(kVS * kTile >= 4 * kQChunk, "dO staging area too small");
 constexpr int kSmem = oBar + 512 + 1024;
@@ -190,8 +188,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint64_t *kfull = bars + 0, *kempty = bars + kKS, *vfull = bars + 2 * kKS, *vempty = bars + 2 * kKS + kVS;
-    uint64_t *sfull = bars + 2 * (kKS + kVS), *sfree = sfull + 1, *dsready = sfull + 2, *dqdone = sfull + 4,
-             *qfull = sfull + 6, *drain = sfull + 7, *dotmem = sfull + 8;
+    uint64_t *sfull = bars + 2 * (kKS + kVS), *dsready = sfull + 2, *dqdone = sfull + 4, *qfull = sfull + 6,
+             *drain = sfull + 7, *dotmem = sfull + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + 9);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 10);
     int *counters = reinterpret_cast<int *>(sfull + 11);  // K issued, V issued, K consumed, V consumed, q issued
@@ -229,11 +227,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             mbar_init(&vempty[s], 1);
         }
         mbar_init(sfull, 1);
-        mbar_init(sfree, 4);
-        for (int s = 0; s < 2; s++) {
-            mbar_init(&dsready[s], 4);
-            mbar_init(&dqdone[s], 1);
-        }
+        mbar_init(dsready, 4);
+        for (int s = 0; s < 2; s++) mbar_init(&dqdone[s], 1);
         mbar_init(qfull, 1);
         mbar_init(drain, 1);
         mbar_init(dotmem, 4);
@@ -355,17 +350,16 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 mma_commit(&vempty[t % kVS]);
             };
             // Issue whichever is ready first: S/dP of tile ns (its K and V
-            // landed and the row warps have copied out S/dP of tile ns - 1) or
-            // dQ of tile nq (its dS is written). Neither waits for the other's
-            // inputs.
+            // landed, and the dQ of tile ns - 1, which reads the dS written
+            // over the S columns, is issued) or dQ of tile nq (its dS is in
+            // TMEM).
             int ns = 0, nq = 0;
             uint64_t t_idle = 0;
             if (ok) tc_fence_after();
             while (ok && nq < T) {
                 bool issued = false;
-                if (ns < T && ns <= nq + 2) {
-                    if ((ns == 0 || mbar_test(sfree, (ns - 1) & 1)) && mbar_test(&kfull[ns % kKS], (ns / kKS) & 1) &&
-                        mbar_test(&vfull[ns % kVS], (ns / kVS) & 1)) {
+                if (ns < T && ns <= nq) {
+                    if (mbar_test(&kfull[ns % kKS], (ns / kKS) & 1) && mbar_test(&vfull[ns % kVS], (ns / kVS) & 1)) {
                         counters[2] = ns + 1;
                         counters[3] = ns + 1;
                         tc_fence_after();
@@ -374,24 +368,24 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                         issued = true;
                     }
                 }
-                if (!issued && nq < ns && mbar_test(&dsready[nq & 1], (nq >> 1) & 1)) {
+                if (!issued && nq < ns && mbar_test(dsready, nq & 1)) {
                     const int s = nq & 1;
                     tc_fence_after();
-                    const SDesc dd = sdesc_split(sdesc_noswz(smem_u32(sm + (s ? oS1 : oS0)), 128, 1024));
+                    const uint32_t da = tmem + kColS;  // dS: 64 keys as 32 columns of bf16 pairs
                     const uint32_t kb = smem_u32(sm + oK + (nq % kKS) * kTile);
                     if (nq < n_ctx) {  // B: all 256 columns, slices 8 KB apart, 16 keys = 2 KB
                         const SDesc kd = sdesc_split(sdesc_sw128(kb, kKChunk, 1024));
-                        mma_bf16_ss(tmem + kColDQ, dd.at(0), kd.at(0), idQ, nq > 0 ? 1u : 0u);
+                        mma_bf16_ts(tmem + kColDQ, da, kd.at(0), idQ, nq > 0 ? 1u : 0u);
 #pragma unroll
-                        for (int k = 1; k < kBN / 16; ++k) mma_bf16_ss(tmem + kColDQ, dd.at(16 * k), kd.at(128 * k), idQ, 1u);
+                        for (int k = 1; k < kBN / 16; ++k) mma_bf16_ts(tmem + kColDQ, da + 8 * k, kd.at(128 * k), idQ, 1u);
                     } else {  // block-major: K^C (slices 1 KB apart, 2 blocks = 6 KB) and K^R (2 KB)
                         const SDesc kdc = sdesc_split(sdesc_sw128(kb, 1024, kDraftKcBlock));
                         const SDesc kdr = sdesc_split(sdesc_sw128(kb + kDraftKr, 1024, 1024));
 #pragma unroll
                         for (int k = 0; k < kBN / 16; ++k) {
                             const uint32_t acc = (nq > 0 || k > 0) ? 1u : 0u;
-                            mma_bf16_ss(tmem + kColDQ, dd.at(16 * k), kdc.at(((2 * kDraftKcBlock) >> 4) * k), idQc, acc);
-                            mma_bf16_ss(tmem + kColDQ + kDC, dd.at(16 * k), kdr.at(128 * k), idQr, acc);
+                            mma_bf16_ts(tmem + kColDQ, da + 8 * k, kdc.at(((2 * kDraftKcBlock) >> 4) * k), idQc, acc);
+                            mma_bf16_ts(tmem + kColDQ + kDC, da + 8 * k, kdr.at(128 * k), idQr, acc);
                         }
                     }
                     mma_commit(&kempty[nq % kKS]);
@@ -472,15 +466,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     pv[32 + c] = b1[c];
                 }
             }
-            // S and dP are in registers: the MMA warp may overwrite them
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sfree);
-            if (t >= 2) {
-                ok = warp_all(mbar_wait(&dqdone[s], ((t - 2) >> 1) & 1, abort_flag));
-                if (!ok) break;
-            }
-            uint8_t *drow = sm + (s ? oS1 : oS0);
+            (void)s;
             // the row's keys in this tile: one contiguous column range [clo, chi)
             int clo, chi;
             if (t < n_ctx) {
@@ -492,23 +478,22 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 chi = clo + kBlock;
             }
             if (!live) chi = clo;
+            uint32_t dsw[kBN / 2];  // dS as bf16 pairs, over the S columns just read
 #pragma unroll
-            for (int u = 0; u < kBN / 8; u++) {
-                float e[8];
+            for (int c = 0; c < kBN; c += 2) {
+                float e[2];
 #pragma unroll
-                for (int k = 0; k < 8; k++) {
-                    const int c = u * 8 + k;
-                    const float pp = (c >= clo && c < chi) ? ex2(fmaf(sv[c], p.scale_log2, -lse2)) : 0.f;
-                    e[k] = pp * (pv[c] - Dr) * p.scale;
+                for (int d = 0; d < 2; d++) {
+                    const float pp = (c + d >= clo && c + d < chi) ? ex2(fmaf(sv[c + d], p.scale_log2, -lse2)) : 0.f;
+                    e[d] = pp * (pv[c + d] - Dr) * p.scale;
                 }
-                *reinterpret_cast<uint4 *>(drow + (r >> 3) * 1024 + u * 128 + (r & 7) * 16) =
-                    make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
-                               pack_bf16x2(e[6], e[7]));
+                dsw[c / 2] = pack_bf16x2(e[0], e[1]);
             }
-            fence_proxy_async_smem();
+            tmem_st32u(trow + kColS, dsw);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dsready[s]);
+            if (lane == 0) mbar_arrive(dsready);
         }
         if (ok) ok = warp_all(mbar_wait(&dqdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
         if (ok) {
