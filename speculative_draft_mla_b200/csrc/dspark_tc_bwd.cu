@@ -14,22 +14,20 @@
 //                      anchor-sorted row order, D, LSE*log2(e); padding rows 0.
 //   2. k_bwd_pad       zeros for padding blocks' rows and draft keys.
 //   3. k_bwd_dq_tc     query-major, one CTA per (b, h, 25 sorted blocks):
-//                      32-key tiles of the group's key set; S and dP in TMEM,
-//                      dS through shared memory, dQ += dS K in TMEM.
-//   4. k_bwd_kv_tc     key-major, one CTA per (b, 128-key tile, role, head
-//                      group): rows of the blocks whose key sets meet the tile,
-//                      in chunks of 32: S^T = K Q^T (and dP^T = V dO^T) in
-//                      TMEM, P^T (dS^T) through shared memory, dV += P^T dO
-//                      (dK += dS^T Q) accumulated in TMEM over the rows. A
-//                      128-key tile's dV and dK accumulators would need all
-//                      512 TMEM columns together, so they are produced by two
-//                      CTA roles that each recompute S^T; the two are adjacent
-//                      in launch order so one of them reads K from L2.
+//                      64-key tiles of the group's key set; S and dP in TMEM,
+//                      dS written over the S columns, dQ += dS K in TMEM.
+//   4. k_bwd_kv_tc     key-major, one CTA per (b, 64-key tile, head group):
+//                      rows of the blocks whose key sets meet the tile, in
+//                      chunks of 64: S^T = K Q^T and dP^T = V dO^T in TMEM,
+//                      P^T and dS^T through shared memory, dV += P^T dO and
+//                      dK += dS^T Q accumulated in TMEM over the rows (M = 64
+//                      accumulators: dK and dV share TMEM columns, one in each
+//                      half of the lanes).
 //   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
 //                      them back and writes dK^R.
-// Key tiles are either context tiles [t0, t0+128) or the draft keys of one
-// group of 25 blocks; the blocks whose windows meet a context tile are a
-// contiguous run of the anchor-sorted list (t0 < A <= t0 + 127 + W - 1).
+// Key tiles are either context tiles [t0, t0+64) or the draft keys of one
+// group of 8 blocks; the blocks whose windows meet a context tile are a
+// contiguous run of the anchor-sorted list (t0 < A <= t0 + 63 + W - 1).
 #include <algorithm>
 
 #include "dspark_tc_common.cuh"
@@ -42,7 +40,7 @@ using namespace tc;
 
 constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
 constexpr int kG = 25;   // blocks per query group (query-major kernel)
-constexpr int kGD = 16;  // blocks per draft-key tile of the key-major kernel (8 slots each)
+constexpr int kGD = 8;   // blocks per draft-key tile of the key-major kernel (8 slots each: 64 keys)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
@@ -561,70 +559,68 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
 }
 
 // ============================================================== dK / dV
-// Key tile = 128 keys (MMA M); the rows that see it stream through in chunks
-// (MMA N of S^T). Each chunk's two row operands have different lifetimes: the
-// one read only by the S^T-stage MMAs (dO for role K, Q for role V) is
-// released as soon as they complete; the one also read by the accumulation
-// (Q for role K, dO for role V) is held until it. P^T / dS^T go to tensor
-// memory, where the accumulation MMA reads them as its A operand.
-// Role K (dK = dS^T Q) needs K and V tiles and S^T, dP^T, dS^T: 32-row chunks,
-// 2 + 3 stages. Role V (dV = P^T dO) needs only K and S^T, P^T written over
-// its own S^T columns: 64-row chunks (half the chunks, the per-chunk latency
-// being what bounds a CTA), 2 + 2 stages.
+// Key tile = 64 keys (MMA M = 64); dK and dV of the tile in one CTA, so K, V
+// and every row of Q and dO that sees the tile cross into shared memory once.
+// With M = 64 an accumulator occupies lanes 0-15 of each 32-lane TMEM
+// sub-partition, and a second one addressed at lane offset 16 the lanes 16-31
+// of the same columns: dK (offset 0) and dV (offset 16) share columns 0..255,
+// S^T (0) and dP^T (16) share a 64-column buffer (two buffers, columns 256 and
+// 320). dK's columns 192..255 are the rope slice: it is summed over the heads
+// of the group, so that part of the accumulator is never reset between heads.
+// Per head: the K^C and V tiles (one stage, reloaded once the head's last
+// S^T / dP^T completed; the rope-key tile is the same for all heads and is
+// loaded once), then the rows that see the tile in chunks of 64 (Q and dO,
+// two stages): S^T = K Q^T and dP^T = V dO^T, P^T and dS^T (bf16) through one
+// shared-memory buffer, dV += P^T dO, dK += dS^T Q.
+// Key warps: warp w covers keys 16 (w & 3) .. + 15 (TMEM sub-partition w & 3)
+// and rows 32 (w >> 2) .. + 31 of a chunk. Lane l < 16 loads S^T of its key,
+// lane l + 16 dP^T of the same key; the two swap halves, so each lane holds
+// both for 16 rows.
 namespace kv {
-constexpr int kMK = 128;                 // keys per tile (MMA M)
-constexpr int kKChunk = kMK * 128;       // 16 KB: 128 keys x 64 columns
-// Draft items are loaded block-major: block bb's 8 K^C rows (3 x 1 KB
-// swizzled slices) at bb * 3 KB, its K^R rows at 48 KB + bb * 1 KB, its V rows
-// (4 x 1 KB) at bb * 4 KB: as MMA A operands, K^C / V with 8-key groups 3 KB /
-// 4 KB apart and 64-column slices 1 KB apart.
+constexpr int kMK = 64;                    // keys per tile (MMA M)
+constexpr int kRC = 64;                    // rows per chunk (MMA N of S^T / dP^T, K of the accumulations)
+constexpr int kSlice = 64 * 128;           // 8 KB: 64 keys or rows x 64 columns, 128-byte swizzled
+// Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
+// slices) at bb * 3 KB, its K^R rows at bb * 1 KB of the rope-key tile, its V
+// rows (4 x 1 KB) at bb * 4 KB: 8-key groups 3 KB / 4 KB apart, 64-column
+// slices 1 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftVBlock = 4 * 1024;
-constexpr int kStageBytes = 8 * 32 * 64; // epilogue staging: 8 warps x 32 keys x 32 columns bf16
-constexpr int oK = 0, oV = oK + 4 * kKChunk;
-template <bool RK> struct KvCfg {
-    static constexpr int kRC = RK ? 32 : 64;  // rows per chunk
-    static constexpr int kES = 2, kLS = RK ? 3 : 2;
-    static constexpr int kRBuf = 4 * kRC * 128;
-    static constexpr int oE = RK ? oV + 4 * kKChunk : oV;  // role V has no V tile
-    static constexpr int oL = oE + kES * kRBuf, oStage = oL + kLS * kRBuf;
-    static constexpr int oMeta = oStage + kStageBytes, oBar = oMeta + kLS * kRC * 12;
-    static constexpr int kSmem = oBar + 256 + 1024;
-    static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
-};
-constexpr int kSmem = KvCfg<true>::kSmem > KvCfg<false>::kSmem ? KvCfg<true>::kSmem : KvCfg<false>::kSmem;
-constexpr int kKeyWarps = 8;             // two per TMEM sub-partition, each half of a chunk's rows
-constexpr int kWarpL = kKeyWarps, kWarpMma = kKeyWarps + 1, kWarpE = kKeyWarps + 2;
+constexpr int oKr = 0, oKc = oKr + kSlice, oV = oKc + 3 * kSlice;
+constexpr int kRowStage = 8 * kSlice;      // Q chunk (4 slices), then dO chunk (4 slices)
+constexpr int oRow = oV + 4 * kSlice;
+constexpr int oPT = oRow + 2 * kRowStage;  // P^T, then dS^T: [64 keys][64 rows] bf16 each
+constexpr int oStage = oPT + 2 * kSlice;   // epilogue staging, 2 KB per key warp
+constexpr int oMeta = oStage + 8 * 2048;   // per row stage: (LSE * log2 e, D) of each row
+constexpr int oBar = oMeta + 2 * kRC * 8;
+constexpr int kSmem = oBar + 128 + 1024;
+static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+constexpr int kKeyWarps = 8;
+constexpr int kWarpKV = kKeyWarps, kWarpRow = kKeyWarps + 1, kWarpMma = kKeyWarps + 2;
 constexpr int kThreads = (kKeyWarps + 3) * 32;
-constexpr uint32_t kColAcc = 0;
+constexpr uint32_t kColAcc = 0, kColS = 256;  // S^T / dP^T buffer s at kColS + 64 s
+constexpr uint32_t kHi = 16u << 16;           // lane offset of the second M = 64 accumulator
 }  // namespace kv
 
-// One CTA per (key tile, role, head group, batch). Role 0 accumulates dV =
-// P^T dO, role 1 dK = dS^T Q; the two roles of a tile are adjacent in launch
-// order so the second reads K and the row chunks from L2.
-template <bool RK>
-__device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensorMap &tm_kr, const CUtensorMap &tm_v,
-                                        const CUtensorMap &tm_qs, const CUtensorMap &tm_dos, const CUtensorMap &tm_kc8,
-                                        const CUtensorMap &tm_kr8, const CUtensorMap &tm_v8, const BwdArgs &p) {
+// One CTA per (64-key tile, head group, batch row).
+__global__ void __launch_bounds__(kv::kThreads, 1)
+    k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
+                const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
+                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8,
+                const BwdArgs p) {
     using namespace kv;
-    using C = KvCfg<RK>;
-    constexpr int kRC = C::kRC, kRChunk = kRC * 128, kRBuf = 4 * kRChunk, kES = C::kES, kLS = C::kLS;
-    constexpr int oE = C::oE, oL = C::oL, oStage = C::oStage, oMeta = C::oMeta, oBar = C::oBar;
-    constexpr uint32_t kColS = 256, kColP = 320, kColPT = 384;  // dP^T and a separate P^T buffer: role K only
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *efull = bars + 2, *efree = efull + kES, *lfull = efree + kES,
-             *lfree = lfull + kLS, *sfull = lfree + kLS, *dsready = sfull + 2, *ptfree = dsready + 2,
-             *accdone = ptfree + 2, *epidone = accdone + 1, *drain = epidone + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(drain + 2);
-    // kv issued, L issued, kv consumed, chunks consumed, E issued
-    int *counters = reinterpret_cast<int *>(drain + 3);
-    int *band = counters + 6;  // first sorted row, row count
+    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *rowfull = bars + 2, *rowfree = bars + 4, *sfull = bars + 6,
+             *dsready = bars + 8, *ptfree = bars + 9, *drain = bars + 10;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // K/V heads issued, row chunks issued, K/V heads consumed, row chunks consumed
+    int *counters = reinterpret_cast<int *>(tmem_slot + 2);
+    int *band = counters + 4;  // first sorted row, row count
 
-    const int item = blockIdx.x >> 1;
-    constexpr bool role_k = RK;
-    const int hg = blockIdx.y, b = blockIdx.z;
+    const int item = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cnt = p.cnt[b];
     const bool is_ctx = item < p.n_ctx_items;
@@ -667,67 +663,59 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
     const int nchunks = (nrows + kRC - 1) / kRC;
     const int h0 = hg * p.hpg;
     const int H = p.hpg;
-    // the key this thread stands for (key warps): TMEM lane = key slot
-    const int k = (threadIdx.x & 127);
-    const int half = warp >> 2;  // which half of a chunk's rows / of the accumulator columns
+    // the key this thread stands for (key warps): TMEM lane (l & 15) of its
+    // sub-partition's two halves
+    const int kk = 16 * (warp & 3) + (lane & 15);
+    const int hr = (warp >> 2) & 1;  // row half of a chunk / column half of the accumulators
+    const bool dlane = lane >= 16;   // lane of the dP^T / dV half
     bool key_valid = false;
     size_t key_pos = 0;
     if (warp < kKeyWarps) {
         if (is_ctx) {
-            key_valid = t0 + k < p.S;
-            key_pos = (size_t)t0 + k;
+            key_valid = t0 + kk < p.S;
+            key_pos = (size_t)t0 + kk;
         } else {  // 8 key slots per block: its 5 keys, then 3 masked rows
-            key_valid = k / 8 < gcnt && k % 8 < kBlock;
-            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + k / 8] + k % 8;
+            key_valid = kk / 8 < gcnt && kk % 8 < kBlock;
+            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + kk / 8] + kk % 8;
         }
     }
     float *dkr_part_row = p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR;
 
     if (nrows == 0) {
         // no row sees these keys: zero gradients for every head of the group
+        // (four threads per key)
         if (warp < kKeyWarps && key_valid) {
+            const int part = 2 * hr + (dlane ? 1 : 0);
             const uint4 z = make_uint4(0, 0, 0, 0);
             for (int hh = 0; hh < H; hh++) {
                 const size_t bh = (size_t)b * p.n_h + h0 + hh;
-                if (role_k) {
-                    uint4 *d = reinterpret_cast<uint4 *>(p.dkc + (bh * p.L + key_pos) * kDC);
-                    for (int e = half; e < kDC / 8; e += 2) d[e] = z;
-                } else {
-                    uint4 *d = reinterpret_cast<uint4 *>(p.dv + (bh * p.L + key_pos) * kDV);
-                    for (int e = half; e < kDV / 8; e += 2) d[e] = z;
-                }
+                uint4 *dk = reinterpret_cast<uint4 *>(p.dkc + (bh * p.L + key_pos) * kDC);
+                for (int e = part; e < kDC / 8; e += 4) dk[e] = z;
+                uint4 *dvv = reinterpret_cast<uint4 *>(p.dv + (bh * p.L + key_pos) * kDV);
+                for (int e = part; e < kDV / 8; e += 4) dvv[e] = z;
             }
-            if (role_k && half == 0)
-                for (int e = 0; e < kDR / 4; e++)
-                    reinterpret_cast<float4 *>(dkr_part_row)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = part; e < kDR / 4; e += 4)
+                reinterpret_cast<float4 *>(dkr_part_row)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
 
-    // K/V tiles start zeroed (masked key slots must hold finite values)
-    for (int e = threadIdx.x; e < (oE - oK) / 16; e += blockDim.x)
-        reinterpret_cast<uint4 *>(sm + oK)[e] = make_uint4(0, 0, 0, 0);
+    // K/V tiles start zeroed (key slots no load reaches must hold finite values)
+    for (int e = threadIdx.x; e < (oRow - oKr) / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + oKr)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         mbar_init(kvfull, 1);
         mbar_init(kvfree, 1);
-        for (int s = 0; s < kES; s++) {
-            mbar_init(&efull[s], 1);
-            mbar_init(&efree[s], 1);
-        }
-        for (int s = 0; s < kLS; s++) {
-            mbar_init(&lfull[s], 1);
-            mbar_init(&lfree[s], 1);
-        }
         for (int s = 0; s < 2; s++) {
+            mbar_init(&rowfull[s], 1);
+            mbar_init(&rowfree[s], 1);
             mbar_init(&sfull[s], 1);
-            mbar_init(&dsready[s], kKeyWarps);
-            mbar_init(&ptfree[s], 1);
         }
-        mbar_init(accdone, 1);
-        mbar_init(epidone, kKeyWarps);
+        mbar_init(dsready, kKeyWarps);
+        mbar_init(ptfree, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
-        for (int c = 0; c < 6; c++) counters[c] = 0;
+        for (int c = 0; c < 4; c++) counters[c] = 0;
         fence_barrier_init();
     }
     if (warp == kWarpMma) {
@@ -740,75 +728,54 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int QT = H * nchunks;  // chunks over all heads of the group
-    // row operands: L = read by the accumulation too (Q for role K, dO for
-    // role V), E = read only by the S^T stage (dO for role K, Q for role V)
-    const CUtensorMap *tm_l = role_k ? &tm_qs : &tm_dos;
-    const CUtensorMap *tm_e = role_k ? &tm_dos : &tm_qs;
 
-    if (warp == kWarpE) {
-        // ------------------------------------------- producer of E operands
-        for (int q = 0; q < QT; ++q) {
-            const int hh = q / nchunks, c = q % nchunks, es = q % kES;
-            const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            const int r0 = row0 + c * kRC;
-            if (q >= kES && !warp_all(mbar_wait(&efree[es], ((q / kES) - 1) & 1, abort_flag))) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&efull[es], kRBuf);
-                tma_load_3d(sm + oE + es * kRBuf, tm_e, &efull[es], 0, (int)(bh * p.R + r0), 0);
-                counters[4] = q + 1;
-            }
-        }
-    } else if (warp == kWarpL) {
-        // ------------------------- producer of K/V tiles and L operands
+    if (warp == kWarpKV) {
+        // ------------------------------------------- producer of K/V tiles
         const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
-        for (int q = 0; q < QT; ++q) {
-            const int hh = q / nchunks, c = q % nchunks;
-            const int ls = q % kLS;
+        for (int hh = 0; hh < H; ++hh) {
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            if (c == 0) {
-                if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
-                if (is_ctx) {
+            if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
+            if (is_ctx) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(kvfull, (hh == 0 ? 8 : 7) * kSlice);
+                    if (hh == 0) tma_load_2d(sm + oKr, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
+                    tma_load_3d(sm + oKc, &tm_kc, kvfull, 0, (int)(bh * p.L + t0), 0);
+                    tma_load_3d(sm + oV, &tm_v, kvfull, 0, (int)(bh * p.L + t0), 0);
+                }
+            } else {
+                if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * ((hh == 0 ? kDQK : kDC) + kDV) * 2);
+                for (int bb = 0; bb < gcnt; ++bb) {
+                    const int nb = __shfl_sync(0xffffffffu, my_n, bb);
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(kvfull, (role_k ? 8 : 4) * kKChunk);
-                        tma_load_3d(sm + oK, &tm_kc, kvfull, 0, (int)(bh * p.L + t0), 0);
-                        tma_load_2d(sm + oK + 3 * kKChunk, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
-                        if (role_k) tma_load_3d(sm + oV, &tm_v, kvfull, 0, (int)(bh * p.L + t0), 0);
-                    }
-                } else {
-                    if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * (role_k ? 2 : 1) * kDQK * 2);
-                    for (int bb = 0; bb < gcnt; ++bb) {
-                        const int nb = __shfl_sync(0xffffffffu, my_n, bb);
-                        if (lane == 0) {
-                            const int row = p.S + kBlock * nb;
-                            tma_load_3d(sm + oK + bb * kDraftKcBlock, &tm_kc8, kvfull, 0, (int)(bh * p.L + row), 0);
-                            tma_load_2d(sm + oK + 3 * kKChunk + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
-                            if (role_k)
-                                tma_load_3d(sm + oV + bb * kDraftVBlock, &tm_v8, kvfull, 0, (int)(bh * p.L + row), 0);
-                        }
+                        const int row = p.S + kBlock * nb;
+                        tma_load_3d(sm + oKc + bb * kDraftKcBlock, &tm_kc8, kvfull, 0, (int)(bh * p.L + row), 0);
+                        if (hh == 0)
+                            tma_load_2d(sm + oKr + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
+                        tma_load_3d(sm + oV + bb * kDraftVBlock, &tm_v8, kvfull, 0, (int)(bh * p.L + row), 0);
                     }
                 }
-                if (lane == 0) counters[0] = hh + 1;
             }
+            if (lane == 0) counters[0] = hh + 1;
+        }
+    } else if (warp == kWarpRow) {
+        // ---------------------------- producer of Q / dO chunks and row data
+        for (int q = 0; q < QT; ++q) {
+            const int hh = q / nchunks, c = q % nchunks, s = q & 1;
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
             const int r0 = row0 + c * kRC;
-            // L operand and the chunk metadata: anchor (INT_MAX past the
-            // band), LSE*log2(e), D
-            if (q >= kLS && !warp_all(mbar_wait(&lfree[ls], ((q / kLS) - 1) & 1, abort_flag))) break;
-            {
-                int *mA = reinterpret_cast<int *>(sm + oMeta + ls * kRC * 12);
-                float2 *mLD = reinterpret_cast<float2 *>(mA + kRC);
+            if (q >= 2 && !warp_all(mbar_wait(&rowfree[s], ((q >> 1) - 1) & 1, abort_flag))) break;
+            float2 *mLD = reinterpret_cast<float2 *>(sm + oMeta + s * kRC * 8);
 #pragma unroll
-                for (int jj = 0; jj < kRC; jj += 32) {
-                    const int rowi = r0 + jj + lane;
-                    const bool in = rowi < row0 + nrows;
-                    mA[jj + lane] = in ? sa[rowi / kBlock] : 0x7fffffff;
-                    mLD[jj + lane] =
-                        in ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi]) : make_float2(0.f, 0.f);
-                }
+            for (int jj = 0; jj < kRC; jj += 32) {
+                const int rowi = r0 + jj + lane;
+                mLD[jj + lane] = rowi < row0 + nrows ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi])
+                                                     : make_float2(0.f, 0.f);
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(&lfull[ls], kRBuf);
-                tma_load_3d(sm + oL + ls * kRBuf, tm_l, &lfull[ls], 0, (int)(bh * p.R + r0), 0);
+                mbar_arrive_expect_tx(&rowfull[s], kRowStage);
+                tma_load_3d(sm + oRow + s * kRowStage, &tm_qs, &rowfull[s], 0, (int)(bh * p.R + r0), 0);
+                tma_load_3d(sm + oRow + s * kRowStage + 4 * kSlice, &tm_dos, &rowfull[s], 0, (int)(bh * p.R + r0), 0);
                 counters[1] = q + 1;
             }
         }
@@ -816,79 +783,73 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kMK, kRC, 0);   // S^T, dP^T: B = Q / dO chunk, K-major
-            const uint32_t idA = idesc_bf16(kMK, 256, 1);   // acc: B = dO / Q chunk, MN-major
+            const uint32_t idV = idesc_bf16(kMK, kDV, 1);   // dV: B = dO chunk, MN-major
+            const uint32_t idKc = idesc_bf16(kMK, kDC, 1);  // dK^C: B = Q^C columns
+            const uint32_t idKr = idesc_bf16(kMK, kDR, 1);  // dK^R: B = Q^R columns
             // A operands: K^C / V slices kcStep / vStep bytes apart (context
-            // tile: 16 KB slices of 128 keys; draft item: block-major); the
-            // K^R slice at 48 KB in both
-            const uint32_t kcStep = is_ctx ? kKChunk : 1024, vStep = is_ctx ? kKChunk : 1024;
-            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + oK), 16, is_ctx ? 1024 : kDraftKcBlock));
-            const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + oK + 3 * kKChunk), 16, 1024));
+            // tile: 8 KB slices of 64 keys; draft tile: block-major)
+            const uint32_t kcStep = is_ctx ? kSlice : 1024, vStep = is_ctx ? kSlice : 1024;
+            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + oKc), 16, is_ctx ? 1024 : kDraftKcBlock));
+            const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + oKr), 16, 1024));
             const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + oV), 16, is_ctx ? 1024 : kDraftVBlock));
+            const SDesc ptd = sdesc_split(sdesc_sw128(smem_u32(sm + oPT), 16, 1024));
+            const SDesc dsd = sdesc_split(sdesc_sw128(smem_u32(sm + oPT + kSlice), 16, 1024));
             bool ok = true;
             auto issue_s = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
-                const SDesc ld_ = sdesc_split(sdesc_sw128(smem_u32(sm + oL + (q % kLS) * kRBuf), 16, 1024));
-                const SDesc ed = sdesc_split(sdesc_sw128(smem_u32(sm + oE + (q % kES) * kRBuf), 16, 1024));
-                const uint32_t dS = tmem + kColS + s * kRC, dP = tmem + kColP + s * kRC;
-                if (role_k) {
-                    // S^T = K Q^T and dP^T = V dO^T interleaved: two independent chains
+                const uint32_t rs = smem_u32(sm + oRow + s * kRowStage);
+                const SDesc qd = sdesc_split(sdesc_sw128(rs, 16, 1024));
+                const SDesc dod = sdesc_split(sdesc_sw128(rs + 4 * kSlice, 16, 1024));
+                const uint32_t dS = tmem + kColS + 64 * s, dP = dS + kHi;
+                // S^T = K Q^T and dP^T = V dO^T interleaved: two independent chains
 #pragma unroll
-                    for (int kk = 0; kk < kDQK / 16; ++kk) {
-                        const int cc = kk >> 2;
-                        const uint32_t sub = (kk & 3) * 2;  // 32 bytes, in 16-byte units
-                        const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
-                        const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(dS, ka, ld_.at(ro), idS, kk > 0 ? 1u : 0u);
-                        mma_bf16_ss(dP, vad.at(((cc * vStep) >> 4) + sub), ed.at(ro), idS, kk > 0 ? 1u : 0u);
-                    }
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < kDQK / 16; ++kk) {
-                        const int cc = kk >> 2;
-                        const uint32_t sub = (kk & 3) * 2;
-                        const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
-                        const uint32_t ro = ((kk >> 2) * kRChunk + (kk & 3) * 32) >> 4;
-                        mma_bf16_ss(dS, ka, ed.at(ro), idS, kk > 0 ? 1u : 0u);
-                    }
+                for (int k16 = 0; k16 < kDQK / 16; ++k16) {
+                    const int cc = k16 >> 2;
+                    const uint32_t sub = (k16 & 3) * 2;  // 32 bytes, in 16-byte units
+                    const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
+                    const uint32_t ro = (cc * kSlice + (k16 & 3) * 32) >> 4;
+                    mma_bf16_ss(dS, ka, qd.at(ro), idS, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(dP, vad.at(((cc * vStep) >> 4) + sub), dod.at(ro), idS, k16 > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[s]);
-                mma_commit(&efree[q % kES]);
                 if (c == nchunks - 1) mma_commit(kvfree);
             };
             auto issue_acc = [&](int q) {
                 const int c = q % nchunks, s = q & 1;
                 tc_fence_after();
-                const SDesc bd = sdesc_split(sdesc_sw128(smem_u32(sm + oL + (q % kLS) * kRBuf), kRChunk, 1024));
-                if constexpr (RK) {  // dS^T in its own buffer: rows 0..15, 16..31
-                    const uint32_t pa = tmem + kColPT + s * (kRC / 2);
-                    mma_bf16_ts(tmem + kColAcc, pa, bd.at(0), idA, c > 0 ? 1u : 0u);
-                    mma_bf16_ts(tmem + kColAcc, pa + 8, bd.at(128), idA, 1u);
-                } else {  // P^T over the first 16 columns of each 32-row half of the S^T buffer
-                    const uint32_t pa = tmem + kColS + s * kRC;
-                    mma_bf16_ts(tmem + kColAcc, pa, bd.at(0), idA, c > 0 ? 1u : 0u);
-                    mma_bf16_ts(tmem + kColAcc, pa + 8, bd.at(128), idA, 1u);
-                    mma_bf16_ts(tmem + kColAcc, pa + 32, bd.at(256), idA, 1u);
-                    mma_bf16_ts(tmem + kColAcc, pa + 40, bd.at(384), idA, 1u);
-                }
-                mma_commit(&lfree[q % kLS]);
-                mma_commit(&ptfree[s]);
-                if (c == nchunks - 1) mma_commit(accdone);
+                const uint32_t rs = smem_u32(sm + oRow + s * kRowStage);
+                const SDesc qb = sdesc_split(sdesc_sw128(rs, kSlice, 1024));            // MN-major
+                const SDesc dob = sdesc_split(sdesc_sw128(rs + 4 * kSlice, kSlice, 1024));
+                // 16 rows per MMA: 32 bytes along the K-major P^T / dS^T rows,
+                // 2 KB (16 rows of 128 bytes) in the row chunk
+#pragma unroll
+                for (int k16 = 0; k16 < kRC / 16; ++k16)
+                    mma_bf16_ss(tmem + kColAcc + kHi, ptd.at(2 * k16), dob.at(128 * k16), idV,
+                                (c > 0 || k16 > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k16 = 0; k16 < kRC / 16; ++k16)
+                    mma_bf16_ss(tmem + kColAcc, dsd.at(2 * k16), qb.at(128 * k16), idKc, (c > 0 || k16 > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k16 = 0; k16 < kRC / 16; ++k16)
+                    mma_bf16_ss(tmem + kColAcc + kDC, dsd.at(2 * k16), qb.at(((3 * kSlice) >> 4) + 128 * k16), idKr,
+                                (q > 0 || k16 > 0) ? 1u : 0u);
+                mma_commit(&rowfree[s]);
+                mma_commit(ptfree);
             };
             // Issue whichever is ready: the S^T stage of chunk ns (its K/V tile
             // and row operands landed; at most one chunk ahead, so its S^T /
-            // dP^T buffer was released by the accumulation of chunk ns - 2) or
-            // the accumulation of chunk na (its P^T / dS^T is in TMEM and, at a
-            // head's first chunk, the previous head's epilogue has read the
-            // accumulator).
+            // dP^T buffer was read by the key warps before they signalled chunk
+            // ns - 2) or the accumulation of chunk na (P^T / dS^T written; at a
+            // head's first chunk the key warps have also read the previous
+            // head's accumulators, which precedes that signal).
             int ns = 0, na = 0;
             uint64_t t_idle = 0;
             while (ok && na < QT) {
                 bool issued = false;
                 if (ns < QT && ns <= na + 1) {
                     const int hh = ns / nchunks, c = ns % nchunks;
-                    if ((c != 0 || mbar_test(kvfull, hh & 1)) && mbar_test(&lfull[ns % kLS], (ns / kLS) & 1) &&
-                        mbar_test(&efull[ns % kES], (ns / kES) & 1)) {
+                    if ((c != 0 || mbar_test(kvfull, hh & 1)) && mbar_test(&rowfull[ns & 1], (ns >> 1) & 1)) {
                         if (c == 0) counters[2] = hh + 1;
                         counters[3] = ns + 1;
                         issue_s(ns);
@@ -896,14 +857,10 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
                         issued = true;
                     }
                 }
-                if (!issued && na < ns) {
-                    const int hh = na / nchunks, c = na % nchunks, s = na & 1;
-                    if (mbar_test(&dsready[s], (na >> 1) & 1) &&
-                        (c != 0 || hh == 0 || mbar_test(epidone, (hh - 1) & 1))) {
-                        issue_acc(na);
-                        ++na;
-                        issued = true;
-                    }
+                if (!issued && na < ns && mbar_test(dsready, na & 1)) {
+                    issue_acc(na);
+                    ++na;
+                    issued = true;
                 }
                 if (issued) {
                     t_idle = 0;
@@ -921,9 +878,8 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
     } else {
         // ------------------------------------------ key warps (0..7)
         const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const int kpos = t0 + k;               // context position of this key (context tiles)
-        const int kblk = k / 8;                // draft tiles: the key's block within the group
-        const int col0 = half * (kRC / 2);     // this warp's rows within a chunk
+        const int rb = 32 * hr + 16 * (lane >> 4);  // first chunk row of this lane after the swap
+        const int kpos = t0 + kk;                   // context position of this key (context tiles)
         // The rows that see this key, in sorted-row order relative to the band:
         // one range [rlo, rhi), the same for every head. Context key: blocks
         // with kpos < A <= kpos + W - 1; draft key slot: its own block.
@@ -944,132 +900,131 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
                 }
                 rhi = kBlock * lo - row0;
             } else {
-                rlo = kBlock * kblk;
+                rlo = kBlock * (kk / 8);
                 rhi = rlo + kBlock;
             }
         }
-        uint8_t *stage = sm + oStage + warp * (32 * 64);
-        float racc[kDR];                       // rope slice of dK summed over heads (half-1 warps)
-#pragma unroll
-        for (int i = 0; i < kDR; i++) racc[i] = 0.f;
+        // this key's row of the P^T / dS^T tiles (128-byte swizzle) and the
+        // two 16-byte units that hold rows rb .. rb + 15
+        const uint32_t prow = (uint32_t)((kk >> 3) * 1024 + (kk & 7) * 128);
+        const uint32_t pu0 = prow + ((((uint32_t)rb >> 3) ^ (kk & 7)) << 4);
+        const uint32_t pu1 = prow + (((((uint32_t)rb >> 3) + 1) ^ (kk & 7)) << 4);
+        uint8_t *stage = sm + oStage + warp * 2048;
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks, s = q & 1;
-            ok = warp_all(mbar_wait(&lfull[q % kLS], (q / kLS) & 1, abort_flag));  // chunk metadata
+            ok = warp_all(mbar_wait(&rowfull[s], (q >> 1) & 1, abort_flag));  // row data
             if (ok) ok = warp_all(mbar_wait(&sfull[s], (q >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            constexpr int RH = kRC / 2;  // rows of the chunk per warp
-            float sv[RH], pv[RH];
-            if constexpr (RK) {
-                float a[32], bq[32];
-                tmem_ld32(trow + kColS + s * kRC, a);  // all 32 rows; this warp uses its half
-                tmem_ld32(trow + kColP + s * kRC, bq);
-                tmem_wait_ld();
+            float v[32];
+            tmem_ld32(trow + kColS + 64 * s + 32 * hr, v);
+            tmem_wait_ld();
+            float sv[16], pv[16];
 #pragma unroll
-                for (int i = 0; i < RH; i++) {
-                    sv[i] = half ? a[RH + i] : a[i];
-                    pv[i] = half ? bq[RH + i] : bq[i];
-                }
-            } else {
-                tmem_ld32(trow + kColS + s * kRC + 32 * half, *reinterpret_cast<float(*)[32]>(&sv[0]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < RH; i++) pv[i] = 0.f;
+            for (int i = 0; i < 16; i++) {
+                const float send = dlane ? v[i] : v[16 + i];
+                const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+                sv[i] = dlane ? recv : v[i];
+                pv[i] = dlane ? v[16 + i] : recv;
             }
-            // rows of the chunk that see this key: [jlo, jhi)
-            const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + (q % kLS) * kRC * 12 + kRC * 4);
-            const int jlo = rlo - c * kRC, jhi = rhi - c * kRC;
-            uint32_t w[RH / 2];
+            const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + s * kRC * 8) + rb;
+            const int jlo = rlo - c * kRC - rb, jhi = rhi - c * kRC - rb;  // visible rows, relative to rb
+            uint32_t pw[8], dw[8];
 #pragma unroll
-            for (int i = 0; i < RH; i += 2) {
-                float e2[2];
+            for (int i = 0; i < 16; i += 2) {
+                float ep[2], ed[2];
 #pragma unroll
                 for (int d = 0; d < 2; d++) {
-                    const int j = col0 + i + d;
+                    const int j = i + d;
                     const float2 ldv = mLD[j];
-                    const float pp = (j >= jlo && j < jhi) ? ex2(fmaf(sv[i + d], p.scale_log2, -ldv.x)) : 0.f;
-                    e2[d] = role_k ? pp * (pv[i + d] - ldv.y) * p.scale : pp;
+                    const float pp = (j >= jlo && j < jhi) ? ex2(fmaf(sv[j], p.scale_log2, -ldv.x)) : 0.f;
+                    ep[d] = pp;
+                    ed[d] = pp * (pv[j] - ldv.y) * p.scale;
                 }
-                w[i / 2] = pack_bf16x2(e2[0], e2[1]);
+                pw[i / 2] = pack_bf16x2(ep[0], ep[1]);
+                dw[i / 2] = pack_bf16x2(ed[0], ed[1]);
             }
-            if constexpr (RK) {
-                // the dS^T buffer s is free once the accumulation of chunk q - 2 completed
-                if (q >= 2) {
-                    ok = warp_all(mbar_wait(&ptfree[s], ((q >> 1) - 1) & 1, abort_flag));
-                    if (!ok) break;
-                }
-                tmem_st8u(trow + kColPT + s * (kRC / 2) + half * 8, *reinterpret_cast<uint32_t(*)[8]>(&w[0]));
-            } else {
-                // over this half's S^T columns (already read; the S^T buffer
-                // is rewritten only after the accumulation that reads P^T)
-                tmem_st16u(trow + kColS + s * kRC + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
+            // the P^T / dS^T buffer is free once the accumulation of chunk q - 1 completed
+            if (q >= 1) {
+                ok = warp_all(mbar_wait(ptfree, (q - 1) & 1, abort_flag));
+                if (!ok) break;
             }
-            tmem_wait_st();
+            *reinterpret_cast<uint4 *>(sm + oPT + pu0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            *reinterpret_cast<uint4 *>(sm + oPT + pu1) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+            *reinterpret_cast<uint4 *>(sm + oPT + kSlice + pu0) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+            *reinterpret_cast<uint4 *>(sm + oPT + kSlice + pu1) = make_uint4(dw[4], dw[5], dw[6], dw[7]);
+            fence_proxy_async_smem();  // visible to the MMAs that read them
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dsready[s]);
+            if (lane == 0) mbar_arrive(dsready);
             if (c != nchunks - 1) continue;
-            // head epilogue: accumulator columns [128 * half, 128 * half + 128)
-            ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag));
+            // head epilogue, once its accumulations completed: accumulator
+            // columns [128 hr, 128 hr + 128); lanes 0-15 hold dK, 16-31 dV
+            ok = warp_all(mbar_wait(ptfree, q & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            // Four rounds of 32 columns: each thread stages its key's 32
-            // values (bf16, 16-byte unit u at u ^ (key & 3)), then the warp
-            // writes 8 keys' 64-byte row segments per instruction.
+            // Four rounds of 32 columns: each thread stages its 32 values
+            // (bf16, 16-byte unit u at u ^ (lane & 3)), then the warp writes 8
+            // rows' 64-byte segments per instruction.
 #pragma unroll
             for (int rd = 0; rd < 4; rd++) {
-                const int col = half * 128 + rd * 32;
-                float v[32];
+                const int col = hr * 128 + rd * 32;
+                const bool rope = col >= kDC;  // dK columns 192..255 stay in TMEM (summed over heads)
                 tmem_ld32(trow + kColAcc + col, v);
                 tmem_wait_ld();
-                if (role_k && half == 1 && rd >= 2) {  // rope slice of dK (columns 192..255): summed over heads
-#pragma unroll
-                    for (int i = 0; i < 32; i++) racc[(rd - 2) * 32 + i] += v[i];
-                    continue;
-                }
 #pragma unroll
                 for (int u = 0; u < 4; u++)
                     *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
                         make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
                                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
                 __syncwarp();
-                const int rowstride = role_k ? kDC : kDV;
-                __nv_bfloat16 *base = role_k ? p.dkc : p.dv;
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
-                    const int kl = 8 * i + (lane >> 2), u = lane & 3;   // key within the warp, unit
-                    const int kkv = __shfl_sync(0xffffffffu, (int)key_valid, kl);
+                    const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
+                    const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
                     const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
-                    if (kkv) {
+                    const bool is_v = kl >= 16;
+                    if (kvl && (is_v || !rope)) {
                         const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
-                        *reinterpret_cast<uint4 *>(base + (bh * p.L + (size_t)kposl) * rowstride + col + 8 * u) = val;
+                        __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
+                                                  : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
+                        *reinterpret_cast<uint4 *>(dst) = val;
                     }
                 }
                 __syncwarp();
             }
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(epidone);
         }
-        if (ok && role_k && key_valid && half == 1) {
-            // this warp held accumulator columns 128..255: dK^C 128..191 and the rope slice 192..255
-            float4 *d = reinterpret_cast<float4 *>(dkr_part_row);
+        if (ok && hr == 1) {
+            // rope slice of dK (columns 192..255 of the lanes 0-15), summed over
+            // the group's heads by the MMAs
+            float *d = dkr_part_row;
+            const bool w_ = key_valid && !dlane;
 #pragma unroll
-            for (int i = 0; i < kDR / 4; i++) d[i] = make_float4(racc[4 * i], racc[4 * i + 1], racc[4 * i + 2], racc[4 * i + 3]);
+            for (int half2 = 0; half2 < 2; half2++) {
+                float v[32];
+                tmem_ld32(trow + kColAcc + kDC + 32 * half2, v);
+                tmem_wait_ld();
+                if (w_)
+#pragma unroll
+                    for (int i = 0; i < 8; i++)
+                        reinterpret_cast<float4 *>(d + 32 * half2)[i] =
+                            make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
         }
     }
 
     __syncthreads();
     if (*abort_flag) {
         volatile int never = 0;
-        if (warp == kWarpL && lane == 0) {
+        if (warp == kWarpKV && lane == 0) {
             for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(kvfull, t & 1, (volatile int *)&never);
+        }
+        if (warp == kWarpRow && lane == 0) {
             for (int t = counters[3]; t < counters[1]; ++t)
-                mbar_wait(&lfull[t % kLS], (t / kLS) & 1, (volatile int *)&never);
-            for (int t = counters[3]; t < counters[4]; ++t)
-                mbar_wait(&efull[t % kES], (t / kES) & 1, (volatile int *)&never);
+                mbar_wait(&rowfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
         }
         if (warp == kWarpMma && lane == 0) {
             mma_commit(drain);
@@ -1085,19 +1040,6 @@ __device__ __forceinline__ void kv_role(const CUtensorMap &tm_kc, const CUtensor
     if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
 }
 
-__global__ void __launch_bounds__(kv::kThreads, 1)
-    k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs32,
-                const __grid_constant__ CUtensorMap tm_dos32, const __grid_constant__ CUtensorMap tm_qs64,
-                const __grid_constant__ CUtensorMap tm_dos64, const __grid_constant__ CUtensorMap tm_kc8,
-                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
-    if (blockIdx.x & 1)
-        kv_role<true>(tm_kc, tm_kr, tm_v, tm_qs32, tm_dos32, tm_kc8, tm_kr8, tm_v8, p);
-    else
-        kv_role<false>(tm_kc, tm_kr, tm_v, tm_qs64, tm_dos64, tm_kc8, tm_kr8, tm_v8, p);
-}
-
-// ------------------------------------------------------------ dK^R reduce
 // ------------------------------------------------------------ dK^R reduce
 // One warp per (b, key): sum the head-group partials (rotated frame), rotate
 // back by the key's position, write dkr. Draft keys of padding blocks: 0.
@@ -1141,11 +1083,9 @@ bool bwd_tc_supported(const Prob &p) {
 
 int bwd_head_groups(const Prob &p) {
     const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kGD - 1) / kGD) * p.B;
-    // two CTA roles per key tile; aim for about eight waves on 148 SMs (shorter
-    // CTAs, smaller tail; measured better than four or sixteen at the
-    // 8192-context workload)
+    // aim for about eight waves on 148 SMs (shorter CTAs, smaller tail)
     int hg = 1;
-    while (hg < p.n_h && 2 * items * hg < 8 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
+    while (hg < p.n_h && items * hg < 8 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
     return hg;
 }
 
@@ -1163,30 +1103,21 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_kr128, m_qs3_32, m_dos3_32, m_kr8;
-    CUtensorMap m_kc3_128, m_v3_128, m_kc3_8, m_v3_8, m_qs3_64, m_dos3_64;
+    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_qs3_64, m_dos3_64, m_kr8, m_kc3_8, m_v3_8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     const void *qs = ws.qs, *dos = ws.dos;
-    if (p.N > 0 && q_rows > 0) {
-        if (!make_map3_bf16(&m_kc3_64, kc, kDC, kv_rows, 64) ||
-            !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
-            !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64) || !make_map3_bf16(&m_qs3_128, qs, kDQK, q_rows, 128) ||
-            !make_map3_bf16(&m_dos3_128, dos, kDV, q_rows, 128) || !make_map3_bf16(&m_qs3_32, qs, kDQK, q_rows, 32) ||
-            !make_map3_bf16(&m_dos3_32, dos, kDV, q_rows, 32) || !make_map3_bf16(&m_qs3_64, qs, kDQK, q_rows, 64) ||
-            !make_map3_bf16(&m_dos3_64, dos, kDV, q_rows, 64))
-            return cudaErrorInvalidValue;
-    }
-    if (!make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
-        !make_map3_bf16(&m_kc3_128, kc, kDC, kv_rows, 128) ||
-        !make_map_bf16(&m_kr128, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 128) ||
-        !make_map3_bf16(&m_v3_128, v, kDV, kv_rows, 128) || !make_map3_bf16(&m_kc3_8, kc, kDC, kv_rows, 8) ||
-        !make_map3_bf16(&m_v3_8, v, kDV, kv_rows, 8))
+    if (!make_map3_bf16(&m_kc3_64, kc, kDC, kv_rows, 64) ||
+        !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
+        !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64) ||
+        !make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
+        !make_map3_bf16(&m_kc3_8, kc, kDC, kv_rows, 8) || !make_map3_bf16(&m_v3_8, v, kDV, kv_rows, 8))
         return cudaErrorInvalidValue;
-    if (p.N == 0 || q_rows == 0) {  // maps over Q rows are never read: any valid map will do
-        m_qs3_32 = m_kc3_128;
-        m_dos3_32 = m_kc3_128;
-        m_qs3_64 = m_kc3_128;
-        m_dos3_64 = m_kc3_128;
+    if (p.N > 0 && q_rows > 0) {
+        if (!make_map3_bf16(&m_qs3_128, qs, kDQK, q_rows, 128) || !make_map3_bf16(&m_dos3_128, dos, kDV, q_rows, 128) ||
+            !make_map3_bf16(&m_qs3_64, qs, kDQK, q_rows, 64) || !make_map3_bf16(&m_dos3_64, dos, kDV, q_rows, 64))
+            return cudaErrorInvalidValue;
+    } else {  // maps over Q rows are never read: any valid map will do
+        m_qs3_128 = m_dos3_128 = m_qs3_64 = m_dos3_64 = m_kc3_64;
     }
     BwdArgs a;
     a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
@@ -1218,12 +1149,12 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
             m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_kc3_8, m_kr8, m_v3_8, a);
     }
-    const dim3 kv_grid(2 * (a.n_ctx_items + (p.N + kGD - 1) / kGD), HG, p.B);
+    const dim3 kv_grid(a.n_ctx_items + (p.N + kGD - 1) / kGD, HG, p.B);
     e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc3_128, m_kr128, m_v3_128, m_qs3_32, m_dos3_32,
-                                                        m_qs3_64, m_dos3_64, m_kc3_8, m_kr8, m_v3_8, a);
+    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kc3_8,
+                                                        m_kr8, m_v3_8, a);
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
     k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
