@@ -910,6 +910,41 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         const uint32_t pu0 = prow + ((((uint32_t)rb >> 3) ^ (kk & 7)) << 4);
         const uint32_t pu1 = prow + (((((uint32_t)rb >> 3) + 1) ^ (kk & 7)) << 4);
         uint8_t *stage = sm + oStage + warp * 2048;
+        uint32_t accp[64];  // a drained head's accumulator columns of this thread, bf16 pairs
+        bool pending = false;
+        int pend_hh = 0;
+        // Write a drained head's dK^C / dV columns: four rounds of 32 columns;
+        // each thread stages its 32 values (16-byte unit u at u ^ (lane & 3)),
+        // then the warp writes 8 rows' 64-byte segments per instruction. dK
+        // columns 192..255 (the rope slice) stay in TMEM, summed over heads.
+        auto store_head = [&](int hh2) {
+            const size_t bh = (size_t)b * p.n_h + h0 + hh2;
+#pragma unroll
+            for (int rd = 0; rd < 4; rd++) {
+                const int col = hr * 128 + rd * 32;
+                const bool rope = col >= kDC;
+#pragma unroll
+                for (int u = 0; u < 4; u++)
+                    *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
+                        make_uint4(accp[16 * rd + 4 * u], accp[16 * rd + 4 * u + 1], accp[16 * rd + 4 * u + 2],
+                                   accp[16 * rd + 4 * u + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
+                    const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
+                    const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
+                    const bool is_v = kl >= 16;
+                    if (kvl && (is_v || !rope)) {
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
+                        __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
+                                                  : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
+                        *reinterpret_cast<uint4 *>(dst) = val;
+                    }
+                }
+                __syncwarp();
+            }
+        };
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks, s = q & 1;
@@ -958,45 +993,30 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dsready);
+            if (pending) {  // the previous head's gradients, while this chunk's accumulation runs
+                store_head(pend_hh);
+                pending = false;
+            }
             if (c != nchunks - 1) continue;
-            // head epilogue, once its accumulations completed: accumulator
-            // columns [128 hr, 128 hr + 128); lanes 0-15 hold dK, 16-31 dV
+            // head end, once its accumulations completed: copy accumulator
+            // columns [128 hr, 128 hr + 128) (lanes 0-15 dK, 16-31 dV) to
+            // registers as bf16, which frees the accumulator for the next
+            // head; they are written out after the next chunk's P^T / dS^T.
             ok = warp_all(mbar_wait(ptfree, q & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            // Four rounds of 32 columns: each thread stages its 32 values
-            // (bf16, 16-byte unit u at u ^ (lane & 3)), then the warp writes 8
-            // rows' 64-byte segments per instruction.
 #pragma unroll
             for (int rd = 0; rd < 4; rd++) {
-                const int col = hr * 128 + rd * 32;
-                const bool rope = col >= kDC;  // dK columns 192..255 stay in TMEM (summed over heads)
-                tmem_ld32(trow + kColAcc + col, v);
+                tmem_ld32(trow + kColAcc + hr * 128 + rd * 32, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 4; u++)
-                    *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
-                        make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                                   pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
-                    const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
-                    const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
-                    const bool is_v = kl >= 16;
-                    if (kvl && (is_v || !rope)) {
-                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
-                        __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
-                                                  : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
-                        *reinterpret_cast<uint4 *>(dst) = val;
-                    }
-                }
-                __syncwarp();
+                for (int i = 0; i < 16; i++) accp[16 * rd + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
             }
             tc_fence_before();
+            pending = true;
+            pend_hh = hh;
         }
+        if (ok && pending) store_head(pend_hh);
         if (ok && hr == 1) {
             // rope slice of dK (columns 192..255 of the lanes 0-15), summed over
             // the group's heads by the MMAs
