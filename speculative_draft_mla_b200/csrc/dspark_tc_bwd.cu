@@ -575,7 +575,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
 // Key warps: warp w covers keys 16 (w & 3) .. + 15 (TMEM sub-partition w & 3)
 // and rows 32 (w >> 2) .. + 31 of a chunk. Lane l < 16 loads S^T of its key,
 // lane l + 16 dP^T of the same key; the two swap halves, so each lane holds
-// both for 16 rows.
+// both for 16 rows. At a head's end they copy the accumulators, as bf16, into
+// the 128 free TMEM columns (the stash), which frees them for the next head;
+// four store warps write the stash out to dK^C / dV while the next head runs.
 namespace kv {
 constexpr int kMK = 64;                    // keys per tile (MMA M)
 constexpr int kRC = 64;                    // rows per chunk (MMA N of S^T / dP^T, K of the accumulations)
@@ -589,15 +591,17 @@ constexpr int oKr = 0, oKc = oKr + kSlice, oV = oKc + 3 * kSlice;
 constexpr int kRowStage = 8 * kSlice;      // Q chunk (4 slices), then dO chunk (4 slices)
 constexpr int oRow = oV + 4 * kSlice;
 constexpr int oPT = oRow + 2 * kRowStage;  // P^T, then dS^T: [64 keys][64 rows] bf16 each
-constexpr int oStage = oPT + 2 * kSlice;   // epilogue staging, 2 KB per key warp
-constexpr int oMeta = oStage + 8 * 2048;   // per row stage: (LSE * log2 e, D) of each row
+constexpr int oStage = oPT + 2 * kSlice;   // epilogue staging, 2 KB per store warp
+constexpr int oMeta = oStage + 4 * 2048;   // per row stage: (LSE * log2 e, D) of each row
 constexpr int oBar = oMeta + 2 * kRC * 8;
-constexpr int kSmem = oBar + 128 + 1024;
+constexpr int kSmem = oBar + 256 + 1024;
 static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 constexpr int kKeyWarps = 8;
 constexpr int kWarpKV = kKeyWarps, kWarpRow = kKeyWarps + 1, kWarpMma = kKeyWarps + 2;
-constexpr int kThreads = (kKeyWarps + 3) * 32;
+constexpr int kWarpSt = kKeyWarps + 3;     // four store warps, one per TMEM sub-partition
+constexpr int kThreads = (kKeyWarps + 7) * 32;
 constexpr uint32_t kColAcc = 0, kColS = 256;  // S^T / dP^T buffer s at kColS + 64 s
+constexpr uint32_t kColStash = 384;           // a finished head's dK / dV as bf16 pairs (128 columns)
 constexpr uint32_t kHi = 16u << 16;           // lane offset of the second M = 64 accumulator
 }  // namespace kv
 
@@ -613,8 +617,9 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *rowfull = bars + 2, *rowfree = bars + 4, *sfull = bars + 6,
-             *dsready = bars + 8, *ptfree = bars + 9, *drain = bars + 10;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+             *dsready = bars + 8, *ptfree = bars + 9, *drain = bars + 10, *stashfull = bars + 11,
+             *stashfree = bars + 12;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     // K/V heads issued, row chunks issued, K/V heads consumed, row chunks consumed
     int *counters = reinterpret_cast<int *>(tmem_slot + 2);
@@ -670,7 +675,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     const bool dlane = lane >= 16;   // lane of the dP^T / dV half
     bool key_valid = false;
     size_t key_pos = 0;
-    if (warp < kKeyWarps) {
+    if (warp < kKeyWarps || warp >= kWarpSt) {
         if (is_ctx) {
             key_valid = t0 + kk < p.S;
             key_pos = (size_t)t0 + kk;
@@ -714,6 +719,8 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         mbar_init(dsready, kKeyWarps);
         mbar_init(ptfree, 1);
         mbar_init(drain, 1);
+        mbar_init(stashfull, kKeyWarps);
+        mbar_init(stashfree, 4);
         *abort_flag = 0;
         for (int c = 0; c < 4; c++) counters[c] = 0;
         fence_barrier_init();
@@ -875,6 +882,60 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 }
             }
         }
+    } else if (warp >= kWarpSt) {
+        // ------------------------------------------------ store warps
+        // Sub-partition warp & 3: keys 16 (warp & 3) .. + 15, lanes 0-15 their
+        // dK, lanes 16-31 their dV. Per head: the stash (128 columns of bf16
+        // pairs: accumulator columns 128 hr + 32 rd .. + 31 at stash column
+        // 64 hr + 16 rd) in eight rounds of 32 values; each thread stages its
+        // 64 bytes (16-byte unit u at u ^ (lane & 3)), then the warp writes 8
+        // rows' 64-byte segments per instruction. dK columns 192..255 (the
+        // rope slice) are not written: they stay in TMEM, summed over heads.
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        uint8_t *stage = sm + oStage + (warp - kWarpSt) * 2048;
+        for (int hh = 0; hh < H; ++hh) {
+            if (!warp_all(mbar_wait(stashfull, hh & 1, abort_flag))) break;
+            tc_fence_after();
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+#pragma unroll 1
+            for (int rr = 0; rr < 4; rr++) {
+                float v[32];
+                tmem_ld32(trow + kColStash + 32 * rr, v);
+                tmem_wait_ld();
+                if (rr == 3) {  // the stash is free for the next head
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(stashfree);
+                }
+#pragma unroll
+                for (int sub = 0; sub < 2; sub++) {
+                    const int col = (rr >> 1) * 128 + ((rr & 1) * 2 + sub) * 32;
+                    const bool rope = col >= kDC;
+#pragma unroll
+                    for (int u = 0; u < 4; u++)
+                        *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
+                            make_uint4(__float_as_uint(v[16 * sub + 4 * u]), __float_as_uint(v[16 * sub + 4 * u + 1]),
+                                       __float_as_uint(v[16 * sub + 4 * u + 2]),
+                                       __float_as_uint(v[16 * sub + 4 * u + 3]));
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
+                        const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
+                        const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
+                        const bool is_v = kl >= 16;
+                        if (kvl && (is_v || !rope)) {
+                            const uint4 val =
+                                *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
+                            __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
+                                                      : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
+                            *reinterpret_cast<uint4 *>(dst) = val;
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+        }
     } else {
         // ------------------------------------------ key warps (0..7)
         const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -909,42 +970,6 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         const uint32_t prow = (uint32_t)((kk >> 3) * 1024 + (kk & 7) * 128);
         const uint32_t pu0 = prow + ((((uint32_t)rb >> 3) ^ (kk & 7)) << 4);
         const uint32_t pu1 = prow + (((((uint32_t)rb >> 3) + 1) ^ (kk & 7)) << 4);
-        uint8_t *stage = sm + oStage + warp * 2048;
-        uint32_t accp[64];  // a drained head's accumulator columns of this thread, bf16 pairs
-        bool pending = false;
-        int pend_hh = 0;
-        // Write a drained head's dK^C / dV columns: four rounds of 32 columns;
-        // each thread stages its 32 values (16-byte unit u at u ^ (lane & 3)),
-        // then the warp writes 8 rows' 64-byte segments per instruction. dK
-        // columns 192..255 (the rope slice) stay in TMEM, summed over heads.
-        auto store_head = [&](int hh2) {
-            const size_t bh = (size_t)b * p.n_h + h0 + hh2;
-#pragma unroll
-            for (int rd = 0; rd < 4; rd++) {
-                const int col = hr * 128 + rd * 32;
-                const bool rope = col >= kDC;
-#pragma unroll
-                for (int u = 0; u < 4; u++)
-                    *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
-                        make_uint4(accp[16 * rd + 4 * u], accp[16 * rd + 4 * u + 1], accp[16 * rd + 4 * u + 2],
-                                   accp[16 * rd + 4 * u + 3]);
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
-                    const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
-                    const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
-                    const bool is_v = kl >= 16;
-                    if (kvl && (is_v || !rope)) {
-                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
-                        __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
-                                                  : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
-                        *reinterpret_cast<uint4 *>(dst) = val;
-                    }
-                }
-                __syncwarp();
-            }
-        };
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks, s = q & 1;
@@ -993,30 +1018,30 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dsready);
-            if (pending) {  // the previous head's gradients, while this chunk's accumulation runs
-                store_head(pend_hh);
-                pending = false;
-            }
             if (c != nchunks - 1) continue;
-            // head end, once its accumulations completed: copy accumulator
-            // columns [128 hr, 128 hr + 128) (lanes 0-15 dK, 16-31 dV) to
-            // registers as bf16, which frees the accumulator for the next
-            // head; they are written out after the next chunk's P^T / dS^T.
+            // head end, once its accumulations completed and the store warps
+            // have read the previous head's stash: accumulator columns
+            // [128 hr, 128 hr + 128) (lanes 0-15 dK, 16-31 dV) -> bf16 pairs in
+            // stash columns [64 hr, 64 hr + 64). The accumulator is then free
+            // for the next head.
             ok = warp_all(mbar_wait(ptfree, q & 1, abort_flag));
+            if (ok && hh >= 1) ok = warp_all(mbar_wait(stashfree, (hh - 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int rd = 0; rd < 4; rd++) {
                 tmem_ld32(trow + kColAcc + hr * 128 + rd * 32, v);
                 tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; i++) accp[16 * rd + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                for (int i = 0; i < 16; i++) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                tmem_st16u(trow + kColStash + hr * 64 + rd * 16, pk);
             }
+            tmem_wait_st();
             tc_fence_before();
-            pending = true;
-            pend_hh = hh;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stashfull);
         }
-        if (ok && pending) store_head(pend_hh);
         if (ok && hr == 1) {
             // rope slice of dK (columns 192..255 of the lanes 0-15), summed over
             // the group's heads by the MMAs
