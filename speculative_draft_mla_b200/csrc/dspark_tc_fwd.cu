@@ -1,42 +1,48 @@
 // Tensor-core (tcgen05 / TMEM / TMA) forward of the DSpark draft attention for
 // the page's head widths (d_c = 192, d_r = 64, d_v = 256), bf16.
 //
-// Work unit: one CTA per (batch b, head h, group of up to 25 kept blocks that
-// are consecutive in anchor order) = up to 125 query rows, the M = 128 of one
+// Work item: (batch b, head h, group of up to 25 kept blocks that are
+// consecutive in anchor order) = up to 125 query rows, the M = 128 of one
 // MMA. The group's key set is the union of its blocks' context windows,
 // [max(0, A_first - W + 1), A_last), walked in 64-key tiles, followed by the
 // group's own draft keys (5 per block) gathered into one or two more tiles.
 // Each row masks every key that is not in its own key set (page "GLM 5.2
 // DSpark speculative-training design", §3: window [A-W+1, A) shared by the 5
 // offsets, own block bidirectional, other blocks invisible). Because blocks
-// are sorted by anchor, neighbouring groups (adjacent blockIdx.x) read
-// overlapping windows close together in time, so the overlap is served by L2.
+// are sorted by anchor, neighbouring items read overlapping windows close
+// together in time, so the overlap is served by L2.
 //
-// The kernel is bound by how many key/value bytes each SM keeps in flight, so
-// shared memory holds only K and V stages (three each): Q lives in tensor
-// memory (A operand of S = Q K^T read from TMEM), and P is written over its
-// own S columns (A operand of O += P V read from TMEM). TMEM: O 0..255,
-// S 256..319 / 320..383, Q 384..511.
+// Persistent: one CTA per SM walks the items blockIdx.x, + gridDim.x, ...
+// K/V tiles, S buffers and pipeline phases are counted over all of a CTA's
+// items, so the K/V stream runs on across item boundaries; the next item's
+// raw Q rows are staged while the current item runs, moved into TMEM as soon
+// as its last QK has completed, and the finished item's O leaves TMEM through
+// the same staging area while the next item's first QK runs.
+// Q lives in tensor memory (A operand of S = Q K^T read from TMEM), and P is
+// written over its own S columns (A operand of O += P V read from TMEM).
+// TMEM: O 0..255, S 256..319 / 320..383, Q 384..511. Shared memory: two K
+// and two V stages, the 64 KB staging area, the softmax pair exchange.
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warps 0-7  softmax: warps w and w + 4 share TMEM sub-partition w % 4, so
 //              query rows 32 (w % 4) .. + 31 (thread = row = TMEM lane), and
 //              split each 64-key tile into two 32-column halves. They move
-//              the row's half of Q into TMEM (RoPE-rotating the rope slice)
-//              at the start, turn each S tile into P with an online softmax
-//              whose row max the pair exchanges through shared memory,
-//              rescale their half of the O row when the running max grows by
-//              more than 2^8, and write O and LSE.
-//   warp 8     K producer: the group's raw Q rows (one bulk copy per row),
-//              TMA loads of context K tiles (K^C as one 3-D box, plus the
-//              pre-rotated shared K^R) and of draft-key tiles (per block one
-//              3-D box of its 8 K^C rows and one of its K^R rows), L2
-//              prefetch of the K and V tiles three tiles ahead.
+//              the row's half of Q into TMEM (RoPE-rotating the rope slice),
+//              turn each S tile into P with an online softmax whose row max
+//              the pair exchanges through shared memory, rescale their half
+//              of the O row when the running max grows by more than 2^8, and
+//              write O and LSE.
+//   warp 8     K producer: TMA loads of context K tiles (K^C as one 3-D box,
+//              plus the pre-rotated shared K^R) and of draft-key tiles (per
+//              block one 3-D box of its 8 K^C rows and one of its K^R rows).
 //   warp 9     TMEM owner and MMA issuer (one thread): S = Q K^T into two
 //              alternating S buffers, O += P V, each issued as soon as its
 //              inputs are ready (an S buffer is reused only after the P V
-//              that reads the P written over it).
+//              that reads the P written over it; an item's first QK after
+//              its Q is in TMEM, its first P V after the previous item's O
+//              has been read out).
 //   warp 10    V producer.
+//   warp 11    raw Q loader (one bulk copy per block of 5 rows).
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait, TMEM is freed and the workspace error word gets kErrTimeout.
@@ -50,28 +56,31 @@ namespace {
 
 using namespace tc;
 
-constexpr int kG = 25;    // blocks per CTA
-constexpr int kM = 128;   // query rows per CTA (MMA M)
+constexpr int kG = 25;    // blocks per work item
+constexpr int kM = 128;   // query rows per work item (MMA M)
 constexpr int kBN = 64;   // keys per tile
 constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
 
 constexpr int kKChunk = kBN * 128;  // one 64-column slice of a K or V tile
 constexpr int kKBytes = 4 * kKChunk;
 constexpr int kVBytes = 4 * kKChunk;
-constexpr int kKS = 3, kVS = 3;     // K and V stages
+constexpr int kKS = 2, kVS = 2;     // K and V stages
 
-// Stage order K0 K1 V0 K2 V1 V2: the raw Q rows are staged over K2 and V1,
-// so the first two K tiles and the first V tile load while Q is moved.
-constexpr int oStage = 3 * kKBytes;
-constexpr int oX = 6 * kKBytes;  // pair exchange: tile max [2][2][128], row sum [2][128] (floats)
+// Shared memory: K0 K1 V0 V1, then the staging area (the next item's raw Q
+// rows; then, once they are in TMEM, the finished item's O rows on their way
+// to global memory), then the softmax pair exchange and the barriers.
+constexpr int oStage = 4 * kKBytes;
+constexpr int kStageBytes = 64 * 1024;
+constexpr int oX = oStage + kStageBytes;  // pair exchange: tile max [2][2][128], row sum [2][128] (floats)
 constexpr int oBar = oX + 3 * 1024;
-__device__ __forceinline__ int k_stage_off(int s) { return s == 0 ? 0 : (s == 1 ? kKBytes : 3 * kKBytes); }
-__device__ __forceinline__ int v_stage_off(int s) { return s == 0 ? 2 * kKBytes : (s == 1 ? 4 * kKBytes : 5 * kKBytes); }
+__device__ __forceinline__ int k_stage_off(int s) { return s * kKBytes; }
+__device__ __forceinline__ int v_stage_off(int s) { return (2 + s) * kKBytes; }
 // Raw Q: one bulk copy per block (5 rows of 512 B), blocks 2576 B apart, so
 // the rows that the threads of a warp read at once fall on at most 5 rows
 // per bank group.
 constexpr int kStageBlockPitch = kBlock * kDQK * 2 + 16;
-static_assert(kG * kStageBlockPitch <= 2 * kKBytes, "staging area too small");
+static_assert(kG * kStageBlockPitch <= kStageBytes, "staging area too small for raw Q");
+static_assert(8 * 32 * 256 <= kStageBytes, "staging area too small for O rows");
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 // Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
 // slices) at bb * 3 KB, its K^R rows at 24 KB + bb * 1 KB; its V rows (4 x 1 KB)
@@ -79,11 +88,13 @@ constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 // 64-column slices 1 KB apart and 8-key groups 4 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
+// barrier words: K and V full/empty per stage, 26 more, then 6 counters
+static_assert((2 * (kKS + kVS) + 26) * 8 + 6 * 4 <= 512, "barrier area too small");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 constexpr int kSoftWarps = 8;
-constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10;
-constexpr int kThreads = 352;
+constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10, kWarpQ = 11;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;  // two S buffers: 256..319, 320..383 (P over the first 16 columns of each half)
@@ -100,8 +111,44 @@ struct FwdArgs {
     __nv_bfloat16 *o;
     float *lse;
     uint32_t *err;
+    int n_groups;  // groups of kG blocks per batch row (work items per (b, h))
+    int n_items;   // n_groups * n_h * B
 };
 
+// Work item w = (group g, head h, batch b), g fastest (neighbouring items read
+// overlapping context windows of one head close together in time).
+struct Item {
+    int b, gcnt, nrows, ctx_lo, n_ctx, T;
+    size_t bh;
+    const int32_t *sa, *sn;
+};
+__device__ __forceinline__ bool item_at(const FwdArgs &p, int w, Item &it) {
+    const int g = w % p.n_groups, h = (w / p.n_groups) % p.n_h, b = w / (p.n_groups * p.n_h);
+    const int cnt = p.cnt[b];
+    const int i0 = g * kG;
+    if (i0 >= cnt) return false;  // this batch row has fewer groups
+    it.b = b;
+    it.gcnt = min(kG, cnt - i0);
+    it.nrows = kBlock * it.gcnt;
+    it.sa = p.sorted_a + (size_t)b * p.N + i0;
+    it.sn = p.sorted_n + (size_t)b * p.N + i0;
+    it.ctx_lo = max(0, it.sa[0] - p.W + 1);
+    const int ctx_hi = it.sa[it.gcnt - 1];
+    it.n_ctx = ctx_hi > it.ctx_lo ? (ctx_hi - it.ctx_lo + kBN - 1) / kBN : 0;
+    it.T = it.n_ctx + (it.gcnt + kDraftBlocksPerTile - 1) / kDraftBlocksPerTile;
+    it.bh = (size_t)b * p.n_h + h;
+    return true;
+}
+// The next valid item of this CTA at or after w (w advances by gridDim.x).
+__device__ __forceinline__ bool next_item(const FwdArgs &p, int &w, Item &it) {
+    for (; w < p.n_items; w += gridDim.x)
+        if (item_at(p, w, it)) return true;
+    return false;
+}
+
+// Persistent: one CTA per SM walks its work items (blockIdx.x, + gridDim.x,
+// ...). Tiles, S buffers and pipeline phases are counted over all of the
+// CTA's items, so K/V loads run on across item boundaries.
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc3, const __grid_constant__ CUtensorMap tm_kr,
              const __grid_constant__ CUtensorMap tm_v3, const __grid_constant__ CUtensorMap tm_kc38,
@@ -109,40 +156,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kfull = bars + 0, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 9;
-    uint64_t *sfull = bars + 12, *pready = bars + 14, *pvdone = bars + 16, *qready = bars + 18;
-    uint64_t *drain = bars + 19, *qraw = bars + 20, *qstaged = bars + 21;
+    uint64_t *kfull = bars, *kempty = kfull + kKS, *vfull = kempty + kKS, *vempty = vfull + kVS;
+    uint64_t *sfull = vempty + kVS, *pready = sfull + 2, *pvdone = sfull + 4;
+    // per item: raw Q landed, Q in TMEM, raw Q read (all softmax warps), O
+    // read out of TMEM, staging area free again
+    uint64_t *qraw = sfull + 6, *qready = sfull + 7, *qdone = sfull + 8, *ofree = sfull + 9, *stgfree = sfull + 10;
+    uint64_t *drain = sfull + 11;
     // softmax pair exchange: per TMEM sub-partition and S buffer the tile max,
     // per sub-partition the row sum (two arrivals each: one per warp)
-    uint64_t *xbar = bars + 22, *lbar = bars + 30;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 34);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 35);
+    uint64_t *xbar = sfull + 12, *lbar = sfull + 20;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + 24);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 25);
     // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
-    // [4] raw Q issued
-    int *counters = reinterpret_cast<int *>(bars + 36);
+    // [4] raw Q loads issued, [5] raw Q loads consumed
+    int *counters = reinterpret_cast<int *>(sfull + 26);
     float *xm = reinterpret_cast<float *>(sm + oX);         // [s][half][row]
     float *xl = reinterpret_cast<float *>(sm + oX + 2048);  // [half][row]
-
-    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int cnt = p.cnt[b];
-    const int i0 = g * kG;
-    if (i0 >= cnt) return;  // uniform: this batch row has fewer groups
-    const int gcnt = min(kG, cnt - i0);
-    const int nrows = kBlock * gcnt;
-    const int32_t *sa = p.sorted_a + (size_t)b * p.N + i0;
-    const int32_t *sn = p.sorted_n + (size_t)b * p.N + i0;
-    const int ctx_lo = max(0, sa[0] - p.W + 1);
-    const int ctx_hi = sa[gcnt - 1];
-    const int n_ctx = ctx_hi > ctx_lo ? (ctx_hi - ctx_lo + kBN - 1) / kBN : 0;
-    const int n_draft = (gcnt + kDraftBlocksPerTile - 1) / kDraftBlocksPerTile;
-    const int T = n_ctx + n_draft;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const size_t bh = (size_t)b * p.n_h + h;
 
     // K/V stages start zeroed: masked key slots of a tile are multiplied by a
-    // zero weight, and must not hold stale non-finite bits (the V stages then
-    // hold raw Q rows, finite, until V tiles overwrite them).
-    for (int e = threadIdx.x; e < oX / 16; e += blockDim.x)
+    // zero weight, and must not hold stale non-finite bits.
+    for (int e = threadIdx.x; e < oStage / 16; e += blockDim.x)
         reinterpret_cast<uint4 *>(sm)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKS; s++) {
@@ -158,14 +192,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&pready[s], kSoftWarps);
             mbar_init(&pvdone[s], 1);
         }
-        mbar_init(qready, kSoftWarps);
-        mbar_init(drain, 1);
         mbar_init(qraw, 1);
-        mbar_init(qstaged, kSoftWarps);
+        mbar_init(qready, kSoftWarps);
+        mbar_init(qdone, kSoftWarps);
+        mbar_init(ofree, kSoftWarps);
+        mbar_init(stgfree, kSoftWarps);
+        mbar_init(drain, 1);
         for (int i = 0; i < 8; i++) mbar_init(&xbar[i], 2);
         for (int i = 0; i < 4; i++) mbar_init(&lbar[i], 2);
         *abort_flag = 0;
-        for (int c = 0; c < 5; c++) counters[c] = 0;
+        for (int c = 0; c < 6; c++) counters[c] = 0;
         fence_barrier_init();
     }
     if (warp == kWarpMma) {
@@ -180,115 +216,90 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kWarpK || warp == kWarpV) {
         // ------------------------------------------------------ producers
-        // lane l holds the block index of group block l
-        const int my_n = lane < gcnt ? sn[lane] : 0;
-        if (warp == kWarpK) {
-            if (lane == 0) {
-                tma_prefetch_desc(&tm_kc3);
-                tma_prefetch_desc(&tm_kr);
-                tma_prefetch_desc(&tm_v3);
-                // raw Q rows of the group: each block's 5 rows are one
-                // contiguous 2560-byte run
-                mbar_arrive_expect_tx(qraw, nrows * kDQK * 2);
-                counters[4] = 1;
-            }
-            __syncwarp();
-            if (lane < gcnt)
-                bulk_load(sm + oStage + lane * kStageBlockPitch, p.q + (bh * p.R + (size_t)kBlock * my_n) * kDQK,
-                          kBlock * kDQK * 2, qraw);
-            // L2 prefetch of tile tt's K and V (context rows, or the 8-row
-            // boxes of the draft tile's blocks, one block per lane)
-            auto prefetch_tile = [&](int tt) {
-                if (tt < n_ctx) {
-                    if (lane == 0) {
-                        const int pos = ctx_lo + tt * kBN;
-                        tma_prefetch_3d(&tm_kc3, 0, (int)(bh * p.L + pos), 0);
-                        tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
-                        tma_prefetch_3d(&tm_v3, 0, (int)(bh * p.L + pos), 0);
-                    }
-                } else {
-                    const int d = tt - n_ctx;
-                    const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
-                    const int n = __shfl_sync(0xffffffffu, my_n, (d * kDraftBlocksPerTile + lane) & 31);
-                    if (lane < nb) {
-                        const int row = p.S + kBlock * n;
-                        tma_prefetch_3d(&tm_kc38, 0, (int)(bh * p.L + row), 0);
-                        tma_prefetch_2d(&tm_kr8, 0, (int)((size_t)b * p.L + row));
-                        tma_prefetch_3d(&tm_v38, 0, (int)(bh * p.L + row), 0);
-                    }
+        const bool isk = warp == kWarpK;
+        if (isk && lane == 0) {
+            tma_prefetch_desc(&tm_kc3);
+            tma_prefetch_desc(&tm_kr);
+            tma_prefetch_desc(&tm_v3);
+        }
+        int tt = 0;  // tiles over all items
+        bool ok = true;
+        Item it;
+        for (int w = blockIdx.x; ok && next_item(p, w, it); w += gridDim.x) {
+            // lane l holds the block index of group block l
+            const int my_n = lane < it.gcnt ? it.sn[lane] : 0;
+            for (int t = 0; t < it.T; ++t, ++tt) {
+                const int nst = isk ? kKS : kVS;
+                const int s = tt % nst;
+                if (tt >= nst && !warp_all(mbar_wait(isk ? &kempty[s] : &vempty[s], ((tt / nst) - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
                 }
-            };
-            int pf_next = kKS;  // next tile to prefetch into L2
-            for (int t = 0; t < T; ++t) {
-                const int s = t % kKS;
-                uint8_t *kt = sm + k_stage_off(s);
-                for (; pf_next <= t + kKS && pf_next < T; ++pf_next) prefetch_tile(pf_next);
-                // the third K stage holds raw Q rows until they are in TMEM
-                if (t == 2 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
-                if (t >= kKS && !warp_all(mbar_wait(&kempty[s], ((t / kKS) - 1) & 1, abort_flag))) break;
-                if (t < n_ctx) {
-                    const int pos0 = ctx_lo + t * kBN;
+                uint64_t *full = isk ? &kfull[s] : &vfull[s];
+                uint8_t *dst = sm + (isk ? k_stage_off(s) : v_stage_off(s));
+                if (t < it.n_ctx) {
+                    const int pos0 = it.ctx_lo + t * kBN;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&kfull[s], kKBytes);
-                        tma_load_3d(kt, &tm_kc3, &kfull[s], 0, (int)(bh * p.L + pos0), 0);
-                        tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[s], 0, (int)((size_t)b * p.L + pos0));
+                        if (isk) {
+                            mbar_arrive_expect_tx(full, kKBytes);
+                            tma_load_3d(dst, &tm_kc3, full, 0, (int)(it.bh * p.L + pos0), 0);
+                            tma_load_2d(dst + 3 * kKChunk, &tm_kr, full, 0, (int)((size_t)it.b * p.L + pos0));
+                        } else {
+                            mbar_arrive_expect_tx(full, kVBytes);
+                            tma_load_3d(dst, &tm_v3, full, 0, (int)(it.bh * p.L + pos0), 0);
+                        }
                     }
                 } else {
                     // draft tile: 8 key slots per block, its 5 keys first (the 3
                     // rows after them are other keys, masked out)
-                    const int d = t - n_ctx;
-                    const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
-                    if (lane == 0) mbar_arrive_expect_tx(&kfull[s], nb * 8 * kDQK * 2);
+                    const int d = t - it.n_ctx;
+                    const int nb = min(kDraftBlocksPerTile, it.gcnt - d * kDraftBlocksPerTile);
+                    if (lane == 0) mbar_arrive_expect_tx(full, nb * 8 * (isk ? kDQK : kDV) * 2);
                     __syncwarp();
                     for (int bb = 0; bb < nb; ++bb) {
                         const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
                         if (lane == 0) {
                             const int row = p.S + kBlock * n;
-                            tma_load_3d(kt + bb * kDraftKcBlock, &tm_kc38, &kfull[s], 0, (int)(bh * p.L + row), 0);
-                            tma_load_2d(kt + kDraftKr + bb * 1024, &tm_kr8, &kfull[s], 0, (int)((size_t)b * p.L + row));
+                            if (isk) {
+                                tma_load_3d(dst + bb * kDraftKcBlock, &tm_kc38, full, 0, (int)(it.bh * p.L + row), 0);
+                                tma_load_2d(dst + kDraftKr + bb * 1024, &tm_kr8, full, 0,
+                                            (int)((size_t)it.b * p.L + row));
+                            } else {
+                                tma_load_3d(dst + bb * kDraftVBlock, &tm_v38, full, 0, (int)(it.bh * p.L + row), 0);
+                            }
                         }
                     }
                 }
-                if (lane == 0) counters[0] = t + 1;
+                if (lane == 0) counters[isk ? 0 : 1] = tt + 1;
             }
-        } else {
-            for (int t = 0; t < T; ++t) {
-                const int s = t % kVS;
-                uint8_t *vt = sm + v_stage_off(s);
-                // the second V stage holds raw Q rows until they are in TMEM
-                if (t == 1 && !warp_all(mbar_wait(qstaged, 0, abort_flag))) break;
-                if (t >= kVS && !warp_all(mbar_wait(&vempty[s], ((t / kVS) - 1) & 1, abort_flag))) break;
-                if (t < n_ctx) {
-                    const int pos0 = ctx_lo + t * kBN;
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&vfull[s], kVBytes);
-                        tma_load_3d(vt, &tm_v3, &vfull[s], 0, (int)(bh * p.L + pos0), 0);
-                    }
-                } else {
-                    const int d = t - n_ctx;
-                    const int nb = min(kDraftBlocksPerTile, gcnt - d * kDraftBlocksPerTile);
-                    if (lane == 0) mbar_arrive_expect_tx(&vfull[s], nb * 8 * kDV * 2);
-                    __syncwarp();
-                    for (int bb = 0; bb < nb; ++bb) {
-                        const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocksPerTile + bb);
-                        if (lane == 0) {
-                            const int row = p.S + kBlock * n;
-                            tma_load_3d(vt + bb * kDraftVBlock, &tm_v38, &vfull[s], 0, (int)(bh * p.L + row), 0);
-                        }
-                    }
-                }
-                if (lane == 0) counters[1] = t + 1;
+        }
+    } else if (warp == kWarpQ) {
+        // -------------------------------------------------- raw Q loader
+        // Item ic's raw Q rows go to the staging area once it is free: after
+        // item 0's Q is in TMEM (ic = 1), else after item ic - 2's O rows left.
+        int ic = 0;
+        Item it;
+        for (int w = blockIdx.x; next_item(p, w, it); w += gridDim.x, ++ic) {
+            if (ic >= 1 && !warp_all(mbar_wait(stgfree, (ic - 1) & 1, abort_flag))) break;
+            const int my_n = lane < it.gcnt ? it.sn[lane] : 0;
+            if (lane == 0) {
+                // each block's 5 rows are one contiguous 2560-byte run
+                mbar_arrive_expect_tx(qraw, it.nrows * kDQK * 2);
+                counters[4] = ic + 1;
             }
+            __syncwarp();
+            if (lane < it.gcnt)
+                bulk_load(sm + oStage + lane * kStageBlockPitch, p.q + (it.bh * p.R + (size_t)kBlock * my_n) * kDQK,
+                          kBlock * kDQK * 2, qraw);
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(kM, kBN, 0);
             const uint32_t idO = idesc_bf16(kM, kDV, 1);
-            bool ok = mbar_wait(qready, 0, abort_flag);
-            auto issue_qk = [&](int t) {
-                const int s = t & 1;
-                const uint32_t kb = smem_u32(sm + k_stage_off(t % kKS));
+            auto issue_qk = [&](int tg, int t, int n_ctx) {
+                const int s = tg & 1;
+                const uint32_t kb = smem_u32(sm + k_stage_off(tg % kKS));
                 const uint32_t dS = tmem + kColS + s * kBN;
                 if (t < n_ctx) {
                     const SDesc kd = sdesc_split(sdesc_sw128(kb, 16, 1024));
@@ -310,48 +321,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16_ts(dS, tmem + kColQ + 8 * k, kdr.at(((k & 3) * 32) >> 4), idS, 1u);
                 }
                 mma_commit(&sfull[s]);
-                mma_commit(&kempty[t % kKS]);
-                counters[2] = t + 1;
+                mma_commit(&kempty[tg % kKS]);
+                counters[2] = tg + 1;
             };
-            auto issue_pv = [&](int t) {
-                const int s = t & 1;
-                const uint32_t vb = smem_u32(sm + v_stage_off(t % kVS));
+            auto issue_pv = [&](int tg, int t, int n_ctx) {
+                const int s = tg & 1;
+                const uint32_t vb = smem_u32(sm + v_stage_off(tg % kVS));
                 const bool ctx = t < n_ctx;
                 // context tile: 64-column slices 8 KB apart, keys 128 B apart;
                 // draft tile: slices 1 KB apart, 8-key groups 4 KB apart
                 const SDesc vd = sdesc_split(ctx ? sdesc_sw128(vb, kKChunk, 1024) : sdesc_sw128(vb, 1024, kDraftVBlock));
                 const uint32_t kstep = ctx ? 128u : 512u;  // 16 keys, in 16-byte units
                 // P of keys 16 k .. 16 k + 15: half k / 2 of the S buffer, its
-                // columns 8 (k % 2) ..
+                // columns 8 (k % 2) ..; the item's first tile overwrites O
                 const uint32_t pa = tmem + kColS + s * kBN;
                 mma_bf16_ts(tmem + kColO, pa, vd.at(0), idO, t > 0 ? 1u : 0u);
                 mma_bf16_ts(tmem + kColO, pa + 8, vd.at(kstep), idO, 1u);
                 mma_bf16_ts(tmem + kColO, pa + 32, vd.at(2 * kstep), idO, 1u);
                 mma_bf16_ts(tmem + kColO, pa + 40, vd.at(3 * kstep), idO, 1u);
-                mma_commit(&vempty[t % kVS]);
+                mma_commit(&vempty[tg % kVS]);
                 mma_commit(&pvdone[s]);
             };
-            // Issue whichever is ready: QK of tile nk (its K landed, and the
-            // P V of tile nk - 2 that reads the P written over its S buffer
-            // is already issued) or P V of tile np (its P is in TMEM and its
-            // V landed).
-            int nk = 0, np = 0;
+            // Two cursors over the CTA's items: QK of tile nk (item icK, local
+            // tile tK) and P V of tile np (item icP, local tile tP). Issue
+            // whichever is ready: QK when its K landed, the P V that reads the
+            // P written over its S buffer (tile nk - 2) is issued and, at an
+            // item's first tile, the item's Q is in TMEM; P V when its P is in
+            // TMEM and its V landed and, at an item's first tile, the previous
+            // item's O has been read out.
+            Item ik, ip;
+            int wk = blockIdx.x, wp = blockIdx.x;
+            bool hk = next_item(p, wk, ik), hp = next_item(p, wp, ip);
+            int nk = 0, np = 0, icK = 0, icP = 0, tK = 0, tP = 0;
+            bool ok = true;
             uint64_t t_idle = 0;
-            if (ok) tc_fence_after();
-            while (ok && np < T) {
+            while (ok && hp) {
                 bool issued = false;
-                if (nk < T && np >= nk - 1 && mbar_test(&kfull[nk % kKS], (nk / kKS) & 1)) {
+                if (hk && np >= nk - 1 && mbar_test(&kfull[nk % kKS], (nk / kKS) & 1) &&
+                    (tK != 0 || mbar_test(qready, icK & 1))) {
                     tc_fence_after();
-                    issue_qk(nk);
+                    issue_qk(nk, tK, ik.n_ctx);
                     ++nk;
+                    if (++tK == ik.T) {
+                        tK = 0;
+                        ++icK;
+                        wk += gridDim.x;
+                        hk = next_item(p, wk, ik);
+                    }
                     issued = true;
                 }
                 if (!issued && np < nk && mbar_test(&pready[np & 1], (np >> 1) & 1) &&
-                    mbar_test(&vfull[np % kVS], (np / kVS) & 1)) {
+                    mbar_test(&vfull[np % kVS], (np / kVS) & 1) && (tP != 0 || icP == 0 || mbar_test(ofree, (icP - 1) & 1))) {
                     counters[3] = np + 1;
                     tc_fence_after();
-                    issue_pv(np);
+                    issue_pv(np, tP, ip.n_ctx);
                     ++np;
+                    if (++tP == ip.T) {
+                        tP = 0;
+                        ++icP;
+                        wp += gridDim.x;
+                        hp = next_item(p, wp, ip);
+                    }
                     issued = true;
                 }
                 if (issued) {
@@ -367,32 +397,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else {
+    } else if (warp < kSoftWarps) {
         // ------------------------------------------------ softmax (rows)
         const int q4 = warp & 3, hf = warp >> 2;  // TMEM sub-partition, column half
         const int r = q4 * 32 + lane;               // query row = TMEM lane
-        const bool live = r < nrows;
-        int A = 0, n = 0, j = 0, lo = 0;
-        if (live) {
-            A = sa[r / kBlock];
-            n = sn[r / kBlock];
-            j = r % kBlock;
-            lo = max(0, A - p.W + 1);
-        }
-        bool ok = true;
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
-        {
-            // Q row r, this thread's half (columns 128 hf .. + 127) -> TMEM
-            // lane r, columns kColQ + 64 hf .. + 63; the rope slice (the last
-            // 64 columns, half 1) is rotated to position A + j first. Rows
-            // past the group are zero.
+        bool ok = true;
+        // Q row r of an item, this thread's half (columns 128 hf .. + 127),
+        // from the staging area -> TMEM lane r, columns kColQ + 64 hf .. + 63;
+        // the rope slice (the last 64 columns, half 1) is rotated to position
+        // A + j first. Rows past the item's blocks are zero.
+        auto move_q = [&](const Item &q_it, int ic) {
+            const bool live = r < q_it.nrows;
             float4 cs[16];  // (cos, sin) of the 32 rope frequencies at A + j (half 1)
             if (hf == 1) {
-                const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)(live ? A + j : 0) * (kDR / 2));
+                const int pos = live ? q_it.sa[r / kBlock] + r % kBlock : 0;
+                const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)pos * (kDR / 2));
 #pragma unroll
                 for (int k = 0; k < 16; k++) cs[k] = __ldg(tp + k);
             }
-            ok = warp_all(mbar_wait(qraw, 0, abort_flag));
+            ok = warp_all(mbar_wait(qraw, ic & 1, abort_flag));
+            if (ok && threadIdx.x == 0) counters[5] = ic + 1;
             const bool have = live && ok;
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + (r / kBlock) * kStageBlockPitch +
                                                                (r % kBlock) * (kDQK * 2) + hf * 256);
@@ -422,127 +447,155 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(qstaged);  // staging area free for V tiles
-                mbar_arrive(qready);
-            }
-        }
+            if (lane == 0) mbar_arrive(qready);
+        };
 
-        float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
-        for (int t = 0; t < T && ok; ++t) {
-            const int s = t & 1;
-            ok = warp_all(mbar_wait(&sfull[s], (t >> 1) & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            // every row's keys in a tile form one contiguous column range
-            // [clo, chi): the window [lo, A) for context tiles, its block's 5
-            // key slots for draft tiles; this warp holds columns 32 hf .. +31
-            int clo, chi;
-            if (t < n_ctx) {
-                const int c0 = ctx_lo + t * kBN;
-                clo = lo - c0;
-                chi = A - c0;
-            } else {
-                clo = 8 * (r / kBlock) - (t - n_ctx) * kBN;
-                chi = clo + kBlock;
-            }
-            if (!live) chi = clo;
-            clo -= 32 * hf;
-            chi -= 32 * hf;
-            // Rows are anchor-sorted, so for most (warp, half tile) pairs no
-            // row of the warp sees any of the 32 keys: such a half tile only
-            // contributes P = 0 (uniform over the warp, no S read).
-            const bool act = __any_sync(0xffffffffu, clo < chi && clo < 32 && chi > 0);
-            float sv[32];
-            float mx[4];
-#pragma unroll
-            for (int k = 0; k < 4; k++) mx[k] = -INFINITY;
-            if (act) {
-                tmem_ld32(trow + kColS + s * kBN + 32 * hf, sv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; c++) {
-                    sv[c] = (c >= clo && c < chi) ? sv[c] : -INFINITY;
-                    mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
-                }
-            }
-            // the pair's tile max, exchanged through shared memory
-            const float mhalf = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            xm[(s * 2 + hf) * kM + r] = mhalf;
+        int tg = 0;  // tiles over all items
+        int ic = 0;
+        Item it, nx;
+        int w = blockIdx.x;
+        bool has = next_item(p, w, it);
+        if (has) {
+            move_q(it, 0);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&xbar[2 * q4 + s]);
-            ok = warp_all(mbar_wait(&xbar[2 * q4 + s], (t >> 1) & 1, abort_flag));
-            if (!ok) break;
-            const float mother = xm[(s * 2 + (hf ^ 1)) * kM + r];
-            const float mt = fmaxf(mhalf, mother) * p.scale_log2;
-            bool resc = false;
-            float alpha = 1.f;
-            if (mt > m_used + kRescaleThreshold) {
-                if (m_used != -INFINITY) {
-                    resc = true;
-                    alpha = ex2(m_used - mt);
-                }
-                m_used = mt;
+            if (lane == 0) mbar_arrive(stgfree);  // item 1's raw Q may load
+        }
+        while (ok && has) {
+            const bool live = r < it.nrows;
+            int A = 0, n = 0, j = 0, lo = 0;
+            if (live) {
+                A = it.sa[r / kBlock];
+                n = it.sn[r / kBlock];
+                j = r % kBlock;
+                lo = max(0, A - p.W + 1);
             }
-            float psum[4];
-#pragma unroll
-            for (int k = 0; k < 4; k++) psum[k] = 0.f;
-            const bool any = m_used != -INFINITY;
-            const float mneg = any ? -m_used : 0.f;
-            uint32_t pw[16];  // this half's 32 P values as bf16 pairs
-            if (act) {
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float e0 = any ? ex2(fmaf(sv[c], p.scale_log2, mneg)) : 0.f;
-                    const float e1 = any ? ex2(fmaf(sv[c + 1], p.scale_log2, mneg)) : 0.f;
-                    psum[c & 3] += e0;
-                    psum[(c + 1) & 3] += e1;
-                    pw[c / 2] = pack_bf16x2(e0, e1);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 16; c++) pw[c] = 0u;
-            }
-            // P over this half's first 16 S columns (the S values are in registers)
-            tmem_st16u(trow + kColS + s * kBN + 32 * hf, pw);
-            l = l * alpha + ((psum[0] + psum[1]) + (psum[2] + psum[3]));
-            if (__any_sync(0xffffffffu, resc)) {
-                if (t >= 1) {
-                    ok = warp_all(mbar_wait(&pvdone[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag));
-                    if (!ok) break;
-                }
+            float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
+            for (int t = 0; t < it.T && ok; ++t, ++tg) {
+                const int s = tg & 1;
+                ok = warp_all(mbar_wait(&sfull[s], (tg >> 1) & 1, abort_flag));
+                if (!ok) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 128 * hf; c < 128 * hf + 128; c += 32) {  // this half's O columns
-                    float ov[32];
-                    tmem_ld32(trow + kColO + c, ov);
+                // every row's keys in a tile form one contiguous column range
+                // [clo, chi): the window [lo, A) for context tiles, its block's 5
+                // key slots for draft tiles; this warp holds columns 32 hf .. +31
+                int clo, chi;
+                if (t < it.n_ctx) {
+                    const int c0 = it.ctx_lo + t * kBN;
+                    clo = lo - c0;
+                    chi = A - c0;
+                } else {
+                    clo = 8 * (r / kBlock) - (t - it.n_ctx) * kBN;
+                    chi = clo + kBlock;
+                }
+                if (!live) chi = clo;
+                clo -= 32 * hf;
+                chi -= 32 * hf;
+                // Rows are anchor-sorted, so for most (warp, half tile) pairs no
+                // row of the warp sees any of the 32 keys: such a half tile only
+                // contributes P = 0 (uniform over the warp, no S read).
+                const bool act = __any_sync(0xffffffffu, clo < chi && clo < 32 && chi > 0);
+                float sv[32];
+                float mx[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) mx[k] = -INFINITY;
+                if (act) {
+                    tmem_ld32(trow + kColS + s * kBN + 32 * hf, sv);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; i++) ov[i] *= alpha;
-                    tmem_st32(trow + kColO + c, ov);
+                    for (int c = 0; c < 32; c++) {
+                        sv[c] = (c >= clo && c < chi) ? sv[c] : -INFINITY;
+                        mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+                    }
                 }
+                // the pair's tile max, exchanged through shared memory
+                const float mhalf = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                xm[(s * 2 + hf) * kM + r] = mhalf;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xbar[2 * q4 + s]);
+                ok = warp_all(mbar_wait(&xbar[2 * q4 + s], (tg >> 1) & 1, abort_flag));
+                if (!ok) break;
+                const float mother = xm[(s * 2 + (hf ^ 1)) * kM + r];
+                const float mt = fmaxf(mhalf, mother) * p.scale_log2;
+                bool resc = false;
+                float alpha = 1.f;
+                if (mt > m_used + kRescaleThreshold) {
+                    if (m_used != -INFINITY) {
+                        resc = true;
+                        alpha = ex2(m_used - mt);
+                    }
+                    m_used = mt;
+                }
+                float psum[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) psum[k] = 0.f;
+                const bool any = m_used != -INFINITY;
+                const float mneg = any ? -m_used : 0.f;
+                uint32_t pw[16];  // this half's 32 P values as bf16 pairs
+                if (act) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        const float e0 = any ? ex2(fmaf(sv[c], p.scale_log2, mneg)) : 0.f;
+                        const float e1 = any ? ex2(fmaf(sv[c + 1], p.scale_log2, mneg)) : 0.f;
+                        psum[c & 3] += e0;
+                        psum[(c + 1) & 3] += e1;
+                        pw[c / 2] = pack_bf16x2(e0, e1);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; c++) pw[c] = 0u;
+                }
+                // P over this half's first 16 S columns (the S values are in registers)
+                tmem_st16u(trow + kColS + s * kBN + 32 * hf, pw);
+                l = l * alpha + ((psum[0] + psum[1]) + (psum[2] + psum[3]));
+                if (__any_sync(0xffffffffu, resc)) {
+                    // (never at an item's first tile: m_used starts at -inf)
+                    ok = warp_all(mbar_wait(&pvdone[(tg - 1) & 1], ((tg - 1) >> 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 128 * hf; c < 128 * hf + 128; c += 32) {  // this half's O columns
+                        float ov[32];
+                        tmem_ld32(trow + kColO + c, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; i++) ov[i] *= alpha;
+                        tmem_st32(trow + kColO + c, ov);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pready[s]);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&pready[s]);
-        }
-        if (ok) ok = warp_all(mbar_wait(&pvdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
-        if (ok) {
-            // the row sum: both halves' shares, exchanged like the tile max
-            xl[hf * kM + r] = l;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&lbar[q4]);
-            ok = warp_all(mbar_wait(&lbar[q4], 0, abort_flag));
-        }
-        if (ok) {
+            if (!ok) break;
+            // The next item's Q into TMEM (its raw rows are staged; every QK of
+            // this item has completed, as all its S tiles have been read), so
+            // that its QK can start while this item's O is written out.
+            int wn = w + gridDim.x;
+            const bool hasn = next_item(p, wn, nx);
+            if (hasn) {
+                move_q(nx, ic + 1);
+                if (!ok) break;
+                if (lane == 0) mbar_arrive(qdone);
+            }
+            ok = warp_all(mbar_wait(&pvdone[(tg - 1) & 1], ((tg - 1) >> 1) & 1, abort_flag));
+            if (ok) {
+                // the row sum: both halves' shares, exchanged like the tile max
+                xl[hf * kM + r] = l;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&lbar[q4]);
+                ok = warp_all(mbar_wait(&lbar[q4], ic & 1, abort_flag));
+            }
+            // the staging area: every warp has read the next item's raw Q rows
+            if (ok && hasn) ok = warp_all(mbar_wait(qdone, ic & 1, abort_flag));
+            if (!ok) break;
             tc_fence_after();
             const float ltot = l + xl[(hf ^ 1) * kM + r];
             const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-            // this half of the O row (columns 128 hf .. +127) -> staging in the
-            // idle K0, K1 stages (row i of the warp at 256 i, unit u at
-            // u ^ (i & 15)) -> two half rows per warp instruction
-            uint8_t *stage = sm + warp * (32 * 256);
+            // this half of the O row (columns 128 hf .. +127) -> staging (row i
+            // of the warp at 256 i, unit u at u ^ (i & 15)) -> two half rows
+            // per warp instruction
+            uint8_t *stage = sm + oStage + warp * (32 * 256);
 #pragma unroll 1
             for (int c = 0; c < 128; c += 32) {
                 float ov[32];
@@ -558,17 +611,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
                 }
             }
+            // O is out of TMEM: the next item's first P V may overwrite it
+            tc_fence_before();
             __syncwarp();
+            if (lane == 0) mbar_arrive(ofree);
             for (int i = 0; i < 16; i++) {
                 const int wr = 2 * i + (lane >> 4), u = lane & 15;  // row within the warp, unit
                 const int rr = q4 * 32 + wr;
                 const int ni = __shfl_sync(0xffffffffu, n, wr), ji = __shfl_sync(0xffffffffu, j, wr);
-                if (rr < nrows) {
+                if (rr < it.nrows) {
                     const uint4 val = *reinterpret_cast<const uint4 *>(stage + wr * 256 + ((u ^ (wr & 15)) << 4));
-                    *reinterpret_cast<uint4 *>(p.o + (bh * p.R + kBlock * ni + ji) * kDV + 128 * hf + 8 * u) = val;
+                    *reinterpret_cast<uint4 *>(p.o + (it.bh * p.R + kBlock * ni + ji) * kDV + 128 * hf + 8 * u) = val;
                 }
             }
-            if (live && hf == 0) p.lse[bh * p.R + kBlock * n + j] = (m_used + log2f(ltot)) * kLn2;
+            if (live && hf == 0) p.lse[it.bh * p.R + kBlock * n + j] = (m_used + log2f(ltot)) * kLn2;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stgfree);  // the raw Q of the item after next may load
+            ++ic;
+            w = wn;
+            it = nx;
+            has = hasn;
         }
     }
 
@@ -578,12 +640,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Drain what may still be in flight, each wait bounded on its own.
         volatile int never = 0;
         if (warp == kWarpK && lane == 0) {
-            if (counters[4]) mbar_wait(qraw, 0, (volatile int *)&never);
             // loads issued but not yet consumed complete in order, one phase each
             for (int t = counters[2]; t < counters[0]; ++t)
                 mbar_wait(&kfull[t % kKS], (t / kKS) & 1, (volatile int *)&never);
             for (int t = counters[3]; t < counters[1]; ++t)
                 mbar_wait(&vfull[t % kVS], (t / kVS) & 1, (volatile int *)&never);
+            for (int t = counters[5]; t < counters[4]; ++t) mbar_wait(qraw, t & 1, (volatile int *)&never);
         }
         if (warp == kWarpMma && lane == 0) {
             mma_commit(drain);
@@ -649,9 +711,13 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.o = (__nv_bfloat16 *)o;
     a.lse = lse;
     a.err = ws.err;
-    dim3 grid((p.N + kG - 1) / kG, p.n_h, p.B);
+    a.n_groups = (p.N + kG - 1) / kG;
+    a.n_items = a.n_groups * p.n_h * p.B;
+    int dev = 0, nsm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     count_launch();
-    k_fwd_tc<<<grid, kThreads, kSmemBytes, st>>>(m_kc3, m_kr, m_v3, m_kc38, m_kr8, m_v38, a);
+    k_fwd_tc<<<std::min(a.n_items, nsm), kThreads, kSmemBytes, st>>>(m_kc3, m_kr, m_v3, m_kc38, m_kr8, m_v38, a);
     return cudaGetLastError();
 }
 
