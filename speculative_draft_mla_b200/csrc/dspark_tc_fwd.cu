@@ -88,8 +88,8 @@ constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 // 64-column slices 1 KB apart and 8-key groups 4 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
-// barrier words: K and V full/empty per stage, 26 more, then 6 counters
-static_assert((2 * (kKS + kVS) + 26) * 8 + 6 * 4 <= 512, "barrier area too small");
+// barrier words: K and V full/empty per stage, 28 more, then 6 counters
+static_assert((2 * (kKS + kVS) + 28) * 8 + 6 * 4 <= 512, "barrier area too small");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 constexpr int kSoftWarps = 8;
@@ -161,7 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // per item: raw Q landed, Q in TMEM, raw Q read (all softmax warps), O
     // read out of TMEM, staging area free again
     uint64_t *qraw = sfull + 6, *qready = sfull + 7, *qdone = sfull + 8, *ofree = sfull + 9, *stgfree = sfull + 10;
-    uint64_t *drain = sfull + 11;
+    // per item: O rows staged (softmax warps), O rows read out (loader warp)
+    uint64_t *drain = sfull + 11, *ostaged = sfull + 26, *oread = sfull + 27;
     // softmax pair exchange: per TMEM sub-partition and S buffer the tile max,
     // per sub-partition the row sum (two arrivals each: one per warp)
     uint64_t *xbar = sfull + 12, *lbar = sfull + 20;
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 25);
     // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
     // [4] raw Q loads issued, [5] raw Q loads consumed
-    int *counters = reinterpret_cast<int *>(sfull + 26);
+    int *counters = reinterpret_cast<int *>(sfull + 28);
     float *xm = reinterpret_cast<float *>(sm + oX);         // [s][half][row]
     float *xl = reinterpret_cast<float *>(sm + oX + 2048);  // [half][row]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(qdone, kSoftWarps);
         mbar_init(ofree, kSoftWarps);
         mbar_init(stgfree, kSoftWarps);
+        mbar_init(ostaged, kSoftWarps);
+        mbar_init(oread, 1);
         mbar_init(drain, 1);
         for (int i = 0; i < 8; i++) mbar_init(&xbar[i], 2);
         for (int i = 0; i < 4; i++) mbar_init(&lbar[i], 2);
@@ -274,23 +277,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == kWarpQ) {
-        // -------------------------------------------------- raw Q loader
-        // Item ic's raw Q rows go to the staging area once it is free: after
-        // item 0's Q is in TMEM (ic = 1), else after item ic - 2's O rows left.
-        int ic = 0;
-        Item it;
-        for (int w = blockIdx.x; next_item(p, w, it); w += gridDim.x, ++ic) {
-            if (ic >= 1 && !warp_all(mbar_wait(stgfree, (ic - 1) & 1, abort_flag))) break;
-            const int my_n = lane < it.gcnt ? it.sn[lane] : 0;
+        // ------------------------------------ raw Q loader and O writer
+        // The staging area holds item ic's raw Q rows until they are in TMEM,
+        // then item ic - 1's O rows (staged by the softmax warps), which this
+        // warp writes out before loading item ic + 1's raw Q rows.
+        auto load_q = [&](const Item &q_it, int ic) {
+            const int my_n = lane < q_it.gcnt ? q_it.sn[lane] : 0;
+            fence_proxy_async_smem();  // this warp's reads of the staging area precede the copy
+            __syncwarp();
             if (lane == 0) {
                 // each block's 5 rows are one contiguous 2560-byte run
-                mbar_arrive_expect_tx(qraw, it.nrows * kDQK * 2);
+                mbar_arrive_expect_tx(qraw, q_it.nrows * kDQK * 2);
                 counters[4] = ic + 1;
             }
             __syncwarp();
-            if (lane < it.gcnt)
-                bulk_load(sm + oStage + lane * kStageBlockPitch, p.q + (it.bh * p.R + (size_t)kBlock * my_n) * kDQK,
+            if (lane < q_it.gcnt)
+                bulk_load(sm + oStage + lane * kStageBlockPitch, p.q + (q_it.bh * p.R + (size_t)kBlock * my_n) * kDQK,
                           kBlock * kDQK * 2, qraw);
+        };
+        Item it, nx;
+        int w = blockIdx.x, ic = 0;
+        bool has = next_item(p, w, it), ok = true;
+        if (has) load_q(it, 0);
+        int wn = w + gridDim.x;
+        bool hasn = has && next_item(p, wn, nx);
+        if (hasn) {  // item 1's raw Q once item 0's is in TMEM
+            ok = warp_all(mbar_wait(stgfree, 0, abort_flag));
+            if (ok) load_q(nx, 1);
+        }
+        while (ok && has) {
+            // item ic's O rows: row i of softmax warp wv's region at 256 i,
+            // 16-byte unit u at u ^ (i & 15); two half rows per instruction
+            ok = warp_all(mbar_wait(ostaged, ic & 1, abort_flag));
+            if (!ok) break;
+            for (int wv = 0; wv < kSoftWarps; ++wv) {
+                const uint8_t *stage = sm + oStage + wv * (32 * 256);
+                const int hfv = wv >> 2;
+#pragma unroll 4
+                for (int i = 0; i < 16; i++) {
+                    const int wr = 2 * i + (lane >> 4), u = lane & 15;  // row within the warp, unit
+                    const int rr = (wv & 3) * 32 + wr;
+                    if (rr < it.nrows) {
+                        const int ni = it.sn[rr / kBlock], ji = rr % kBlock;
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + wr * 256 + ((u ^ (wr & 15)) << 4));
+                        *reinterpret_cast<uint4 *>(p.o + (it.bh * p.R + kBlock * ni + ji) * kDV + 128 * hfv + 8 * u) = val;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(oread);
+            // the item after next: its raw Q into the staging area
+            int w2 = wn + gridDim.x;
+            Item n2;
+            const bool has2 = hasn && next_item(p, w2, n2);
+            if (has2) load_q(n2, ic + 2);
+            ++ic;
+            w = wn;
+            it = nx;
+            has = hasn;
+            wn = w2;
+            nx = n2;
+            hasn = has2;
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer
@@ -586,8 +633,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&lbar[q4]);
                 ok = warp_all(mbar_wait(&lbar[q4], ic & 1, abort_flag));
             }
-            // the staging area: every warp has read the next item's raw Q rows
+            // the staging area: every warp has read the next item's raw Q rows,
+            // and the loader warp has written out the previous item's O rows
             if (ok && hasn) ok = warp_all(mbar_wait(qdone, ic & 1, abort_flag));
+            if (ok && ic >= 1) ok = warp_all(mbar_wait(oread, (ic - 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
             const float ltot = l + xl[(hf ^ 1) * kM + r];
@@ -611,22 +660,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
                 }
             }
-            // O is out of TMEM: the next item's first P V may overwrite it
+            // O is out of TMEM: the next item's first P V may overwrite it; the
+            // loader warp writes the staged rows to global memory
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(ofree);
-            for (int i = 0; i < 16; i++) {
-                const int wr = 2 * i + (lane >> 4), u = lane & 15;  // row within the warp, unit
-                const int rr = q4 * 32 + wr;
-                const int ni = __shfl_sync(0xffffffffu, n, wr), ji = __shfl_sync(0xffffffffu, j, wr);
-                if (rr < it.nrows) {
-                    const uint4 val = *reinterpret_cast<const uint4 *>(stage + wr * 256 + ((u ^ (wr & 15)) << 4));
-                    *reinterpret_cast<uint4 *>(p.o + (it.bh * p.R + kBlock * ni + ji) * kDV + 128 * hf + 8 * u) = val;
-                }
+            if (lane == 0) {
+                mbar_arrive(ofree);
+                mbar_arrive(ostaged);
             }
             if (live && hf == 0) p.lse[it.bh * p.R + kBlock * n + j] = (m_used + log2f(ltot)) * kLn2;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(stgfree);  // the raw Q of the item after next may load
             ++ic;
             w = wn;
             it = nx;
