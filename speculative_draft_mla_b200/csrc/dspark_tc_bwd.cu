@@ -254,19 +254,10 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         }
         // lane l holds the block index of group block l (l < gcnt)
         const int my_n = lane < gcnt ? sn[lane] : 0;
-        int pf_next = 2;
         for (int t = 0; t < T; ++t) {
             const int ks = t % kKS, vs = t % kVS;
             uint8_t *kt = sm + oK + ks * kTile;
             uint8_t *vt = sm + oV + vs * kTile;
-            if (lane == 0) {
-                for (; pf_next <= t + 4 && pf_next < n_ctx; ++pf_next) {
-                    const int pos = ctx_lo + pf_next * kBN;
-                    tma_prefetch_3d(&tm_kc, 0, (int)(bh * p.L + pos), 0);
-                    tma_prefetch_2d(&tm_kr, 0, (int)((size_t)b * p.L + pos));
-                    tma_prefetch_3d(&tm_v, 0, (int)(bh * p.L + pos), 0);
-                }
-            }
             if (t >= kKS && !warp_all(mbar_wait(&kempty[ks], ((t / kKS) - 1) & 1, abort_flag))) break;
             if (t < n_ctx) {
                 const int pos0 = ctx_lo + t * kBN;
