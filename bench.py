@@ -79,6 +79,28 @@ def algorithmic_work(wl, anchors, keep):
                 union_positions=union, rows=rows)
 
 
+def measured_traffic(call):
+    """DRAM bytes of one call (sum over its kernels) from the committed ncu capture of the
+    benchmark workload, or None when the kernel sources have changed since it was taken."""
+    import glob
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic_s8192_n512_b2.json")) as f:
+            d = json.load(f)
+        h = hashlib.sha256()
+        srcs = glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cu")) + \
+            glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cuh"))
+        for path in sorted(srcs, key=os.path.basename):
+            h.update(os.path.basename(path).encode())
+            with open(path, "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != d["sources_sha256"]:
+            return None
+        return sum(k["dram_read_bytes"] + k["dram_write_bytes"] for k in d["calls"][call])
+    except Exception:
+        return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -346,7 +368,8 @@ def main():
     roof_ms = max((work["fwd_bytes"] + work["bwd_bytes"]) / (hbm * 1e9),
                   (work["fwd_flops"] + work["bwd_flops"]) / (tfl_sus * 1e12)) * 1e3
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": None, "kernel": "attn_%s call (all its kernels)" % dominant,
+                "traffic": (measured_traffic(dominant) if wl.name == "s8192_n512_b2" else None),
+                "kernel": "attn_%s call (all its kernels)" % dominant,
                 "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % src if src == "measured" else "fallback",
                 "step_frac": roof_ms / ms_max, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
                 "fwd_bytes": work["fwd_bytes"], "bwd_bytes": work["bwd_bytes"],
