@@ -79,22 +79,33 @@ def algorithmic_work(wl, anchors, keep):
                 union_positions=union, rows=rows)
 
 
-def measured_traffic(call):
-    """DRAM bytes of one call (sum over its kernels) from the committed ncu capture of the
-    benchmark workload, or None when the kernel sources have changed since it was taken."""
+# The tensor-core kernel file of the other call plays no part in a call's DRAM traffic.
+_OTHER_CALL_SOURCE = {"fwd": "dspark_tc_bwd.cu", "bwd": "dspark_tc_fwd.cu"}
+
+
+def sources_sha256(call):
+    """sha256 over (basename, content) of the kernel sources one C-ABI call is built from."""
     import glob
     import hashlib
+    h = hashlib.sha256()
+    srcs = glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cu")) + \
+        glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cuh"))
+    for path in sorted(srcs, key=os.path.basename):
+        if os.path.basename(path) == _OTHER_CALL_SOURCE[call]:
+            continue
+        h.update(os.path.basename(path).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(call):
+    """DRAM bytes of one call (sum over its kernels) from the committed ncu capture of the
+    benchmark workload, or None when that call's kernel sources have changed since it was taken."""
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic_s8192_n512_b2.json")) as f:
             d = json.load(f)
-        h = hashlib.sha256()
-        srcs = glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cu")) + \
-            glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cuh"))
-        for path in sorted(srcs, key=os.path.basename):
-            h.update(os.path.basename(path).encode())
-            with open(path, "rb") as f:
-                h.update(f.read())
-        if h.hexdigest() != d["sources_sha256"]:
+        if sources_sha256(call) != d["sources_sha256"][call]:
             return None
         return sum(k["dram_read_bytes"] + k["dram_write_bytes"] for k in d["calls"][call])
     except Exception:
