@@ -15,9 +15,10 @@
 // Persistent: one CTA per SM walks the items blockIdx.x, + gridDim.x, ...
 // K/V tiles, S buffers and pipeline phases are counted over all of a CTA's
 // items, so the K/V stream runs on across item boundaries; the next item's
-// raw Q rows are staged while the current item runs, moved into TMEM as soon
-// as its last QK has completed, and the finished item's O leaves TMEM through
-// the same staging area while the next item's first QK runs.
+// raw Q rows are staged (and their rope slice rotated) while the current item
+// runs, moved into TMEM as soon as its last QK has completed, and the finished
+// item's O leaves TMEM through the same staging area, one bulk copy per block,
+// while the next item's first QK runs.
 // Q lives in tensor memory (A operand of S = Q K^T read from TMEM), and P is
 // written over its own S columns (A operand of O += P V read from TMEM).
 // TMEM: O 0..255, S 256..319 / 320..383, Q 384..511. Shared memory: two K
@@ -27,11 +28,11 @@
 //   warps 0-7  softmax: warps w and w + 4 share TMEM sub-partition w % 4, so
 //              query rows 32 (w % 4) .. + 31 (thread = row = TMEM lane), and
 //              split each 64-key tile into two 32-column halves. They move
-//              the row's half of Q into TMEM (RoPE-rotating the rope slice),
+//              the row's half of Q from the staging area into TMEM,
 //              turn each S tile into P with an online softmax whose row max
 //              the pair exchanges through shared memory, rescale their half
-//              of the O row when the running max grows by more than 2^8, and
-//              write O and LSE.
+//              of the O row when the running max grows by more than 2^8,
+//              stage O and write LSE.
 //   warp 8     K producer: TMA loads of context K tiles (K^C as one 3-D box,
 //              plus the pre-rotated shared K^R) and of draft-key tiles (per
 //              block one 3-D box of its 8 K^C rows and one of its K^R rows).
@@ -42,7 +43,9 @@
 //              its Q is in TMEM, its first P V after the previous item's O
 //              has been read out).
 //   warp 10    V producer.
-//   warp 11    raw Q loader (one bulk copy per block of 5 rows).
+//   warp 11    raw Q loader (one bulk copy per block of 5 rows), which then
+//              RoPE-rotates the staged rows' rope slice in place, and O writer
+//              (one bulk copy per block of 5 staged O rows).
 // Every mbarrier wait is bounded; on time-out the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained with a
 // bounded wait, TMEM is freed and the workspace error word gets kErrTimeout.
@@ -68,19 +71,20 @@ constexpr int kKS = 2, kVS = 2;     // K and V stages
 
 // Shared memory: K0 K1 V0 V1, then the staging area (the next item's raw Q
 // rows; then, once they are in TMEM, the finished item's O rows on their way
-// to global memory), then the softmax pair exchange and the barriers.
+// to global memory, in the same layout), then the softmax pair exchange and
+// the barriers.
 constexpr int oStage = 4 * kKBytes;
 constexpr int kStageBytes = 64 * 1024;
 constexpr int oX = oStage + kStageBytes;  // pair exchange: tile max [2][2][128], row sum [2][128] (floats)
 constexpr int oBar = oX + 3 * 1024;
 __device__ __forceinline__ int k_stage_off(int s) { return s * kKBytes; }
 __device__ __forceinline__ int v_stage_off(int s) { return (2 + s) * kKBytes; }
-// Raw Q: one bulk copy per block (5 rows of 512 B), blocks 2576 B apart, so
-// the rows that the threads of a warp read at once fall on at most 5 rows
-// per bank group.
+// Raw Q and O: one bulk copy per block (5 rows of 512 B), blocks 2576 B
+// apart, so the rows that the threads of a warp access at once fall on at
+// most 5 rows per bank group.
 constexpr int kStageBlockPitch = kBlock * kDQK * 2 + 16;
-static_assert(kG * kStageBlockPitch <= kStageBytes, "staging area too small for raw Q");
-static_assert(8 * 32 * 256 <= kStageBytes, "staging area too small for O rows");
+static_assert(kG * kStageBlockPitch <= kStageBytes, "staging area too small for raw Q and O rows");
+static_assert(kDQK == kDV, "raw Q and O rows share the staging layout");
 constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 // Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
 // slices) at bb * 3 KB, its K^R rows at 24 KB + bb * 1 KB; its V rows (4 x 1 KB)
@@ -88,8 +92,8 @@ constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 // 64-column slices 1 KB apart and 8-key groups 4 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
-// barrier words: K and V full/empty per stage, 28 more, then 6 counters
-static_assert((2 * (kKS + kVS) + 28) * 8 + 6 * 4 <= 512, "barrier area too small");
+// barrier words: K and V full/empty per stage, 28 more, 6 counters, then one more barrier
+static_assert((2 * (kKS + kVS) + 32) * 8 <= 512, "barrier area too small");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 constexpr int kSoftWarps = 8;
@@ -114,6 +118,24 @@ struct FwdArgs {
     int n_groups;  // groups of kG blocks per batch row (work items per (b, h))
     int n_items;   // n_groups * n_h * B
 };
+
+// A bf16 pair (x0 low, x1 high) of a rope slice rotated by (c, s).
+__device__ __forceinline__ uint32_t rope_rot(uint32_t w, float c, float s) {
+    const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
+    return pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+}
+// 1-D bulk copy shared -> global (16-byte aligned addresses, size a multiple
+// of 16), tracked by this thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's bulk stores have read their shared-memory source
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Work item w = (group g, head h, batch b), g fastest (neighbouring items read
 // overlapping context windows of one head close together in time).
@@ -171,6 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
     // [4] raw Q loads issued, [5] raw Q loads consumed
     int *counters = reinterpret_cast<int *>(sfull + 28);
+    // per item: the staged raw Q rows' rope slice rotated (loader warp)
+    uint64_t *qrot = sfull + 31;
     float *xm = reinterpret_cast<float *>(sm + oX);         // [s][half][row]
     float *xl = reinterpret_cast<float *>(sm + oX + 2048);  // [half][row]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -194,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&pvdone[s], 1);
         }
         mbar_init(qraw, 1);
+        mbar_init(qrot, 1);
         mbar_init(qready, kSoftWarps);
         mbar_init(qdone, kSoftWarps);
         mbar_init(ofree, kSoftWarps);
@@ -280,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------ raw Q loader and O writer
         // The staging area holds item ic's raw Q rows until they are in TMEM,
         // then item ic - 1's O rows (staged by the softmax warps), which this
-        // warp writes out before loading item ic + 1's raw Q rows.
+        // warp stores before loading item ic + 1's raw Q rows.
         auto load_q = [&](const Item &q_it, int ic) {
             const int my_n = lane < q_it.gcnt ? q_it.sn[lane] : 0;
             fence_proxy_async_smem();  // this warp's reads of the staging area precede the copy
@@ -295,42 +320,78 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bulk_load(sm + oStage + lane * kStageBlockPitch, p.q + (q_it.bh * p.R + (size_t)kBlock * my_n) * kDQK,
                           kBlock * kDQK * 2, qraw);
         };
-        Item it, nx;
-        int w = blockIdx.x, ic = 0;
-        bool has = next_item(p, w, it), ok = true;
-        if (has) load_q(it, 0);
-        int wn = w + gridDim.x;
-        bool hasn = has && next_item(p, wn, nx);
-        if (hasn) {  // item 1's raw Q once item 0's is in TMEM
-            ok = warp_all(mbar_wait(stgfree, 0, abort_flag));
-            if (ok) load_q(nx, 1);
-        }
-        while (ok && has) {
-            // item ic's O rows: row i of softmax warp wv's region at 256 i,
-            // 16-byte unit u at u ^ (i & 15); two half rows per instruction
-            ok = warp_all(mbar_wait(ostaged, ic & 1, abort_flag));
-            if (!ok) break;
-            for (int wv = 0; wv < kSoftWarps; ++wv) {
-                const uint8_t *stage = sm + oStage + wv * (32 * 256);
-                const int hfv = wv >> 2;
-#pragma unroll 4
-                for (int i = 0; i < 16; i++) {
-                    const int wr = 2 * i + (lane >> 4), u = lane & 15;  // row within the warp, unit
-                    const int rr = (wv & 3) * 32 + wr;
-                    if (rr < it.nrows) {
-                        const int ni = it.sn[rr / kBlock], ji = rr % kBlock;
-                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + wr * 256 + ((u ^ (wr & 15)) << 4));
-                        *reinterpret_cast<uint4 *>(p.o + (it.bh * p.R + kBlock * ni + ji) * kDV + 128 * hfv + 8 * u) = val;
+        // Once they have landed, the rope slice (the last 64 columns) of every
+        // staged row is rotated in place to the row's position A + j: lane i
+        // turns frequency i (one bf16 pair) of each row, 25 rows per round of
+        // table loads. This runs while the item before is still in flight, so
+        // the softmax warps only copy the rows into TMEM at the item switch.
+        auto rotate_q = [&](const Item &q_it, int ic) -> bool {
+            if (!warp_all(mbar_wait(qraw, ic & 1, abort_flag))) return false;
+            if (lane == 0) counters[5] = ic + 1;
+            const int my_a = lane < q_it.gcnt ? q_it.sa[lane] : 0;
+            for (int b0 = 0; b0 < q_it.gcnt; b0 += 5) {
+                float2 cs[5][kBlock];
+#pragma unroll
+                for (int bb = 0; bb < 5; bb++) {
+                    const int a = __shfl_sync(0xffffffffu, my_a, b0 + bb);  // b0 + bb <= 28
+#pragma unroll
+                    for (int j = 0; j < kBlock; j++)
+                        cs[bb][j] = b0 + bb < q_it.gcnt ? __ldg(p.tab + (size_t)(a + j) * (kDR / 2) + lane)
+                                                        : make_float2(1.f, 0.f);
+                }
+#pragma unroll
+                for (int bb = 0; bb < 5; bb++) {
+                    if (b0 + bb < q_it.gcnt) {
+                        uint32_t *row = reinterpret_cast<uint32_t *>(sm + oStage + (b0 + bb) * kStageBlockPitch + kDC * 2);
+#pragma unroll
+                        for (int j = 0; j < kBlock; j++) {
+                            uint32_t *wp = row + j * (kDQK / 2) + lane;
+                            *wp = rope_rot(*wp, cs[bb][j].x, cs[bb][j].y);
+                        }
                     }
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(qrot);
+            return true;
+        };
+        Item it, nx;
+        int w = blockIdx.x, ic = 0;
+        bool has = next_item(p, w, it), ok = true;
+        if (has) {
+            load_q(it, 0);
+            ok = rotate_q(it, 0);
+        }
+        int wn = w + gridDim.x;
+        bool hasn = has && next_item(p, wn, nx);
+        if (ok && hasn) {  // item 1's raw Q once item 0's is in TMEM
+            ok = warp_all(mbar_wait(stgfree, 0, abort_flag));
+            if (ok) {
+                load_q(nx, 1);
+                ok = rotate_q(nx, 1);
+            }
+        }
+        while (ok && has) {
+            // item ic's O rows: each block's 5 rows (contiguous in global
+            // memory) with one bulk copy; the staging area is free again once
+            // the copies have read it
+            ok = warp_all(mbar_wait(ostaged, ic & 1, abort_flag));
+            if (!ok) break;
+            if (lane < it.gcnt)
+                bulk_store(p.o + (it.bh * p.R + (size_t)kBlock * it.sn[lane]) * kDV, sm + oStage + lane * kStageBlockPitch,
+                           kBlock * kDV * 2);
+            bulk_commit();
+            bulk_wait_read_all();
             __syncwarp();
             if (lane == 0) mbar_arrive(oread);
             // the item after next: its raw Q into the staging area
             int w2 = wn + gridDim.x;
             Item n2;
             const bool has2 = hasn && next_item(p, w2, n2);
-            if (has2) load_q(n2, ic + 2);
+            if (has2) {
+                load_q(n2, ic + 2);
+                ok = rotate_q(n2, ic + 2);
+            }
             ++ic;
             w = wn;
             it = nx;
@@ -339,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             nx = n2;
             hasn = has2;
         }
+        bulk_wait_all();  // the O stores are complete before the CTA ends
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
@@ -451,39 +513,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         bool ok = true;
         // Q row r of an item, this thread's half (columns 128 hf .. + 127),
-        // from the staging area -> TMEM lane r, columns kColQ + 64 hf .. + 63;
-        // the rope slice (the last 64 columns, half 1) is rotated to position
-        // A + j first. Rows past the item's blocks are zero.
+        // from the staging area (rope slice already rotated by the loader
+        // warp) -> TMEM lane r, columns kColQ + 64 hf .. + 63. Rows past the
+        // item's blocks are zero.
         auto move_q = [&](const Item &q_it, int ic) {
             const bool live = r < q_it.nrows;
-            float4 cs[16];  // (cos, sin) of the 32 rope frequencies at A + j (half 1)
-            if (hf == 1) {
-                const int pos = live ? q_it.sa[r / kBlock] + r % kBlock : 0;
-                const float4 *tp = reinterpret_cast<const float4 *>(p.tab + (size_t)pos * (kDR / 2));
-#pragma unroll
-                for (int k = 0; k < 16; k++) cs[k] = __ldg(tp + k);
-            }
-            ok = warp_all(mbar_wait(qraw, ic & 1, abort_flag));
-            if (ok && threadIdx.x == 0) counters[5] = ic + 1;
+            ok = warp_all(mbar_wait(qrot, ic & 1, abort_flag));
             const bool have = live && ok;
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + (r / kBlock) * kStageBlockPitch +
                                                                (r % kBlock) * (kDQK * 2) + hf * 256);
-            // a bf16 pair (x0 low, x1 high) rotated by (c, s)
-            auto rot = [](uint32_t w, float c, float s_) {
-                const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
-                return pack_bf16x2(x0 * c - x1 * s_, x0 * s_ + x1 * c);
-            };
 #pragma unroll
             for (int part = 0; part < 2; part++) {  // 8 units (64 bf16) per TMEM store
                 uint32_t w[32];
 #pragma unroll
                 for (int uu = 0; uu < 8; uu++) {
-                    uint4 val = have ? src[part * 8 + uu] : make_uint4(0, 0, 0, 0);
-                    if (hf == 1 && part == 1) {  // rope unit uu: frequencies 4 uu .. 4 uu + 3
-                        const float4 c01 = cs[2 * uu], c23 = cs[2 * uu + 1];
-                        val = make_uint4(rot(val.x, c01.x, c01.y), rot(val.y, c01.z, c01.w), rot(val.z, c23.x, c23.y),
-                                         rot(val.w, c23.z, c23.w));
-                    }
+                    const uint4 val = have ? src[part * 8 + uu] : make_uint4(0, 0, 0, 0);
                     w[4 * uu + 0] = val.x;
                     w[4 * uu + 1] = val.y;
                     w[4 * uu + 2] = val.z;
@@ -634,34 +678,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = warp_all(mbar_wait(&lbar[q4], ic & 1, abort_flag));
             }
             // the staging area: every warp has read the next item's raw Q rows,
-            // and the loader warp has written out the previous item's O rows
+            // and the loader warp's bulk copies have read the previous item's O rows
             if (ok && hasn) ok = warp_all(mbar_wait(qdone, ic & 1, abort_flag));
             if (ok && ic >= 1) ok = warp_all(mbar_wait(oread, (ic - 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
             const float ltot = l + xl[(hf ^ 1) * kM + r];
             const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-            // this half of the O row (columns 128 hf .. +127) -> staging (row i
-            // of the warp at 256 i, unit u at u ^ (i & 15)) -> two half rows
-            // per warp instruction
-            uint8_t *stage = sm + oStage + warp * (32 * 256);
+            // this half of the O row (columns 128 hf .. +127) -> the staging
+            // area in the raw Q layout (block r / 5 at r / 5 * 2576, row r % 5
+            // at + 512 (r % 5)); rows past the item's blocks are not staged
+            uint8_t *orow = sm + oStage + (live ? (r / kBlock) * kStageBlockPitch + (r % kBlock) * (kDV * 2) : 0) + hf * 256;
 #pragma unroll 1
             for (int c = 0; c < 128; c += 32) {
                 float ov[32];
                 tmem_ld32(trow + kColO + 128 * hf + c, ov);
                 tmem_wait_ld();
+                if (live) {
 #pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const int u = c / 8 + k;
-                    *reinterpret_cast<uint4 *>(stage + lane * 256 + ((u ^ (lane & 15)) << 4)) =
-                        make_uint4(pack_bf16x2(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv),
-                                   pack_bf16x2(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv),
-                                   pack_bf16x2(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv),
-                                   pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
+                    for (int k = 0; k < 4; k++)
+                        *reinterpret_cast<uint4 *>(orow + (c / 8 + k) * 16) =
+                            make_uint4(pack_bf16x2(ov[8 * k + 0] * inv, ov[8 * k + 1] * inv),
+                                       pack_bf16x2(ov[8 * k + 2] * inv, ov[8 * k + 3] * inv),
+                                       pack_bf16x2(ov[8 * k + 4] * inv, ov[8 * k + 5] * inv),
+                                       pack_bf16x2(ov[8 * k + 6] * inv, ov[8 * k + 7] * inv));
                 }
             }
             // O is out of TMEM: the next item's first P V may overwrite it; the
-            // loader warp writes the staged rows to global memory
+            // loader warp stores the staged rows with bulk copies (async proxy)
+            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
