@@ -1,4 +1,5 @@
-"""Multi-process host logic of the benchmark on CPU (gloo, world size 2).
+"""Host logic of the benchmark on CPU: the multi-process steps (gloo, world
+size 2), the work model and the lookup of the stored DRAM traffic.
 
 The attention shards by batch with no collective on the data path; the only
 cross-rank steps are the barrier around the timed region, the max over ranks
@@ -65,3 +66,27 @@ def test_work_model_counts():
     assert w["union_positions"] == 3
     pairs = 5 * (0 + 5) + 5 * (3 + 5)
     assert w["fwd_flops"] == 2 * pairs * (4 + 4)
+
+
+def test_traffic_follows_each_calls_sources(tmp_path, monkeypatch):
+    """A call's stored DRAM traffic is reported while the sources it is built
+    from are unchanged, whatever happens to the other call's kernel file."""
+    import json
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "speculative_draft_mla_b200" / "csrc"
+    shutil.copytree(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc"), csrc)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    calls = {c: [{"kernel": "k", "dram_read_bytes": 100 * (i + 1), "dram_write_bytes": 7}]
+             for i, c in enumerate(("fwd", "bwd"))}
+    stored = {"sources_sha256": {c: bench.sources_sha256(c) for c in calls}, "calls": calls}
+    (tmp_path / "profiles" / "dram_traffic_s8192_n512_b2.json").write_text(json.dumps(stored))
+    assert bench.measured_traffic("fwd") == 107 and bench.measured_traffic("bwd") == 207
+    with open(csrc / "dspark_tc_fwd.cu", "a") as f:
+        f.write("\n// edited\n")
+    assert bench.measured_traffic("fwd") is None and bench.measured_traffic("bwd") == 207
+    with open(csrc / "dspark_tc_common.cuh", "a") as f:
+        f.write("\n// edited\n")
+    assert bench.measured_traffic("bwd") is None
