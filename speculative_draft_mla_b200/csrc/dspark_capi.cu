@@ -151,7 +151,7 @@ dspark_status dspark_build_descriptor(const dspark_problem *pp, const int32_t *a
     dspark_status why;
     if (!make_prob(pp, &p, &why)) return why;
     DSPARK_TRY(check_ws(p, workspace, workspace_bytes, false));
-    if ((size_t)p.B * p.N && (!anchors || !keep)) return DSPARK_ERR_NULL;
+    if ((size_t)p.B * p.N != 0 && (!anchors || !keep)) return DSPARK_ERR_NULL;
     cudaStream_t st = (cudaStream_t)stream;
     return build(p, anchors, keep, ws_view(p, workspace), st);
 }
