@@ -326,16 +326,18 @@ def main():
     stream = torch.cuda.current_stream(device)
     R = capi.FLAG_REUSE_DESCRIPTOR
 
-    def step(ev=None):
+    def step(ev=None, d=None, outs=None):
+        d = dev if d is None else d
+        o_, lse_, g_ = (o, lse, grads) if outs is None else outs
         if ev is not None:
             ev[0].record(stream)
-        capi.build_descriptor(prob, dev["anchors"], dev["keep"], ws)
-        capi.attn_fwd(dev["q"], dev["kc"], dev["kr"], dev["v"], dev["anchors"], dev["keep"], wl.S, wl.W,
-                      wl.rope_base, workspace=ws, flags=R, out=(o, lse))
+        capi.build_descriptor(prob, d["anchors"], d["keep"], ws)
+        capi.attn_fwd(d["q"], d["kc"], d["kr"], d["v"], d["anchors"], d["keep"], wl.S, wl.W,
+                      wl.rope_base, workspace=ws, flags=R, out=(o_, lse_))
         if ev is not None:
             ev[1].record(stream)
-        capi.attn_bwd(dev["q"], dev["kc"], dev["kr"], dev["v"], dev["anchors"], dev["keep"], o, lse, dev["dout"],
-                      wl.S, wl.W, wl.rope_base, workspace=ws, flags=R, out=grads)
+        capi.attn_bwd(d["q"], d["kc"], d["kr"], d["v"], d["anchors"], d["keep"], o_, lse_, d["dout"],
+                      wl.S, wl.W, wl.rope_base, workspace=ws, flags=R, out=g_)
         if ev is not None:
             ev[2].record(stream)
 
@@ -386,35 +388,60 @@ def main():
                 "fwd_bytes": work["fwd_bytes"], "bwd_bytes": work["bwd_bytes"],
                 "fwd_flops": work["fwd_flops"], "bwd_flops": work["bwd_flops"]}
 
-    # end to end through the public API with host buffers
+    # End to end through the public API with host buffers: every step copies
+    # its inputs in from pinned host memory and all of its outputs back. As a
+    # training loop would, the copies run on their own streams into and out of
+    # two device buffer sets, so that step i+1's inputs arrive and step i's
+    # outputs leave while a step computes.
     e2e = None
     if not args.no_e2e:
         ins = ("q", "kc", "kr", "v", "anchors", "keep", "dout")
         outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse) + grads]
         h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in ins)
         d2h = sum(t.numel() * t.element_size() for t in outs_host)
+        dsets = [dev, {k: (torch.empty_like(dev[k]) if k in ins else dev[k]) for k in dev}]
+        osets = [(o, lse, grads), (torch.empty_like(o), torch.empty_like(lse), tuple(torch.empty_like(g) for g in grads))]
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        in_done = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for k in ins:
-                dev[k].copy_(pinned[k], non_blocking=True)
-            step()
-            for hdst, src_t in zip(outs_host, (o, lse) + grads):
-                hdst.copy_(src_t, non_blocking=True)
+        def e2e_run(n, a=None, b=None):
+            if a is not None:
+                a.record(s_in)
+            for i in range(n):
+                j = i & 1
+                if i >= 2:  # set j's inputs were last read by step i - 2
+                    s_in.wait_event(comp_done[j])
+                with torch.cuda.stream(s_in):
+                    for k in ins:
+                        dsets[j][k].copy_(pinned[k], non_blocking=True)
+                in_done[j].record(s_in)
+                stream.wait_event(in_done[j])
+                if i >= 2:  # set j's outputs were last read by step i - 2's copy out
+                    stream.wait_event(out_done[j])
+                step(d=dsets[j], outs=(osets[j][0], osets[j][1], osets[j][2]))
+                comp_done[j].record(stream)
+                s_out.wait_event(comp_done[j])
+                with torch.cuda.stream(s_out):
+                    for hdst, src_t in zip(outs_host, (osets[j][0], osets[j][1]) + osets[j][2]):
+                        hdst.copy_(src_t, non_blocking=True)
+                out_done[j].record(s_out)
+            if b is not None:
+                b.record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         ke = max(2, min(args.steps, 5))
         barrier(world)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        b.record(stream)
+        e2e_run(ke, a, b)
         torch.cuda.synchronize()
         ems = reduce_max(a.elapsed_time(b) / ke, device, world)
         e2e = {"value": aggregate(wl.rows, world, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems,
+               "copies": "own streams, two device buffer sets: step i+1's inputs in and step i's outputs out "
+                         "while a step computes"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
