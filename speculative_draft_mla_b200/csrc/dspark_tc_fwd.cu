@@ -5,7 +5,8 @@
 // consecutive in anchor order) = up to 125 query rows, the M = 128 of one
 // MMA. The group's key set is the union of its blocks' context windows,
 // [max(0, A_first - W + 1), A_last), walked in 64-key tiles, followed by the
-// group's own draft keys (5 per block) gathered into one or two more tiles.
+// group's own draft keys (5 per block, in 8 key slots) gathered into tiles of
+// 8 blocks (up to 4 more tiles).
 // Each row masks every key that is not in its own key set (page "GLM 5.2
 // DSpark speculative-training design", §3: window [A-W+1, A) shared by the 5
 // offsets, own block bidirectional, other blocks invisible). Because blocks
