@@ -160,7 +160,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device, period=0.01):
+    def __init__(self, device, period=0.002):
         self.samples, self.reasons, self.period = [], set(), period
         self.max_mhz = None
         self._stop = threading.Event()
