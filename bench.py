@@ -79,22 +79,22 @@ def algorithmic_work(wl, anchors, keep):
                 union_positions=union, rows=rows)
 
 
-# The tensor-core kernel file of the other call plays no part in a call's DRAM traffic.
-_OTHER_CALL_SOURCE = {"fwd": "dspark_tc_bwd.cu", "bwd": "dspark_tc_fwd.cu"}
+# The device sources each C-ABI call's kernels at the benchmark workload are
+# built from (the host-side argument checks, the SIMT family, the no-workspace
+# entry point and the host sampler play no part in a call's DRAM traffic).
+_CALL_SOURCES = {
+    "fwd": ("dspark_internal.cuh", "dspark_prep.cu", "dspark_tc_common.cuh", "dspark_tc_fwd.cu"),
+    "bwd": ("dspark_internal.cuh", "dspark_prep.cu", "dspark_tc_common.cuh", "dspark_tc_bwd.cu"),
+}
 
 
 def sources_sha256(call):
     """sha256 over (basename, content) of the kernel sources one C-ABI call is built from."""
-    import glob
     import hashlib
     h = hashlib.sha256()
-    srcs = glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cu")) + \
-        glob.glob(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", "*.cuh"))
-    for path in sorted(srcs, key=os.path.basename):
-        if os.path.basename(path) == _OTHER_CALL_SOURCE[call]:
-            continue
-        h.update(os.path.basename(path).encode())
-        with open(path, "rb") as f:
+    for name in sorted(_CALL_SOURCES[call]):
+        h.update(name.encode())
+        with open(os.path.join(ROOT, "speculative_draft_mla_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 

@@ -132,9 +132,11 @@ DSPARK_API dspark_status dspark_attn_fwd(const dspark_problem *p, const void *q,
  *     bit 1: a bounded device-side wait gave up).
  *   - Returns DSPARK_ERR_UNSUPPORTED when the forward needs more scratch than
  *     the array holds; other statuses as dspark_attn_fwd.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make that
- *     first call before any stream capture.
+ *   - Every call outside a stream capture looks up the array's device address
+ *     (cudaGetSymbolAddress, with the stream's device current), so a
+ *     cudaDeviceReset between calls is harmless; a call on a stream that is
+ *     being captured reuses the address of the last uncaptured call on that
+ *     device. Make the first call on a device before any stream capture.
  *   - All calls share the one array, which keeps the last call's contents: two
  *     calls whose work overlaps on the GPU (different streams, or different
  *     host threads on the same device) race on it. Serialise them. */

@@ -30,13 +30,20 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
-dspark_status scratch_address(void **out) {
+// Device address of the scratch array on the current device. Outside a
+// stream capture it is looked up on every call (cudaGetSymbolAddress, with the
+// device current), so that an address cached before a cudaDeviceReset (which
+// reloads the module and may move the array) is never used again. While the
+// stream is being captured the address cached by the last uncaptured call on
+// this device is used; a capture before any uncaptured call on the device
+// attempts the lookup as well.
+dspark_status scratch_address(cudaStream_t st, void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSPARK_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return DSPARK_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone || !g_addr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSPARK_ERR_CUDA;
         g_addr[dev] = p;
@@ -59,7 +66,7 @@ extern "C" dspark_status dspark_attn_fwd_noalloc(const dspark_problem *p, const 
     }
     if (need > kScratchBytes) return DSPARK_ERR_UNSUPPORTED;
     void *scratch = nullptr;
-    const dspark_status s0 = scratch_address(&scratch);
+    const dspark_status s0 = scratch_address((cudaStream_t)stream, &scratch);
     if (s0 != DSPARK_OK) return s0;
     // The descriptor is rebuilt on every call (which also clears the error
     // word); everything else the forward reads from the scratch is fully

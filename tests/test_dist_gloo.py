@@ -69,8 +69,9 @@ def test_work_model_counts():
 
 
 def test_traffic_follows_each_calls_sources(tmp_path, monkeypatch):
-    """A call's stored DRAM traffic is reported while the sources it is built
-    from are unchanged, whatever happens to the other call's kernel file."""
+    """A call's stored DRAM traffic is reported while the device sources it is
+    built from are unchanged, whatever happens to host-only files or to the
+    other call's kernel file."""
     import json
     import shutil
     sys.path.insert(0, ROOT)
@@ -83,6 +84,11 @@ def test_traffic_follows_each_calls_sources(tmp_path, monkeypatch):
              for i, c in enumerate(("fwd", "bwd"))}
     stored = {"sources_sha256": {c: bench.sources_sha256(c) for c in calls}, "calls": calls}
     (tmp_path / "profiles" / "dram_traffic_s8192_n512_b2.json").write_text(json.dumps(stored))
+    assert bench.measured_traffic("fwd") == 107 and bench.measured_traffic("bwd") == 207
+    # host-only and unrelated sources do not invalidate either call's figure
+    for name in ("dspark_capi.cu", "dspark_noalloc.cu", "dspark_simt.cu", "dspark_host.cpp"):
+        with open(csrc / name, "a") as f:
+            f.write("\n// edited\n")
     assert bench.measured_traffic("fwd") == 107 and bench.measured_traffic("bwd") == 207
     with open(csrc / "dspark_tc_fwd.cu", "a") as f:
         f.write("\n// edited\n")

@@ -46,6 +46,9 @@ EDGE = [
     ("page_dims_small", 40, 1, 300, 20, 128, 2, 192, 64, 256, 1.0, False),
     ("page_dims_dense", 41, 1, 200, 60, 128, 2, 192, 64, 256, 0.9, True),
     ("page_dims_ragged", 42, 2, 133, 7, 128, 1, 192, 64, 256, 1.0, False),
+    # three batch rows and 20 heads: the key-major kernels split the heads into
+    # groups, so batch-row and head-group indexing is exercised at page dims
+    ("page_dims_b3_heads20", 43, 3, 400, 40, 128, 20, 192, 64, 256, 0.85, True),
 ]
 
 
@@ -126,6 +129,48 @@ def _np(s):
     return [s[k].double().numpy() for k in ("q", "kc", "kr", "v")]
 
 
+def _uncovered(an_b, kp_b, S, W):
+    """Context positions inside no kept block's window [max(0, A-W+1), A)."""
+    cov = np.zeros(S + 1, np.int64)
+    a = an_b[kp_b == 1]
+    np.add.at(cov, np.maximum(0, a - W + 1), 1)
+    np.add.at(cov, a, -1)
+    return np.nonzero(np.cumsum(cov)[:S] == 0)[0]
+
+
+def _sample_keys(rng, an_b, kp_b, S, W, N):
+    """Key positions of one batch row to compare: window edges of a sampled
+    block, the edge of the lowest window, an uncovered position, the ends of
+    the context, random context positions, draft keys of kept blocks and the
+    draft keys of a padding block (their gradients must be zero)."""
+    kept = np.nonzero(kp_b == 1)[0]
+    keys = [0, S - 2, S - 1]
+    far = kept[an_b[kept] >= W]
+    if far.size:
+        a = int(an_b[int(rng.choice(far))])
+        keys += [a - 1, a - W + 1, a - W]
+    low = int(kept[np.argmin(an_b[kept])])
+    if an_b[low] > 0:
+        keys.append(int(an_b[low]) - 1)
+    unc = _uncovered(an_b, kp_b, S, W)
+    if unc.size:
+        keys.append(int(rng.choice(unc)))
+    keys += [int(x) for x in rng.integers(0, S, 5)]
+    for n in rng.choice(kept, 3, replace=False):
+        keys.append(S + 5 * int(n) + int(rng.integers(5)))
+    keys.append(S + 5 * int(kept[-1]) + 4)
+    pads = np.nonzero(kp_b == 0)[0]
+    if pads.size:
+        n = int(rng.choice(pads))
+        keys += [S + 5 * n, S + 5 * n + 4]
+    return sorted(set(keys))
+
+
+# one head of each group of 16 (the key-major kernels split the 64 heads into
+# groups), the first and last head of the first group
+_KEY_HEADS = (0, 15, 16, 47, 63)
+
+
 @pytest.mark.parametrize("wid", [3, 4, 5])
 def test_full_size_sampled(oracle_mod, wid):
     wl = synth.WORKLOADS[wid]
@@ -144,11 +189,14 @@ def test_full_size_sampled(oracle_mod, wid):
             assert torch.count_nonzero(gpu["dq"][b][:, rows]) == 0
     for k in ("o", "dq", "dkc", "dkr", "dv"):
         assert torch.isfinite(gpu[k].float()).all(), k
-    # sampled rows: random ones plus the block with the smallest anchor
+    # sampled rows: random ones, at least four per batch row (heads in each
+    # group), plus the block with the smallest anchor
     picks = []
-    for _ in range(24):
-        b, h = int(rng.integers(wl.B)), int(rng.integers(wl.n_h))
-        picks.append((b, h, int(rng.integers(5 * wl.N))))
+    for b in range(wl.B):
+        for h in rng.choice(_KEY_HEADS, 4, replace=False):
+            picks.append((b, int(h), int(rng.integers(5 * wl.N))))
+    for _ in range(8):
+        picks.append((int(rng.integers(wl.B)), int(rng.integers(wl.n_h)), int(rng.integers(5 * wl.N))))
     b0 = 0
     n_small = int(np.argmin(np.where(kp[b0] == 1, an[b0], 1 << 30)))
     picks += [(b0, 0, 5 * n_small + j) for j in range(5)]
@@ -161,25 +209,30 @@ def test_full_size_sampled(oracle_mod, wid):
         dq_ref = oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
                                            s["dout"].double().numpy(), S, W, BASE, "dq", np.array([[0, 0, r]]))
         assert_close(gpu["dq"][b, h, r][None], dq_ref, torch.bfloat16, "dq[%d,%d,%d]" % (b, h, r))
-    # sampled keys: context (covered, edge and possibly uncovered) and draft keys
-    keys = [0, S - 1, int(an[0][n_small]) - 1 if an[0][n_small] > 0 else 1]
-    keys += [int(x) for x in rng.integers(0, S, 8)]
-    keys += [S + 5 * int(rng.integers(wl.N)) + int(rng.integers(5)) for _ in range(4)]
-    pads = np.nonzero(kp[0] == 0)[0]
-    if pads.size:
-        keys.append(S + 5 * int(pads[0]))
-    for key in keys:
-        b, h = 0, int(rng.integers(wl.n_h))
-        s = _slice(c, b, h)
-        ref = oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
-                                        s["dout"].double().numpy(), S, W, BASE, "dkv", np.array([[0, 0, key]]))
-        assert_close(gpu["dkc"][b, h, key][None], ref[:, :wl.d_c], torch.bfloat16, "dkc[%d]" % key)
-        assert_close(gpu["dv"][b, h, key][None], ref[:, wl.d_c:], torch.bfloat16, "dv[%d]" % key)
-    # rope-key gradient: sum over heads of per-head oracle contributions
-    dkr_keys = np.array([[0, k] for k in keys[:4]])
-    tot = np.zeros((len(dkr_keys), wl.d_r))
-    for h in range(wl.n_h):
-        s = _slice(c, 0, h)
-        tot += oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
-                                         s["dout"].double().numpy(), S, W, BASE, "dkr", dkr_keys)
-    assert_close(gpu["dkr"][0, dkr_keys[:, 1]], tot, torch.bfloat16, "dkr")
+    # key gradients of every batch row: dK^C and dV at each sampled key for one
+    # head of every head group, dK^R (the sum over all heads) at every sampled key
+    for b in range(wl.B):
+        keys = _sample_keys(rng, an[b], kp[b], S, W, wl.N)
+        assert len(keys) >= 16, keys
+        items = np.array([[0, 0, k] for k in keys])
+        for h in _KEY_HEADS:
+            s = _slice(c, b, h)
+            ref = oracle_mod.attn_bwd_items(*_np(s), s["anchors"].numpy(), s["keep"].numpy(),
+                                            s["dout"].double().numpy(), S, W, BASE, "dkv", items)
+            assert_close(gpu["dkc"][b, h, keys], ref[:, :wl.d_c], torch.bfloat16, "dkc[b=%d,h=%d]" % (b, h))
+            assert_close(gpu["dv"][b, h, keys], ref[:, wl.d_c:], torch.bfloat16, "dv[b=%d,h=%d]" % (b, h))
+        dkr_items = np.array([[0, k] for k in keys])
+        tot = np.zeros((len(keys), wl.d_r))
+        kr_b = c["kr"][b:b + 1].double().numpy()
+        for h in range(wl.n_h):
+            s = _slice(c, b, h)
+            tot += oracle_mod.attn_bwd_items(s["q"].double().numpy(), s["kc"].double().numpy(), kr_b,
+                                             s["v"].double().numpy(), s["anchors"].numpy(), s["keep"].numpy(),
+                                             s["dout"].double().numpy(), S, W, BASE, "dkr", dkr_items)
+        assert_close(gpu["dkr"][b, keys], tot, torch.bfloat16, "dkr[b=%d]" % b)
+        pads = np.nonzero(kp[b] == 0)[0]
+        if pads.size:  # draft keys of padding blocks: zero gradients for every head
+            pk = (wl.S + 5 * pads[:, None] + np.arange(5)[None]).ravel()
+            for k in ("dkc", "dv"):
+                assert torch.count_nonzero(gpu[k][b][:, pk]) == 0, k
+            assert torch.count_nonzero(gpu["dkr"][b][pk]) == 0
