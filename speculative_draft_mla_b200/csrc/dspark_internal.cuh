@@ -44,6 +44,7 @@ struct WsLayout {
     size_t qs;        // bf16 [B, n_h, 5N, 256] rotated Q, anchor-sorted rows
     size_t dos;       // bf16 [B, n_h, 5N, 256] dO, anchor-sorted rows
     size_t dkr_part;  // float [HG, B, L, d_r] rope-key gradient per head group
+    size_t dqacc;     // float [B, n_h, 5N, d_c + d_r] dQ accumulator, anchor-sorted rows
     size_t total;
 };
 
@@ -72,6 +73,7 @@ inline WsLayout ws_layout(const Prob &p) {
     w.dos = off;       off = align256(off + 2 * rows * p.d_v);
     w.dkr_part = off;
     off = align256(off + (tc ? sizeof(float) * (size_t)bwd_head_groups(p) * p.B * p.L * p.d_r : 0));
+    w.dqacc = off;     off = align256(off + sizeof(float) * rows * p.dqk);
     w.total = off;
     return w;
 }
@@ -86,6 +88,7 @@ struct Ws {
     float *lses;
     void *qs, *dos;
     float *dkr_part;
+    float *dqacc;
 };
 
 inline Ws ws_view(const Prob &p, void *base) {
@@ -103,6 +106,7 @@ inline Ws ws_view(const Prob &p, void *base) {
     w.qs = (void *)(c + l.qs);
     w.dos = (void *)(c + l.dos);
     w.dkr_part = (float *)(c + l.dkr_part);
+    w.dqacc = (float *)(c + l.dqacc);
     return w;
 }
 

@@ -9,22 +9,27 @@
 // on rotated q and k rope slices; the rope parts of dQ and dK are rotated back,
 // and dK^R, shared by every head (§4), is the sum over heads.
 //
-// Launch sequence (one stream, no atomics, every output element written once):
-//   1. k_bwd_prep      per kept block and head: rotated Q and dO copied into
-//                      anchor-sorted row order, D, LSE*log2(e); padding rows 0.
-//   2. k_bwd_pad       zeros for padding blocks' rows and draft keys.
-//   3. k_bwd_dq_tc     query-major, one CTA per (b, h, 25 sorted blocks):
-//                      64-key tiles of the group's key set; S and dP in TMEM,
-//                      dS written over the S columns, dQ += dS K in TMEM.
-//   4. k_bwd_kv_tc     key-major, one CTA per (b, 64-key tile, head group):
-//                      rows of the blocks whose key sets meet the tile, in
-//                      chunks of 64: S^T = K Q^T and dP^T = V dO^T in TMEM,
-//                      P^T and dS^T through shared memory, dV += P^T dO and
-//                      dK += dS^T Q accumulated in TMEM over the rows (M = 64
-//                      accumulators: dK and dV share TMEM columns, one in each
-//                      half of the lanes).
+// Launch sequence (one stream):
+//   1. k_bwd_prep       per kept block and head: rotated Q and dO copied into
+//                       anchor-sorted row order, D, LSE*log2(e), and the
+//                       block's rows of the fp32 dQ accumulator zeroed.
+//   2. k_bwd_pad        zeros for padding blocks' rows and draft keys.
+//   3. k_bwd_tc         key-major, one CTA per (b, 64-key tile, head group),
+//                       one pass over K and V: rows of the blocks whose key
+//                       sets meet the tile, in chunks of 64. S^T = K Q^T and
+//                       dP^T = V dO^T in TMEM, P^T and dS^T through shared
+//                       memory, dV += P^T dO and dK += dS^T Q accumulated in
+//                       TMEM over the rows (M = 64 accumulators: dK and dV share
+//                       TMEM columns, one in each half of the lanes), and the
+//                       chunk's dQ contribution dS K in TMEM, added into the
+//                       fp32 dQ accumulator with vector reductions. dK and dV
+//                       are written once, by the CTA that owns the keys (no
+//                       atomics); dQ rows receive one contribution per key tile
+//                       that meets their window, plus their draft tile's.
+//   4. k_bwd_dq_out     rotates the rope part of the accumulated dQ back,
+//                       rounds to bf16 and writes dq in the caller's row order.
 //   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
-//                      them back and writes dK^R.
+//                       them back and writes dK^R.
 // Key tiles are either context tiles [t0, t0+64) or the draft keys of one
 // group of 8 blocks; the blocks whose windows meet a context tile are a
 // contiguous run of the anchor-sorted list (t0 < A <= t0 + 63 + W - 1).
@@ -39,14 +44,14 @@ namespace {
 using namespace tc;
 
 constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
-constexpr int kG = 25;   // blocks per query group (query-major kernel)
-constexpr int kGD = 8;   // blocks per draft-key tile of the key-major kernel (8 slots each: 64 keys)
+constexpr int kGD = 8;   // blocks per draft-key tile (8 slots each: 64 keys)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
 // One warp per row of a kept block (5 warps): rotated q -> qs, do -> dos,
-// D = rowsum(dO * O), LSE * log2(e); rows past the kept blocks are zeroed so
-// tiles that overhang them multiply finite values.
+// D = rowsum(dO * O), LSE * log2(e), and the row of the dQ accumulator set to
+// zero; rows past the kept blocks are zeroed so tiles that overhang them
+// multiply finite values.
 __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfloat16 *__restrict__ q,
                                                   const __nv_bfloat16 *__restrict__ o,
                                                   const __nv_bfloat16 *__restrict__ dout,
@@ -55,7 +60,7 @@ __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfl
                                                   const int32_t *__restrict__ sorted_a,
                                                   const float2 *__restrict__ tab, __nv_bfloat16 *__restrict__ qs,
                                                   __nv_bfloat16 *__restrict__ dos, float *__restrict__ ds_,
-                                                  float *__restrict__ lses) {
+                                                  float *__restrict__ lses, float *__restrict__ dqacc) {
     const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
@@ -63,6 +68,9 @@ __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfl
     const size_t srow = bh * R + kBlock * i + j;
     uint4 *qd = reinterpret_cast<uint4 *>(qs + srow * kDQK) + lane;
     uint4 *dd = reinterpret_cast<uint4 *>(dos + srow * kDV) + lane;
+    float4 *acc = reinterpret_cast<float4 *>(dqacc + srow * kDQK) + 2 * lane;
+    acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i >= cnt[b]) {
         *qd = make_uint4(0, 0, 0, 0);
         *dd = make_uint4(0, 0, 0, 0);
@@ -92,17 +100,17 @@ __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfl
     const uint4 ov = __ldg(reinterpret_cast<const uint4 *>(o + orow * kDV) + lane);
     *dd = dv;
     const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
-    float acc = 0.f;
+    float accd = 0.f;
 #pragma unroll
     for (int k = 0; k < 4; k++) {
         const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&dw[k]);
         const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162 *>(&ow[k]);
-        acc = fmaf(__bfloat162float(x.x), __bfloat162float(y.x), acc);
-        acc = fmaf(__bfloat162float(x.y), __bfloat162float(y.y), acc);
+        accd = fmaf(__bfloat162float(x.x), __bfloat162float(y.x), accd);
+        accd = fmaf(__bfloat162float(x.y), __bfloat162float(y.y), accd);
     }
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    for (int off = 16; off > 0; off >>= 1) accd += __shfl_xor_sync(0xffffffffu, accd, off);
     if (lane == 0) {
-        ds_[srow] = acc;
+        ds_[srow] = accd;
         lses[srow] = lse[orow] * kLog2e;
     }
 }
@@ -129,447 +137,49 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
     }
 }
 
-// ================================================================ dQ
-// CTA = (group g of 25 sorted blocks, head h, batch b); warps 0-3 rows
-// (thread t = row t = TMEM lane t), warp 4 producer, warp 5 MMA.
-// Key tiles are 64 keys wide: an M = 128 MMA costs about the same for N = 32
-// and N = 64, so the wider tile halves the MMA count per key.
-// Q stays in shared memory (A operand of S = Q K^T); dO is moved into tensor
-// memory once at the start (A operand of dP = dO V^T read from TMEM). TMEM:
-// dQ 256 columns, S 64, dP 64, dO 128. The row warps write dS (bf16) over the
-// S columns they have read, where dQ += dS K reads it as its A operand; the
-// next tile's S and dP are issued after that MMA. Shared memory then holds
-// only Q and the K / V stages: a K tile is held from its load until the dQ of
-// its tile, so it gets three stages, V two. The 64 KB where dO first lands
-// then holds the two V stages.
-namespace dq {
-constexpr int kM = 128, kBN = 64;
-constexpr int kQChunk = kM * 128;      // 16 KB: 128 rows x 64 columns
-constexpr int kKChunk = kBN * 128;     // 8 KB: 64 keys x 64 columns
-constexpr int kTile = 4 * kKChunk;     // 32 KB
-constexpr int kKS = 3, kVS = 2;        // K and V stages
-// Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
-// slices) at bb * 3 KB, its K^R rows at 24 KB + bb * 1 KB, its V rows
-// (4 x 1 KB) at bb * 4 KB.
-constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
-constexpr int oQ = 0, oK = oQ + 4 * kQChunk, oV = oK + kKS * kTile, oBar = oV + kVS * kTile;
-constexpr int oDOStage = oV;           // dO lands here first
-static_assert(kVS * kTile >= 4 * kQChunk, "dO staging area too small");
-constexpr int kSmem = oBar + 512 + 1024;
-static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
-constexpr int kThreads = 192;
-constexpr uint32_t kColDQ = 0, kColS = 256, kColP = 320, kColDO = 384;  // dO: 384..511
-}  // namespace dq
-
 struct BwdArgs {
     int n_h, S, N, W, L, R;
     float scale_log2, scale;
-    const __nv_bfloat16 *kc, *krr, *v;
-    const __nv_bfloat16 *qs, *dos;
     const float *ds_, *lses;
     const int32_t *cnt, *sorted_n, *sorted_a;
-    const float2 *tab;
-    __nv_bfloat16 *dq, *dkc, *dv;
-    float *dkr_part;
-    int hpg;  // heads per head group (key-major kernel)
+    __nv_bfloat16 *dkc, *dv;
+    float *dkr_part, *dqacc;
+    int hpg;  // heads per head group
     int n_ctx_items;
     uint32_t *err;
 };
 
-__global__ void __launch_bounds__(dq::kThreads, 1)
-    k_bwd_dq_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-                const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
-                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
-    using namespace dq;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kfull = bars + 0, *kempty = bars + kKS, *vfull = bars + 2 * kKS, *vempty = bars + 2 * kKS + kVS;
-    uint64_t *sfull = bars + 2 * (kKS + kVS), *dsready = sfull + 2, *dqdone = sfull + 4, *qfull = sfull + 6,
-             *drain = sfull + 7, *dotmem = sfull + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + 9);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 10);
-    int *counters = reinterpret_cast<int *>(sfull + 11);  // K issued, V issued, K consumed, V consumed, q issued
-
-    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int cnt = p.cnt[b];
-    const int i0 = g * kG;
-    if (i0 >= cnt) return;
-    const int gcnt = min(kG, cnt - i0);
-    const int nrows = kBlock * gcnt;
-    const int32_t *sa = p.sorted_a + (size_t)b * p.N + i0;
-    const int32_t *sn = p.sorted_n + (size_t)b * p.N + i0;
-    const int ctx_lo = max(0, sa[0] - p.W + 1);
-    const int ctx_hi = sa[gcnt - 1];
-    const int n_ctx = ctx_hi > ctx_lo ? (ctx_hi - ctx_lo + kBN - 1) / kBN : 0;
-    constexpr int kDraftBlocks = kBN / 8;  // draft tiles: 8 key slots per block
-    const int n_draft = (gcnt + kDraftBlocks - 1) / kDraftBlocks;
-    const int T = n_ctx + n_draft;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const size_t bh = (size_t)b * p.n_h + h;
-    const size_t srow0 = bh * p.R + (size_t)kBlock * i0;  // first sorted row of the group
-
-    // K stages start zeroed (masked key slots must hold finite values)
-    for (int e = threadIdx.x; e < (oV - oK) / 16; e += blockDim.x)
-        reinterpret_cast<uint4 *>(sm + oK)[e] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kKS; s++) {
-            mbar_init(&kfull[s], 1);
-            mbar_init(&kempty[s], 1);
-        }
-        for (int s = 0; s < kVS; s++) {
-            mbar_init(&vfull[s], 1);
-            mbar_init(&vempty[s], 1);
-        }
-        mbar_init(sfull, 1);
-        mbar_init(dsready, 4);
-        for (int s = 0; s < 2; s++) mbar_init(&dqdone[s], 1);
-        mbar_init(qfull, 1);
-        mbar_init(drain, 1);
-        mbar_init(dotmem, 4);
-        *abort_flag = 0;
-        for (int c = 0; c < 5; c++) counters[c] = 0;
-        fence_barrier_init();
-        fence_proxy_async_smem();
-    }
-    if (warp == 5) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 4) {
-        // ------------------------------------------------------- producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(qfull, 8 * kQChunk);
-            tma_load_3d(sm + oQ, &tm_qs, qfull, 0, (int)srow0, 0);
-            tma_load_3d(sm + oDOStage, &tm_dos, qfull, 0, (int)srow0, 0);
-            counters[4] = 1;
-        }
-        // lane l holds the block index of group block l (l < gcnt)
-        const int my_n = lane < gcnt ? sn[lane] : 0;
-        for (int t = 0; t < T; ++t) {
-            const int ks = t % kKS, vs = t % kVS;
-            uint8_t *kt = sm + oK + ks * kTile;
-            uint8_t *vt = sm + oV + vs * kTile;
-            if (t >= kKS && !warp_all(mbar_wait(&kempty[ks], ((t / kKS) - 1) & 1, abort_flag))) break;
-            if (t < n_ctx) {
-                const int pos0 = ctx_lo + t * kBN;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&kfull[ks], kTile);
-                    tma_load_3d(kt, &tm_kc, &kfull[ks], 0, (int)(bh * p.L + pos0), 0);
-                    tma_load_2d(kt + 3 * kKChunk, &tm_kr, &kfull[ks], 0, (int)((size_t)b * p.L + pos0));
-                }
-            } else {
-                // draft tile: 8 key slots per block (its 5 keys, then 3 masked rows)
-                const int d = t - n_ctx;
-                const int nb = min(kDraftBlocks, gcnt - d * kDraftBlocks);
-                if (lane == 0) mbar_arrive_expect_tx(&kfull[ks], nb * 8 * kDQK * 2);
-                for (int bb = 0; bb < nb; ++bb) {
-                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
-                    if (lane == 0) {
-                        const int row = p.S + kBlock * n;
-                        tma_load_3d(kt + bb * kDraftKcBlock, &tm_kc8, &kfull[ks], 0, (int)(bh * p.L + row), 0);
-                        tma_load_2d(kt + kDraftKr + bb * 1024, &tm_kr8, &kfull[ks], 0, (int)((size_t)b * p.L + row));
-                    }
-                }
-            }
-            if (lane == 0) counters[0] = t + 1;
-            // the V stages hold dO until the row warps have moved it to TMEM
-            if (t == 0 && !warp_all(mbar_wait(dotmem, 0, abort_flag))) break;
-            if (t >= kVS && !warp_all(mbar_wait(&vempty[vs], ((t / kVS) - 1) & 1, abort_flag))) break;
-            if (t < n_ctx) {
-                const int pos0 = ctx_lo + t * kBN;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&vfull[vs], kTile);
-                    tma_load_3d(vt, &tm_v, &vfull[vs], 0, (int)(bh * p.L + pos0), 0);
-                }
-            } else {
-                const int d = t - n_ctx;
-                const int nb = min(kDraftBlocks, gcnt - d * kDraftBlocks);
-                if (lane == 0) mbar_arrive_expect_tx(&vfull[vs], nb * 8 * kDV * 2);
-                for (int bb = 0; bb < nb; ++bb) {
-                    const int n = __shfl_sync(0xffffffffu, my_n, d * kDraftBlocks + bb);
-                    if (lane == 0) {
-                        const int row = p.S + kBlock * n;
-                        tma_load_3d(vt + bb * kDraftVBlock, &tm_v8, &vfull[vs], 0, (int)(bh * p.L + row), 0);
-                    }
-                }
-            }
-            if (lane == 0) counters[1] = t + 1;
-        }
-    } else if (warp == 5) {
-        // ----------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idS = idesc_bf16(kM, kBN, 0);    // S, dP: B = K / V tile, K-major
-            const uint32_t idQ = idesc_bf16(kM, kDQK, 1);   // dQ: B = K tile, MN-major
-            const SDesc qd = sdesc_split(sdesc_sw128(smem_u32(sm + oQ), 16, 1024));
-            bool ok = mbar_wait(qfull, 0, abort_flag);
-            if (ok) ok = mbar_wait(dotmem, 0, abort_flag);
-            const uint32_t idQc = idesc_bf16(kM, kDC, 1);   // draft tiles: dQ^C and dQ^R separately
-            const uint32_t idQr = idesc_bf16(kM, kDR, 1);
-            auto issue_sdp = [&](int t) {
-                const bool ctx = t < n_ctx;
-                const uint32_t kb = smem_u32(sm + oK + (t % kKS) * kTile), vb = smem_u32(sm + oV + (t % kVS) * kTile);
-                // B operands: context tile slices 8 KB apart with keys 128 B
-                // apart; draft tile block-major (K^C / V 8-key groups 3 KB / 4 KB
-                // apart, slices 1 KB apart; K^R at 24 KB)
-                const uint32_t step = ctx ? kKChunk : 1024;
-                const SDesc kd = sdesc_split(sdesc_sw128(kb, 16, ctx ? 1024 : kDraftKcBlock));
-                const SDesc krd = sdesc_split(sdesc_sw128(kb + kDraftKr, 16, 1024));
-                const SDesc vd = sdesc_split(sdesc_sw128(vb, 16, ctx ? 1024 : kDraftVBlock));
-                const uint32_t dS = tmem + kColS, dP = tmem + kColP;
-                // S and dP interleaved: two independent accumulation chains
-#pragma unroll
-                for (int k = 0; k < kDQK / 16; ++k) {
-                    const int c = k >> 2;
-                    const uint32_t sub = (k & 3) * 2;
-                    const uint32_t qo = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
-                    const uint64_t kbd = c < 3 ? kd.at(((c * step) >> 4) + sub) : krd.at(sub);
-                    mma_bf16_ss(dS, qd.at(qo), kbd, idS, k > 0 ? 1u : 0u);
-                    mma_bf16_ts(dP, tmem + kColDO + 8 * k, vd.at(((c * step) >> 4) + sub), idS, k > 0 ? 1u : 0u);
-                }
-                mma_commit(sfull);
-                mma_commit(&vempty[t % kVS]);
-            };
-            // Issue whichever is ready first: S/dP of tile ns (its K and V
-            // landed, and the dQ of tile ns - 1, which reads the dS written
-            // over the S columns, is issued) or dQ of tile nq (its dS is in
-            // TMEM).
-            int ns = 0, nq = 0;
-            uint64_t t_idle = 0;
-            if (ok) tc_fence_after();
-            while (ok && nq < T) {
-                bool issued = false;
-                if (ns < T && ns <= nq) {
-                    if (mbar_test(&kfull[ns % kKS], (ns / kKS) & 1) && mbar_test(&vfull[ns % kVS], (ns / kVS) & 1)) {
-                        counters[2] = ns + 1;
-                        counters[3] = ns + 1;
-                        tc_fence_after();
-                        issue_sdp(ns);
-                        ++ns;
-                        issued = true;
-                    }
-                }
-                if (!issued && nq < ns && mbar_test(dsready, nq & 1)) {
-                    const int s = nq & 1;
-                    tc_fence_after();
-                    const uint32_t da = tmem + kColS;  // dS: 64 keys as 32 columns of bf16 pairs
-                    const uint32_t kb = smem_u32(sm + oK + (nq % kKS) * kTile);
-                    if (nq < n_ctx) {  // B: all 256 columns, slices 8 KB apart, 16 keys = 2 KB
-                        const SDesc kd = sdesc_split(sdesc_sw128(kb, kKChunk, 1024));
-                        mma_bf16_ts(tmem + kColDQ, da, kd.at(0), idQ, nq > 0 ? 1u : 0u);
-#pragma unroll
-                        for (int k = 1; k < kBN / 16; ++k) mma_bf16_ts(tmem + kColDQ, da + 8 * k, kd.at(128 * k), idQ, 1u);
-                    } else {  // block-major: K^C (slices 1 KB apart, 2 blocks = 6 KB) and K^R (2 KB)
-                        const SDesc kdc = sdesc_split(sdesc_sw128(kb, 1024, kDraftKcBlock));
-                        const SDesc kdr = sdesc_split(sdesc_sw128(kb + kDraftKr, 1024, 1024));
-#pragma unroll
-                        for (int k = 0; k < kBN / 16; ++k) {
-                            const uint32_t acc = (nq > 0 || k > 0) ? 1u : 0u;
-                            mma_bf16_ts(tmem + kColDQ, da + 8 * k, kdc.at(((2 * kDraftKcBlock) >> 4) * k), idQc, acc);
-                            mma_bf16_ts(tmem + kColDQ + kDC, da + 8 * k, kdr.at(128 * k), idQr, acc);
-                        }
-                    }
-                    mma_commit(&kempty[nq % kKS]);
-                    mma_commit(&dqdone[s]);
-                    ++nq;
-                    issued = true;
-                }
-                if (issued) {
-                    t_idle = 0;
-                } else {
-                    const uint64_t now = globaltimer();
-                    if (t_idle == 0) t_idle = now;
-                    if (*abort_flag) ok = false;
-                    else if (now - t_idle > kWaitTimeoutNs) {
-                        *abort_flag = 1;
-                        ok = false;
-                    }
-                }
-            }
-        }
-    } else {
-        // ------------------------------------------------ rows (warps 0-3)
-        const int r = threadIdx.x;
-        const bool live = r < nrows;
-        int A = 0, n = 0, j = 0, lo = 0;
-        float lse2 = 0.f, Dr = 0.f;
-        if (live) {
-            A = sa[r / kBlock];
-            n = sn[r / kBlock];
-            j = r % kBlock;
-            lo = max(0, A - p.W + 1);
-            lse2 = p.lses[srow0 + r];
-            Dr = p.ds_[srow0 + r];
-        }
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        bool ok = warp_all(mbar_wait(qfull, 0, abort_flag));
-        {
-            // dO row r: shared memory (128-byte swizzled, 64-column chunks) ->
-            // TMEM lane r, columns kColDO.. (bf16 pairs, 8 per 16-byte unit)
-#pragma unroll 1
-            for (int c = 0; c < 4; c++) {
-                uint32_t w[32];
-#pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    const uint4 val = *reinterpret_cast<const uint4 *>(sm + oDOStage + c * kQChunk + sw128(r, u));
-                    w[4 * u + 0] = val.x;
-                    w[4 * u + 1] = val.y;
-                    w[4 * u + 2] = val.z;
-                    w[4 * u + 3] = val.w;
-                }
-                tmem_st32u(trow + kColDO + 32 * c, w);
-            }
-            // the V stages now hold dO rows or zero fill: finite, as masked
-            // key slots of draft tiles need
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dotmem);
-        }
-        for (int t = 0; t < T && ok; ++t) {
-            const int s = t & 1;
-            ok = warp_all(mbar_wait(sfull, t & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            float sv[64], pv[64];
-            {
-                float a0[32], a1[32], b0[32], b1[32];
-                tmem_ld32(trow + kColS, a0);
-                tmem_ld32(trow + kColS + 32, a1);
-                tmem_ld32(trow + kColP, b0);
-                tmem_ld32(trow + kColP + 32, b1);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; c++) {
-                    sv[c] = a0[c];
-                    sv[32 + c] = a1[c];
-                    pv[c] = b0[c];
-                    pv[32 + c] = b1[c];
-                }
-            }
-            (void)s;
-            // the row's keys in this tile: one contiguous column range [clo, chi)
-            int clo, chi;
-            if (t < n_ctx) {
-                const int c0 = ctx_lo + t * kBN;
-                clo = lo - c0;
-                chi = A - c0;
-            } else {
-                clo = 8 * (r / kBlock) - (t - n_ctx) * kBN;
-                chi = clo + kBlock;
-            }
-            if (!live) chi = clo;
-            uint32_t dsw[kBN / 2];  // dS as bf16 pairs, over the S columns just read
-#pragma unroll
-            for (int c = 0; c < kBN; c += 2) {
-                float e[2];
-#pragma unroll
-                for (int d = 0; d < 2; d++) {
-                    const float pp = (c + d >= clo && c + d < chi) ? ex2(fmaf(sv[c + d], p.scale_log2, -lse2)) : 0.f;
-                    e[d] = pp * (pv[c + d] - Dr) * p.scale;
-                }
-                dsw[c / 2] = pack_bf16x2(e[0], e[1]);
-            }
-            tmem_st32u(trow + kColS, dsw);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dsready);
-        }
-        if (ok) ok = warp_all(mbar_wait(&dqdone[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag));
-        if (ok) {
-            tc_fence_after();
-            // dQ row (rope slice rotated back by A + j) -> staging in the idle
-            // K stages (unit u of row r at u ^ (r & 31)) -> one 512-byte row
-            // per warp instruction
-            uint8_t *stage = sm + oK + warp * (32 * kDQK * 2);
-#pragma unroll 1
-            for (int c = 0; c < kDQK; c += 32) {
-                float v[32];
-                tmem_ld32(trow + kColDQ + c, v);
-                tmem_wait_ld();
-                if (c >= kDC) {  // rope slice: rotate back by the query position A + j
-                    const float2 *cs = p.tab + (size_t)(A + j) * (kDR / 2) + (c - kDC) / 2;
-#pragma unroll
-                    for (int k = 0; k < 16; k++) {
-                        const float2 t2 = live ? __ldg(cs + k) : make_float2(1.f, 0.f);
-                        const float x0 = v[2 * k], x1 = v[2 * k + 1];
-                        v[2 * k] = x0 * t2.x + x1 * t2.y;
-                        v[2 * k + 1] = x1 * t2.x - x0 * t2.y;
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const int u = c / 8 + k;
-                    *reinterpret_cast<uint4 *>(stage + lane * 512 + ((u ^ lane) << 4)) = make_uint4(
-                        pack_bf16x2(v[8 * k + 0], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
-                        pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
-                }
-            }
-            __syncwarp();
-            for (int i = 0; i < 32; i++) {
-                const int rr = warp * 32 + i;
-                if (rr >= nrows) break;  // uniform
-                const int ni = __shfl_sync(0xffffffffu, n, i), ji = __shfl_sync(0xffffffffu, j, i);
-                const uint4 val = *reinterpret_cast<const uint4 *>(stage + i * 512 + ((lane ^ i) << 4));
-                *reinterpret_cast<uint4 *>(p.dq + (bh * p.R + kBlock * ni + ji) * kDQK + 8 * lane) = val;
-            }
-        }
-    }
-
-    __syncthreads();
-    if (*abort_flag) {
-        volatile int never = 0;
-        if (warp == 4 && lane == 0) {
-            if (counters[4]) mbar_wait(qfull, 0, (volatile int *)&never);
-            for (int t = counters[2]; t < counters[0]; ++t)
-                mbar_wait(&kfull[t % kKS], (t / kKS) & 1, (volatile int *)&never);
-            for (int t = counters[3]; t < counters[1]; ++t)
-                mbar_wait(&vfull[t % kVS], (t / kVS) & 1, (volatile int *)&never);
-        }
-        if (warp == 5 && lane == 0) {
-            mma_commit(drain);
-            mbar_wait(drain, 0, (volatile int *)&never);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 5) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-    if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
+__device__ __forceinline__ void red_add_v4(float *addr, const uint4 &v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(v.x)),
+                 "f"(__uint_as_float(v.y)), "f"(__uint_as_float(v.z)), "f"(__uint_as_float(v.w))
+                 : "memory");
 }
 
-// ============================================================== dK / dV
-// Key tile = 64 keys (MMA M = 64); dK and dV of the tile in one CTA, so K, V
-// and every row of Q and dO that sees the tile cross into shared memory once.
-// With M = 64 an accumulator occupies lanes 0-15 of each 32-lane TMEM
-// sub-partition, and a second one addressed at lane offset 16 the lanes 16-31
-// of the same columns: dK (offset 0) and dV (offset 16) share columns 0..255,
-// S^T (0) and dP^T (16) share a 64-column buffer (two buffers, columns 256 and
-// 320). dK's columns 192..255 are the rope slice: it is summed over the heads
-// of the group, so that part of the accumulator is never reset between heads.
-// Per head: the K^C and V tiles (one stage, reloaded once the head's last
-// S^T / dP^T completed; the rope-key tile is the same for all heads and is
-// loaded once), then the rows that see the tile in chunks of 64 (Q and dO,
-// two stages): S^T = K Q^T and dP^T = V dO^T, P^T and dS^T (bf16) through one
-// shared-memory buffer, dV += P^T dO, dK += dS^T Q.
+// ============================================================= one pass
+// Key tile = 64 keys (MMA M = 64); dK, dV and the dQ contributions of the
+// tile in one CTA, so K, V and every row of Q and dO that sees the tile cross
+// into shared memory once per head. With M = 64 an accumulator occupies lanes
+// 0-15 of each 32-lane TMEM sub-partition, and a second one addressed at lane
+// offset 16 the lanes 16-31 of the same columns:
+//   columns   0..255  dK (offset 0; 192..255 the rope slice, summed over the
+//                     group's heads, never reset between heads) and dV (16);
+//   columns 256..383  S^T (0) and dP^T (16), two buffers of 64 columns;
+//   columns 384..511  the chunk's dQ contribution: M = 64 rows, dims 0..127 at
+//                     offset 0, dims 128..255 at offset 16.
+// Per head: the K^C and V tiles (KVS stages; the rope-key tile is the same
+// for all heads and is loaded once), then the rows that see the tile in chunks
+// of 64 (Q and dO, RS stages): S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
+// (bf16) through one shared-memory buffer, dV += P^T dO, dK += dS^T Q, and
+// dQ_c = dS K with dS read as an MN-major A operand from the dS^T tile.
 // Key warps: warp w covers keys 16 (w & 3) .. + 15 (TMEM sub-partition w & 3)
 // and rows 32 (w >> 2) .. + 31 of a chunk. Lane l < 16 loads S^T of its key,
 // lane l + 16 dP^T of the same key; the two swap halves, so each lane holds
-// both for 16 rows. At a head's end they copy the accumulators, as bf16, into
-// the 128 free TMEM columns (the stash), which frees them for the next head;
-// four store warps write the stash out to dK^C / dV while the next head runs.
-namespace kv {
+// both for 16 rows. At a head's end they read the accumulators, round them to
+// bf16 and store dK^C and dV through a staging area in the P^T / dS^T buffer.
+// dQ warps (one per TMEM sub-partition) read each chunk's dQ contribution and
+// add it into the fp32 accumulator (four 128-byte row segments per vector
+// reduction instruction).
+namespace bw {
 constexpr int kMK = 64;                    // keys per tile (MMA M)
 constexpr int kRC = 64;                    // rows per chunk (MMA N of S^T / dP^T, K of the accumulations)
 constexpr int kSlice = 64 * 128;           // 8 KB: 64 keys or rows x 64 columns, 128-byte swizzled
@@ -578,39 +188,48 @@ constexpr int kSlice = 64 * 128;           // 8 KB: 64 keys or rows x 64 columns
 // rows (4 x 1 KB) at bb * 4 KB: 8-key groups 3 KB / 4 KB apart, 64-column
 // slices 1 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftVBlock = 4 * 1024;
-constexpr int oKr = 0, oKc = oKr + kSlice, oV = oKc + 3 * kSlice;
+constexpr int kKV = 7 * kSlice;            // one head's K^C (3 slices) then V (4 slices)
 constexpr int kRowStage = 8 * kSlice;      // Q chunk (4 slices), then dO chunk (4 slices)
-constexpr int oRow = oV + 4 * kSlice;
-constexpr int oPT = oRow + 2 * kRowStage;  // P^T, then dS^T: [64 keys][64 rows] bf16 each
-constexpr int oStage = oPT + 2 * kSlice;   // epilogue staging, 2 KB per store warp
-constexpr int oMeta = oStage + 4 * 2048;   // per row stage: (LSE * log2 e, D) of each row
-constexpr int oBar = oMeta + 2 * kRC * 8;
-constexpr int kSmem = oBar + 256 + 1024;
-static_assert(kSmem <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+constexpr int kPT = 2 * kSlice;            // P^T, then dS^T: [64 keys][64 rows] bf16 each
+constexpr int kDqStage = 32 * 64;          // per dQ warp: 32 lanes x 16 fp32
 constexpr int kKeyWarps = 8;
 constexpr int kWarpKV = kKeyWarps, kWarpRow = kKeyWarps + 1, kWarpMma = kKeyWarps + 2;
-constexpr int kWarpSt = kKeyWarps + 3;     // four store warps, one per TMEM sub-partition
+constexpr int kWarpDq = kKeyWarps + 3;     // four dQ warps, one per TMEM sub-partition
 constexpr int kThreads = (kKeyWarps + 7) * 32;
-constexpr uint32_t kColAcc = 0, kColS = 256;  // S^T / dP^T buffer s at kColS + 64 s
-constexpr uint32_t kColStash = 384;           // a finished head's dK / dV as bf16 pairs (128 columns)
-constexpr uint32_t kHi = 16u << 16;           // lane offset of the second M = 64 accumulator
-}  // namespace kv
+constexpr uint32_t kColAcc = 0, kColS = 256, kColDQ = 384;  // S^T / dP^T buffer s at kColS + 64 s
+constexpr uint32_t kHi = 16u << 16;        // lane offset of the second M = 64 accumulator
+
+// Shared memory for KVS K/V stages and RS row stages.
+template <int KVS, int RS>
+struct Smem {
+    static constexpr int oKr = 0;                          // rope-key tile (8 KB)
+    static constexpr int oKV = oKr + kSlice;               // K/V stage s at oKV + s * kKV
+    static constexpr int oRow = oKV + KVS * kKV;           // row stage s at oRow + s * kRowStage
+    static constexpr int oPT = oRow + RS * kRowStage;      // P^T / dS^T buffer u at oPT + u * kPT
+    static constexpr int oStage = oPT + 2 * kPT;           // dQ warps' staging
+    static constexpr int oMeta = oStage + 4 * kDqStage;    // per row stage: (LSE * log2 e, D) of each row
+    static constexpr int oBar = oMeta + RS * kRC * 8;
+    static constexpr int kBytes = oBar + 256 + 1024;       // barriers, counters, alignment slack
+    static_assert(kBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
+};
+}  // namespace bw
 
 // One CTA per (64-key tile, head group, batch row).
-__global__ void __launch_bounds__(kv::kThreads, 1)
-    k_bwd_kv_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-                const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
-                const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8,
-                const BwdArgs p) {
-    using namespace kv;
+template <int KVS, int RS>
+__global__ void __launch_bounds__(bw::kThreads, 1)
+    k_bwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
+             const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
+             const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
+    using namespace bw;
+    using L = Smem<KVS, RS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
-    uint64_t *kvfull = bars + 0, *kvfree = bars + 1, *rowfull = bars + 2, *rowfree = bars + 4, *sfull = bars + 6,
-             *dsready = bars + 8, *ptfree = bars + 9, *drain = bars + 10, *stashfull = bars + 11,
-             *stashfree = bars + 12;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::oBar);
+    uint64_t *kvfull = bars + 0, *kvfree = bars + 2, *rowfull = bars + 4, *rowfree = bars + 6, *sfull = bars + 8,
+             *ptfree = bars + 10, *dsready = bars + 12, *dqfull = bars + 13, *dqfree = bars + 14, *kdrain = bars + 15,
+             *accdone = bars + 16, *drain = bars + 17;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     // K/V heads issued, row chunks issued, K/V heads consumed, row chunks consumed
     int *counters = reinterpret_cast<int *>(tmem_slot + 2);
@@ -666,7 +285,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     const bool dlane = lane >= 16;   // lane of the dP^T / dV half
     bool key_valid = false;
     size_t key_pos = 0;
-    if (warp < kKeyWarps || warp >= kWarpSt) {
+    if (warp < kKeyWarps) {
         if (is_ctx) {
             key_valid = t0 + kk < p.S;
             key_pos = (size_t)t0 + kk;
@@ -697,21 +316,27 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     }
 
     // K/V tiles start zeroed (key slots no load reaches must hold finite values)
-    for (int e = threadIdx.x; e < (oRow - oKr) / 16; e += blockDim.x)
-        reinterpret_cast<uint4 *>(sm + oKr)[e] = make_uint4(0, 0, 0, 0);
+    for (int e = threadIdx.x; e < (L::oRow - L::oKr) / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + L::oKr)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        mbar_init(kvfull, 1);
-        mbar_init(kvfree, 1);
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < KVS; s++) {
+            mbar_init(&kvfull[s], 1);
+            mbar_init(&kvfree[s], 1);
+        }
+        for (int s = 0; s < RS; s++) {
             mbar_init(&rowfull[s], 1);
             mbar_init(&rowfree[s], 1);
+        }
+        for (int s = 0; s < 2; s++) {
             mbar_init(&sfull[s], 1);
+            mbar_init(&ptfree[s], 1);
         }
         mbar_init(dsready, kKeyWarps);
-        mbar_init(ptfree, 1);
+        mbar_init(accdone, 1);
+        mbar_init(dqfull, 1);
+        mbar_init(dqfree, 4);
+        mbar_init(kdrain, kKeyWarps);
         mbar_init(drain, 1);
-        mbar_init(stashfull, kKeyWarps);
-        mbar_init(stashfree, 4);
         *abort_flag = 0;
         for (int c = 0; c < 4; c++) counters[c] = 0;
         fence_barrier_init();
@@ -731,25 +356,28 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         // ------------------------------------------- producer of K/V tiles
         const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
         for (int hh = 0; hh < H; ++hh) {
+            const int s = hh % KVS;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            if (hh >= 1 && !warp_all(mbar_wait(kvfree, (hh - 1) & 1, abort_flag))) break;
+            if (hh >= KVS && !warp_all(mbar_wait(&kvfree[s], ((hh / KVS) - 1) & 1, abort_flag))) break;
+            uint8_t *kv = sm + L::oKV + s * kKV;
             if (is_ctx) {
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(kvfull, (hh == 0 ? 8 : 7) * kSlice);
-                    if (hh == 0) tma_load_2d(sm + oKr, &tm_kr, kvfull, 0, (int)((size_t)b * p.L + t0));
-                    tma_load_3d(sm + oKc, &tm_kc, kvfull, 0, (int)(bh * p.L + t0), 0);
-                    tma_load_3d(sm + oV, &tm_v, kvfull, 0, (int)(bh * p.L + t0), 0);
+                    mbar_arrive_expect_tx(&kvfull[s], (hh == 0 ? 8 : 7) * kSlice);
+                    if (hh == 0) tma_load_2d(sm + L::oKr, &tm_kr, &kvfull[s], 0, (int)((size_t)b * p.L + t0));
+                    tma_load_3d(kv, &tm_kc, &kvfull[s], 0, (int)(bh * p.L + t0), 0);
+                    tma_load_3d(kv + 3 * kSlice, &tm_v, &kvfull[s], 0, (int)(bh * p.L + t0), 0);
                 }
             } else {
-                if (lane == 0) mbar_arrive_expect_tx(kvfull, gcnt * 8 * ((hh == 0 ? kDQK : kDC) + kDV) * 2);
+                if (lane == 0) mbar_arrive_expect_tx(&kvfull[s], gcnt * 8 * ((hh == 0 ? kDQK : kDC) + kDV) * 2);
                 for (int bb = 0; bb < gcnt; ++bb) {
                     const int nb = __shfl_sync(0xffffffffu, my_n, bb);
                     if (lane == 0) {
                         const int row = p.S + kBlock * nb;
-                        tma_load_3d(sm + oKc + bb * kDraftKcBlock, &tm_kc8, kvfull, 0, (int)(bh * p.L + row), 0);
+                        tma_load_3d(kv + bb * kDraftKcBlock, &tm_kc8, &kvfull[s], 0, (int)(bh * p.L + row), 0);
                         if (hh == 0)
-                            tma_load_2d(sm + oKr + bb * 1024, &tm_kr8, kvfull, 0, (int)((size_t)b * p.L + row));
-                        tma_load_3d(sm + oV + bb * kDraftVBlock, &tm_v8, kvfull, 0, (int)(bh * p.L + row), 0);
+                            tma_load_2d(sm + L::oKr + bb * 1024, &tm_kr8, &kvfull[s], 0, (int)((size_t)b * p.L + row));
+                        tma_load_3d(kv + 3 * kSlice + bb * kDraftVBlock, &tm_v8, &kvfull[s], 0, (int)(bh * p.L + row),
+                                    0);
                     }
                 }
             }
@@ -757,23 +385,49 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         }
     } else if (warp == kWarpRow) {
         // ---------------------------- producer of Q / dO chunks and row data
-        for (int q = 0; q < QT; ++q) {
-            const int hh = q / nchunks, c = q % nchunks, s = q & 1;
+        // The row data of chunk q + 1 (LSE * log2 e and D, one value per lane
+        // and 32 rows) is read into registers, and its Q / dO rows prefetched
+        // into L2, while chunk q is in use, so that once the stage is free only
+        // the shared-memory copy remains.
+        auto meta_of = [&](int q, float2 (&m)[kRC / 32]) {
+            const int hh = q / nchunks, c = q % nchunks;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
             const int r0 = row0 + c * kRC;
-            if (q >= 2 && !warp_all(mbar_wait(&rowfree[s], ((q >> 1) - 1) & 1, abort_flag))) break;
-            float2 *mLD = reinterpret_cast<float2 *>(sm + oMeta + s * kRC * 8);
 #pragma unroll
-            for (int jj = 0; jj < kRC; jj += 32) {
-                const int rowi = r0 + jj + lane;
-                mLD[jj + lane] = rowi < row0 + nrows ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi])
-                                                     : make_float2(0.f, 0.f);
+            for (int jj = 0; jj < kRC / 32; jj++) {
+                const int rowi = r0 + 32 * jj + lane;
+                m[jj] = rowi < row0 + nrows ? make_float2(p.lses[bh * p.R + rowi], p.ds_[bh * p.R + rowi])
+                                            : make_float2(0.f, 0.f);
             }
+        };
+        float2 mnext[kRC / 32];
+        meta_of(0, mnext);
+        for (int q = 0; q < QT; ++q) {
+            const int hh = q / nchunks, c = q % nchunks, s = q % RS;
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+            const int r0 = row0 + c * kRC;
+            float2 mcur[kRC / 32];
+#pragma unroll
+            for (int jj = 0; jj < kRC / 32; jj++) mcur[jj] = mnext[jj];
+            if (q + 1 < QT) {
+                meta_of(q + 1, mnext);
+                if (lane == 0) {
+                    const int hn = (q + 1) / nchunks, cn = (q + 1) % nchunks;
+                    const int rn = (int)(((size_t)b * p.n_h + h0 + hn) * p.R + row0 + cn * kRC);
+                    tma_prefetch_l2_3d(&tm_qs, 0, rn, 0);
+                    tma_prefetch_l2_3d(&tm_dos, 0, rn, 0);
+                }
+            }
+            if (q >= RS && !warp_all(mbar_wait(&rowfree[s], ((q / RS) - 1) & 1, abort_flag))) break;
+            float2 *mLD = reinterpret_cast<float2 *>(sm + L::oMeta + s * kRC * 8);
+#pragma unroll
+            for (int jj = 0; jj < kRC / 32; jj++) mLD[32 * jj + lane] = mcur[jj];
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(&rowfull[s], kRowStage);
-                tma_load_3d(sm + oRow + s * kRowStage, &tm_qs, &rowfull[s], 0, (int)(bh * p.R + r0), 0);
-                tma_load_3d(sm + oRow + s * kRowStage + 4 * kSlice, &tm_dos, &rowfull[s], 0, (int)(bh * p.R + r0), 0);
+                tma_load_3d(sm + L::oRow + s * kRowStage, &tm_qs, &rowfull[s], 0, (int)(bh * p.R + r0), 0);
+                tma_load_3d(sm + L::oRow + s * kRowStage + 4 * kSlice, &tm_dos, &rowfull[s], 0, (int)(bh * p.R + r0),
+                            0);
                 counters[1] = q + 1;
             }
         }
@@ -784,22 +438,36 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
             const uint32_t idV = idesc_bf16(kMK, kDV, 1);   // dV: B = dO chunk, MN-major
             const uint32_t idKc = idesc_bf16(kMK, kDC, 1);  // dK^C: B = Q^C columns
             const uint32_t idKr = idesc_bf16(kMK, kDR, 1);  // dK^R: B = Q^R columns
-            // A operands: K^C / V slices kcStep / vStep bytes apart (context
-            // tile: 8 KB slices of 64 keys; draft tile: block-major)
-            const uint32_t kcStep = is_ctx ? kSlice : 1024, vStep = is_ctx ? kSlice : 1024;
-            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + oKc), 16, is_ctx ? 1024 : kDraftKcBlock));
-            const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + oKr), 16, 1024));
-            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + oV), 16, is_ctx ? 1024 : kDraftVBlock));
-            const SDesc ptd = sdesc_split(sdesc_sw128(smem_u32(sm + oPT), 16, 1024));
-            const SDesc dsd = sdesc_split(sdesc_sw128(smem_u32(sm + oPT + kSlice), 16, 1024));
+            // dQ_c = dS K: A = dS (M = 64 rows, K = keys) read MN-major from the
+            // dS^T tile, B = the key tile (N = dims, K = keys), MN-major
+            const uint32_t idQ128 = idesc_bf16_ab(kRC, 128, 1, 1);
+            const uint32_t idQ64 = idesc_bf16_ab(kRC, 64, 1, 1);
+            // A operands of S^T / dP^T: K^C / V slices kcStep bytes apart
+            // (context tile: 8 KB slices of 64 keys; draft tile: block-major)
+            const uint32_t kcStep = is_ctx ? kSlice : 1024;
+            const uint32_t kOff = is_ctx ? 1024 : kDraftKcBlock, vOff = is_ctx ? 1024 : kDraftVBlock;
+            const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), 16, 1024));
+            // P^T / dS^T buffer u: descriptors of buffer 0 plus kPT / 16 * u
+            const SDesc ptd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT), 16, 1024));
+            const SDesc dsd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT + kSlice), 16, 1024));
+            const SDesc dsq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT + kSlice), kSlice, 1024));
+            constexpr uint32_t kPTu = kPT >> 4;
+            // B operands of dQ_c, MN-major: dims 0..127 of K^C (two slices),
+            // dims 128..191 (third slice), the rope key (dims 192..255); 16 keys
+            // are 2 KB in every case (context: 16 rows of 128 B; draft: 2 blocks)
+            const SDesc krq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), is_ctx ? kSlice : 1024, 1024));
+            const uint32_t kcq_step = is_ctx ? 128u : (uint32_t)((2 * kDraftKcBlock) >> 4);
             bool ok = true;
             auto issue_s = [&](int q) {
-                const int c = q % nchunks, s = q & 1;
+                const int hh = q / nchunks, s = q % RS, bsel = q & 1;
                 tc_fence_after();
-                const uint32_t rs = smem_u32(sm + oRow + s * kRowStage);
+                const uint32_t kb = smem_u32(sm + L::oKV + (hh % KVS) * kKV);
+                const SDesc kad = sdesc_split(sdesc_sw128(kb, 16, kOff));
+                const SDesc vad = sdesc_split(sdesc_sw128(kb + 3 * kSlice, 16, vOff));
+                const uint32_t rs = smem_u32(sm + L::oRow + s * kRowStage);
                 const SDesc qd = sdesc_split(sdesc_sw128(rs, 16, 1024));
                 const SDesc dod = sdesc_split(sdesc_sw128(rs + 4 * kSlice, 16, 1024));
-                const uint32_t dS = tmem + kColS + 64 * s, dP = dS + kHi;
+                const uint32_t dS = tmem + kColS + 64 * bsel, dP = dS + kHi;
                 // S^T = K Q^T and dP^T = V dO^T interleaved: two independent chains
 #pragma unroll
                 for (int k16 = 0; k16 < kDQK / 16; ++k16) {
@@ -808,46 +476,67 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                     const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
                     const uint32_t ro = (cc * kSlice + (k16 & 3) * 32) >> 4;
                     mma_bf16_ss(dS, ka, qd.at(ro), idS, k16 > 0 ? 1u : 0u);
-                    mma_bf16_ss(dP, vad.at(((cc * vStep) >> 4) + sub), dod.at(ro), idS, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(dP, vad.at(((cc * kcStep) >> 4) + sub), dod.at(ro), idS, k16 > 0 ? 1u : 0u);
                 }
-                mma_commit(&sfull[s]);
-                if (c == nchunks - 1) mma_commit(kvfree);
+                mma_commit(&sfull[bsel]);
             };
             auto issue_acc = [&](int q) {
-                const int c = q % nchunks, s = q & 1;
+                const int c = q % nchunks, s = q % RS;
+                const uint32_t pu = kPTu * (q & 1);
                 tc_fence_after();
-                const uint32_t rs = smem_u32(sm + oRow + s * kRowStage);
-                const SDesc qb = sdesc_split(sdesc_sw128(rs, kSlice, 1024));            // MN-major
+                const uint32_t rs = smem_u32(sm + L::oRow + s * kRowStage);
+                const SDesc qb = sdesc_split(sdesc_sw128(rs, kSlice, 1024));  // MN-major
                 const SDesc dob = sdesc_split(sdesc_sw128(rs + 4 * kSlice, kSlice, 1024));
                 // 16 rows per MMA: 32 bytes along the K-major P^T / dS^T rows,
                 // 2 KB (16 rows of 128 bytes) in the row chunk
 #pragma unroll
                 for (int k16 = 0; k16 < kRC / 16; ++k16)
-                    mma_bf16_ss(tmem + kColAcc + kHi, ptd.at(2 * k16), dob.at(128 * k16), idV,
+                    mma_bf16_ss(tmem + kColAcc + kHi, ptd.at(pu + 2 * k16), dob.at(128 * k16), idV,
                                 (c > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
                 for (int k16 = 0; k16 < kRC / 16; ++k16)
-                    mma_bf16_ss(tmem + kColAcc, dsd.at(2 * k16), qb.at(128 * k16), idKc, (c > 0 || k16 > 0) ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColAcc, dsd.at(pu + 2 * k16), qb.at(128 * k16), idKc, (c > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
                 for (int k16 = 0; k16 < kRC / 16; ++k16)
-                    mma_bf16_ss(tmem + kColAcc + kDC, dsd.at(2 * k16), qb.at(((3 * kSlice) >> 4) + 128 * k16), idKr,
+                    mma_bf16_ss(tmem + kColAcc + kDC, dsd.at(pu + 2 * k16), qb.at(((3 * kSlice) >> 4) + 128 * k16), idKr,
                                 (q > 0 || k16 > 0) ? 1u : 0u);
                 mma_commit(&rowfree[s]);
-                mma_commit(ptfree);
+                if (c == nchunks - 1) mma_commit(accdone);  // the head's accumulators are final
+            };
+            auto issue_dq = [&](int q) {
+                const int hh = q / nchunks, c = q % nchunks;
+                const uint32_t pu = kPTu * (q & 1);
+                tc_fence_after();
+                const uint32_t kb = smem_u32(sm + L::oKV + (hh % KVS) * kKV);
+                const SDesc kq0 = sdesc_split(sdesc_sw128(kb, is_ctx ? kSlice : 1024, kOff));
+                const SDesc kq1 = sdesc_split(sdesc_sw128(kb + (is_ctx ? 2 * kSlice : 2048), kSlice, kOff));
+#pragma unroll
+                for (int k16 = 0; k16 < kMK / 16; ++k16) {
+                    const uint64_t a = dsq.at(pu + 128 * k16);  // 16 keys = 16 rows of the dS^T tile
+                    mma_bf16_ss(tmem + kColDQ, a, kq0.at(kcq_step * k16), idQ128, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColDQ + kHi, a, kq1.at(kcq_step * k16), idQ64, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColDQ + kHi + 64, a, krq.at(128 * k16), idQ64, k16 > 0 ? 1u : 0u);
+                }
+                mma_commit(dqfull);
+                mma_commit(&ptfree[q & 1]);
+                if (c == nchunks - 1) mma_commit(&kvfree[hh % KVS]);
             };
             // Issue whichever is ready: the S^T stage of chunk ns (its K/V tile
-            // and row operands landed; at most one chunk ahead, so its S^T /
-            // dP^T buffer was read by the key warps before they signalled chunk
-            // ns - 2) or the accumulation of chunk na (P^T / dS^T written; at a
-            // head's first chunk the key warps have also read the previous
-            // head's accumulators, which precedes that signal).
-            int ns = 0, na = 0;
+            // and row operands landed; at most one chunk ahead of the
+            // accumulations, so its S^T / dP^T buffer was read by the key
+            // warps before they signalled chunk ns - 2), the accumulation of
+            // chunk na (P^T / dS^T written; at a head's first chunk the key
+            // warps have also read out the previous head's accumulators, which
+            // precedes that signal), or the dQ contribution of chunk nd (its
+            // accumulation issued, the dQ warps have read chunk nd - 1's).
+            int ns = 0, na = 0, nd = 0;
             uint64_t t_idle = 0;
-            while (ok && na < QT) {
+            while (ok && nd < QT) {
                 bool issued = false;
                 if (ns < QT && ns <= na + 1) {
                     const int hh = ns / nchunks, c = ns % nchunks;
-                    if ((c != 0 || mbar_test(kvfull, hh & 1)) && mbar_test(&rowfull[ns & 1], (ns >> 1) & 1)) {
+                    if ((c != 0 || mbar_test(&kvfull[hh % KVS], (hh / KVS) & 1)) &&
+                        mbar_test(&rowfull[ns % RS], (ns / RS) & 1)) {
                         if (c == 0) counters[2] = hh + 1;
                         counters[3] = ns + 1;
                         issue_s(ns);
@@ -858,6 +547,11 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 if (!issued && na < ns && mbar_test(dsready, na & 1)) {
                     issue_acc(na);
                     ++na;
+                    issued = true;
+                }
+                if (!issued && nd < na && (nd == 0 || mbar_test(dqfree, (nd - 1) & 1))) {
+                    issue_dq(nd);
+                    ++nd;
                     issued = true;
                 }
                 if (issued) {
@@ -873,54 +567,50 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 }
             }
         }
-    } else if (warp >= kWarpSt) {
-        // ------------------------------------------------ store warps
-        // Sub-partition warp & 3: keys 16 (warp & 3) .. + 15, lanes 0-15 their
-        // dK, lanes 16-31 their dV. Per head: the stash (128 columns of bf16
-        // pairs: accumulator columns 128 hr + 32 rd .. + 31 at stash column
-        // 64 hr + 16 rd) in eight rounds of 32 values; each thread stages its
-        // 64 bytes (16-byte unit u at u ^ (lane & 3)), then the warp writes 8
-        // rows' 64-byte segments per instruction. dK columns 192..255 (the
-        // rope slice) are not written: they stay in TMEM, summed over heads.
-        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        uint8_t *stage = sm + oStage + (warp - kWarpSt) * 2048;
-        for (int hh = 0; hh < H; ++hh) {
-            if (!warp_all(mbar_wait(stashfull, hh & 1, abort_flag))) break;
+    } else if (warp >= kWarpDq) {
+        // --------------------------------------------------- dQ warps
+        // Sub-partition sp: lanes 0-15 hold dims 0..127 of chunk rows
+        // 16 sp .. + 15, lanes 16-31 dims 128..255 of the same rows. Per chunk:
+        // four loads of 32 columns, each staged in two halves (each thread its
+        // 64 bytes, 16-byte unit u at u ^ (lane & 3)); the warp adds eight rows'
+        // 64-byte segments per instruction into the accumulator (sorted rows).
+        const int sp = warp & 3;  // a warp reaches the TMEM lanes of sub-partition warp % 4 only
+        const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
+        uint8_t *stage = sm + L::oStage + sp * kDqStage;
+        bool ok = true;
+        for (int q = 0; q < QT && ok; ++q) {
+            const int hh = q / nchunks, c = q % nchunks;
+            ok = warp_all(mbar_wait(dqfull, q & 1, abort_flag));
+            if (!ok) break;
             tc_fence_after();
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
+            const int cr0 = c * kRC + 16 * sp;  // chunk-relative band row of lane 0
+            float *acc_rows = p.dqacc + (bh * p.R + row0) * kDQK;
 #pragma unroll 1
-            for (int rr = 0; rr < 4; rr++) {
+            for (int rd = 0; rd < 4; rd++) {
                 float v[32];
-                tmem_ld32(trow + kColStash + 32 * rr, v);
+                tmem_ld32(trow + kColDQ + 32 * rd, v);
                 tmem_wait_ld();
-                if (rr == 3) {  // the stash is free for the next head
+                if (rd == 3) {  // the dQ columns are free for the next chunk
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(stashfree);
+                    if (lane == 0) mbar_arrive(dqfree);
                 }
 #pragma unroll
-                for (int sub = 0; sub < 2; sub++) {
-                    const int col = (rr >> 1) * 128 + ((rr & 1) * 2 + sub) * 32;
-                    const bool rope = col >= kDC;
+                for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
                     for (int u = 0; u < 4; u++)
                         *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
-                            make_uint4(__float_as_uint(v[16 * sub + 4 * u]), __float_as_uint(v[16 * sub + 4 * u + 1]),
-                                       __float_as_uint(v[16 * sub + 4 * u + 2]),
-                                       __float_as_uint(v[16 * sub + 4 * u + 3]));
+                            make_uint4(__float_as_uint(v[16 * hf + 4 * u]), __float_as_uint(v[16 * hf + 4 * u + 1]),
+                                       __float_as_uint(v[16 * hf + 4 * u + 2]), __float_as_uint(v[16 * hf + 4 * u + 3]));
                     __syncwarp();
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
-                        const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
-                        const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
-                        const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
-                        const bool is_v = kl >= 16;
-                        if (kvl && (is_v || !rope)) {
-                            const uint4 val =
-                                *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
-                            __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
-                                                      : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
-                            *reinterpret_cast<uint4 *>(dst) = val;
+                        const int sl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
+                        const int br = cr0 + (sl & 15);                    // band row
+                        if (br < nrows) {
+                            const uint4 val = *reinterpret_cast<const uint4 *>(stage + sl * 64 + ((u ^ (sl & 3)) << 4));
+                            red_add_v4(acc_rows + (size_t)br * kDQK + (sl >> 4) * 128 + 32 * rd + 16 * hf + 4 * u, val);
                         }
                     }
                     __syncwarp();
@@ -963,13 +653,13 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         const uint32_t pu1 = prow + (((((uint32_t)rb >> 3) + 1) ^ (kk & 7)) << 4);
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
-            const int hh = q / nchunks, c = q % nchunks, s = q & 1;
-            ok = warp_all(mbar_wait(&rowfull[s], (q >> 1) & 1, abort_flag));  // row data
-            if (ok) ok = warp_all(mbar_wait(&sfull[s], (q >> 1) & 1, abort_flag));
+            const int hh = q / nchunks, c = q % nchunks, s = q % RS, bsel = q & 1;
+            ok = warp_all(mbar_wait(&rowfull[s], (q / RS) & 1, abort_flag));  // row data
+            if (ok) ok = warp_all(mbar_wait(&sfull[bsel], (q >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
             float v[32];
-            tmem_ld32(trow + kColS + 64 * s + 32 * hr, v);
+            tmem_ld32(trow + kColS + 64 * bsel + 32 * hr, v);
             tmem_wait_ld();
             float sv[16], pv[16];
 #pragma unroll
@@ -979,7 +669,7 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 sv[i] = dlane ? recv : v[i];
                 pv[i] = dlane ? v[16 + i] : recv;
             }
-            const float2 *mLD = reinterpret_cast<const float2 *>(sm + oMeta + s * kRC * 8) + rb;
+            const float2 *mLD = reinterpret_cast<const float2 *>(sm + L::oMeta + s * kRC * 8) + rb;
             const int jlo = rlo - c * kRC - rb, jhi = rhi - c * kRC - rb;  // visible rows, relative to rb
             uint32_t pw[8], dw[8];
 #pragma unroll
@@ -996,42 +686,68 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
                 pw[i / 2] = pack_bf16x2(ep[0], ep[1]);
                 dw[i / 2] = pack_bf16x2(ed[0], ed[1]);
             }
-            // the P^T / dS^T buffer is free once the accumulation of chunk q - 1 completed
-            if (q >= 1) {
-                ok = warp_all(mbar_wait(ptfree, (q - 1) & 1, abort_flag));
-                if (!ok) break;
-            }
-            *reinterpret_cast<uint4 *>(sm + oPT + pu0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-            *reinterpret_cast<uint4 *>(sm + oPT + pu1) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-            *reinterpret_cast<uint4 *>(sm + oPT + kSlice + pu0) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
-            *reinterpret_cast<uint4 *>(sm + oPT + kSlice + pu1) = make_uint4(dw[4], dw[5], dw[6], dw[7]);
+            // P^T / dS^T buffer q & 1 is free once the accumulation and the dQ
+            // contribution of chunk q - 2 completed; at a head's first chunk,
+            // every key warp has also read its staged rows of the previous
+            // head's accumulators (staged in this same buffer)
+            uint8_t *pt = sm + L::oPT + (q & 1) * kPT;
+            if (q >= 2) ok = warp_all(mbar_wait(&ptfree[q & 1], ((q - 2) >> 1) & 1, abort_flag));
+            if (ok && c == 0 && hh >= 1) ok = warp_all(mbar_wait(kdrain, (hh - 1) & 1, abort_flag));
+            if (!ok) break;
+            *reinterpret_cast<uint4 *>(pt + pu0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            *reinterpret_cast<uint4 *>(pt + pu1) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+            *reinterpret_cast<uint4 *>(pt + kSlice + pu0) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+            *reinterpret_cast<uint4 *>(pt + kSlice + pu1) = make_uint4(dw[4], dw[5], dw[6], dw[7]);
             fence_proxy_async_smem();  // visible to the MMAs that read them
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dsready);
             if (c != nchunks - 1) continue;
-            // head end, once its accumulations completed and the store warps
-            // have read the previous head's stash: accumulator columns
-            // [128 hr, 128 hr + 128) (lanes 0-15 dK, 16-31 dV) -> bf16 pairs in
-            // stash columns [64 hr, 64 hr + 64). The accumulator is then free
-            // for the next head.
-            ok = warp_all(mbar_wait(ptfree, q & 1, abort_flag));
-            if (ok && hh >= 1) ok = warp_all(mbar_wait(stashfree, (hh - 1) & 1, abort_flag));
+            // head end, once its accumulations completed (its last dQ
+            // contribution may still run): accumulator columns
+            // [128 hr, 128 hr + 128) (lanes 0-15 dK, 16-31 dV) -> bf16 -> dK^C /
+            // dV rows, staged 32 columns at a time in the other P^T / dS^T
+            // buffer (free once chunk q - 1's MMAs completed; 2 KB per warp, each
+            // thread its 64 bytes, 16-byte unit u at u ^ (lane & 3)), the warp
+            // writing 8 rows' 64-byte segments per instruction. dK columns
+            // 192..255 (the rope slice) stay in TMEM, summed over heads. The
+            // accumulator is then free for the next head.
+            ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag));
+            if (ok && q >= 1) ok = warp_all(mbar_wait(&ptfree[(q + 1) & 1], ((q - 1) >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-#pragma unroll
+            uint8_t *stage = sm + L::oPT + ((q + 1) & 1) * kPT + warp * 2048;
+            const size_t bh = (size_t)b * p.n_h + h0 + hh;
+#pragma unroll 1
             for (int rd = 0; rd < 4; rd++) {
                 tmem_ld32(trow + kColAcc + hr * 128 + rd * 32, v);
                 tmem_wait_ld();
-                uint32_t pk[16];
+                const int col = hr * 128 + rd * 32;
+                const bool rope = col >= kDC;
 #pragma unroll
-                for (int i = 0; i < 16; i++) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-                tmem_st16u(trow + kColStash + hr * 64 + rd * 16, pk);
+                for (int u = 0; u < 4; u++)
+                    *reinterpret_cast<uint4 *>(stage + lane * 64 + ((u ^ (lane & 3)) << 4)) =
+                        make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                   pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int kl = 8 * i + (lane >> 2), u = lane & 3;  // source lane, unit
+                    const int kvl = __shfl_sync(0xffffffffu, (int)key_valid, kl);
+                    const long long kposl = __shfl_sync(0xffffffffu, (long long)key_pos, kl);
+                    const bool is_v = kl >= 16;
+                    if (kvl && (is_v || !rope)) {
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stage + kl * 64 + ((u ^ (kl & 3)) << 4));
+                        __nv_bfloat16 *dst = is_v ? p.dv + (bh * p.L + (size_t)kposl) * kDV + col + 8 * u
+                                                  : p.dkc + (bh * p.L + (size_t)kposl) * kDC + col + 8 * u;
+                        *reinterpret_cast<uint4 *>(dst) = val;
+                    }
+                }
+                __syncwarp();
             }
-            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(stashfull);
+            if (lane == 0) mbar_arrive(kdrain);
         }
         if (ok && hr == 1) {
             // rope slice of dK (columns 192..255 of the lanes 0-15), summed over
@@ -1056,11 +772,12 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     if (*abort_flag) {
         volatile int never = 0;
         if (warp == kWarpKV && lane == 0) {
-            for (int t = counters[2]; t < counters[0]; ++t) mbar_wait(kvfull, t & 1, (volatile int *)&never);
+            for (int t = counters[2]; t < counters[0]; ++t)
+                mbar_wait(&kvfull[t % KVS], (t / KVS) & 1, (volatile int *)&never);
         }
         if (warp == kWarpRow && lane == 0) {
             for (int t = counters[3]; t < counters[1]; ++t)
-                mbar_wait(&rowfull[t & 1], (t >> 1) & 1, (volatile int *)&never);
+                mbar_wait(&rowfull[t % RS], (t / RS) & 1, (volatile int *)&never);
         }
         if (warp == kWarpMma && lane == 0) {
             mma_commit(drain);
@@ -1074,6 +791,39 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         tmem_dealloc(tmem, 512);
     }
     if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
+}
+
+// ------------------------------------------------------------- dQ output
+// One warp per row of a kept block (5 warps): the accumulated dQ row (sorted
+// order; lane l holds dims 8 l .. 8 l + 7), its rope slice (lanes 24-31)
+// rotated back by the query position A + j, rounded to bf16 and written to the
+// caller's row 5 n + j.
+__global__ void __launch_bounds__(160) k_bwd_dq_out(int n_h, int N, const int32_t *__restrict__ cnt,
+                                                    const int32_t *__restrict__ sorted_n,
+                                                    const int32_t *__restrict__ sorted_a,
+                                                    const float2 *__restrict__ tab, const float *__restrict__ dqacc,
+                                                    __nv_bfloat16 *__restrict__ dq) {
+    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if (i >= cnt[b]) return;
+    const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int R = kBlock * N;
+    const size_t bh = (size_t)b * n_h + h;
+    const int n = sorted_n[(size_t)b * N + i], a = sorted_a[(size_t)b * N + i];
+    const float4 *src = reinterpret_cast<const float4 *>(dqacc + (bh * R + kBlock * i + j) * kDQK) + 2 * lane;
+    const float4 x = src[0], y = src[1];
+    float v[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    if (lane >= 24) {  // rope slice: rotate back by the query position A + j
+        const float2 *cs = tab + (size_t)(a + j) * (kDR / 2) + (lane - 24) * 4;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const float2 t2 = __ldg(cs + k);
+            const float x0 = v[2 * k], x1 = v[2 * k + 1];
+            v[2 * k] = x0 * t2.x + x1 * t2.y;
+            v[2 * k + 1] = x1 * t2.x - x0 * t2.y;
+        }
+    }
+    *(reinterpret_cast<uint4 *>(dq + (bh * R + kBlock * n + j) * kDQK) + lane) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
 // ------------------------------------------------------------ dK^R reduce
@@ -1110,6 +860,9 @@ __global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int
     *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
 }
 
+// Stage counts of the one-pass kernel: K/V of two heads in flight, one row stage.
+constexpr int kKVS = 2, kRS = 1;
+
 }  // namespace
 
 bool bwd_tc_supported(const Prob &p) {
@@ -1118,7 +871,7 @@ bool bwd_tc_supported(const Prob &p) {
 }
 
 int bwd_head_groups(const Prob &p) {
-    const long long items = (long long)((p.S + kv::kMK - 1) / kv::kMK + (p.N + kGD - 1) / kGD) * p.B;
+    const long long items = (long long)((p.S + bw::kMK - 1) / bw::kMK + (p.N + kGD - 1) / kGD) * p.B;
     // aim for about eight waves on 148 SMs (shorter CTAs, smaller tail)
     int hg = 1;
     while (hg < p.n_h && items * hg < 8 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
@@ -1134,14 +887,14 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         count_launch();
         k_bwd_prep<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(
             p.n_h, p.N, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dout, lse, ws.cnt,
-            ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs, (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses);
+            ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs, (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses,
+            ws.dqacc);
         count_launch();
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_qs3_64, m_dos3_64, m_kr8, m_kc3_8, m_v3_8;
+    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kr8, m_kc3_8, m_v3_8;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
-    const void *qs = ws.qs, *dos = ws.dos;
     if (!make_map3_bf16(&m_kc3_64, kc, kDC, kv_rows, 64) ||
         !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
         !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64) ||
@@ -1149,48 +902,39 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         !make_map3_bf16(&m_kc3_8, kc, kDC, kv_rows, 8) || !make_map3_bf16(&m_v3_8, v, kDV, kv_rows, 8))
         return cudaErrorInvalidValue;
     if (p.N > 0 && q_rows > 0) {
-        if (!make_map3_bf16(&m_qs3_128, qs, kDQK, q_rows, 128) || !make_map3_bf16(&m_dos3_128, dos, kDV, q_rows, 128) ||
-            !make_map3_bf16(&m_qs3_64, qs, kDQK, q_rows, 64) || !make_map3_bf16(&m_dos3_64, dos, kDV, q_rows, 64))
+        if (!make_map3_bf16(&m_qs3_64, ws.qs, kDQK, q_rows, 64) || !make_map3_bf16(&m_dos3_64, ws.dos, kDV, q_rows, 64))
             return cudaErrorInvalidValue;
     } else {  // maps over Q rows are never read: any valid map will do
-        m_qs3_128 = m_dos3_128 = m_qs3_64 = m_dos3_64 = m_kc3_64;
+        m_qs3_64 = m_dos3_64 = m_kc3_64;
     }
     BwdArgs a;
     a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
     a.scale_log2 = p.scale_log2;
     a.scale = p.scale;
-    a.kc = (const __nv_bfloat16 *)kc;
-    a.krr = (const __nv_bfloat16 *)ws.kr_rot;
-    a.v = (const __nv_bfloat16 *)v;
-    a.qs = (const __nv_bfloat16 *)ws.qs;
-    a.dos = (const __nv_bfloat16 *)ws.dos;
     a.ds_ = ws.dvec;
     a.lses = ws.lses;
     a.cnt = ws.cnt;
     a.sorted_n = ws.sorted_n;
     a.sorted_a = ws.sorted_a;
-    a.tab = ws.rope;
-    a.dq = (__nv_bfloat16 *)dq;
     a.dkc = (__nv_bfloat16 *)dkc;
     a.dv = (__nv_bfloat16 *)dv;
     a.dkr_part = ws.dkr_part;
+    a.dqacc = ws.dqacc;
     a.hpg = p.n_h / HG;
-    a.n_ctx_items = (p.S + kv::kMK - 1) / kv::kMK;
+    a.n_ctx_items = (p.S + bw::kMK - 1) / bw::kMK;
     a.err = ws.err;
-    cudaError_t e;
-    if (p.N > 0) {
-        e = cudaFuncSetAttribute(k_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, dq::kSmem);
-        if (e != cudaSuccess) return e;
-        count_launch();
-        k_bwd_dq_tc<<<dim3((p.N + kG - 1) / kG, p.n_h, p.B), dq::kThreads, dq::kSmem, st>>>(
-            m_kc3_64, m_kr64, m_v3_64, m_qs3_128, m_dos3_128, m_kc3_8, m_kr8, m_v3_8, a);
-    }
-    const dim3 kv_grid(a.n_ctx_items + (p.N + kGD - 1) / kGD, HG, p.B);
-    e = cudaFuncSetAttribute(k_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmem);
+    const dim3 grid(a.n_ctx_items + (p.N + kGD - 1) / kGD, HG, p.B);
+    constexpr int smem = bw::Smem<kKVS, kRS>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<kKVS, kRS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_kv_tc<<<kv_grid, kv::kThreads, kv::kSmem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kc3_8,
-                                                        m_kr8, m_v3_8, a);
+    k_bwd_tc<kKVS, kRS><<<grid, bw::kThreads, smem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kc3_8,
+                                                          m_kr8, m_v3_8, a);
+    if (p.N > 0) {
+        count_launch();
+        k_bwd_dq_out<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(p.n_h, p.N, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope,
+                                                             ws.dqacc, (__nv_bfloat16 *)dq);
+    }
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
     k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,

@@ -110,6 +110,12 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
         "l"((uint64_t)m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// Prefetch of a 3-D tile into L2 (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *m, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"((uint64_t)m), "r"(x),
+                 "r"(y), "r"(z)
+                 : "memory");
+}
 // 1-D bulk copy of `bytes` contiguous bytes (16-byte aligned addresses, size a
 // multiple of 16) completing on bar's transaction count.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -246,6 +252,11 @@ __device__ __forceinline__ SDesc sdesc_split(uint64_t d) { return SDesc{(uint32_
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
+}
+// The same with A MN-major as well (a_mn = 1: A's M index runs along its
+// 128-byte rows, its K index across them).
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, int a_mn, int b_mn) {
+    return idesc_bf16(M, N, b_mn) | ((uint32_t)a_mn << 15);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {

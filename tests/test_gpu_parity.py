@@ -111,12 +111,24 @@ def test_s2048_workload_full(oracle_mod):
 
 
 def test_deterministic():
+    """O, LSE, dK^C, dK^R and dV are bitwise reproducible (every element is
+    written once, by one thread, in a fixed order). dQ is the sum of one
+    contribution per key tile that meets the row's window, added in fp32 in
+    whatever order the tiles finish, so two runs may differ by the rounding of
+    that sum: at most one bf16 unit in the last place."""
     wl = synth.WORKLOADS[2]
     c = synth.make_inputs(wl)
     a = run_gpu(c, wl.S, wl.W)
     b = run_gpu(c, wl.S, wl.W)
     for k in a:
-        assert torch.equal(a[k], b[k]), k
+        if k == "dq":
+            x, y = a[k].float(), b[k].float()
+            # one bf16 unit of the larger value, plus the fp32 rounding of a sum
+            # of O(1) terms where the value itself is near zero
+            ulp = torch.maximum(x.abs(), y.abs()) * 2.0 ** -7 + 1e-6
+            assert ((x - y).abs() <= ulp).all(), k
+        else:
+            assert torch.equal(a[k], b[k]), k
 
 
 def _slice(c, b, h):
