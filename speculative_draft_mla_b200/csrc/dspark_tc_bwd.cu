@@ -11,8 +11,7 @@
 //
 // Launch sequence (one stream):
 //   1. k_bwd_prep       per kept block and head: rotated Q and dO copied into
-//                       anchor-sorted row order, D, LSE*log2(e), and the
-//                       block's rows of the fp32 dQ accumulator zeroed.
+//                       anchor-sorted row order, D, LSE*log2(e).
 //   2. k_bwd_pad        zeros for padding blocks' rows and draft keys.
 //   3. k_bwd_tc         key-major, one CTA per (b, 64-key tile, head group),
 //                       one pass over K and V: rows of the blocks whose key
@@ -21,11 +20,16 @@
 //                       memory, dV += P^T dO and dK += dS^T Q accumulated in
 //                       TMEM over the rows (M = 64 accumulators: dK and dV share
 //                       TMEM columns, one in each half of the lanes), and the
-//                       chunk's dQ contribution dS K in TMEM, added into the
-//                       fp32 dQ accumulator with vector reductions. dK and dV
-//                       are written once, by the CTA that owns the keys (no
-//                       atomics); dQ rows receive one contribution per key tile
-//                       that meets their window, plus their draft tile's.
+//                       chunk's dQ contribution dS K in TMEM. dK and dV are
+//                       written once, by the CTA that owns the keys (no
+//                       atomics). dQ goes through an fp32 accumulator in
+//                       anchor-sorted row order: the draft-key tiles come first
+//                       in the grid; each stores its rows' draft-key
+//                       contribution (every kept row belongs to exactly one draft
+//                       tile, so the accumulator needs no clearing) and raises a
+//                       flag; the context tiles wait for the flags of the rows
+//                       they meet, then add their contributions with vector
+//                       reductions.
 //   4. k_bwd_dq_out     rotates the rope part of the accumulated dQ back,
 //                       rounds to bf16 and writes dq in the caller's row order.
 //   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
@@ -49,9 +53,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
 // One warp per row of a kept block (5 warps): rotated q -> qs, do -> dos,
-// D = rowsum(dO * O), LSE * log2(e), and the row of the dQ accumulator set to
-// zero; rows past the kept blocks are zeroed so tiles that overhang them
-// multiply finite values.
+// D = rowsum(dO * O), LSE * log2(e); rows past the kept blocks are zeroed so
+// tiles that overhang them multiply finite values.
 __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfloat16 *__restrict__ q,
                                                   const __nv_bfloat16 *__restrict__ o,
                                                   const __nv_bfloat16 *__restrict__ dout,
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfl
                                                   const int32_t *__restrict__ sorted_a,
                                                   const float2 *__restrict__ tab, __nv_bfloat16 *__restrict__ qs,
                                                   __nv_bfloat16 *__restrict__ dos, float *__restrict__ ds_,
-                                                  float *__restrict__ lses, float *__restrict__ dqacc) {
+                                                  float *__restrict__ lses) {
     const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
@@ -68,9 +71,6 @@ __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfl
     const size_t srow = bh * R + kBlock * i + j;
     uint4 *qd = reinterpret_cast<uint4 *>(qs + srow * kDQK) + lane;
     uint4 *dd = reinterpret_cast<uint4 *>(dos + srow * kDV) + lane;
-    float4 *acc = reinterpret_cast<float4 *>(dqacc + srow * kDQK) + 2 * lane;
-    acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i >= cnt[b]) {
         *qd = make_uint4(0, 0, 0, 0);
         *dd = make_uint4(0, 0, 0, 0);
@@ -138,16 +138,24 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
 }
 
 struct BwdArgs {
-    int n_h, S, N, W, L, R;
+    int B, n_h, S, N, W, L, R;
     float scale_log2, scale;
     const float *ds_, *lses;
     const int32_t *cnt, *sorted_n, *sorted_a;
-    __nv_bfloat16 *dkc, *dv;
+    const float2 *tab;
+    __nv_bfloat16 *dq, *dkc, *dv;
     float *dkr_part, *dqacc;
-    int hpg;  // heads per head group
-    int n_ctx_items;
+    int32_t *dqflag;
+    int HG, hpg;  // head groups, heads per group
+    int n_ctx, n_draft;  // context / draft-key tiles per (batch row, head group)
     uint32_t *err;
 };
+
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ void red_add_v4(float *addr, const uint4 &v) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(v.x)),
@@ -188,7 +196,6 @@ constexpr int kSlice = 64 * 128;           // 8 KB: 64 keys or rows x 64 columns
 // rows (4 x 1 KB) at bb * 4 KB: 8-key groups 3 KB / 4 KB apart, 64-column
 // slices 1 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftVBlock = 4 * 1024;
-constexpr int kKV = 7 * kSlice;            // one head's K^C (3 slices) then V (4 slices)
 constexpr int kRowStage = 8 * kSlice;      // Q chunk (4 slices), then dO chunk (4 slices)
 constexpr int kPT = 2 * kSlice;            // P^T, then dS^T: [64 keys][64 rows] bf16 each
 constexpr int kDqStage = 32 * 64;          // per dQ warp: 32 lanes x 16 fp32
@@ -199,14 +206,19 @@ constexpr int kThreads = (kKeyWarps + 7) * 32;
 constexpr uint32_t kColAcc = 0, kColS = 256, kColDQ = 384;  // S^T / dP^T buffer s at kColS + 64 s
 constexpr uint32_t kHi = 16u << 16;        // lane offset of the second M = 64 accumulator
 
-// Shared memory for KVS K/V stages and RS row stages.
-template <int KVS, int RS>
+// Shared memory: the rope-key tile, one K^C and one V stage (V is free as
+// soon as a head's last dP^T completed, K^C after its last dQ contribution,
+// so the next head's tiles load while the current one finishes), RS row
+// stages, the P^T / dS^T buffer (also the staging area of the head-end
+// dK / dV readout), the dQ warps' staging, the per-row data.
+template <int RS>
 struct Smem {
     static constexpr int oKr = 0;                          // rope-key tile (8 KB)
-    static constexpr int oKV = oKr + kSlice;               // K/V stage s at oKV + s * kKV
-    static constexpr int oRow = oKV + KVS * kKV;           // row stage s at oRow + s * kRowStage
-    static constexpr int oPT = oRow + RS * kRowStage;      // P^T / dS^T buffer u at oPT + u * kPT
-    static constexpr int oStage = oPT + 2 * kPT;           // dQ warps' staging
+    static constexpr int oKc = oKr + kSlice;               // K^C (3 slices)
+    static constexpr int oV = oKc + 3 * kSlice;            // V (4 slices)
+    static constexpr int oRow = oV + 4 * kSlice;           // row stage s at oRow + s * kRowStage
+    static constexpr int oPT = oRow + RS * kRowStage;      // P^T, then dS^T
+    static constexpr int oStage = oPT + kPT;               // dQ warps' staging
     static constexpr int oMeta = oStage + 4 * kDqStage;    // per row stage: (LSE * log2 e, D) of each row
     static constexpr int oBar = oMeta + RS * kRC * 8;
     static constexpr int kBytes = oBar + 256 + 1024;       // barriers, counters, alignment slack
@@ -215,35 +227,42 @@ struct Smem {
 }  // namespace bw
 
 // One CTA per (64-key tile, head group, batch row).
-template <int KVS, int RS>
+template <int RS>
 __global__ void __launch_bounds__(bw::kThreads, 1)
     k_bwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
              const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
              const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
     using namespace bw;
-    using L = Smem<KVS, RS>;
+    using L = Smem<RS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::oBar);
-    uint64_t *kvfull = bars + 0, *kvfree = bars + 2, *rowfull = bars + 4, *rowfree = bars + 6, *sfull = bars + 8,
-             *ptfree = bars + 10, *dsready = bars + 12, *dqfull = bars + 13, *dqfree = bars + 14, *kdrain = bars + 15,
-             *accdone = bars + 16, *drain = bars + 17;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    uint64_t *kfull = bars + 0, *kfree = bars + 1, *vfull = bars + 2, *vfree = bars + 3, *rowfull = bars + 4,
+             *rowfree = bars + 6, *sfull = bars + 8, *ptfree = bars + 10, *dsready = bars + 11, *dqfull = bars + 12,
+             *dqfree = bars + 13, *kdrain = bars + 14, *accdone = bars + 15, *drain = bars + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    // K/V heads issued, row chunks issued, K/V heads consumed, row chunks consumed
+    // K heads issued, V heads issued, row chunks issued, heads consumed, row chunks consumed
     int *counters = reinterpret_cast<int *>(tmem_slot + 2);
-    int *band = counters + 4;  // first sorted row, row count
+    int *band = counters + 5;  // first sorted row, row count
 
-    const int item = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    // Items: all draft-key tiles (region-major, region = (b, head group)),
+    // then all context tiles, so that a context tile starts after the draft
+    // tiles of its rows were dispatched.
+    const int n_draft_all = p.B * p.HG * p.n_draft;
+    const bool is_ctx = (int)blockIdx.x >= n_draft_all;
+    const int rel = is_ctx ? (int)blockIdx.x - n_draft_all : (int)blockIdx.x;
+    const int per = is_ctx ? p.n_ctx : p.n_draft;
+    const int region = rel / per, item = rel % per;
+    const int b = region / p.HG, hg = region % p.HG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cnt = p.cnt[b];
-    const bool is_ctx = item < p.n_ctx_items;
     int t0 = 0, gcnt = 0, i0 = 0;
     if (is_ctx) {
         t0 = item * kMK;
     } else {
-        i0 = (item - p.n_ctx_items) * kGD;
+        i0 = item * kGD;
         if (i0 >= cnt) return;  // uniform: fewer draft tiles in this batch row
         gcnt = min(kGD, cnt - i0);
     }
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + kk / 8] + kk % 8;
         }
     }
-    float *dkr_part_row = p.dkr_part + (((size_t)hg * gridDim.z + b) * p.L + key_pos) * kDR;
+    float *dkr_part_row = p.dkr_part + (((size_t)hg * p.B + b) * p.L + key_pos) * kDR;
 
     if (nrows == 0) {
         // no row sees these keys: zero gradients for every head of the group
@@ -319,18 +338,16 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     for (int e = threadIdx.x; e < (L::oRow - L::oKr) / 16; e += blockDim.x)
         reinterpret_cast<uint4 *>(sm + L::oKr)[e] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < KVS; s++) {
-            mbar_init(&kvfull[s], 1);
-            mbar_init(&kvfree[s], 1);
-        }
+        mbar_init(kfull, 1);
+        mbar_init(kfree, 1);
+        mbar_init(vfull, 1);
+        mbar_init(vfree, 1);
         for (int s = 0; s < RS; s++) {
             mbar_init(&rowfull[s], 1);
             mbar_init(&rowfree[s], 1);
         }
-        for (int s = 0; s < 2; s++) {
-            mbar_init(&sfull[s], 1);
-            mbar_init(&ptfree[s], 1);
-        }
+        for (int s = 0; s < 2; s++) mbar_init(&sfull[s], 1);
+        mbar_init(ptfree, 1);
         mbar_init(dsready, kKeyWarps);
         mbar_init(accdone, 1);
         mbar_init(dqfull, 1);
@@ -338,7 +355,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         mbar_init(kdrain, kKeyWarps);
         mbar_init(drain, 1);
         *abort_flag = 0;
-        for (int c = 0; c < 4; c++) counters[c] = 0;
+        for (int c = 0; c < 5; c++) counters[c] = 0;
         fence_barrier_init();
     }
     if (warp == kWarpMma) {
@@ -354,34 +371,66 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
 
     if (warp == kWarpKV) {
         // ------------------------------------------- producer of K/V tiles
+        // Per head: V once the previous head's last dP^T completed, then K^C
+        // (and, for the first head, the rope-key tile) once the previous head's
+        // last dQ contribution completed.
         const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
         for (int hh = 0; hh < H; ++hh) {
-            const int s = hh % KVS;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            if (hh >= KVS && !warp_all(mbar_wait(&kvfree[s], ((hh / KVS) - 1) & 1, abort_flag))) break;
-            uint8_t *kv = sm + L::oKV + s * kKV;
+            if (hh >= 1 && !warp_all(mbar_wait(vfree, (hh - 1) & 1, abort_flag))) break;
             if (is_ctx) {
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&kvfull[s], (hh == 0 ? 8 : 7) * kSlice);
-                    if (hh == 0) tma_load_2d(sm + L::oKr, &tm_kr, &kvfull[s], 0, (int)((size_t)b * p.L + t0));
-                    tma_load_3d(kv, &tm_kc, &kvfull[s], 0, (int)(bh * p.L + t0), 0);
-                    tma_load_3d(kv + 3 * kSlice, &tm_v, &kvfull[s], 0, (int)(bh * p.L + t0), 0);
+                    mbar_arrive_expect_tx(vfull, 4 * kSlice);
+                    tma_load_3d(sm + L::oV, &tm_v, vfull, 0, (int)(bh * p.L + t0), 0);
                 }
             } else {
-                if (lane == 0) mbar_arrive_expect_tx(&kvfull[s], gcnt * 8 * ((hh == 0 ? kDQK : kDC) + kDV) * 2);
+                if (lane == 0) mbar_arrive_expect_tx(vfull, gcnt * 8 * kDV * 2);
+                for (int bb = 0; bb < gcnt; ++bb) {
+                    const int nb = __shfl_sync(0xffffffffu, my_n, bb);
+                    if (lane == 0)
+                        tma_load_3d(sm + L::oV + bb * kDraftVBlock, &tm_v8, vfull, 0, (int)(bh * p.L + p.S + kBlock * nb),
+                                    0);
+                }
+            }
+            if (lane == 0) counters[1] = hh + 1;
+            if (hh >= 1 && !warp_all(mbar_wait(kfree, (hh - 1) & 1, abort_flag))) break;
+            if (is_ctx) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(kfull, (hh == 0 ? 4 : 3) * kSlice);
+                    if (hh == 0) tma_load_2d(sm + L::oKr, &tm_kr, kfull, 0, (int)((size_t)b * p.L + t0));
+                    tma_load_3d(sm + L::oKc, &tm_kc, kfull, 0, (int)(bh * p.L + t0), 0);
+                }
+            } else {
+                if (lane == 0) mbar_arrive_expect_tx(kfull, gcnt * 8 * (hh == 0 ? kDQK : kDC) * 2);
                 for (int bb = 0; bb < gcnt; ++bb) {
                     const int nb = __shfl_sync(0xffffffffu, my_n, bb);
                     if (lane == 0) {
                         const int row = p.S + kBlock * nb;
-                        tma_load_3d(kv + bb * kDraftKcBlock, &tm_kc8, &kvfull[s], 0, (int)(bh * p.L + row), 0);
-                        if (hh == 0)
-                            tma_load_2d(sm + L::oKr + bb * 1024, &tm_kr8, &kvfull[s], 0, (int)((size_t)b * p.L + row));
-                        tma_load_3d(kv + 3 * kSlice + bb * kDraftVBlock, &tm_v8, &kvfull[s], 0, (int)(bh * p.L + row),
-                                    0);
+                        tma_load_3d(sm + L::oKc + bb * kDraftKcBlock, &tm_kc8, kfull, 0, (int)(bh * p.L + row), 0);
+                        if (hh == 0) tma_load_2d(sm + L::oKr + bb * 1024, &tm_kr8, kfull, 0, (int)((size_t)b * p.L + row));
                     }
                 }
             }
             if (lane == 0) counters[0] = hh + 1;
+            // the next head's tiles into L2, so that their loads (issued once
+            // this head's tiles are free) wait on L2 rather than on DRAM
+            if (hh + 1 < H) {
+                const size_t bn = bh + 1;
+                if (is_ctx) {
+                    if (lane == 0) {
+                        tma_prefetch_l2_3d(&tm_kc, 0, (int)(bn * p.L + t0), 0);
+                        tma_prefetch_l2_3d(&tm_v, 0, (int)(bn * p.L + t0), 0);
+                    }
+                } else {
+                    for (int bb = 0; bb < gcnt; ++bb) {
+                        const int nb = __shfl_sync(0xffffffffu, my_n, bb);
+                        if (lane == 0) {
+                            tma_prefetch_l2_3d(&tm_kc8, 0, (int)(bn * p.L + p.S + kBlock * nb), 0);
+                            tma_prefetch_l2_3d(&tm_v8, 0, (int)(bn * p.L + p.S + kBlock * nb), 0);
+                        }
+                    }
+                }
+            }
         }
     } else if (warp == kWarpRow) {
         // ---------------------------- producer of Q / dO chunks and row data
@@ -428,7 +477,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                 tma_load_3d(sm + L::oRow + s * kRowStage, &tm_qs, &rowfull[s], 0, (int)(bh * p.R + r0), 0);
                 tma_load_3d(sm + L::oRow + s * kRowStage + 4 * kSlice, &tm_dos, &rowfull[s], 0, (int)(bh * p.R + r0),
                             0);
-                counters[1] = q + 1;
+                counters[2] = q + 1;
             }
         }
     } else if (warp == kWarpMma) {
@@ -447,23 +496,20 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             const uint32_t kcStep = is_ctx ? kSlice : 1024;
             const uint32_t kOff = is_ctx ? 1024 : kDraftKcBlock, vOff = is_ctx ? 1024 : kDraftVBlock;
             const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), 16, 1024));
-            // P^T / dS^T buffer u: descriptors of buffer 0 plus kPT / 16 * u
             const SDesc ptd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT), 16, 1024));
             const SDesc dsd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT + kSlice), 16, 1024));
             const SDesc dsq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT + kSlice), kSlice, 1024));
-            constexpr uint32_t kPTu = kPT >> 4;
             // B operands of dQ_c, MN-major: dims 0..127 of K^C (two slices),
             // dims 128..191 (third slice), the rope key (dims 192..255); 16 keys
             // are 2 KB in every case (context: 16 rows of 128 B; draft: 2 blocks)
             const SDesc krq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), is_ctx ? kSlice : 1024, 1024));
             const uint32_t kcq_step = is_ctx ? 128u : (uint32_t)((2 * kDraftKcBlock) >> 4);
             bool ok = true;
+            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKc), 16, kOff));
+            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + L::oV), 16, vOff));
             auto issue_s = [&](int q) {
-                const int hh = q / nchunks, s = q % RS, bsel = q & 1;
+                const int c = q % nchunks, s = q % RS, bsel = q & 1;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(sm + L::oKV + (hh % KVS) * kKV);
-                const SDesc kad = sdesc_split(sdesc_sw128(kb, 16, kOff));
-                const SDesc vad = sdesc_split(sdesc_sw128(kb + 3 * kSlice, 16, vOff));
                 const uint32_t rs = smem_u32(sm + L::oRow + s * kRowStage);
                 const SDesc qd = sdesc_split(sdesc_sw128(rs, 16, 1024));
                 const SDesc dod = sdesc_split(sdesc_sw128(rs + 4 * kSlice, 16, 1024));
@@ -479,10 +525,10 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                     mma_bf16_ss(dP, vad.at(((cc * kcStep) >> 4) + sub), dod.at(ro), idS, k16 > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[bsel]);
+                if (c == nchunks - 1) mma_commit(vfree);  // the head's V tile is no longer read
             };
             auto issue_acc = [&](int q) {
                 const int c = q % nchunks, s = q % RS;
-                const uint32_t pu = kPTu * (q & 1);
                 tc_fence_after();
                 const uint32_t rs = smem_u32(sm + L::oRow + s * kRowStage);
                 const SDesc qb = sdesc_split(sdesc_sw128(rs, kSlice, 1024));  // MN-major
@@ -491,67 +537,67 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                 // 2 KB (16 rows of 128 bytes) in the row chunk
 #pragma unroll
                 for (int k16 = 0; k16 < kRC / 16; ++k16)
-                    mma_bf16_ss(tmem + kColAcc + kHi, ptd.at(pu + 2 * k16), dob.at(128 * k16), idV,
+                    mma_bf16_ss(tmem + kColAcc + kHi, ptd.at(2 * k16), dob.at(128 * k16), idV,
                                 (c > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
                 for (int k16 = 0; k16 < kRC / 16; ++k16)
-                    mma_bf16_ss(tmem + kColAcc, dsd.at(pu + 2 * k16), qb.at(128 * k16), idKc, (c > 0 || k16 > 0) ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColAcc, dsd.at(2 * k16), qb.at(128 * k16), idKc, (c > 0 || k16 > 0) ? 1u : 0u);
 #pragma unroll
                 for (int k16 = 0; k16 < kRC / 16; ++k16)
-                    mma_bf16_ss(tmem + kColAcc + kDC, dsd.at(pu + 2 * k16), qb.at(((3 * kSlice) >> 4) + 128 * k16), idKr,
+                    mma_bf16_ss(tmem + kColAcc + kDC, dsd.at(2 * k16), qb.at(((3 * kSlice) >> 4) + 128 * k16), idKr,
                                 (q > 0 || k16 > 0) ? 1u : 0u);
                 mma_commit(&rowfree[s]);
+                mma_commit(ptfree);  // after the chunk's dQ contribution, issued before
                 if (c == nchunks - 1) mma_commit(accdone);  // the head's accumulators are final
             };
             auto issue_dq = [&](int q) {
-                const int hh = q / nchunks, c = q % nchunks;
-                const uint32_t pu = kPTu * (q & 1);
+                const int c = q % nchunks;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(sm + L::oKV + (hh % KVS) * kKV);
+                const uint32_t kb = smem_u32(sm + L::oKc);
                 const SDesc kq0 = sdesc_split(sdesc_sw128(kb, is_ctx ? kSlice : 1024, kOff));
                 const SDesc kq1 = sdesc_split(sdesc_sw128(kb + (is_ctx ? 2 * kSlice : 2048), kSlice, kOff));
 #pragma unroll
                 for (int k16 = 0; k16 < kMK / 16; ++k16) {
-                    const uint64_t a = dsq.at(pu + 128 * k16);  // 16 keys = 16 rows of the dS^T tile
+                    const uint64_t a = dsq.at(128 * k16);  // 16 keys = 16 rows of the dS^T tile
                     mma_bf16_ss(tmem + kColDQ, a, kq0.at(kcq_step * k16), idQ128, k16 > 0 ? 1u : 0u);
                     mma_bf16_ss(tmem + kColDQ + kHi, a, kq1.at(kcq_step * k16), idQ64, k16 > 0 ? 1u : 0u);
                     mma_bf16_ss(tmem + kColDQ + kHi + 64, a, krq.at(128 * k16), idQ64, k16 > 0 ? 1u : 0u);
                 }
                 mma_commit(dqfull);
-                mma_commit(&ptfree[q & 1]);
-                if (c == nchunks - 1) mma_commit(&kvfree[hh % KVS]);
+                if (c == nchunks - 1) mma_commit(kfree);  // the head's K^C / K^R tiles are no longer read
             };
-            // Issue whichever is ready: the S^T stage of chunk ns (its K/V tile
-            // and row operands landed; at most one chunk ahead of the
-            // accumulations, so its S^T / dP^T buffer was read by the key
-            // warps before they signalled chunk ns - 2), the accumulation of
-            // chunk na (P^T / dS^T written; at a head's first chunk the key
-            // warps have also read out the previous head's accumulators, which
-            // precedes that signal), or the dQ contribution of chunk nd (its
-            // accumulation issued, the dQ warps have read chunk nd - 1's).
+            // Issue whichever is ready: the S^T / dP^T stage of chunk ns (its K,
+            // V and row operands landed; at most one chunk ahead of the dQ
+            // contributions, so its S^T / dP^T buffer was read by the key warps
+            // before they signalled chunk ns - 2), the dQ contribution of chunk
+            // nd (P^T / dS^T written, the dQ warps have read chunk nd - 1's; it
+            // goes first so that the head's K^C tile is freed early), or the
+            // accumulation of chunk na (after its dQ contribution; at a head's
+            // first chunk the key warps have also read out the previous head's
+            // accumulators, which precedes their dS^T signal).
             int ns = 0, na = 0, nd = 0;
             uint64_t t_idle = 0;
-            while (ok && nd < QT) {
+            while (ok && na < QT) {
                 bool issued = false;
-                if (ns < QT && ns <= na + 1) {
+                if (ns < QT && ns <= nd + 1) {
                     const int hh = ns / nchunks, c = ns % nchunks;
-                    if ((c != 0 || mbar_test(&kvfull[hh % KVS], (hh / KVS) & 1)) &&
+                    if ((c != 0 || (mbar_test(kfull, hh & 1) && mbar_test(vfull, hh & 1))) &&
                         mbar_test(&rowfull[ns % RS], (ns / RS) & 1)) {
-                        if (c == 0) counters[2] = hh + 1;
-                        counters[3] = ns + 1;
+                        if (c == 0) counters[3] = hh + 1;
+                        counters[4] = ns + 1;
                         issue_s(ns);
                         ++ns;
                         issued = true;
                     }
                 }
-                if (!issued && na < ns && mbar_test(dsready, na & 1)) {
-                    issue_acc(na);
-                    ++na;
-                    issued = true;
-                }
-                if (!issued && nd < na && (nd == 0 || mbar_test(dqfree, (nd - 1) & 1))) {
+                if (!issued && nd < ns && mbar_test(dsready, nd & 1) && (nd == 0 || mbar_test(dqfree, (nd - 1) & 1))) {
                     issue_dq(nd);
                     ++nd;
+                    issued = true;
+                }
+                if (!issued && na < nd) {
+                    issue_acc(na);
+                    ++na;
                     issued = true;
                 }
                 if (issued) {
@@ -572,12 +618,32 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         // Sub-partition sp: lanes 0-15 hold dims 0..127 of chunk rows
         // 16 sp .. + 15, lanes 16-31 dims 128..255 of the same rows. Per chunk:
         // four loads of 32 columns, each staged in two halves (each thread its
-        // 64 bytes, 16-byte unit u at u ^ (lane & 3)); the warp adds eight rows'
-        // 64-byte segments per instruction into the accumulator (sorted rows).
+        // 64 bytes, 16-byte unit u at u ^ (lane & 3)); the warp writes eight
+        // rows' 64-byte segments per instruction into the accumulator (sorted
+        // rows): plain stores in a draft tile (the first contribution), vector
+        // reductions in a context tile.
         const int sp = warp & 3;  // a warp reaches the TMEM lanes of sub-partition warp % 4 only
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
         uint8_t *stage = sm + L::oStage + sp * kDqStage;
+        int32_t *flags = p.dqflag + (size_t)region * p.n_draft;
         bool ok = true;
+        if (is_ctx) {
+            // the draft tiles holding the band's rows have stored them
+            const int d0 = (row0 / kBlock) / kGD, d1 = ((row0 + nrows) / kBlock - 1) / kGD;
+            const uint64_t tw = globaltimer();
+            for (int d = d0 + lane; ok && d <= d1; d += 32) {
+                while (ld_acquire(flags + d) < 4) {
+                    if (*abort_flag) { ok = false; break; }
+                    if (globaltimer() - tw > kWaitTimeoutNs) {
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(256);
+                }
+            }
+            ok = warp_all(ok);
+        }
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks;
             ok = warp_all(mbar_wait(dqfull, q & 1, abort_flag));
@@ -610,11 +676,21 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                         const int br = cr0 + (sl & 15);                    // band row
                         if (br < nrows) {
                             const uint4 val = *reinterpret_cast<const uint4 *>(stage + sl * 64 + ((u ^ (sl & 3)) << 4));
-                            red_add_v4(acc_rows + (size_t)br * kDQK + (sl >> 4) * 128 + 32 * rd + 16 * hf + 4 * u, val);
+                            float *dst = acc_rows + (size_t)br * kDQK + (sl >> 4) * 128 + 32 * rd + 16 * hf + 4 * u;
+                            if (is_ctx)
+                                red_add_v4(dst, val);
+                            else
+                                *reinterpret_cast<uint4 *>(dst) = val;
                         }
                     }
                     __syncwarp();
                 }
+            }
+            if (!is_ctx && q == QT - 1) {
+                // every row of the tile stored for every head
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(flags + item, 1);
             }
         }
     } else {
@@ -686,12 +762,12 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                 pw[i / 2] = pack_bf16x2(ep[0], ep[1]);
                 dw[i / 2] = pack_bf16x2(ed[0], ed[1]);
             }
-            // P^T / dS^T buffer q & 1 is free once the accumulation and the dQ
-            // contribution of chunk q - 2 completed; at a head's first chunk,
+            // the P^T / dS^T buffer is free once the dQ contribution and the
+            // accumulation of chunk q - 1 completed; at a head's first chunk,
             // every key warp has also read its staged rows of the previous
             // head's accumulators (staged in this same buffer)
-            uint8_t *pt = sm + L::oPT + (q & 1) * kPT;
-            if (q >= 2) ok = warp_all(mbar_wait(&ptfree[q & 1], ((q - 2) >> 1) & 1, abort_flag));
+            uint8_t *pt = sm + L::oPT;
+            if (q >= 1) ok = warp_all(mbar_wait(ptfree, (q - 1) & 1, abort_flag));
             if (ok && c == 0 && hh >= 1) ok = warp_all(mbar_wait(kdrain, (hh - 1) & 1, abort_flag));
             if (!ok) break;
             *reinterpret_cast<uint4 *>(pt + pu0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
@@ -703,20 +779,18 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(dsready);
             if (c != nchunks - 1) continue;
-            // head end, once its accumulations completed (its last dQ
-            // contribution may still run): accumulator columns
-            // [128 hr, 128 hr + 128) (lanes 0-15 dK, 16-31 dV) -> bf16 -> dK^C /
-            // dV rows, staged 32 columns at a time in the other P^T / dS^T
-            // buffer (free once chunk q - 1's MMAs completed; 2 KB per warp, each
+            // head end, once its accumulations (and, issued before them, its dQ
+            // contributions) completed: accumulator columns [128 hr, 128 hr + 128)
+            // (lanes 0-15 dK, 16-31 dV) -> bf16 -> dK^C / dV rows, staged 32
+            // columns at a time in the P^T / dS^T buffer (2 KB per warp, each
             // thread its 64 bytes, 16-byte unit u at u ^ (lane & 3)), the warp
             // writing 8 rows' 64-byte segments per instruction. dK columns
             // 192..255 (the rope slice) stay in TMEM, summed over heads. The
             // accumulator is then free for the next head.
             ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag));
-            if (ok && q >= 1) ok = warp_all(mbar_wait(&ptfree[(q + 1) & 1], ((q - 1) >> 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            uint8_t *stage = sm + L::oPT + ((q + 1) & 1) * kPT + warp * 2048;
+            uint8_t *stage = sm + L::oPT + warp * 2048;
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
 #pragma unroll 1
             for (int rd = 0; rd < 4; rd++) {
@@ -772,11 +846,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     if (*abort_flag) {
         volatile int never = 0;
         if (warp == kWarpKV && lane == 0) {
-            for (int t = counters[2]; t < counters[0]; ++t)
-                mbar_wait(&kvfull[t % KVS], (t / KVS) & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[0]; ++t) mbar_wait(kfull, t & 1, (volatile int *)&never);
+            for (int t = counters[3]; t < counters[1]; ++t) mbar_wait(vfull, t & 1, (volatile int *)&never);
         }
         if (warp == kWarpRow && lane == 0) {
-            for (int t = counters[3]; t < counters[1]; ++t)
+            for (int t = counters[4]; t < counters[2]; ++t)
                 mbar_wait(&rowfull[t % RS], (t / RS) & 1, (volatile int *)&never);
         }
         if (warp == kWarpMma && lane == 0) {
@@ -860,8 +934,8 @@ __global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int
     *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
 }
 
-// Stage counts of the one-pass kernel: K/V of two heads in flight, one row stage.
-constexpr int kKVS = 2, kRS = 1;
+// Row stages of the one-pass kernel.
+constexpr int kRS = 2;
 
 }  // namespace
 
@@ -887,8 +961,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         count_launch();
         k_bwd_prep<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(
             p.n_h, p.N, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dout, lse, ws.cnt,
-            ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs, (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses,
-            ws.dqacc);
+            ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs, (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses);
         count_launch();
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
@@ -908,7 +981,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         m_qs3_64 = m_dos3_64 = m_kc3_64;
     }
     BwdArgs a;
-    a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
+    a.B = p.B; a.n_h = p.n_h; a.S = p.S; a.N = p.N; a.W = p.W; a.L = p.L; a.R = p.R;
     a.scale_log2 = p.scale_log2;
     a.scale = p.scale;
     a.ds_ = ws.dvec;
@@ -916,19 +989,29 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.cnt = ws.cnt;
     a.sorted_n = ws.sorted_n;
     a.sorted_a = ws.sorted_a;
+    a.tab = ws.rope;
+    a.dq = (__nv_bfloat16 *)dq;
     a.dkc = (__nv_bfloat16 *)dkc;
     a.dv = (__nv_bfloat16 *)dv;
     a.dkr_part = ws.dkr_part;
     a.dqacc = ws.dqacc;
+    a.dqflag = ws.dqflag;
+    a.HG = HG;
     a.hpg = p.n_h / HG;
-    a.n_ctx_items = (p.S + bw::kMK - 1) / bw::kMK;
+    a.n_ctx = (p.S + bw::kMK - 1) / bw::kMK;
+    a.n_draft = (p.N + kGD - 1) / kGD;
     a.err = ws.err;
-    const dim3 grid(a.n_ctx_items + (p.N + kGD - 1) / kGD, HG, p.B);
-    constexpr int smem = bw::Smem<kKVS, kRS>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<kKVS, kRS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const size_t nflags = (size_t)p.B * HG * a.n_draft;
+    if (nflags) {
+        cudaError_t ee = cudaMemsetAsync(ws.dqflag, 0, nflags * sizeof(int32_t), st);
+        if (ee != cudaSuccess) return ee;
+    }
+    const unsigned grid = (unsigned)((size_t)p.B * HG * (a.n_draft + a.n_ctx));
+    constexpr int smem = bw::Smem<kRS>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<kRS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_tc<kKVS, kRS><<<grid, bw::kThreads, smem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kc3_8,
+    k_bwd_tc<kRS><<<grid, bw::kThreads, smem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kc3_8,
                                                           m_kr8, m_v3_8, a);
     if (p.N > 0) {
         count_launch();

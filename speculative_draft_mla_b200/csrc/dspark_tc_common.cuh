@@ -116,6 +116,10 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *m, int x, 
                  "r"(y), "r"(z)
                  : "memory");
 }
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *m, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)m), "r"(x), "r"(y)
+                 : "memory");
+}
 // 1-D bulk copy of `bytes` contiguous bytes (16-byte aligned addresses, size a
 // multiple of 16) completing on bar's transaction count.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
