@@ -45,7 +45,6 @@ struct WsLayout {
     size_t dos;       // bf16 [B, n_h, 5N, 256] dO, anchor-sorted rows
     size_t dkr_part;  // float [HG, B, L, d_r] rope-key gradient per head group
     size_t dqacc;     // float [B, n_h, 5N, d_c + d_r] dQ accumulator, anchor-sorted rows
-    size_t dqflag;    // int32 [B, HG, ceil(N / 8)] draft tiles whose dQ rows are stored
     size_t total;
 };
 
@@ -75,8 +74,6 @@ inline WsLayout ws_layout(const Prob &p) {
     w.dkr_part = off;
     off = align256(off + (tc ? sizeof(float) * (size_t)bwd_head_groups(p) * p.B * p.L * p.d_r : 0));
     w.dqacc = off;     off = align256(off + sizeof(float) * rows * p.dqk);
-    w.dqflag = off;
-    off = align256(off + (tc ? sizeof(int32_t) * (size_t)p.B * bwd_head_groups(p) * ((p.N + 7) / 8) : 0));
     w.total = off;
     return w;
 }
@@ -92,7 +89,6 @@ struct Ws {
     void *qs, *dos;
     float *dkr_part;
     float *dqacc;
-    int32_t *dqflag;
 };
 
 inline Ws ws_view(const Prob &p, void *base) {
@@ -111,7 +107,6 @@ inline Ws ws_view(const Prob &p, void *base) {
     w.dos = (void *)(c + l.dos);
     w.dkr_part = (float *)(c + l.dkr_part);
     w.dqacc = (float *)(c + l.dqacc);
-    w.dqflag = (int32_t *)(c + l.dqflag);
     return w;
 }
 

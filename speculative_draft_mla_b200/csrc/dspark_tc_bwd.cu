@@ -10,33 +10,31 @@
 // and dK^R, shared by every head (§4), is the sum over heads.
 //
 // Launch sequence (one stream):
-//   1. k_bwd_prep       per kept block and head: rotated Q and dO copied into
-//                       anchor-sorted row order, D, LSE*log2(e).
+//   1. k_bwd_prep       per kept block, looping over the heads: rotated Q and
+//                       dO copied into anchor-sorted row order, D, LSE*log2(e),
+//                       and the whole backward of the block's own 5 draft keys
+//                       (5 x 5 per head, on the CUDA cores): their dK^C, dV and
+//                       dK^R (summed over heads), and the rows' draft-key dQ
+//                       contribution, stored as the first value of the fp32 dQ
+//                       accumulator (anchor-sorted rows).
 //   2. k_bwd_pad        zeros for padding blocks' rows and draft keys.
-//   3. k_bwd_tc         key-major, one CTA per (b, 64-key tile, head group),
-//                       one pass over K and V: rows of the blocks whose key
-//                       sets meet the tile, in chunks of 64. S^T = K Q^T and
-//                       dP^T = V dO^T in TMEM, P^T and dS^T through shared
-//                       memory, dV += P^T dO and dK += dS^T Q accumulated in
-//                       TMEM over the rows (M = 64 accumulators: dK and dV share
-//                       TMEM columns, one in each half of the lanes), and the
-//                       chunk's dQ contribution dS K in TMEM. dK and dV are
-//                       written once, by the CTA that owns the keys (no
-//                       atomics). dQ goes through an fp32 accumulator in
-//                       anchor-sorted row order: the draft-key tiles come first
-//                       in the grid; each stores its rows' draft-key
-//                       contribution (every kept row belongs to exactly one draft
-//                       tile, so the accumulator needs no clearing) and raises a
-//                       flag; the context tiles wait for the flags of the rows
-//                       they meet, then add their contributions with vector
-//                       reductions.
+//   3. k_bwd_tc         key-major over the context, one CTA per (b, 64-key
+//                       tile, head group), one pass over K and V: rows of the
+//                       blocks whose windows meet the tile, in chunks of 64.
+//                       S^T = K Q^T and dP^T = V dO^T in TMEM, P^T and dS^T
+//                       through shared memory, dV += P^T dO and dK += dS^T Q
+//                       accumulated in TMEM over the rows (M = 64 accumulators:
+//                       dK and dV share TMEM columns, one in each half of the
+//                       lanes), and the chunk's dQ contribution dS K in TMEM,
+//                       added into the dQ accumulator with vector reductions.
+//                       dK and dV are written once, by the CTA that owns the
+//                       keys (no atomics).
 //   4. k_bwd_dq_out     rotates the rope part of the accumulated dQ back,
 //                       rounds to bf16 and writes dq in the caller's row order.
-//   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
-//                       them back and writes dK^R.
-// Key tiles are either context tiles [t0, t0+64) or the draft keys of one
-// group of 8 blocks; the blocks whose windows meet a context tile are a
-// contiguous run of the anchor-sorted list (t0 < A <= t0 + 63 + W - 1).
+//   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials of the
+//                       context keys, rotates them back and writes dK^R.
+// The blocks whose windows meet a context tile [t0, t0 + 64) are a contiguous
+// run of the anchor-sorted list (t0 < A <= t0 + 63 + W - 1).
 #include <algorithm>
 
 #include "dspark_tc_common.cuh"
@@ -48,14 +46,57 @@ namespace {
 using namespace tc;
 
 constexpr int kDC = 192, kDR = 64, kDQK = 256, kDV = 256;
-constexpr int kGD = 8;   // blocks per draft-key tile (8 slots each: 64 keys)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
-// One warp per row of a kept block (5 warps): rotated q -> qs, do -> dos,
-// D = rowsum(dO * O), LSE * log2(e); rows past the kept blocks are zeroed so
-// tiles that overhang them multiply finite values.
-__global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfloat16 *__restrict__ q,
+// The row-wise preparation and the draft-key part of the backward, one CTA
+// per kept block (anchor-sorted index i) and batch row, looping over the
+// heads. A producer warp stages each head's inputs into shared memory with
+// bulk copies, kPrepStages heads ahead: the block's 5 rows of q, O and dO and
+// its 5 draft keys' K^C and V (the rotated rope keys of the draft keys are the
+// same for all heads and are staged once). Compute warp j handles row 5 n + j,
+// lane l dims 8 l .. 8 l + 7. Per head:
+//   - rotated q -> qs, do -> dos (anchor-sorted rows), D = rowsum(dO * O),
+//     LSE * log2(e);
+//   - the block's own 5 draft keys, which no other row sees (page §3):
+//     S = q_rot k_rot^T s and dP = dO V^T over the 5 keys, P = exp(S - LSE),
+//     dS = P (dP - D) s; the rows' draft-key dQ contribution dS K_rot is
+//     stored as the first value of the fp32 dQ accumulator (the context tiles
+//     add theirs later, in stream order), and the draft keys' gradients
+//     dK = dS^T q_rot, dV = P^T dO are complete here: warp j then stands for
+//     draft key j, writes its dK^C and dV, and sums the rope part of dK over
+//     the heads in registers, written rotated back after the last head.
+// q_rot is rounded to bf16 as the tensor-core kernels see it (the forward's
+// LSE was formed from the same rounded operands). Rows past the kept blocks
+// are zeroed so that tiles overhanging them multiply finite values. Every
+// wait is bounded; on time-out the CTA stops issuing, waits (bounded) for its
+// copies in flight and sets the timeout bit of the error word.
+namespace pr {
+// Barrier 1 of the five compute warps with an OR over their predicates: every
+// warp gets the same answer from one barrier instance.
+__device__ __forceinline__ bool compute_warps_or(bool x) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 160, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)x)
+        : "memory");
+    return r != 0;
+}
+constexpr int kStages = 3;
+constexpr int kRowsB = kBlock * kDQK * 2;  // 5 rows of 256 bf16 (q, O, dO, V)
+constexpr int kKcB = kBlock * kDC * 2;     // 5 rows of K^C
+constexpr int oQ = 0, oO = kRowsB, oDO = 2 * kRowsB, oV = 3 * kRowsB, oKc = 4 * kRowsB;
+constexpr int kStageB = 4 * kRowsB + kKcB;  // 12160
+constexpr int kThreads = 6 * 32;           // 5 compute warps + the producer
+}  // namespace pr
+
+__global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, int N, int L, float scale, float scale_log2,
+                                                  const __nv_bfloat16 *__restrict__ q,
+                                                  const __nv_bfloat16 *__restrict__ kc,
+                                                  const __nv_bfloat16 *__restrict__ krr,
+                                                  const __nv_bfloat16 *__restrict__ v,
                                                   const __nv_bfloat16 *__restrict__ o,
                                                   const __nv_bfloat16 *__restrict__ dout,
                                                   const float *__restrict__ lse, const int32_t *__restrict__ cnt,
@@ -63,64 +104,234 @@ __global__ void __launch_bounds__(160) k_bwd_prep(int n_h, int N, const __nv_bfl
                                                   const int32_t *__restrict__ sorted_a,
                                                   const float2 *__restrict__ tab, __nv_bfloat16 *__restrict__ qs,
                                                   __nv_bfloat16 *__restrict__ dos, float *__restrict__ ds_,
-                                                  float *__restrict__ lses) {
-    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+                                                  float *__restrict__ lses, float *__restrict__ dqacc,
+                                                  __nv_bfloat16 *__restrict__ dkc, __nv_bfloat16 *__restrict__ dkr,
+                                                  __nv_bfloat16 *__restrict__ dv, uint32_t *err) {
+    using namespace pr;
+    __shared__ __align__(128) uint8_t st[kStages][kStageB];
+    __shared__ __align__(16) uint4 s_kr[kBlock][8];                // rotated rope keys of the draft keys
+    __shared__ __align__(16) uint4 s_q[kBlock][32], s_do[kBlock][32];  // the head's rotated q and dO rows
+    __shared__ float s_p[kBlock][kBlock], s_ds[kBlock][kBlock];  // [row][key]
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], krbar;
+    __shared__ int abort_s;
+    const int i = blockIdx.x, b = blockIdx.y;
     const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
-    const size_t bh = (size_t)b * n_h + h;
-    const size_t srow = bh * R + kBlock * i + j;
-    uint4 *qd = reinterpret_cast<uint4 *>(qs + srow * kDQK) + lane;
-    uint4 *dd = reinterpret_cast<uint4 *>(dos + srow * kDV) + lane;
     if (i >= cnt[b]) {
-        *qd = make_uint4(0, 0, 0, 0);
-        *dd = make_uint4(0, 0, 0, 0);
-        if (lane == 0) {
-            ds_[srow] = 0.f;
-            lses[srow] = 0.f;
-        }
+        if (j < kBlock)
+            for (int h = 0; h < n_h; h++) {
+                const size_t srow = ((size_t)b * n_h + h) * R + kBlock * i + j;
+                reinterpret_cast<uint4 *>(qs + srow * kDQK)[lane] = make_uint4(0, 0, 0, 0);
+                reinterpret_cast<uint4 *>(dos + srow * kDV)[lane] = make_uint4(0, 0, 0, 0);
+                if (lane == 0) {
+                    ds_[srow] = 0.f;
+                    lses[srow] = 0.f;
+                }
+            }
         return;
     }
     const int n = sorted_n[(size_t)b * N + i], a = sorted_a[(size_t)b * N + i];
-    const size_t orow = bh * R + kBlock * n + j;
-    uint4 qv = __ldg(reinterpret_cast<const uint4 *>(q + orow * kDQK) + lane);
-    if (lane >= 24) {
-        const float2 *cs = tab + (size_t)(a + j) * (kDR / 2) + (lane - 24) * 4;
-        uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&w[k]);
-            const float x0 = __bfloat162float(pr.x), x1 = __bfloat162float(pr.y);
-            const float2 c = __ldg(cs + k);
-            w[k] = pack_bf16x2(x0 * c.x - x1 * c.y, x0 * c.y + x1 * c.x);
+    const size_t key0 = (size_t)S + kBlock * n;  // the block's first draft key
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; s++) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], kBlock);
         }
-        qv = make_uint4(w[0], w[1], w[2], w[3]);
+        tc::mbar_init(&krbar, 1);
+        abort_s = 0;
+        tc::fence_barrier_init();
     }
-    *qd = qv;
-    const uint4 dv = __ldg(reinterpret_cast<const uint4 *>(dout + orow * kDV) + lane);
-    const uint4 ov = __ldg(reinterpret_cast<const uint4 *>(o + orow * kDV) + lane);
-    *dd = dv;
-    const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
-    float accd = 0.f;
+    __syncthreads();
+    volatile int *abort_flag = &abort_s;
+    if (j == kBlock) {
+        // ---------------------------------------------------- producer
+        int issued = 0;
+        if (lane == 0) {
+            tc::mbar_arrive_expect_tx(&krbar, kBlock * kDR * 2);
+            tc::bulk_load(&s_kr[0][0], krr + ((size_t)b * L + key0) * kDR, kBlock * kDR * 2, &krbar);
+            for (int h = 0; h < n_h; h++) {
+                const int s = h % kStages;
+                if (h >= kStages && !tc::mbar_wait(&empty[s], ((h / kStages) - 1) & 1, abort_flag)) break;
+                const size_t bh = (size_t)b * n_h + h;
+                const size_t orow = (bh * R + kBlock * n) * kDQK, krow = bh * L + key0;
+                uint8_t *d = st[s];
+                tc::mbar_arrive_expect_tx(&full[s], kStageB);
+                tc::bulk_load(d + oQ, q + orow, kRowsB, &full[s]);
+                tc::bulk_load(d + oO, o + orow, kRowsB, &full[s]);
+                tc::bulk_load(d + oDO, dout + orow, kRowsB, &full[s]);
+                tc::bulk_load(d + oV, v + krow * kDV, kRowsB, &full[s]);
+                tc::bulk_load(d + oKc, kc + krow * kDC, kKcB, &full[s]);
+                issued = h + 1;
+            }
+        }
+        // every copy issued has landed before the CTA may end (each wait bounded)
+        __syncwarp();
+        if (lane == 0) {
+            volatile int never = 0;
+            tc::mbar_wait(&krbar, 0, &never);
+            for (int h = max(0, issued - kStages); h < issued; h++)
+                tc::mbar_wait(&full[h % kStages], (h / kStages) & 1, &never);
+        }
+    } else {
+        // ------------------------------------------------ compute warps
+        // RoPE (cos, sin) of this lane's 4 frequencies at the row's position
+        // a + j (query rotation) and at the key position a + j (warp j as a key)
+        float2 cq[4] = {};
+        if (lane >= 24)
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&dw[k]);
-        const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162 *>(&ow[k]);
-        accd = fmaf(__bfloat162float(x.x), __bfloat162float(y.x), accd);
-        accd = fmaf(__bfloat162float(x.y), __bfloat162float(y.y), accd);
+            for (int f = 0; f < 4; f++) cq[f] = __ldg(tab + (size_t)(a + j) * (kDR / 2) + (lane - 24) * 4 + f);
+        float dkr_acc[8] = {};  // warp j = draft key j: rope part of dK, summed over heads (lanes 24-31)
+        // The compute warps leave together: each bounded wait is followed by a
+        // barrier of the five warps that ORs their "give up" predicates, so no
+        // warp is left waiting at a barrier the others have abandoned.
+        bool ok = !compute_warps_or(!tc::mbar_wait(&krbar, 0, abort_flag) || *abort_flag);
+        float lse_n = ok ? lse[((size_t)b * n_h) * R + kBlock * n + j] : 0.f;
+        for (int h = 0; h < n_h && ok; h++) {
+            const int s = h % kStages;
+            const size_t bh = (size_t)b * n_h + h;
+            const size_t srow = bh * R + kBlock * i + j;
+            const float lse_r = lse_n;
+            if (h + 1 < n_h) lse_n = lse[(bh + 1) * R + kBlock * n + j];  // the next head's, ahead of need
+            if (compute_warps_or(!tc::mbar_wait(&full[s], (h / kStages) & 1, abort_flag) || *abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint8_t *d = st[s];
+            uint4 qv = reinterpret_cast<const uint4 *>(d + oQ + j * kDQK * 2)[lane];
+            if (lane >= 24) {
+                uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                for (int f = 0; f < 4; f++) {
+                    const float x0 = __uint_as_float(w[f] << 16), x1 = __uint_as_float(w[f] & 0xffff0000u);
+                    w[f] = pack_bf16x2(x0 * cq[f].x - x1 * cq[f].y, x0 * cq[f].y + x1 * cq[f].x);
+                }
+                qv = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            const uint4 dv4 = reinterpret_cast<const uint4 *>(d + oDO + j * kDV * 2)[lane];
+            const uint4 ov4 = reinterpret_cast<const uint4 *>(d + oO + j * kDV * 2)[lane];
+            reinterpret_cast<uint4 *>(qs + srow * kDQK)[lane] = qv;
+            reinterpret_cast<uint4 *>(dos + srow * kDV)[lane] = dv4;
+            s_q[j][lane] = qv;
+            s_do[j][lane] = dv4;
+            float sc[kBlock], dp[kBlock], dd = 0.f;
+            {
+                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+                const uint32_t ow[4] = {ov4.x, ov4.y, ov4.z, ov4.w};
+#pragma unroll
+                for (int f = 0; f < 4; f++) {
+                    dd = fmaf(__uint_as_float(dw[f] << 16), __uint_as_float(ow[f] << 16), dd);
+                    dd = fmaf(__uint_as_float(dw[f] & 0xffff0000u), __uint_as_float(ow[f] & 0xffff0000u), dd);
+                }
+#pragma unroll
+                for (int k = 0; k < kBlock; k++) {
+                    const uint4 kq = lane < 24 ? reinterpret_cast<const uint4 *>(d + oKc + k * kDC * 2)[lane]
+                                               : s_kr[k][lane - 24];
+                    const uint4 vv = reinterpret_cast<const uint4 *>(d + oV + k * kDV * 2)[lane];
+                    const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                    float s1 = 0.f, p1 = 0.f;
+#pragma unroll
+                    for (int f = 0; f < 4; f++) {
+                        s1 = fmaf(__uint_as_float(qw[f] << 16), __uint_as_float(kw[f] << 16), s1);
+                        s1 = fmaf(__uint_as_float(qw[f] & 0xffff0000u), __uint_as_float(kw[f] & 0xffff0000u), s1);
+                        p1 = fmaf(__uint_as_float(dw[f] << 16), __uint_as_float(vw[f] << 16), p1);
+                        p1 = fmaf(__uint_as_float(dw[f] & 0xffff0000u), __uint_as_float(vw[f] & 0xffff0000u), p1);
+                    }
+                    sc[k] = s1;
+                    dp[k] = p1;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                dd += __shfl_xor_sync(0xffffffffu, dd, off);
+#pragma unroll
+                for (int k = 0; k < kBlock; k++) {
+                    sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], off);
+                    dp[k] += __shfl_xor_sync(0xffffffffu, dp[k], off);
+                }
+            }
+            const float lse2 = lse_r * kLog2e;
+            if (lane == 0) {
+                ds_[srow] = dd;
+                lses[srow] = lse2;
+            }
+            // the row's draft-key dQ contribution, dims 8 lane .. + 7
+            float dqv[8] = {};
+#pragma unroll
+            for (int k = 0; k < kBlock; k++) {
+                const float pk = exp2f(fmaf(sc[k], scale_log2, -lse2));
+                const float dsk = pk * (dp[k] - dd) * scale;
+                if (lane == 0) {
+                    s_p[j][k] = pk;
+                    s_ds[j][k] = dsk;
+                }
+                const uint4 kq = lane < 24 ? reinterpret_cast<const uint4 *>(d + oKc + k * kDC * 2)[lane] : s_kr[k][lane - 24];
+                const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w};
+#pragma unroll
+                for (int f = 0; f < 4; f++) {
+                    dqv[2 * f] = fmaf(dsk, __uint_as_float(kw[f] << 16), dqv[2 * f]);
+                    dqv[2 * f + 1] = fmaf(dsk, __uint_as_float(kw[f] & 0xffff0000u), dqv[2 * f + 1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
+            float4 *acc = reinterpret_cast<float4 *>(dqacc + srow * kDQK) + 2 * lane;
+            acc[0] = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
+            acc[1] = make_float4(dqv[4], dqv[5], dqv[6], dqv[7]);
+            asm volatile("bar.sync 1, 160;" ::: "memory");  // the compute warps' rows and weights are staged
+            // warp j now stands for draft key j: dK = sum_r dS[r][j] q_rot[r],
+            // dV = sum_r P[r][j] dO[r]
+            float dk[8] = {}, dvv[8] = {};
+#pragma unroll
+            for (int r = 0; r < kBlock; r++) {
+                const float pr = s_p[r][j], dsr = s_ds[r][j];
+                const uint4 qa = s_q[r][lane], da = s_do[r][lane];
+                const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, dw[4] = {da.x, da.y, da.z, da.w};
+#pragma unroll
+                for (int f = 0; f < 4; f++) {
+                    dk[2 * f] = fmaf(dsr, __uint_as_float(qw[f] << 16), dk[2 * f]);
+                    dk[2 * f + 1] = fmaf(dsr, __uint_as_float(qw[f] & 0xffff0000u), dk[2 * f + 1]);
+                    dvv[2 * f] = fmaf(pr, __uint_as_float(dw[f] << 16), dvv[2 * f]);
+                    dvv[2 * f + 1] = fmaf(pr, __uint_as_float(dw[f] & 0xffff0000u), dvv[2 * f + 1]);
+                }
+            }
+            asm volatile("bar.sync 1, 160;" ::: "memory");  // read before the next head overwrites them
+            const size_t krow = bh * L + key0 + j;
+            reinterpret_cast<uint4 *>(dv + krow * kDV)[lane] =
+                make_uint4(pack_bf16x2(dvv[0], dvv[1]), pack_bf16x2(dvv[2], dvv[3]), pack_bf16x2(dvv[4], dvv[5]),
+                           pack_bf16x2(dvv[6], dvv[7]));
+            if (lane < 24) {
+                reinterpret_cast<uint4 *>(dkc + krow * kDC)[lane] =
+                    make_uint4(pack_bf16x2(dk[0], dk[1]), pack_bf16x2(dk[2], dk[3]), pack_bf16x2(dk[4], dk[5]),
+                               pack_bf16x2(dk[6], dk[7]));
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; e++) dkr_acc[e] += dk[e];
+            }
+        }
+        // the draft keys' rope gradient (sum over heads, rotated frame) rotated
+        // back by the key position a + j
+        if (ok && lane >= 24) {
+            float y[8];
+#pragma unroll
+            for (int f = 0; f < 4; f++) {
+                const float x0 = dkr_acc[2 * f], x1 = dkr_acc[2 * f + 1];
+                y[2 * f] = x0 * cq[f].x + x1 * cq[f].y;
+                y[2 * f + 1] = x1 * cq[f].x - x0 * cq[f].y;
+            }
+            reinterpret_cast<uint4 *>(dkr + ((size_t)b * L + key0 + j) * kDR)[lane - 24] = make_uint4(
+                pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+        }
     }
-    for (int off = 16; off > 0; off >>= 1) accd += __shfl_xor_sync(0xffffffffu, accd, off);
-    if (lane == 0) {
-        ds_[srow] = accd;
-        lses[srow] = lse[orow] * kLog2e;
-    }
+    __syncthreads();
+    if (threadIdx.x == 0 && abort_s) atomicOr(err, kErrTimeout);
 }
 
 // -------------------------------------------------------------- padding
 // Padding blocks (keep = 0 or invalid anchor): dq rows and the block's own
-// draft keys' dkc / dv get zeros (their dkr is zeroed by the reduction).
+// draft keys' dkc / dv / dkr get zeros.
 __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, const int32_t *anchors,
                                                  const uint8_t *keep, __nv_bfloat16 *dq, __nv_bfloat16 *dkc,
-                                                 __nv_bfloat16 *dv) {
+                                                 __nv_bfloat16 *dkr, __nv_bfloat16 *dv) {
     const int n = blockIdx.x, b = blockIdx.y;
     const int a = anchors[(size_t)b * N + n];
     if (keep[(size_t)b * N + n] && a >= 0 && a <= S - 2) return;
@@ -135,6 +346,8 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
         for (int e = threadIdx.x; e < kBlock * kDC / 8; e += blockDim.x) k4[e] = z;
         for (int e = threadIdx.x; e < kBlock * kDV / 8; e += blockDim.x) v4[e] = z;
     }
+    uint4 *r4 = reinterpret_cast<uint4 *>(dkr + ((size_t)b * L + S + kBlock * n) * kDR);
+    for (int e = threadIdx.x; e < kBlock * kDR / 8; e += blockDim.x) r4[e] = z;
 }
 
 struct BwdArgs {
@@ -145,17 +358,10 @@ struct BwdArgs {
     const float2 *tab;
     __nv_bfloat16 *dq, *dkc, *dv;
     float *dkr_part, *dqacc;
-    int32_t *dqflag;
     int HG, hpg;  // head groups, heads per group
-    int n_ctx, n_draft;  // context / draft-key tiles per (batch row, head group)
+    int n_ctx;    // context tiles per batch row
     uint32_t *err;
 };
-
-__device__ __forceinline__ int ld_acquire(const int32_t *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
 __device__ __forceinline__ void red_add_v4(float *addr, const uint4 &v) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(v.x)),
@@ -191,11 +397,6 @@ namespace bw {
 constexpr int kMK = 64;                    // keys per tile (MMA M)
 constexpr int kRC = 64;                    // rows per chunk (MMA N of S^T / dP^T, K of the accumulations)
 constexpr int kSlice = 64 * 128;           // 8 KB: 64 keys or rows x 64 columns, 128-byte swizzled
-// Draft tiles are block-major: block bb's 8 K^C rows (3 x 1 KB swizzled
-// slices) at bb * 3 KB, its K^R rows at bb * 1 KB of the rope-key tile, its V
-// rows (4 x 1 KB) at bb * 4 KB: 8-key groups 3 KB / 4 KB apart, 64-column
-// slices 1 KB apart.
-constexpr int kDraftKcBlock = 3 * 1024, kDraftVBlock = 4 * 1024;
 constexpr int kRowStage = 8 * kSlice;      // Q chunk (4 slices), then dO chunk (4 slices)
 constexpr int kPT = 2 * kSlice;            // P^T, then dS^T: [64 keys][64 rows] bf16 each
 constexpr int kDqStage = 32 * 64;          // per dQ warp: 32 lanes x 16 fp32
@@ -231,8 +432,7 @@ template <int RS>
 __global__ void __launch_bounds__(bw::kThreads, 1)
     k_bwd_tc(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-             const __grid_constant__ CUtensorMap tm_dos, const __grid_constant__ CUtensorMap tm_kc8,
-             const __grid_constant__ CUtensorMap tm_kr8, const __grid_constant__ CUtensorMap tm_v8, const BwdArgs p) {
+             const __grid_constant__ CUtensorMap tm_dos, const BwdArgs p) {
     using namespace bw;
     using L = Smem<RS>;
     extern __shared__ uint8_t smem_raw[];
@@ -247,50 +447,29 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     int *counters = reinterpret_cast<int *>(tmem_slot + 2);
     int *band = counters + 5;  // first sorted row, row count
 
-    // Items: all draft-key tiles (region-major, region = (b, head group)),
-    // then all context tiles, so that a context tile starts after the draft
-    // tiles of its rows were dispatched.
-    const int n_draft_all = p.B * p.HG * p.n_draft;
-    const bool is_ctx = (int)blockIdx.x >= n_draft_all;
-    const int rel = is_ctx ? (int)blockIdx.x - n_draft_all : (int)blockIdx.x;
-    const int per = is_ctx ? p.n_ctx : p.n_draft;
-    const int region = rel / per, item = rel % per;
+    // item = (region = (b, head group), context tile)
+    const int region = (int)blockIdx.x / p.n_ctx, item = (int)blockIdx.x % p.n_ctx;
     const int b = region / p.HG, hg = region % p.HG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cnt = p.cnt[b];
-    int t0 = 0, gcnt = 0, i0 = 0;
-    if (is_ctx) {
-        t0 = item * kMK;
-    } else {
-        i0 = item * kGD;
-        if (i0 >= cnt) return;  // uniform: fewer draft tiles in this batch row
-        gcnt = min(kGD, cnt - i0);
-    }
+    const int t0 = item * kMK;
     const int32_t *sa = p.sorted_a + (size_t)b * p.N;
     const int32_t *sn = p.sorted_n + (size_t)b * p.N;
     if (threadIdx.x == 0) {
-        int r0, nr;
-        if (is_ctx) {
-            // blocks with t0 < A <= t0 + kMK - 1 + W - 1
-            int lo = 0, hi = cnt;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (sa[mid] > t0) hi = mid; else lo = mid + 1;
-            }
-            const long long lim = (long long)t0 + kMK - 1 + p.W - 1;
-            int lo2 = lo, hi2 = cnt;
-            while (lo2 < hi2) {
-                const int mid = (lo2 + hi2) >> 1;
-                if ((long long)sa[mid] > lim) hi2 = mid; else lo2 = mid + 1;
-            }
-            r0 = kBlock * lo;
-            nr = kBlock * (lo2 - lo);
-        } else {
-            r0 = kBlock * i0;
-            nr = kBlock * gcnt;
+        // blocks with t0 < A <= t0 + kMK - 1 + W - 1
+        int lo = 0, hi = cnt;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sa[mid] > t0) hi = mid; else lo = mid + 1;
         }
-        band[0] = r0;
-        band[1] = nr;
+        const long long lim = (long long)t0 + kMK - 1 + p.W - 1;
+        int lo2 = lo, hi2 = cnt;
+        while (lo2 < hi2) {
+            const int mid = (lo2 + hi2) >> 1;
+            if ((long long)sa[mid] > lim) hi2 = mid; else lo2 = mid + 1;
+        }
+        band[0] = kBlock * lo;
+        band[1] = kBlock * (lo2 - lo);
     }
     __syncthreads();
     const int row0 = band[0], nrows = band[1];
@@ -302,17 +481,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     const int kk = 16 * (warp & 3) + (lane & 15);
     const int hr = (warp >> 2) & 1;  // row half of a chunk / column half of the accumulators
     const bool dlane = lane >= 16;   // lane of the dP^T / dV half
-    bool key_valid = false;
-    size_t key_pos = 0;
-    if (warp < kKeyWarps) {
-        if (is_ctx) {
-            key_valid = t0 + kk < p.S;
-            key_pos = (size_t)t0 + kk;
-        } else {  // 8 key slots per block: its 5 keys, then 3 masked rows
-            key_valid = kk / 8 < gcnt && kk % 8 < kBlock;
-            if (key_valid) key_pos = (size_t)p.S + kBlock * sn[i0 + kk / 8] + kk % 8;
-        }
-    }
+    const bool key_valid = warp < kKeyWarps && t0 + kk < p.S;
+    const size_t key_pos = key_valid ? (size_t)t0 + kk : 0;
     float *dkr_part_row = p.dkr_part + (((size_t)hg * p.B + b) * p.L + key_pos) * kDR;
 
     if (nrows == 0) {
@@ -373,62 +543,25 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         // ------------------------------------------- producer of K/V tiles
         // Per head: V once the previous head's last dP^T completed, then K^C
         // (and, for the first head, the rope-key tile) once the previous head's
-        // last dQ contribution completed.
-        const int my_n = (!is_ctx && lane < gcnt) ? sn[i0 + lane] : 0;
+        // last dQ contribution completed; then the next head's tiles into L2, so
+        // that those loads wait on L2 rather than on DRAM.
         for (int hh = 0; hh < H; ++hh) {
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
             if (hh >= 1 && !warp_all(mbar_wait(vfree, (hh - 1) & 1, abort_flag))) break;
-            if (is_ctx) {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(vfull, 4 * kSlice);
-                    tma_load_3d(sm + L::oV, &tm_v, vfull, 0, (int)(bh * p.L + t0), 0);
-                }
-            } else {
-                if (lane == 0) mbar_arrive_expect_tx(vfull, gcnt * 8 * kDV * 2);
-                for (int bb = 0; bb < gcnt; ++bb) {
-                    const int nb = __shfl_sync(0xffffffffu, my_n, bb);
-                    if (lane == 0)
-                        tma_load_3d(sm + L::oV + bb * kDraftVBlock, &tm_v8, vfull, 0, (int)(bh * p.L + p.S + kBlock * nb),
-                                    0);
-                }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(vfull, 4 * kSlice);
+                tma_load_3d(sm + L::oV, &tm_v, vfull, 0, (int)(bh * p.L + t0), 0);
+                counters[1] = hh + 1;
             }
-            if (lane == 0) counters[1] = hh + 1;
             if (hh >= 1 && !warp_all(mbar_wait(kfree, (hh - 1) & 1, abort_flag))) break;
-            if (is_ctx) {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(kfull, (hh == 0 ? 4 : 3) * kSlice);
-                    if (hh == 0) tma_load_2d(sm + L::oKr, &tm_kr, kfull, 0, (int)((size_t)b * p.L + t0));
-                    tma_load_3d(sm + L::oKc, &tm_kc, kfull, 0, (int)(bh * p.L + t0), 0);
-                }
-            } else {
-                if (lane == 0) mbar_arrive_expect_tx(kfull, gcnt * 8 * (hh == 0 ? kDQK : kDC) * 2);
-                for (int bb = 0; bb < gcnt; ++bb) {
-                    const int nb = __shfl_sync(0xffffffffu, my_n, bb);
-                    if (lane == 0) {
-                        const int row = p.S + kBlock * nb;
-                        tma_load_3d(sm + L::oKc + bb * kDraftKcBlock, &tm_kc8, kfull, 0, (int)(bh * p.L + row), 0);
-                        if (hh == 0) tma_load_2d(sm + L::oKr + bb * 1024, &tm_kr8, kfull, 0, (int)((size_t)b * p.L + row));
-                    }
-                }
-            }
-            if (lane == 0) counters[0] = hh + 1;
-            // the next head's tiles into L2, so that their loads (issued once
-            // this head's tiles are free) wait on L2 rather than on DRAM
-            if (hh + 1 < H) {
-                const size_t bn = bh + 1;
-                if (is_ctx) {
-                    if (lane == 0) {
-                        tma_prefetch_l2_3d(&tm_kc, 0, (int)(bn * p.L + t0), 0);
-                        tma_prefetch_l2_3d(&tm_v, 0, (int)(bn * p.L + t0), 0);
-                    }
-                } else {
-                    for (int bb = 0; bb < gcnt; ++bb) {
-                        const int nb = __shfl_sync(0xffffffffu, my_n, bb);
-                        if (lane == 0) {
-                            tma_prefetch_l2_3d(&tm_kc8, 0, (int)(bn * p.L + p.S + kBlock * nb), 0);
-                            tma_prefetch_l2_3d(&tm_v8, 0, (int)(bn * p.L + p.S + kBlock * nb), 0);
-                        }
-                    }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(kfull, (hh == 0 ? 4 : 3) * kSlice);
+                if (hh == 0) tma_load_2d(sm + L::oKr, &tm_kr, kfull, 0, (int)((size_t)b * p.L + t0));
+                tma_load_3d(sm + L::oKc, &tm_kc, kfull, 0, (int)(bh * p.L + t0), 0);
+                counters[0] = hh + 1;
+                if (hh + 1 < H) {
+                    tma_prefetch_l2_3d(&tm_kc, 0, (int)((bh + 1) * p.L + t0), 0);
+                    tma_prefetch_l2_3d(&tm_v, 0, (int)((bh + 1) * p.L + t0), 0);
                 }
             }
         }
@@ -493,20 +626,20 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             const uint32_t idQ64 = idesc_bf16_ab(kRC, 64, 1, 1);
             // A operands of S^T / dP^T: K^C / V slices kcStep bytes apart
             // (context tile: 8 KB slices of 64 keys; draft tile: block-major)
-            const uint32_t kcStep = is_ctx ? kSlice : 1024;
-            const uint32_t kOff = is_ctx ? 1024 : kDraftKcBlock, vOff = is_ctx ? 1024 : kDraftVBlock;
+            // A operands of S^T / dP^T: K^C / V slices of 64 keys, 8 KB apart
             const SDesc krd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), 16, 1024));
             const SDesc ptd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT), 16, 1024));
             const SDesc dsd = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT + kSlice), 16, 1024));
             const SDesc dsq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oPT + kSlice), kSlice, 1024));
             // B operands of dQ_c, MN-major: dims 0..127 of K^C (two slices),
             // dims 128..191 (third slice), the rope key (dims 192..255); 16 keys
-            // are 2 KB in every case (context: 16 rows of 128 B; draft: 2 blocks)
-            const SDesc krq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), is_ctx ? kSlice : 1024, 1024));
-            const uint32_t kcq_step = is_ctx ? 128u : (uint32_t)((2 * kDraftKcBlock) >> 4);
+            // are 16 rows of 128 B (2 KB)
+            const SDesc krq = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKr), kSlice, 1024));
+            const SDesc kq0 = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKc), kSlice, 1024));
+            const SDesc kq1 = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKc + 2 * kSlice), kSlice, 1024));
             bool ok = true;
-            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKc), 16, kOff));
-            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + L::oV), 16, vOff));
+            const SDesc kad = sdesc_split(sdesc_sw128(smem_u32(sm + L::oKc), 16, 1024));
+            const SDesc vad = sdesc_split(sdesc_sw128(smem_u32(sm + L::oV), 16, 1024));
             auto issue_s = [&](int q) {
                 const int c = q % nchunks, s = q % RS, bsel = q & 1;
                 tc_fence_after();
@@ -519,10 +652,10 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                 for (int k16 = 0; k16 < kDQK / 16; ++k16) {
                     const int cc = k16 >> 2;
                     const uint32_t sub = (k16 & 3) * 2;  // 32 bytes, in 16-byte units
-                    const uint64_t ka = cc < 3 ? kad.at(((cc * kcStep) >> 4) + sub) : krd.at(sub);
+                    const uint64_t ka = cc < 3 ? kad.at(((cc * kSlice) >> 4) + sub) : krd.at(sub);
                     const uint32_t ro = (cc * kSlice + (k16 & 3) * 32) >> 4;
                     mma_bf16_ss(dS, ka, qd.at(ro), idS, k16 > 0 ? 1u : 0u);
-                    mma_bf16_ss(dP, vad.at(((cc * kcStep) >> 4) + sub), dod.at(ro), idS, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(dP, vad.at(((cc * kSlice) >> 4) + sub), dod.at(ro), idS, k16 > 0 ? 1u : 0u);
                 }
                 mma_commit(&sfull[bsel]);
                 if (c == nchunks - 1) mma_commit(vfree);  // the head's V tile is no longer read
@@ -553,14 +686,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             auto issue_dq = [&](int q) {
                 const int c = q % nchunks;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(sm + L::oKc);
-                const SDesc kq0 = sdesc_split(sdesc_sw128(kb, is_ctx ? kSlice : 1024, kOff));
-                const SDesc kq1 = sdesc_split(sdesc_sw128(kb + (is_ctx ? 2 * kSlice : 2048), kSlice, kOff));
 #pragma unroll
                 for (int k16 = 0; k16 < kMK / 16; ++k16) {
                     const uint64_t a = dsq.at(128 * k16);  // 16 keys = 16 rows of the dS^T tile
-                    mma_bf16_ss(tmem + kColDQ, a, kq0.at(kcq_step * k16), idQ128, k16 > 0 ? 1u : 0u);
-                    mma_bf16_ss(tmem + kColDQ + kHi, a, kq1.at(kcq_step * k16), idQ64, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColDQ, a, kq0.at(128 * k16), idQ128, k16 > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColDQ + kHi, a, kq1.at(128 * k16), idQ64, k16 > 0 ? 1u : 0u);
                     mma_bf16_ss(tmem + kColDQ + kHi + 64, a, krq.at(128 * k16), idQ64, k16 > 0 ? 1u : 0u);
                 }
                 mma_commit(dqfull);
@@ -620,30 +750,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         // four loads of 32 columns, each staged in two halves (each thread its
         // 64 bytes, 16-byte unit u at u ^ (lane & 3)); the warp writes eight
         // rows' 64-byte segments per instruction into the accumulator (sorted
-        // rows): plain stores in a draft tile (the first contribution), vector
-        // reductions in a context tile.
+        // rows) with vector reductions.
         const int sp = warp & 3;  // a warp reaches the TMEM lanes of sub-partition warp % 4 only
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
         uint8_t *stage = sm + L::oStage + sp * kDqStage;
-        int32_t *flags = p.dqflag + (size_t)region * p.n_draft;
         bool ok = true;
-        if (is_ctx) {
-            // the draft tiles holding the band's rows have stored them
-            const int d0 = (row0 / kBlock) / kGD, d1 = ((row0 + nrows) / kBlock - 1) / kGD;
-            const uint64_t tw = globaltimer();
-            for (int d = d0 + lane; ok && d <= d1; d += 32) {
-                while (ld_acquire(flags + d) < 4) {
-                    if (*abort_flag) { ok = false; break; }
-                    if (globaltimer() - tw > kWaitTimeoutNs) {
-                        *abort_flag = 1;
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(256);
-                }
-            }
-            ok = warp_all(ok);
-        }
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks;
             ok = warp_all(mbar_wait(dqfull, q & 1, abort_flag));
@@ -676,21 +787,11 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                         const int br = cr0 + (sl & 15);                    // band row
                         if (br < nrows) {
                             const uint4 val = *reinterpret_cast<const uint4 *>(stage + sl * 64 + ((u ^ (sl & 3)) << 4));
-                            float *dst = acc_rows + (size_t)br * kDQK + (sl >> 4) * 128 + 32 * rd + 16 * hf + 4 * u;
-                            if (is_ctx)
-                                red_add_v4(dst, val);
-                            else
-                                *reinterpret_cast<uint4 *>(dst) = val;
+                            red_add_v4(acc_rows + (size_t)br * kDQK + (sl >> 4) * 128 + 32 * rd + 16 * hf + 4 * u, val);
                         }
                     }
                     __syncwarp();
                 }
-            }
-            if (!is_ctx && q == QT - 1) {
-                // every row of the tile stored for every head
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicAdd(flags + item, 1);
             }
         }
     } else {
@@ -703,24 +804,19 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         // with kpos < A <= kpos + W - 1; draft key slot: its own block.
         int rlo = 0, rhi = 0;
         if (key_valid) {
-            if (is_ctx) {
-                int lo = row0 / kBlock, hi = (row0 + nrows) / kBlock;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (sa[mid] > kpos) hi = mid; else lo = mid + 1;
-                }
-                rlo = kBlock * lo - row0;
-                const long long lim = (long long)kpos + p.W - 1;
-                hi = (row0 + nrows) / kBlock;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if ((long long)sa[mid] > lim) hi = mid; else lo = mid + 1;
-                }
-                rhi = kBlock * lo - row0;
-            } else {
-                rlo = kBlock * (kk / 8);
-                rhi = rlo + kBlock;
+            int lo = row0 / kBlock, hi = (row0 + nrows) / kBlock;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (sa[mid] > kpos) hi = mid; else lo = mid + 1;
             }
+            rlo = kBlock * lo - row0;
+            const long long lim = (long long)kpos + p.W - 1;
+            hi = (row0 + nrows) / kBlock;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if ((long long)sa[mid] > lim) hi = mid; else lo = mid + 1;
+            }
+            rhi = kBlock * lo - row0;
         }
         // this key's row of the P^T / dS^T tiles (128-byte swizzle) and the
         // two 16-byte units that hold rows rb .. rb + 15
@@ -901,37 +997,24 @@ __global__ void __launch_bounds__(160) k_bwd_dq_out(int n_h, int N, const int32_
 }
 
 // ------------------------------------------------------------ dK^R reduce
-// One warp per (b, key): sum the head-group partials (rotated frame), rotate
-// back by the key's position, write dkr. Draft keys of padding blocks: 0.
-__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int L, int HG,
-                                                        const int32_t *anchors, const uint8_t *keep,
-                                                        const float2 *tab, const float *part,
-                                                        __nv_bfloat16 *dkr) {
+// One warp per (b, context key): sum the head-group partials (rotated frame),
+// rotate back by the key's position, write dkr. (The draft keys' dkr is
+// written by k_bwd_prep and k_bwd_pad.)
+__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int L, int HG, const float2 *tab,
+                                                        const float *part, __nv_bfloat16 *dkr) {
     const size_t wid = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (wid >= (size_t)B * L) return;
-    const int b = (int)(wid / L), key = (int)(wid % L);
-    int pos = key;
-    bool live = true;
-    if (key >= S) {
-        const int n = (key - S) / kBlock, i = (key - S) % kBlock;
-        const int a = anchors[(size_t)b * N + n];
-        live = keep[(size_t)b * N + n] && a >= 0 && a <= S - 2;
-        pos = a + i;
-    }
+    if (wid >= (size_t)B * S) return;
+    const int b = (int)(wid / S), key = (int)(wid % S);
     float x0 = 0.f, x1 = 0.f;
-    if (live) {
-        for (int g = 0; g < HG; g++) {
-            const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
-            x0 += v.x;
-            x1 += v.y;
-        }
-        const float2 cs = tab[(size_t)pos * (kDR / 2) + lane];
-        const float y0 = x0 * cs.x + x1 * cs.y, y1 = x1 * cs.x - x0 * cs.y;
-        x0 = y0;
-        x1 = y1;
+    for (int g = 0; g < HG; g++) {
+        const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
+        x0 += v.x;
+        x1 += v.y;
     }
-    *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
+    const float2 cs = tab[(size_t)key * (kDR / 2) + lane];
+    *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) =
+        __floats2bfloat162_rn(x0 * cs.x + x1 * cs.y, x1 * cs.x - x0 * cs.y);
 }
 
 // Row stages of the one-pass kernel.
@@ -945,10 +1028,10 @@ bool bwd_tc_supported(const Prob &p) {
 }
 
 int bwd_head_groups(const Prob &p) {
-    const long long items = (long long)((p.S + bw::kMK - 1) / bw::kMK + (p.N + kGD - 1) / kGD) * p.B;
-    // aim for about eight waves on 148 SMs (shorter CTAs, smaller tail)
+    const long long items = (long long)((p.S + bw::kMK - 1) / bw::kMK) * p.B;
+    // aim for about six waves on 148 SMs (shorter CTAs, smaller tail)
     int hg = 1;
-    while (hg < p.n_h && items * hg < 8 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
+    while (hg < p.n_h && items * hg < 6 * 148 && p.n_h % (hg * 2) == 0) hg *= 2;
     return hg;
 }
 
@@ -959,20 +1042,20 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     const int HG = bwd_head_groups(p);
     if (p.N > 0) {
         count_launch();
-        k_bwd_prep<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(
-            p.n_h, p.N, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dout, lse, ws.cnt,
-            ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs, (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses);
+        k_bwd_prep<<<dim3(p.N, p.B), pr::kThreads, 0, st>>>(
+            p.n_h, p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
+            (const __nv_bfloat16 *)ws.kr_rot, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)o,
+            (const __nv_bfloat16 *)dout, lse, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs,
+            (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dkr,
+            (__nv_bfloat16 *)dv, ws.err);
         count_launch();
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
-                                                   (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
+                                                   (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dkr, (__nv_bfloat16 *)dv);
     }
-    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kr8, m_kc3_8, m_v3_8;
+    CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
     if (!make_map3_bf16(&m_kc3_64, kc, kDC, kv_rows, 64) ||
-        !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) ||
-        !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64) ||
-        !make_map_bf16(&m_kr8, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 8) ||
-        !make_map3_bf16(&m_kc3_8, kc, kDC, kv_rows, 8) || !make_map3_bf16(&m_v3_8, v, kDV, kv_rows, 8))
+        !make_map_bf16(&m_kr64, ws.kr_rot, kDR, (uint64_t)p.B * p.L, 64) || !make_map3_bf16(&m_v3_64, v, kDV, kv_rows, 64))
         return cudaErrorInvalidValue;
     if (p.N > 0 && q_rows > 0) {
         if (!make_map3_bf16(&m_qs3_64, ws.qs, kDQK, q_rows, 64) || !make_map3_bf16(&m_dos3_64, ws.dos, kDV, q_rows, 64))
@@ -995,33 +1078,25 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.dv = (__nv_bfloat16 *)dv;
     a.dkr_part = ws.dkr_part;
     a.dqacc = ws.dqacc;
-    a.dqflag = ws.dqflag;
     a.HG = HG;
     a.hpg = p.n_h / HG;
     a.n_ctx = (p.S + bw::kMK - 1) / bw::kMK;
-    a.n_draft = (p.N + kGD - 1) / kGD;
     a.err = ws.err;
-    const size_t nflags = (size_t)p.B * HG * a.n_draft;
-    if (nflags) {
-        cudaError_t ee = cudaMemsetAsync(ws.dqflag, 0, nflags * sizeof(int32_t), st);
-        if (ee != cudaSuccess) return ee;
-    }
-    const unsigned grid = (unsigned)((size_t)p.B * HG * (a.n_draft + a.n_ctx));
+    const unsigned grid = (unsigned)((size_t)p.B * HG * a.n_ctx);
     constexpr int smem = bw::Smem<kRS>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<kRS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_tc<kRS><<<grid, bw::kThreads, smem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, m_kc3_8,
-                                                          m_kr8, m_v3_8, a);
+    k_bwd_tc<kRS><<<grid, bw::kThreads, smem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, a);
     if (p.N > 0) {
         count_launch();
         k_bwd_dq_out<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(p.n_h, p.N, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope,
                                                              ws.dqacc, (__nv_bfloat16 *)dq);
     }
-    const size_t warps = (size_t)p.B * p.L;
+    const size_t warps = (size_t)p.B * p.S;
     count_launch();
-    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
-                                                                   ws.dkr_part, (__nv_bfloat16 *)dkr);
+    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.L, HG, ws.rope, ws.dkr_part,
+                                                                   (__nv_bfloat16 *)dkr);
     return cudaGetLastError();
 }
 
