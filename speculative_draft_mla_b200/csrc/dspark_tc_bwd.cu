@@ -10,11 +10,11 @@
 // and dK^R, shared by every head (§4), is the sum over heads.
 //
 // Launch sequence (one stream):
-//   1. k_bwd_prep       per kept block, looping over the heads: rotated Q and
+//   1. k_bwd_prep       per kept block and head group: rotated Q and
 //                       dO copied into anchor-sorted row order, D, LSE*log2(e),
 //                       and the whole backward of the block's own 5 draft keys
 //                       (5 x 5 per head, on the CUDA cores): their dK^C, dV and
-//                       dK^R (summed over heads), and the rows' draft-key dQ
+//                       the group's partial dK^R, and the rows' draft-key dQ
 //                       contribution, stored as the first value of the fp32 dQ
 //                       accumulator (anchor-sorted rows).
 //   2. k_bwd_pad        zeros for padding blocks' rows and draft keys.
@@ -31,8 +31,8 @@
 //                       keys (no atomics).
 //   4. k_bwd_dq_out     rotates the rope part of the accumulated dQ back,
 //                       rounds to bf16 and writes dq in the caller's row order.
-//   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials of the
-//                       context keys, rotates them back and writes dK^R.
+//   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
+//                       them back and writes dK^R.
 // The blocks whose windows meet a context tile [t0, t0 + 64) are a contiguous
 // run of the anchor-sorted list (t0 < A <= t0 + 63 + W - 1).
 #include <algorithm>
@@ -50,8 +50,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
 // The row-wise preparation and the draft-key part of the backward, one CTA
-// per kept block (anchor-sorted index i) and batch row, looping over the
-// heads. A producer warp stages each head's inputs into shared memory with
+// per kept block (anchor-sorted index i), head group and batch row, looping
+// over the group's heads. A producer warp stages each head's inputs into shared memory with
 // bulk copies, kPrepStages heads ahead: the block's 5 rows of q, O and dO and
 // its 5 draft keys' K^C and V (the rotated rope keys of the draft keys are the
 // same for all heads and are staged once). Compute warp j handles row 5 n + j,
@@ -65,7 +65,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 //     add theirs later, in stream order), and the draft keys' gradients
 //     dK = dS^T q_rot, dV = P^T dO are complete here: warp j then stands for
 //     draft key j, writes its dK^C and dV, and sums the rope part of dK over
-//     the heads in registers, written rotated back after the last head.
+//     the group's heads in registers; after the last head that sum goes to the
+//     group's partial rope-key gradient (rotated frame), summed over the
+//     groups and rotated back by k_bwd_dkr_reduce.
 // q_rot is rounded to bf16 as the tensor-core kernels see it (the forward's
 // LSE was formed from the same rounded operands). Rows past the kept blocks
 // are zeroed so that tiles overhanging them multiply finite values. Every
@@ -92,7 +94,8 @@ constexpr int kStageB = 4 * kRowsB + kKcB;  // 12160
 constexpr int kThreads = 6 * 32;           // 5 compute warps + the producer
 }  // namespace pr
 
-__global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, int N, int L, float scale, float scale_log2,
+__global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int hpg, int S, int N, int L, float scale,
+                                                  float scale_log2,
                                                   const __nv_bfloat16 *__restrict__ q,
                                                   const __nv_bfloat16 *__restrict__ kc,
                                                   const __nv_bfloat16 *__restrict__ krr,
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, in
                                                   const float2 *__restrict__ tab, __nv_bfloat16 *__restrict__ qs,
                                                   __nv_bfloat16 *__restrict__ dos, float *__restrict__ ds_,
                                                   float *__restrict__ lses, float *__restrict__ dqacc,
-                                                  __nv_bfloat16 *__restrict__ dkc, __nv_bfloat16 *__restrict__ dkr,
+                                                  __nv_bfloat16 *__restrict__ dkc, float *__restrict__ dkr_part,
                                                   __nv_bfloat16 *__restrict__ dv, uint32_t *err) {
     using namespace pr;
     __shared__ __align__(128) uint8_t st[kStages][kStageB];
@@ -114,12 +117,13 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, in
     __shared__ float s_p[kBlock][kBlock], s_ds[kBlock][kBlock];  // [row][key]
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages], krbar;
     __shared__ int abort_s;
-    const int i = blockIdx.x, b = blockIdx.y;
+    const int i = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
     const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
+    const int h0 = hg * hpg;
     if (i >= cnt[b]) {
         if (j < kBlock)
-            for (int h = 0; h < n_h; h++) {
+            for (int h = h0; h < h0 + hpg; h++) {
                 const size_t srow = ((size_t)b * n_h + h) * R + kBlock * i + j;
                 reinterpret_cast<uint4 *>(qs + srow * kDQK)[lane] = make_uint4(0, 0, 0, 0);
                 reinterpret_cast<uint4 *>(dos + srow * kDV)[lane] = make_uint4(0, 0, 0, 0);
@@ -149,10 +153,10 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, in
         if (lane == 0) {
             tc::mbar_arrive_expect_tx(&krbar, kBlock * kDR * 2);
             tc::bulk_load(&s_kr[0][0], krr + ((size_t)b * L + key0) * kDR, kBlock * kDR * 2, &krbar);
-            for (int h = 0; h < n_h; h++) {
+            for (int h = 0; h < hpg; h++) {
                 const int s = h % kStages;
                 if (h >= kStages && !tc::mbar_wait(&empty[s], ((h / kStages) - 1) & 1, abort_flag)) break;
-                const size_t bh = (size_t)b * n_h + h;
+                const size_t bh = (size_t)b * n_h + h0 + h;
                 const size_t orow = (bh * R + kBlock * n) * kDQK, krow = bh * L + key0;
                 uint8_t *d = st[s];
                 tc::mbar_arrive_expect_tx(&full[s], kStageB);
@@ -185,13 +189,13 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, in
         // barrier of the five warps that ORs their "give up" predicates, so no
         // warp is left waiting at a barrier the others have abandoned.
         bool ok = !compute_warps_or(!tc::mbar_wait(&krbar, 0, abort_flag) || *abort_flag);
-        float lse_n = ok ? lse[((size_t)b * n_h) * R + kBlock * n + j] : 0.f;
-        for (int h = 0; h < n_h && ok; h++) {
+        float lse_n = ok ? lse[((size_t)b * n_h + h0) * R + kBlock * n + j] : 0.f;
+        for (int h = 0; h < hpg && ok; h++) {
             const int s = h % kStages;
-            const size_t bh = (size_t)b * n_h + h;
+            const size_t bh = (size_t)b * n_h + h0 + h;
             const size_t srow = bh * R + kBlock * i + j;
             const float lse_r = lse_n;
-            if (h + 1 < n_h) lse_n = lse[(bh + 1) * R + kBlock * n + j];  // the next head's, ahead of need
+            if (h + 1 < hpg) lse_n = lse[(bh + 1) * R + kBlock * n + j];  // the next head's, ahead of need
             if (compute_warps_or(!tc::mbar_wait(&full[s], (h / kStages) & 1, abort_flag) || *abort_flag)) {
                 ok = false;
                 break;
@@ -308,18 +312,13 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, in
                 for (int e = 0; e < 8; e++) dkr_acc[e] += dk[e];
             }
         }
-        // the draft keys' rope gradient (sum over heads, rotated frame) rotated
-        // back by the key position a + j
+        // the draft key's rope gradient summed over the group's heads
+        // (rotated frame): this group's partial
         if (ok && lane >= 24) {
-            float y[8];
-#pragma unroll
-            for (int f = 0; f < 4; f++) {
-                const float x0 = dkr_acc[2 * f], x1 = dkr_acc[2 * f + 1];
-                y[2 * f] = x0 * cq[f].x + x1 * cq[f].y;
-                y[2 * f + 1] = x1 * cq[f].x - x0 * cq[f].y;
-            }
-            reinterpret_cast<uint4 *>(dkr + ((size_t)b * L + key0 + j) * kDR)[lane - 24] = make_uint4(
-                pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+            float4 *dst = reinterpret_cast<float4 *>(dkr_part + (((size_t)hg * gridDim.z + b) * L + key0 + j) * kDR) +
+                          2 * (lane - 24);
+            dst[0] = make_float4(dkr_acc[0], dkr_acc[1], dkr_acc[2], dkr_acc[3]);
+            dst[1] = make_float4(dkr_acc[4], dkr_acc[5], dkr_acc[6], dkr_acc[7]);
         }
     }
     __syncthreads();
@@ -328,10 +327,10 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, in
 
 // -------------------------------------------------------------- padding
 // Padding blocks (keep = 0 or invalid anchor): dq rows and the block's own
-// draft keys' dkc / dv / dkr get zeros.
+// draft keys' dkc / dv get zeros (their dkr is zeroed by the reduction).
 __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, const int32_t *anchors,
                                                  const uint8_t *keep, __nv_bfloat16 *dq, __nv_bfloat16 *dkc,
-                                                 __nv_bfloat16 *dkr, __nv_bfloat16 *dv) {
+                                                 __nv_bfloat16 *dv) {
     const int n = blockIdx.x, b = blockIdx.y;
     const int a = anchors[(size_t)b * N + n];
     if (keep[(size_t)b * N + n] && a >= 0 && a <= S - 2) return;
@@ -346,8 +345,6 @@ __global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, c
         for (int e = threadIdx.x; e < kBlock * kDC / 8; e += blockDim.x) k4[e] = z;
         for (int e = threadIdx.x; e < kBlock * kDV / 8; e += blockDim.x) v4[e] = z;
     }
-    uint4 *r4 = reinterpret_cast<uint4 *>(dkr + ((size_t)b * L + S + kBlock * n) * kDR);
-    for (int e = threadIdx.x; e < kBlock * kDR / 8; e += blockDim.x) r4[e] = z;
 }
 
 struct BwdArgs {
@@ -997,24 +994,39 @@ __global__ void __launch_bounds__(160) k_bwd_dq_out(int n_h, int N, const int32_
 }
 
 // ------------------------------------------------------------ dK^R reduce
-// One warp per (b, context key): sum the head-group partials (rotated frame),
-// rotate back by the key's position, write dkr. (The draft keys' dkr is
-// written by k_bwd_prep and k_bwd_pad.)
-__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int L, int HG, const float2 *tab,
-                                                        const float *part, __nv_bfloat16 *dkr) {
+// One warp per (b, key): sum the head-group partials of the rope-key gradient
+// (rotated frame; context keys from k_bwd_tc, draft keys from k_bwd_prep),
+// rotate back by the key's position, write dkr. Draft keys of padding blocks:
+// 0.
+__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int L, int HG,
+                                                        const int32_t *anchors, const uint8_t *keep,
+                                                        const float2 *tab, const float *part,
+                                                        __nv_bfloat16 *dkr) {
     const size_t wid = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (wid >= (size_t)B * S) return;
-    const int b = (int)(wid / S), key = (int)(wid % S);
-    float x0 = 0.f, x1 = 0.f;
-    for (int g = 0; g < HG; g++) {
-        const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
-        x0 += v.x;
-        x1 += v.y;
+    if (wid >= (size_t)B * L) return;
+    const int b = (int)(wid / L), key = (int)(wid % L);
+    int pos = key;
+    bool live = true;
+    if (key >= S) {
+        const int n = (key - S) / kBlock, i = (key - S) % kBlock;
+        const int a = anchors[(size_t)b * N + n];
+        live = keep[(size_t)b * N + n] && a >= 0 && a <= S - 2;
+        pos = a + i;
     }
-    const float2 cs = tab[(size_t)key * (kDR / 2) + lane];
-    *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) =
-        __floats2bfloat162_rn(x0 * cs.x + x1 * cs.y, x1 * cs.x - x0 * cs.y);
+    float x0 = 0.f, x1 = 0.f;
+    if (live) {
+        for (int g = 0; g < HG; g++) {
+            const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
+            x0 += v.x;
+            x1 += v.y;
+        }
+        const float2 cs = tab[(size_t)pos * (kDR / 2) + lane];
+        const float y0 = x0 * cs.x + x1 * cs.y, y1 = x1 * cs.x - x0 * cs.y;
+        x0 = y0;
+        x1 = y1;
+    }
+    *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
 }
 
 // Row stages of the one-pass kernel.
@@ -1042,15 +1054,15 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     const int HG = bwd_head_groups(p);
     if (p.N > 0) {
         count_launch();
-        k_bwd_prep<<<dim3(p.N, p.B), pr::kThreads, 0, st>>>(
-            p.n_h, p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
+        k_bwd_prep<<<dim3(p.N, HG, p.B), pr::kThreads, 0, st>>>(
+            p.n_h, p.n_h / HG, p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
             (const __nv_bfloat16 *)ws.kr_rot, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)o,
             (const __nv_bfloat16 *)dout, lse, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs,
-            (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dkr,
+            (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, ws.dkr_part,
             (__nv_bfloat16 *)dv, ws.err);
         count_launch();
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
-                                                   (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dkr, (__nv_bfloat16 *)dv);
+                                                   (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
     CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
@@ -1093,10 +1105,10 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         k_bwd_dq_out<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(p.n_h, p.N, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope,
                                                              ws.dqacc, (__nv_bfloat16 *)dq);
     }
-    const size_t warps = (size_t)p.B * p.S;
+    const size_t warps = (size_t)p.B * p.L;
     count_launch();
-    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.L, HG, ws.rope, ws.dkr_part,
-                                                                   (__nv_bfloat16 *)dkr);
+    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
+                                                                   ws.dkr_part, (__nv_bfloat16 *)dkr);
     return cudaGetLastError();
 }
 
