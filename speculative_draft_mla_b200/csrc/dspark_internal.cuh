@@ -43,13 +43,14 @@ struct WsLayout {
     size_t lses;      // float [B, n_h, 5N] LSE * log2(e), anchor-sorted rows
     size_t qs;        // bf16 [B, n_h, 5N, 256] rotated Q, anchor-sorted rows
     size_t dos;       // bf16 [B, n_h, 5N, 256] dO, anchor-sorted rows
-    size_t dkr_part;  // float [HG, B, L, d_r] rope-key gradient per head group
+    size_t dkr_part;  // float [max(HG, HGd), B, L, d_r] rope-key gradient per head group
     size_t dqacc;     // float [B, n_h, 5N, d_c + d_r] dQ accumulator, anchor-sorted rows
     size_t total;
 };
 
 bool bwd_tc_supported(const Prob &p);
-int bwd_head_groups(const Prob &p);
+int bwd_head_groups(const Prob &p);  // head groups of the tensor-core backward (context keys)
+int bwd_prep_groups(const Prob &p);  // head groups of its preparation (draft keys)
 size_t fwd_workspace_size(const dspark_problem *p);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -72,7 +73,8 @@ inline WsLayout ws_layout(const Prob &p) {
     w.qs = off;        off = align256(off + 2 * rows * p.dqk);
     w.dos = off;       off = align256(off + 2 * rows * p.d_v);
     w.dkr_part = off;
-    off = align256(off + (tc ? sizeof(float) * (size_t)bwd_head_groups(p) * p.B * p.L * p.d_r : 0));
+    const int groups = tc ? (bwd_head_groups(p) > bwd_prep_groups(p) ? bwd_head_groups(p) : bwd_prep_groups(p)) : 0;
+    off = align256(off + sizeof(float) * (size_t)groups * p.B * p.L * p.d_r);
     w.dqacc = off;     off = align256(off + sizeof(float) * rows * p.dqk);
     w.total = off;
     return w;

@@ -50,52 +50,59 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
 // The row-wise preparation and the draft-key part of the backward, one CTA
-// per kept block (anchor-sorted index i), head group and batch row, looping
-// over the group's heads. A producer warp stages each head's inputs into shared memory with
-// bulk copies, kPrepStages heads ahead: the block's 5 rows of q, O and dO and
+// per kept block (anchor-sorted index i), group of up to kHeads heads and
+// batch row. A producer warp stages each head's inputs into shared memory with
+// bulk copies (ring of kStages heads): the block's 5 rows of q, O and dO and
 // its 5 draft keys' K^C and V (the rotated rope keys of the draft keys are the
-// same for all heads and are staged once). Compute warp j handles row 5 n + j,
-// lane l dims 8 l .. 8 l + 7. Per head:
-//   - rotated q -> qs, do -> dos (anchor-sorted rows), D = rowsum(dO * O),
-//     LSE * log2(e);
-//   - the block's own 5 draft keys, which no other row sees (page §3):
-//     S = q_rot k_rot^T s and dP = dO V^T over the 5 keys, P = exp(S - LSE),
-//     dS = P (dP - D) s; the rows' draft-key dQ contribution dS K_rot is
-//     stored as the first value of the fp32 dQ accumulator (the context tiles
-//     add theirs later, in stream order), and the draft keys' gradients
-//     dK = dS^T q_rot, dV = P^T dO are complete here: warp j then stands for
-//     draft key j, writes its dK^C and dV, and sums the rope part of dK over
-//     the group's heads in registers; after the last head that sum goes to the
-//     group's partial rope-key gradient (rotated frame), summed over the
-//     groups and rotated back by k_bwd_dkr_reduce.
+// same for all heads and are staged once). Compute warp w takes the heads
+// w, w + kWarps, ... of the group, one whole block per head, lane l owning
+// dims 8 l .. 8 l + 7 of every row (rows 5 n + r, r = 0..4) and key:
+//   - rotated q -> qs (and back into the stage), dO -> dos (anchor-sorted rows);
+//   - the 55 partial sums of S = q_rot k_rot^T, dP = dO V^T over the block's
+//     own 5 draft keys (which no other row sees, page §3) and D = rowsum(dO * O),
+//     reduced across the warp in one butterfly that leaves sums 2 l, 2 l + 1 in
+//     lane l; then P = exp(S s - LSE), dS = P (dP - D) s for the 25 pairs;
+//   - the rows' draft-key dQ contribution dS K_rot, stored as the first value
+//     of the fp32 dQ accumulator (the context tiles add theirs later, in
+//     stream order), D and LSE * log2(e);
+//   - the draft keys' gradients, complete here: dK^C = dS^T q_rot and
+//     dV = P^T dO written, the rope part of dK summed over the group's heads
+//     in shared memory and written, after the last head, as the group's partial
+//     rope-key gradient (rotated frame; k_bwd_dkr_reduce sums the groups).
 // q_rot is rounded to bf16 as the tensor-core kernels see it (the forward's
 // LSE was formed from the same rounded operands). Rows past the kept blocks
 // are zeroed so that tiles overhanging them multiply finite values. Every
 // wait is bounded; on time-out the CTA stops issuing, waits (bounded) for its
-// copies in flight and sets the timeout bit of the error word.
+// copies in flight and sets the timeout bit of the error word; the compute
+// warps meet at one barrier only, after their loops.
 namespace pr {
-// Barrier 1 of the five compute warps with an OR over their predicates: every
-// warp gets the same answer from one barrier instance.
-__device__ __forceinline__ bool compute_warps_or(bool x) {
+// Barrier 1 of the compute warps with an OR over their predicates: every warp
+// gets the same answer from one barrier instance.
+__device__ __forceinline__ bool compute_warps_or(bool x, int nthreads) {
     uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 160, p;\n\t"
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}\n"
         : "=r"(r)
-        : "r"((uint32_t)x)
+        : "r"((uint32_t)x), "r"(nthreads)
         : "memory");
     return r != 0;
 }
-constexpr int kStages = 3;
+constexpr int kWarps = 4;                  // compute warps
+constexpr int kHeads = 16;                 // heads per CTA at most
+constexpr int kStages = 6;                 // staged heads
 constexpr int kRowsB = kBlock * kDQK * 2;  // 5 rows of 256 bf16 (q, O, dO, V)
 constexpr int kKcB = kBlock * kDC * 2;     // 5 rows of K^C
 constexpr int oQ = 0, oO = kRowsB, oDO = 2 * kRowsB, oV = 3 * kRowsB, oKc = 4 * kRowsB;
 constexpr int kStageB = 4 * kRowsB + kKcB;  // 12160
-constexpr int kThreads = 6 * 32;           // 5 compute warps + the producer
+constexpr int kThreads = (kWarps + 1) * 32;
+constexpr int kSmem = kStages * kStageB + 128;  // dynamic: the stages (+ alignment)
 }  // namespace pr
 
-__global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int hpg, int S, int N, int L, float scale,
-                                                  float scale_log2,
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, int N, int L, float scale, float scale_log2,
                                                   const __nv_bfloat16 *__restrict__ q,
                                                   const __nv_bfloat16 *__restrict__ kc,
                                                   const __nv_bfloat16 *__restrict__ krr,
@@ -111,20 +118,22 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int hpg, 
                                                   __nv_bfloat16 *__restrict__ dkc, float *__restrict__ dkr_part,
                                                   __nv_bfloat16 *__restrict__ dv, uint32_t *err) {
     using namespace pr;
-    __shared__ __align__(128) uint8_t st[kStages][kStageB];
-    __shared__ __align__(16) uint4 s_kr[kBlock][8];                // rotated rope keys of the draft keys
-    __shared__ __align__(16) uint4 s_q[kBlock][32], s_do[kBlock][32];  // the head's rotated q and dO rows
-    __shared__ float s_p[kBlock][kBlock], s_ds[kBlock][kBlock];  // [row][key]
+    extern __shared__ uint8_t prep_smem[];
+    uint8_t *st0 = prep_smem + ((128u - (tc::smem_u32(prep_smem) & 127u)) & 127u);
+    __shared__ __align__(16) uint4 s_kr[kBlock][8];         // rotated rope keys of the draft keys
+    __shared__ __align__(16) float s_tot[kWarps][64];        // the warp's reduced sums
+    __shared__ float s_p[kWarps][kBlock * kBlock], s_ds[kWarps][kBlock * kBlock];  // [row * 5 + key]
+    __shared__ __align__(16) float s_dkr[kWarps][kBlock][kDR];  // rope part of dK, summed over the warp's heads
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages], krbar;
     __shared__ int abort_s;
     const int i = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-    const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
-    const int h0 = hg * hpg;
+    const int h0 = hg * kHeads, nhh = min(kHeads, n_h - h0);  // the group's heads
     if (i >= cnt[b]) {
-        if (j < kBlock)
-            for (int h = h0; h < h0 + hpg; h++) {
-                const size_t srow = ((size_t)b * n_h + h) * R + kBlock * i + j;
+        for (int hh = w; hh < nhh; hh += kWarps + 1)
+            for (int r = 0; r < kBlock; r++) {
+                const size_t srow = ((size_t)b * n_h + h0 + hh) * R + kBlock * i + r;
                 reinterpret_cast<uint4 *>(qs + srow * kDQK)[lane] = make_uint4(0, 0, 0, 0);
                 reinterpret_cast<uint4 *>(dos + srow * kDV)[lane] = make_uint4(0, 0, 0, 0);
                 if (lane == 0) {
@@ -139,33 +148,34 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int hpg, 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; s++) {
             tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&empty[s], kBlock);
+            tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(&krbar, 1);
         abort_s = 0;
         tc::fence_barrier_init();
     }
+    for (int e = threadIdx.x; e < kWarps * kBlock * kDR; e += blockDim.x) (&s_dkr[0][0][0])[e] = 0.f;
     __syncthreads();
     volatile int *abort_flag = &abort_s;
-    if (j == kBlock) {
+    if (w == kWarps) {
         // ---------------------------------------------------- producer
         int issued = 0;
         if (lane == 0) {
             tc::mbar_arrive_expect_tx(&krbar, kBlock * kDR * 2);
             tc::bulk_load(&s_kr[0][0], krr + ((size_t)b * L + key0) * kDR, kBlock * kDR * 2, &krbar);
-            for (int h = 0; h < hpg; h++) {
-                const int s = h % kStages;
-                if (h >= kStages && !tc::mbar_wait(&empty[s], ((h / kStages) - 1) & 1, abort_flag)) break;
-                const size_t bh = (size_t)b * n_h + h0 + h;
+            for (int hh = 0; hh < nhh; hh++) {
+                const int s = hh % kStages;
+                if (hh >= kStages && !tc::mbar_wait(&empty[s], ((hh / kStages) - 1) & 1, abort_flag)) break;
+                const size_t bh = (size_t)b * n_h + h0 + hh;
                 const size_t orow = (bh * R + kBlock * n) * kDQK, krow = bh * L + key0;
-                uint8_t *d = st[s];
+                uint8_t *d = st0 + s * kStageB;
                 tc::mbar_arrive_expect_tx(&full[s], kStageB);
                 tc::bulk_load(d + oQ, q + orow, kRowsB, &full[s]);
                 tc::bulk_load(d + oO, o + orow, kRowsB, &full[s]);
                 tc::bulk_load(d + oDO, dout + orow, kRowsB, &full[s]);
                 tc::bulk_load(d + oV, v + krow * kDV, kRowsB, &full[s]);
                 tc::bulk_load(d + oKc, kc + krow * kDC, kKcB, &full[s]);
-                issued = h + 1;
+                issued = hh + 1;
             }
         }
         // every copy issued has landed before the CTA may end (each wait bounded)
@@ -173,154 +183,188 @@ __global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int hpg, 
         if (lane == 0) {
             volatile int never = 0;
             tc::mbar_wait(&krbar, 0, &never);
-            for (int h = max(0, issued - kStages); h < issued; h++)
-                tc::mbar_wait(&full[h % kStages], (h / kStages) & 1, &never);
+            for (int hh = max(0, issued - kStages); hh < issued; hh++)
+                tc::mbar_wait(&full[hh % kStages], (hh / kStages) & 1, &never);
         }
-    } else {
-        // ------------------------------------------------ compute warps
-        // RoPE (cos, sin) of this lane's 4 frequencies at the row's position
-        // a + j (query rotation) and at the key position a + j (warp j as a key)
-        float2 cq[4] = {};
-        if (lane >= 24)
+        __syncthreads();
+        if (threadIdx.x == kWarps * 32 && abort_s) atomicOr(err, kErrTimeout);
+        return;
+    }
+    // ---------------------------------------------------- compute warps
+    // RoPE (cos, sin) of this lane's 4 frequencies (lanes 24-31) at position a + r
+    const float2 *cs0 = tab + (size_t)a * (kDR / 2) + (lane >= 24 ? (lane - 24) * 4 : 0);
+    bool ok = tc::warp_all(tc::mbar_wait(&krbar, 0, abort_flag));
+    // LSE of the warp's next head (lanes 0-4: rows 0-4), read a head ahead
+    float lse_n = (ok && w < nhh && lane < kBlock) ? lse[((size_t)b * n_h + h0 + w) * R + kBlock * n + lane] : 0.f;
+    for (int hh = w; hh < nhh && ok; hh += kWarps) {
+        const int s = hh % kStages;
+        const size_t bh = (size_t)b * n_h + h0 + hh;
+        const float lse_r = lse_n;
+        if (hh + kWarps < nhh && lane < kBlock) lse_n = lse[(bh + kWarps) * R + kBlock * n + lane];
+        ok = tc::warp_all(tc::mbar_wait(&full[s], (hh / kStages) & 1, abort_flag));
+        if (!ok) break;
+        uint8_t *d = st0 + s * kStageB;
+        // the 55 partial sums: S[r][k] at 5 r + k, dP[r][k] at 25 + 5 r + k, D[r] at 50 + r
+        float acc[64];
 #pragma unroll
-            for (int f = 0; f < 4; f++) cq[f] = __ldg(tab + (size_t)(a + j) * (kDR / 2) + (lane - 24) * 4 + f);
-        float dkr_acc[8] = {};  // warp j = draft key j: rope part of dK, summed over heads (lanes 24-31)
-        // The compute warps leave together: each bounded wait is followed by a
-        // barrier of the five warps that ORs their "give up" predicates, so no
-        // warp is left waiting at a barrier the others have abandoned.
-        bool ok = !compute_warps_or(!tc::mbar_wait(&krbar, 0, abort_flag) || *abort_flag);
-        float lse_n = ok ? lse[((size_t)b * n_h + h0) * R + kBlock * n + j] : 0.f;
-        for (int h = 0; h < hpg && ok; h++) {
-            const int s = h % kStages;
-            const size_t bh = (size_t)b * n_h + h0 + h;
-            const size_t srow = bh * R + kBlock * i + j;
-            const float lse_r = lse_n;
-            if (h + 1 < hpg) lse_n = lse[(bh + 1) * R + kBlock * n + j];  // the next head's, ahead of need
-            if (compute_warps_or(!tc::mbar_wait(&full[s], (h / kStages) & 1, abort_flag) || *abort_flag)) {
-                ok = false;
-                break;
-            }
-            const uint8_t *d = st[s];
-            uint4 qv = reinterpret_cast<const uint4 *>(d + oQ + j * kDQK * 2)[lane];
+        for (int e = 0; e < 64; e++) acc[e] = 0.f;
+#pragma unroll
+        for (int r = 0; r < kBlock; r++) {
+            uint4 qv = reinterpret_cast<const uint4 *>(d + oQ + r * kDQK * 2)[lane];
             if (lane >= 24) {
-                uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+                uint32_t wq[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
                 for (int f = 0; f < 4; f++) {
-                    const float x0 = __uint_as_float(w[f] << 16), x1 = __uint_as_float(w[f] & 0xffff0000u);
-                    w[f] = pack_bf16x2(x0 * cq[f].x - x1 * cq[f].y, x0 * cq[f].y + x1 * cq[f].x);
+                    const float2 c = __ldg(cs0 + r * (kDR / 2) + f);
+                    const float x0 = bf_lo(wq[f]), x1 = bf_hi(wq[f]);
+                    wq[f] = pack_bf16x2(x0 * c.x - x1 * c.y, x0 * c.y + x1 * c.x);
                 }
-                qv = make_uint4(w[0], w[1], w[2], w[3]);
+                qv = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                reinterpret_cast<uint4 *>(d + oQ + r * kDQK * 2)[lane] = qv;  // rotated, for dK below
             }
-            const uint4 dv4 = reinterpret_cast<const uint4 *>(d + oDO + j * kDV * 2)[lane];
-            const uint4 ov4 = reinterpret_cast<const uint4 *>(d + oO + j * kDV * 2)[lane];
+            const uint4 dv4 = reinterpret_cast<const uint4 *>(d + oDO + r * kDV * 2)[lane];
+            const uint4 ov4 = reinterpret_cast<const uint4 *>(d + oO + r * kDV * 2)[lane];
+            const size_t srow = bh * R + kBlock * i + r;
             reinterpret_cast<uint4 *>(qs + srow * kDQK)[lane] = qv;
             reinterpret_cast<uint4 *>(dos + srow * kDV)[lane] = dv4;
-            s_q[j][lane] = qv;
-            s_do[j][lane] = dv4;
-            float sc[kBlock], dp[kBlock], dd = 0.f;
-            {
-                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-                const uint32_t ow[4] = {ov4.x, ov4.y, ov4.z, ov4.w};
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+            const uint32_t ow[4] = {ov4.x, ov4.y, ov4.z, ov4.w};
 #pragma unroll
-                for (int f = 0; f < 4; f++) {
-                    dd = fmaf(__uint_as_float(dw[f] << 16), __uint_as_float(ow[f] << 16), dd);
-                    dd = fmaf(__uint_as_float(dw[f] & 0xffff0000u), __uint_as_float(ow[f] & 0xffff0000u), dd);
-                }
-#pragma unroll
-                for (int k = 0; k < kBlock; k++) {
-                    const uint4 kq = lane < 24 ? reinterpret_cast<const uint4 *>(d + oKc + k * kDC * 2)[lane]
-                                               : s_kr[k][lane - 24];
-                    const uint4 vv = reinterpret_cast<const uint4 *>(d + oV + k * kDV * 2)[lane];
-                    const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
-                    float s1 = 0.f, p1 = 0.f;
-#pragma unroll
-                    for (int f = 0; f < 4; f++) {
-                        s1 = fmaf(__uint_as_float(qw[f] << 16), __uint_as_float(kw[f] << 16), s1);
-                        s1 = fmaf(__uint_as_float(qw[f] & 0xffff0000u), __uint_as_float(kw[f] & 0xffff0000u), s1);
-                        p1 = fmaf(__uint_as_float(dw[f] << 16), __uint_as_float(vw[f] << 16), p1);
-                        p1 = fmaf(__uint_as_float(dw[f] & 0xffff0000u), __uint_as_float(vw[f] & 0xffff0000u), p1);
-                    }
-                    sc[k] = s1;
-                    dp[k] = p1;
-                }
+            for (int f = 0; f < 4; f++) {
+                acc[50 + r] = fmaf(bf_lo(dw[f]), bf_lo(ow[f]), acc[50 + r]);
+                acc[50 + r] = fmaf(bf_hi(dw[f]), bf_hi(ow[f]), acc[50 + r]);
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                dd += __shfl_xor_sync(0xffffffffu, dd, off);
-#pragma unroll
-                for (int k = 0; k < kBlock; k++) {
-                    sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], off);
-                    dp[k] += __shfl_xor_sync(0xffffffffu, dp[k], off);
-                }
-            }
-            const float lse2 = lse_r * kLog2e;
-            if (lane == 0) {
-                ds_[srow] = dd;
-                lses[srow] = lse2;
-            }
-            // the row's draft-key dQ contribution, dims 8 lane .. + 7
-            float dqv[8] = {};
 #pragma unroll
             for (int k = 0; k < kBlock; k++) {
-                const float pk = exp2f(fmaf(sc[k], scale_log2, -lse2));
-                const float dsk = pk * (dp[k] - dd) * scale;
-                if (lane == 0) {
-                    s_p[j][k] = pk;
-                    s_ds[j][k] = dsk;
+                const uint4 kq = lane < 24 ? reinterpret_cast<const uint4 *>(d + oKc + k * kDC * 2)[lane] : s_kr[k][lane - 24];
+                const uint4 vv = reinterpret_cast<const uint4 *>(d + oV + k * kDV * 2)[lane];
+                const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                for (int f = 0; f < 4; f++) {
+                    acc[5 * r + k] = fmaf(bf_lo(qw[f]), bf_lo(kw[f]), acc[5 * r + k]);
+                    acc[5 * r + k] = fmaf(bf_hi(qw[f]), bf_hi(kw[f]), acc[5 * r + k]);
+                    acc[25 + 5 * r + k] = fmaf(bf_lo(dw[f]), bf_lo(vw[f]), acc[25 + 5 * r + k]);
+                    acc[25 + 5 * r + k] = fmaf(bf_hi(dw[f]), bf_hi(vw[f]), acc[25 + 5 * r + k]);
                 }
+            }
+        }
+        // butterfly reduce-scatter over the warp: at each step keep one half of
+        // the values (the upper one if this lane's bit is set) and add the
+        // partner's; lane l ends with the sums of values 2 l and 2 l + 1
+#pragma unroll
+        for (int step = 0; step < 5; step++) {
+            const int bit = 16 >> step, half = 32 >> step;
+            const bool up = lane & bit;
+#pragma unroll
+            for (int e = 0; e < half; e++) {
+                const float send = up ? acc[e] : acc[e + half];
+                const float keep = up ? acc[e + half] : acc[e];
+                acc[e] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+            }
+        }
+        s_tot[w][2 * lane] = acc[0];
+        s_tot[w][2 * lane + 1] = acc[1];
+        __syncwarp();
+        if (lane < kBlock * kBlock) {
+            const int r = lane / kBlock;
+            const float lse2 = __shfl_sync(0x1ffffffu, lse_r, r) * kLog2e;
+            const float pr = exp2f(fmaf(s_tot[w][lane], scale_log2, -lse2));
+            s_p[w][lane] = pr;
+            s_ds[w][lane] = pr * (s_tot[w][25 + lane] - s_tot[w][50 + r]) * scale;
+        }
+        if (lane < kBlock) {
+            const size_t srow = bh * R + kBlock * i + lane;
+            ds_[srow] = s_tot[w][50 + lane];
+            lses[srow] = lse_r * kLog2e;
+        }
+        __syncwarp();
+        // the rows' draft-key dQ contribution: dq[r] = sum_k dS[r][k] k_rot[k]
+        {
+            float kf[kBlock][8];
+#pragma unroll
+            for (int k = 0; k < kBlock; k++) {
                 const uint4 kq = lane < 24 ? reinterpret_cast<const uint4 *>(d + oKc + k * kDC * 2)[lane] : s_kr[k][lane - 24];
                 const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w};
 #pragma unroll
                 for (int f = 0; f < 4; f++) {
-                    dqv[2 * f] = fmaf(dsk, __uint_as_float(kw[f] << 16), dqv[2 * f]);
-                    dqv[2 * f + 1] = fmaf(dsk, __uint_as_float(kw[f] & 0xffff0000u), dqv[2 * f + 1]);
+                    kf[k][2 * f] = bf_lo(kw[f]);
+                    kf[k][2 * f + 1] = bf_hi(kw[f]);
                 }
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
-            float4 *acc = reinterpret_cast<float4 *>(dqacc + srow * kDQK) + 2 * lane;
-            acc[0] = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
-            acc[1] = make_float4(dqv[4], dqv[5], dqv[6], dqv[7]);
-            asm volatile("bar.sync 1, 160;" ::: "memory");  // the compute warps' rows and weights are staged
-            // warp j now stands for draft key j: dK = sum_r dS[r][j] q_rot[r],
-            // dV = sum_r P[r][j] dO[r]
-            float dk[8] = {}, dvv[8] = {};
 #pragma unroll
             for (int r = 0; r < kBlock; r++) {
-                const float pr = s_p[r][j], dsr = s_ds[r][j];
-                const uint4 qa = s_q[r][lane], da = s_do[r][lane];
-                const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, dw[4] = {da.x, da.y, da.z, da.w};
+                float dq8[8] = {};
+#pragma unroll
+                for (int k = 0; k < kBlock; k++) {
+                    const float dsk = s_ds[w][kBlock * r + k];
+#pragma unroll
+                    for (int e = 0; e < 8; e++) dq8[e] = fmaf(dsk, kf[k][e], dq8[e]);
+                }
+                float4 *acc4 = reinterpret_cast<float4 *>(dqacc + (bh * R + kBlock * i + r) * kDQK) + 2 * lane;
+                acc4[0] = make_float4(dq8[0], dq8[1], dq8[2], dq8[3]);
+                acc4[1] = make_float4(dq8[4], dq8[5], dq8[6], dq8[7]);
+            }
+        }
+        // the draft keys' gradients, one pass each: dK[k] = sum_r dS[r][k] q_rot[r],
+        // then dV[k] = sum_r P[r][k] dO[r]
+#pragma unroll
+        for (int pass = 0; pass < 2; pass++) {
+            const int off = pass == 0 ? oQ : oDO;
+            const float *wgt = pass == 0 ? s_ds[w] : s_p[w];
+            float g[kBlock][8] = {};
+#pragma unroll
+            for (int r = 0; r < kBlock; r++) {
+                const uint4 x4 = reinterpret_cast<const uint4 *>(d + off + r * kDQK * 2)[lane];
+                const uint32_t xw[4] = {x4.x, x4.y, x4.z, x4.w};
+                float xf[8];
 #pragma unroll
                 for (int f = 0; f < 4; f++) {
-                    dk[2 * f] = fmaf(dsr, __uint_as_float(qw[f] << 16), dk[2 * f]);
-                    dk[2 * f + 1] = fmaf(dsr, __uint_as_float(qw[f] & 0xffff0000u), dk[2 * f + 1]);
-                    dvv[2 * f] = fmaf(pr, __uint_as_float(dw[f] << 16), dvv[2 * f]);
-                    dvv[2 * f + 1] = fmaf(pr, __uint_as_float(dw[f] & 0xffff0000u), dvv[2 * f + 1]);
+                    xf[2 * f] = bf_lo(xw[f]);
+                    xf[2 * f + 1] = bf_hi(xw[f]);
+                }
+#pragma unroll
+                for (int k = 0; k < kBlock; k++) {
+                    const float wk = wgt[kBlock * r + k];
+#pragma unroll
+                    for (int e = 0; e < 8; e++) g[k][e] = fmaf(wk, xf[e], g[k][e]);
                 }
             }
-            asm volatile("bar.sync 1, 160;" ::: "memory");  // read before the next head overwrites them
-            const size_t krow = bh * L + key0 + j;
-            reinterpret_cast<uint4 *>(dv + krow * kDV)[lane] =
-                make_uint4(pack_bf16x2(dvv[0], dvv[1]), pack_bf16x2(dvv[2], dvv[3]), pack_bf16x2(dvv[4], dvv[5]),
-                           pack_bf16x2(dvv[6], dvv[7]));
-            if (lane < 24) {
-                reinterpret_cast<uint4 *>(dkc + krow * kDC)[lane] =
-                    make_uint4(pack_bf16x2(dk[0], dk[1]), pack_bf16x2(dk[2], dk[3]), pack_bf16x2(dk[4], dk[5]),
-                               pack_bf16x2(dk[6], dk[7]));
-            } else {
+            if (pass == 1) {
+                // the stage is no longer read (and its rotated q, written here,
+                // precedes the bulk copy that will refill it)
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&empty[s]);
+            }
 #pragma unroll
-                for (int e = 0; e < 8; e++) dkr_acc[e] += dk[e];
+            for (int k = 0; k < kBlock; k++) {
+                const size_t krow = bh * L + key0 + k;
+                const uint4 pk = make_uint4(pack_bf16x2(g[k][0], g[k][1]), pack_bf16x2(g[k][2], g[k][3]),
+                                            pack_bf16x2(g[k][4], g[k][5]), pack_bf16x2(g[k][6], g[k][7]));
+                if (pass == 1) {
+                    reinterpret_cast<uint4 *>(dv + krow * kDV)[lane] = pk;
+                } else if (lane < 24) {
+                    reinterpret_cast<uint4 *>(dkc + krow * kDC)[lane] = pk;
+                } else {
+                    float4 *acc4 = reinterpret_cast<float4 *>(&s_dkr[w][k][8 * (lane - 24)]);
+                    const float4 x = acc4[0], y = acc4[1];
+                    acc4[0] = make_float4(x.x + g[k][0], x.y + g[k][1], x.z + g[k][2], x.w + g[k][3]);
+                    acc4[1] = make_float4(y.x + g[k][4], y.y + g[k][5], y.z + g[k][6], y.w + g[k][7]);
+                }
             }
         }
-        // the draft key's rope gradient summed over the group's heads
-        // (rotated frame): this group's partial
-        if (ok && lane >= 24) {
-            float4 *dst = reinterpret_cast<float4 *>(dkr_part + (((size_t)hg * gridDim.z + b) * L + key0 + j) * kDR) +
-                          2 * (lane - 24);
-            dst[0] = make_float4(dkr_acc[0], dkr_acc[1], dkr_acc[2], dkr_acc[3]);
-            dst[1] = make_float4(dkr_acc[4], dkr_acc[5], dkr_acc[6], dkr_acc[7]);
-        }
     }
+    // the compute warps meet once; unless one gave up, the draft keys' rope
+    // gradient summed over the group's heads is this group's partial
+    const bool give_up = compute_warps_or(!ok || *abort_flag, kWarps * 32);
+    if (!give_up)
+        for (int e = threadIdx.x; e < kBlock * kDR; e += kWarps * 32) {
+            const int k = e / kDR, c = e % kDR;
+            float x = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < kWarps; ww++) x += s_dkr[ww][k][c];
+            dkr_part[(((size_t)hg * gridDim.z + b) * L + key0 + k) * kDR + c] = x;
+        }
     __syncthreads();
     if (threadIdx.x == 0 && abort_s) atomicOr(err, kErrTimeout);
 }
@@ -995,10 +1039,11 @@ __global__ void __launch_bounds__(160) k_bwd_dq_out(int n_h, int N, const int32_
 
 // ------------------------------------------------------------ dK^R reduce
 // One warp per (b, key): sum the head-group partials of the rope-key gradient
-// (rotated frame; context keys from k_bwd_tc, draft keys from k_bwd_prep),
+// (rotated frame; context keys from k_bwd_tc's HG groups, draft keys from
+// k_bwd_prep's HGd groups),
 // rotate back by the key's position, write dkr. Draft keys of padding blocks:
 // 0.
-__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int L, int HG,
+__global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int L, int HG, int HGd,
                                                         const int32_t *anchors, const uint8_t *keep,
                                                         const float2 *tab, const float *part,
                                                         __nv_bfloat16 *dkr) {
@@ -1016,7 +1061,8 @@ __global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int
     }
     float x0 = 0.f, x1 = 0.f;
     if (live) {
-        for (int g = 0; g < HG; g++) {
+        const int groups = key < S ? HG : HGd;  // context keys: the tensor-core kernel's groups
+        for (int g = 0; g < groups; g++) {
             const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
             x0 += v.x;
             x1 += v.y;
@@ -1039,6 +1085,8 @@ bool bwd_tc_supported(const Prob &p) {
            (long long)p.B * p.n_h * p.L < (1ll << 31) && (long long)p.B * p.n_h * p.R < (1ll << 31);
 }
 
+int bwd_prep_groups(const Prob &p) { return (p.n_h + pr::kHeads - 1) / pr::kHeads; }
+
 int bwd_head_groups(const Prob &p) {
     const long long items = (long long)((p.S + bw::kMK - 1) / bw::kMK) * p.B;
     // aim for about six waves on 148 SMs (shorter CTAs, smaller tail)
@@ -1054,8 +1102,10 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     const int HG = bwd_head_groups(p);
     if (p.N > 0) {
         count_launch();
-        k_bwd_prep<<<dim3(p.N, HG, p.B), pr::kThreads, 0, st>>>(
-            p.n_h, p.n_h / HG, p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
+        cudaError_t ep = cudaFuncSetAttribute(k_bwd_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, pr::kSmem);
+        if (ep != cudaSuccess) return ep;
+        k_bwd_prep<<<dim3(p.N, bwd_prep_groups(p), p.B), pr::kThreads, pr::kSmem, st>>>(
+            p.n_h, p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
             (const __nv_bfloat16 *)ws.kr_rot, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)o,
             (const __nv_bfloat16 *)dout, lse, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs,
             (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, ws.dkr_part,
@@ -1107,8 +1157,8 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     }
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
-    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, anchors, keep, ws.rope,
-                                                                   ws.dkr_part, (__nv_bfloat16 *)dkr);
+    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, bwd_prep_groups(p), anchors,
+                                                                   keep, ws.rope, ws.dkr_part, (__nv_bfloat16 *)dkr);
     return cudaGetLastError();
 }
 
