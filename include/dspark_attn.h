@@ -167,6 +167,21 @@ DSPARK_API const char *dspark_status_string(dspark_status s);
  * caller count the device work of a timed region. */
 DSPARK_API uint64_t dspark_launch_counter(void);
 
+/* Time after which a bounded wait inside a kernel gives up (ns; default and
+ * maximum 2 s). Every pipeline wait of the tensor-core kernels (a consumer
+ * waiting for a copy or an MMA, a producer waiting for a free stage, the MMA
+ * issuer waiting for any operand) gives up after this long, raises its CTA's
+ * abort flag, and the call then reports DSPARK_ERR_DEVICE through
+ * dspark_get_error; the outputs of such a call are unspecified. The waits that
+ * let copies and MMAs already issued complete before a CTA exits keep the 2 s
+ * limit whatever is set here. Process-wide, read by each fwd / bwd call when
+ * it launches. ns = 0, or a value above 2 s, sets the default. Returns the
+ * limit in effect before the call. A limit far below the kernels' own
+ * latencies makes the waits run out on purpose, so the time-out path (error
+ * report, copies drained, TMEM released, context usable afterwards) can be
+ * exercised without a stalled device. */
+DSPARK_API uint64_t dspark_set_wait_limit_ns(uint64_t ns);
+
 /* Host helper, page §2 "anchor sampling": for each batch row, the candidates
  * are A in [0, S-2] with loss_mask[A] = loss_mask[A+1] = 1, where
  * loss_mask[S-1] is read as 0 (appendix A: the last position is neither an

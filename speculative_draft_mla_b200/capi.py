@@ -18,7 +18,8 @@ FLAG_REUSE_DESCRIPTOR = 1
 STATUS = {0: "OK", 1: "ERR_NULL", 2: "ERR_SHAPE", 3: "ERR_DTYPE", 4: "ERR_ANCHOR", 5: "ERR_WORKSPACE",
           6: "ERR_CUDA", 7: "ERR_DEVICE", 8: "ERR_ALIGN", 9: "ERR_UNSUPPORTED"}
 EXPORTS = ("dspark_workspace_size", "dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd",
-           "dspark_get_error", "dspark_status_string", "dspark_sample_anchors", "dspark_launch_counter")
+           "dspark_get_error", "dspark_status_string", "dspark_sample_anchors", "dspark_launch_counter",
+           "dspark_set_wait_limit_ns")
 
 
 class Problem(ctypes.Structure):
@@ -61,6 +62,8 @@ def load():
     lib.dspark_attn_fwd_noalloc.restype = ctypes.c_int
     lib.dspark_launch_counter.argtypes = []
     lib.dspark_launch_counter.restype = ctypes.c_uint64
+    lib.dspark_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.dspark_set_wait_limit_ns.restype = ctypes.c_uint64
     for f in ("dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd", "dspark_get_error"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -193,6 +196,12 @@ def get_error(workspace, stream=None):
 def launch_counter():
     """Kernels the library has launched in this process so far."""
     return int(load().dspark_launch_counter())
+
+
+def set_wait_limit_ns(ns):
+    """Limit (ns) of the kernels' pipeline waits for later calls; 0 restores
+    the default (2 s). Returns the previous limit."""
+    return int(load().dspark_set_wait_limit_ns(int(ns)))
 
 
 def sample_anchors(loss_mask, N, seed):

@@ -12,6 +12,7 @@ using namespace dspark;
 
 namespace dspark {
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<uint64_t> g_wait_ns{kWaitTimeoutNs};  // pipeline-wait limit of later launches
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 }  // namespace dspark
 
@@ -44,6 +45,7 @@ bool make_prob(const dspark_problem *pp, Prob *out, dspark_status *why) {
     r.dtype = p.dtype;
     r.scale = (float)(1.0 / std::sqrt((double)r.dqk));
     r.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)r.dqk));
+    r.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     *out = r;
     return true;
 }
@@ -223,6 +225,11 @@ dspark_status dspark_get_error(void *workspace, void *stream) {
 }
 
 uint64_t dspark_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
+
+uint64_t dspark_set_wait_limit_ns(uint64_t ns) {
+    if (ns == 0 || ns > kWaitTimeoutNs) ns = kWaitTimeoutNs;
+    return g_wait_ns.exchange(ns, std::memory_order_relaxed);
+}
 
 const char *dspark_status_string(dspark_status s) {
     switch (s) {

@@ -16,6 +16,8 @@ constexpr int kBlock = 5;  // draft block length (block_size = 5)
 // Device error word bits (workspace offset 0).
 constexpr uint32_t kErrAnchor = 1u;   // kept anchor outside [0, S-2]
 constexpr uint32_t kErrTimeout = 2u;  // a bounded mbarrier wait gave up
+// Default (and largest) time a bounded wait lasts before it gives up, in ns.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 
 struct Prob {
     int B, n_h, S, N, W, d_c, d_r, d_v;
@@ -27,6 +29,7 @@ struct Prob {
     int dtype;
     float scale_log2;  // (d_c + d_r)^(-1/2) * log2(e)
     float scale;       // (d_c + d_r)^(-1/2)
+    uint64_t wait_ns;  // limit of the kernels' pipeline waits (ns)
 };
 
 // Workspace layout (byte offsets, each 256-aligned).

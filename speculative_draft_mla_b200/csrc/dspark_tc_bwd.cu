@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, in
                                                   __nv_bfloat16 *__restrict__ dos, float *__restrict__ ds_,
                                                   float *__restrict__ lses, float *__restrict__ dqacc,
                                                   __nv_bfloat16 *__restrict__ dkc, float *__restrict__ dkr_part,
-                                                  __nv_bfloat16 *__restrict__ dv, uint32_t *err) {
+                                                  __nv_bfloat16 *__restrict__ dv, uint32_t *err,
+                                                  uint64_t wlim) {
     using namespace pr;
     extern __shared__ uint8_t prep_smem[];
     uint8_t *st0 = prep_smem + ((128u - (tc::smem_u32(prep_smem) & 127u)) & 127u);
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, in
             tc::bulk_load(&s_kr[0][0], krr + ((size_t)b * L + key0) * kDR, kBlock * kDR * 2, &krbar);
             for (int hh = 0; hh < nhh; hh++) {
                 const int s = hh % kStages;
-                if (hh >= kStages && !tc::mbar_wait(&empty[s], ((hh / kStages) - 1) & 1, abort_flag)) break;
+                if (hh >= kStages && !tc::mbar_wait(&empty[s], ((hh / kStages) - 1) & 1, abort_flag, wlim)) break;
                 const size_t bh = (size_t)b * n_h + h0 + hh;
                 const size_t orow = (bh * R + kBlock * n) * kDQK, krow = bh * L + key0;
                 uint8_t *d = st0 + s * kStageB;
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, in
     // ---------------------------------------------------- compute warps
     // RoPE (cos, sin) of this lane's 4 frequencies (lanes 24-31) at position a + r
     const float2 *cs0 = tab + (size_t)a * (kDR / 2) + (lane >= 24 ? (lane - 24) * 4 : 0);
-    bool ok = tc::warp_all(tc::mbar_wait(&krbar, 0, abort_flag));
+    bool ok = tc::warp_all(tc::mbar_wait(&krbar, 0, abort_flag, wlim));
     // LSE of the warp's next head (lanes 0-4: rows 0-4), read a head ahead
     float lse_n = (ok && w < nhh && lane < kBlock) ? lse[((size_t)b * n_h + h0 + w) * R + kBlock * n + lane] : 0.f;
     for (int hh = w; hh < nhh && ok; hh += kWarps) {
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, in
         const size_t bh = (size_t)b * n_h + h0 + hh;
         const float lse_r = lse_n;
         if (hh + kWarps < nhh && lane < kBlock) lse_n = lse[(bh + kWarps) * R + kBlock * n + lane];
-        ok = tc::warp_all(tc::mbar_wait(&full[s], (hh / kStages) & 1, abort_flag));
+        ok = tc::warp_all(tc::mbar_wait(&full[s], (hh / kStages) & 1, abort_flag, wlim));
         if (!ok) break;
         uint8_t *d = st0 + s * kStageB;
         // the 55 partial sums: S[r][k] at 5 r + k, dP[r][k] at 25 + 5 r + k, D[r] at 50 + r
@@ -402,6 +403,7 @@ struct BwdArgs {
     int HG, hpg;  // head groups, heads per group
     int n_ctx;    // context tiles per batch row
     uint32_t *err;
+    uint64_t wait_ns;  // limit of the pipeline waits (ns)
 };
 
 __device__ __forceinline__ void red_add_v4(float *addr, const uint4 &v) {
@@ -484,6 +486,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
              *dqfree = bars + 13, *kdrain = bars + 14, *accdone = bars + 15, *drain = bars + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint64_t wlim = p.wait_ns;
     // K heads issued, V heads issued, row chunks issued, heads consumed, row chunks consumed
     int *counters = reinterpret_cast<int *>(tmem_slot + 2);
     int *band = counters + 5;  // first sorted row, row count
@@ -588,13 +591,13 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         // that those loads wait on L2 rather than on DRAM.
         for (int hh = 0; hh < H; ++hh) {
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
-            if (hh >= 1 && !warp_all(mbar_wait(vfree, (hh - 1) & 1, abort_flag))) break;
+            if (hh >= 1 && !warp_all(mbar_wait(vfree, (hh - 1) & 1, abort_flag, wlim))) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(vfull, 4 * kSlice);
                 tma_load_3d(sm + L::oV, &tm_v, vfull, 0, (int)(bh * p.L + t0), 0);
                 counters[1] = hh + 1;
             }
-            if (hh >= 1 && !warp_all(mbar_wait(kfree, (hh - 1) & 1, abort_flag))) break;
+            if (hh >= 1 && !warp_all(mbar_wait(kfree, (hh - 1) & 1, abort_flag, wlim))) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(kfull, (hh == 0 ? 4 : 3) * kSlice);
                 if (hh == 0) tma_load_2d(sm + L::oKr, &tm_kr, kfull, 0, (int)((size_t)b * p.L + t0));
@@ -641,7 +644,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                     tma_prefetch_l2_3d(&tm_dos, 0, rn, 0);
                 }
             }
-            if (q >= RS && !warp_all(mbar_wait(&rowfree[s], ((q / RS) - 1) & 1, abort_flag))) break;
+            if (q >= RS && !warp_all(mbar_wait(&rowfree[s], ((q / RS) - 1) & 1, abort_flag, wlim))) break;
             float2 *mLD = reinterpret_cast<float2 *>(sm + L::oMeta + s * kRC * 8);
 #pragma unroll
             for (int jj = 0; jj < kRC / 32; jj++) mLD[32 * jj + lane] = mcur[jj];
@@ -777,7 +780,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
                     const uint64_t now = globaltimer();
                     if (t_idle == 0) t_idle = now;
                     if (*abort_flag) ok = false;
-                    else if (now - t_idle > kWaitTimeoutNs) {
+                    else if (now - t_idle > wlim) {
                         *abort_flag = 1;
                         ok = false;
                     }
@@ -798,7 +801,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks;
-            ok = warp_all(mbar_wait(dqfull, q & 1, abort_flag));
+            ok = warp_all(mbar_wait(dqfull, q & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             const size_t bh = (size_t)b * p.n_h + h0 + hh;
@@ -867,8 +870,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
         bool ok = true;
         for (int q = 0; q < QT && ok; ++q) {
             const int hh = q / nchunks, c = q % nchunks, s = q % RS, bsel = q & 1;
-            ok = warp_all(mbar_wait(&rowfull[s], (q / RS) & 1, abort_flag));  // row data
-            if (ok) ok = warp_all(mbar_wait(&sfull[bsel], (q >> 1) & 1, abort_flag));
+            ok = warp_all(mbar_wait(&rowfull[s], (q / RS) & 1, abort_flag, wlim));  // row data
+            if (ok) ok = warp_all(mbar_wait(&sfull[bsel], (q >> 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             float v[32];
@@ -904,8 +907,8 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             // every key warp has also read its staged rows of the previous
             // head's accumulators (staged in this same buffer)
             uint8_t *pt = sm + L::oPT;
-            if (q >= 1) ok = warp_all(mbar_wait(ptfree, (q - 1) & 1, abort_flag));
-            if (ok && c == 0 && hh >= 1) ok = warp_all(mbar_wait(kdrain, (hh - 1) & 1, abort_flag));
+            if (q >= 1) ok = warp_all(mbar_wait(ptfree, (q - 1) & 1, abort_flag, wlim));
+            if (ok && c == 0 && hh >= 1) ok = warp_all(mbar_wait(kdrain, (hh - 1) & 1, abort_flag, wlim));
             if (!ok) break;
             *reinterpret_cast<uint4 *>(pt + pu0) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
             *reinterpret_cast<uint4 *>(pt + pu1) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
@@ -924,7 +927,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
             // writing 8 rows' 64-byte segments per instruction. dK columns
             // 192..255 (the rope slice) stay in TMEM, summed over heads. The
             // accumulator is then free for the next head.
-            ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag));
+            ok = warp_all(mbar_wait(accdone, hh & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             uint8_t *stage = sm + L::oPT + warp * 2048;
@@ -1109,7 +1112,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
             (const __nv_bfloat16 *)ws.kr_rot, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)o,
             (const __nv_bfloat16 *)dout, lse, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs,
             (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, ws.dkr_part,
-            (__nv_bfloat16 *)dv, ws.err);
+            (__nv_bfloat16 *)dv, ws.err, p.wait_ns);
         count_launch();
         k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
                                                    (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
@@ -1144,6 +1147,7 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.hpg = p.n_h / HG;
     a.n_ctx = (p.S + bw::kMK - 1) / bw::kMK;
     a.err = ws.err;
+    a.wait_ns = p.wait_ns;
     const unsigned grid = (unsigned)((size_t)p.B * HG * a.n_ctx);
     constexpr int smem = bw::Smem<kRS>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<kRS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

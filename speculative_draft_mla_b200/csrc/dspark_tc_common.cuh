@@ -19,9 +19,6 @@
 namespace dspark {
 namespace tc {
 
-// A bounded wait gives up after this long (ns) and raises the CTA's abort flag.
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -70,16 +67,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 // Wait for the completion of the phase with the given parity. Gives up when
-// the CTA's abort flag is raised or after kWaitTimeoutNs (then raises it).
-// Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// the CTA's abort flag is raised or after limit_ns (then raises it). Returns
+// false when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kWaitTimeoutNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 return false;
             }

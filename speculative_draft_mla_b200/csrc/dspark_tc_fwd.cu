@@ -118,6 +118,7 @@ struct FwdArgs {
     uint32_t *err;
     int n_groups;  // groups of kG blocks per batch row (work items per (b, h))
     int n_items;   // n_groups * n_h * B
+    uint64_t wait_ns;  // limit of the pipeline waits (ns)
 };
 
 // A bf16 pair (x0 low, x1 high) of a rope slice rotated by (c, s).
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *xbar = sfull + 12, *lbar = sfull + 20;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + 24);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sfull + 25);
+    const uint64_t wlim = p.wait_ns;
     // [0] K tiles issued, [1] V tiles issued, [2] K tiles consumed by an MMA, [3] V tiles consumed,
     // [4] raw Q loads issued, [5] raw Q loads consumed
     int *counters = reinterpret_cast<int *>(sfull + 28);
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = 0; t < it.T; ++t, ++tt) {
                 const int nst = isk ? kKS : kVS;
                 const int s = tt % nst;
-                if (tt >= nst && !warp_all(mbar_wait(isk ? &kempty[s] : &vempty[s], ((tt / nst) - 1) & 1, abort_flag))) {
+                if (tt >= nst && !warp_all(mbar_wait(isk ? &kempty[s] : &vempty[s], ((tt / nst) - 1) & 1, abort_flag, wlim))) {
                     ok = false;
                     break;
                 }
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // table loads. This runs while the item before is still in flight, so
         // the softmax warps only copy the rows into TMEM at the item switch.
         auto rotate_q = [&](const Item &q_it, int ic) -> bool {
-            if (!warp_all(mbar_wait(qraw, ic & 1, abort_flag))) return false;
+            if (!warp_all(mbar_wait(qraw, ic & 1, abort_flag, wlim))) return false;
             if (lane == 0) counters[5] = ic + 1;
             const int my_a = lane < q_it.gcnt ? q_it.sa[lane] : 0;
             for (int b0 = 0; b0 < q_it.gcnt; b0 += 5) {
@@ -366,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int wn = w + gridDim.x;
         bool hasn = has && next_item(p, wn, nx);
         if (ok && hasn) {  // item 1's raw Q once item 0's is in TMEM
-            ok = warp_all(mbar_wait(stgfree, 0, abort_flag));
+            ok = warp_all(mbar_wait(stgfree, 0, abort_flag, wlim));
             if (ok) {
                 load_q(nx, 1);
                 ok = rotate_q(nx, 1);
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // item ic's O rows: each block's 5 rows (contiguous in global
             // memory) with one bulk copy; the staging area is free again once
             // the copies have read it
-            ok = warp_all(mbar_wait(ostaged, ic & 1, abort_flag));
+            ok = warp_all(mbar_wait(ostaged, ic & 1, abort_flag, wlim));
             if (!ok) break;
             if (lane < it.gcnt)
                 bulk_store(p.o + (it.bh * p.R + (size_t)kBlock * it.sn[lane]) * kDV, sm + oStage + lane * kStageBlockPitch,
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t now = globaltimer();
                     if (t_idle == 0) t_idle = now;
                     if (*abort_flag) ok = false;
-                    else if (now - t_idle > kWaitTimeoutNs) {
+                    else if (now - t_idle > wlim) {
                         *abort_flag = 1;
                         ok = false;
                     }
@@ -519,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // item's blocks are zero.
         auto move_q = [&](const Item &q_it, int ic) {
             const bool live = r < q_it.nrows;
-            ok = warp_all(mbar_wait(qrot, ic & 1, abort_flag));
+            ok = warp_all(mbar_wait(qrot, ic & 1, abort_flag, wlim));
             const bool have = live && ok;
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + oStage + (r / kBlock) * kStageBlockPitch +
                                                                (r % kBlock) * (kDQK * 2) + hf * 256);
@@ -564,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
             for (int t = 0; t < it.T && ok; ++t, ++tg) {
                 const int s = tg & 1;
-                ok = warp_all(mbar_wait(&sfull[s], (tg >> 1) & 1, abort_flag));
+                ok = warp_all(mbar_wait(&sfull[s], (tg >> 1) & 1, abort_flag, wlim));
                 if (!ok) break;
                 tc_fence_after();
                 // every row's keys in a tile form one contiguous column range
@@ -604,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 xm[(s * 2 + hf) * kM + r] = mhalf;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xbar[2 * q4 + s]);
-                ok = warp_all(mbar_wait(&xbar[2 * q4 + s], (tg >> 1) & 1, abort_flag));
+                ok = warp_all(mbar_wait(&xbar[2 * q4 + s], (tg >> 1) & 1, abort_flag, wlim));
                 if (!ok) break;
                 const float mother = xm[(s * 2 + (hf ^ 1)) * kM + r];
                 const float mt = fmaxf(mhalf, mother) * p.scale_log2;
@@ -641,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l = l * alpha + ((psum[0] + psum[1]) + (psum[2] + psum[3]));
                 if (__any_sync(0xffffffffu, resc)) {
                     // (never at an item's first tile: m_used starts at -inf)
-                    ok = warp_all(mbar_wait(&pvdone[(tg - 1) & 1], ((tg - 1) >> 1) & 1, abort_flag));
+                    ok = warp_all(mbar_wait(&pvdone[(tg - 1) & 1], ((tg - 1) >> 1) & 1, abort_flag, wlim));
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll 1
@@ -670,18 +672,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 if (lane == 0) mbar_arrive(qdone);
             }
-            ok = warp_all(mbar_wait(&pvdone[(tg - 1) & 1], ((tg - 1) >> 1) & 1, abort_flag));
+            ok = warp_all(mbar_wait(&pvdone[(tg - 1) & 1], ((tg - 1) >> 1) & 1, abort_flag, wlim));
             if (ok) {
                 // the row sum: both halves' shares, exchanged like the tile max
                 xl[hf * kM + r] = l;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&lbar[q4]);
-                ok = warp_all(mbar_wait(&lbar[q4], ic & 1, abort_flag));
+                ok = warp_all(mbar_wait(&lbar[q4], ic & 1, abort_flag, wlim));
             }
             // the staging area: every warp has read the next item's raw Q rows,
             // and the loader warp's bulk copies have read the previous item's O rows
-            if (ok && hasn) ok = warp_all(mbar_wait(qdone, ic & 1, abort_flag));
-            if (ok && ic >= 1) ok = warp_all(mbar_wait(oread, (ic - 1) & 1, abort_flag));
+            if (ok && hasn) ok = warp_all(mbar_wait(qdone, ic & 1, abort_flag, wlim));
+            if (ok && ic >= 1) ok = warp_all(mbar_wait(oread, (ic - 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             const float ltot = l + xl[(hf ^ 1) * kM + r];
@@ -799,6 +801,7 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.o = (__nv_bfloat16 *)o;
     a.lse = lse;
     a.err = ws.err;
+    a.wait_ns = p.wait_ns;
     a.n_groups = (p.N + kG - 1) / kG;
     a.n_items = a.n_groups * p.n_h * p.B;
     int dev = 0, nsm = 0;

@@ -126,3 +126,15 @@ def test_sampler_uniform(lib):
     expect = trials * N / cand
     chi2 = ((counts[:cand] - expect) ** 2 / expect).sum()
     assert chi2 < 30.0, chi2  # 9 degrees of freedom; p ~ 5e-4 at 30
+
+
+def test_wait_limit_setter(lib):
+    """The pipeline-wait limit is process-wide; 0 and values above the 2 s
+    default restore the default; each call returns the limit it replaced."""
+    default = 2_000_000_000
+    prev = capi.set_wait_limit_ns(0)
+    assert prev == default
+    assert capi.set_wait_limit_ns(1000) == default
+    assert capi.set_wait_limit_ns(5 * default) == 1000
+    assert capi.set_wait_limit_ns(0) == default
+    assert capi.set_wait_limit_ns(0) == default
