@@ -332,6 +332,8 @@ def main():
         if ev is not None:
             ev[0].record(stream)
         capi.build_descriptor(prob, d["anchors"], d["keep"], ws)
+        if ev is not None:
+            ev[3].record(stream)
         capi.attn_fwd(d["q"], d["kc"], d["kr"], d["v"], d["anchors"], d["keep"], wl.S, wl.W,
                       wl.rope_base, workspace=ws, flags=R, out=(o_, lse_))
         if ev is not None:
@@ -347,7 +349,7 @@ def main():
     torch.cuda.synchronize()
 
     # timed region: exactly K steps, events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(device) as clk:
         barrier(world)
@@ -370,6 +372,7 @@ def main():
     ms_max = reduce_max(ms, device, world)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    desc_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in evs)  # the descriptor build, inside fwd_ms
     value = aggregate(wl.rows, world, ms_max)
 
     work = algorithmic_work(wl, host["anchors"], host["keep"])
@@ -384,7 +387,7 @@ def main():
                 "traffic": (measured_traffic(dominant) if wl.name == "s8192_n512_b2" else None),
                 "kernel": "attn_%s call (all its kernels)" % dominant,
                 "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % src if src == "measured" else "fallback",
-                "step_frac": roof_ms / ms_max, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                "step_frac": roof_ms / ms_max, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "desc_ms": desc_ms,
                 "fwd_bytes": work["fwd_bytes"], "bwd_bytes": work["bwd_bytes"],
                 "fwd_flops": work["fwd_flops"], "bwd_flops": work["bwd_flops"]}
 

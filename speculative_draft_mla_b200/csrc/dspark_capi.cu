@@ -172,8 +172,15 @@ dspark_status dspark_attn_fwd(const dspark_problem *pp, const void *q, const voi
     cudaStream_t st = (cudaStream_t)stream;
     const Ws w = ws_view(p, workspace);
     if (!(flags & DSPARK_FLAG_REUSE_DESCRIPTOR)) DSPARK_TRY(build(p, anchors, keep, w, st));
-    DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, w, st));
-    if (fwd_tc_supported(p))
+    const bool tc = fwd_tc_supported(p);
+    // the tensor-core forward leaves padding blocks' rows to this launch: O = 0, LSE = -inf
+    PadRows pad{};
+    pad.t[0] = o;
+    pad.rows[0] = p.R;
+    pad.width[0] = p.d_v;
+    pad.lse = lse;
+    DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, keep, tc ? &pad : nullptr, w, st));
+    if (tc)
         DSPARK_CUDA(launch_fwd_tc(p, q, kc, v, anchors, keep, o, lse, w, st));
     else
         DSPARK_CUDA(launch_fwd_simt(p, q, kc, v, anchors, keep, o, lse, w, st));
@@ -200,8 +207,24 @@ dspark_status dspark_attn_bwd(const dspark_problem *pp, const void *q, const voi
     cudaStream_t st = (cudaStream_t)stream;
     const Ws w = ws_view(p, workspace);
     if (!(flags & DSPARK_FLAG_REUSE_DESCRIPTOR)) DSPARK_TRY(build(p, anchors, keep, w, st));
-    DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, w, st));
-    if (bwd_tc_supported(p))
+    const bool tc = bwd_tc_supported(p);
+    // the tensor-core backward leaves padding blocks' dq rows and their own
+    // draft keys' dK^C and dV to this launch (zeros; their dK^R is zeroed by the
+    // backward's rope-key reduction)
+    PadRows pad{};
+    pad.t[0] = dq;
+    pad.rows[0] = p.R;
+    pad.width[0] = p.dqk;
+    pad.t[1] = dkc;
+    pad.rows[1] = p.L;
+    pad.first[1] = p.S;
+    pad.width[1] = p.d_c;
+    pad.t[2] = dv;
+    pad.rows[2] = p.L;
+    pad.first[2] = p.S;
+    pad.width[2] = p.d_v;
+    DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, keep, tc ? &pad : nullptr, w, st));
+    if (tc)
         DSPARK_CUDA(launch_bwd_tc(p, q, kc, v, anchors, keep, o, lse, do_, dq, dkc, dkr, dv, w, st));
     else
         DSPARK_CUDA(launch_bwd_simt(p, q, kc, v, anchors, keep, o, lse, do_, dq, dkc, dkr, dv, w, st));

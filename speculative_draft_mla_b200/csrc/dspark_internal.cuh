@@ -131,8 +131,23 @@ void count_launch(unsigned n = 1);
 // descriptor: sort kept blocks by anchor, validate anchors, rope table
 cudaError_t launch_build_descriptor(const Prob &p, const int32_t *anchors, const uint8_t *keep, const Ws &ws,
                                     cudaStream_t st);
-// rotated rope keys for all kv positions
-cudaError_t launch_rotate_kr(const Prob &p, const void *kr, const int32_t *anchors, const Ws &ws, cudaStream_t st);
+// Rows of padding blocks (keep = 0 or an invalid anchor, page §3: such a block
+// sees nothing) that the rope-key rotation launch zeroes as well, so that the
+// tensor-core paths need no launch of their own for them. Up to three bf16
+// tensors laid out [B, n_h, rows, width]; block n owns rows first + 5 n ..
+// first + 5 n + 4 of each. Unused entries have t = NULL.
+struct PadRows {
+    void *t[3];
+    int rows[3];   // rows per (b, h)
+    int first[3];  // row of block 0's first position (0 for query rows, S for draft keys)
+    int width[3];  // elements per row, a multiple of 8
+    float *lse;    // [B, n_h, 5N] fp32: -inf for the block's rows (NULL = none)
+};
+
+// rotated rope keys for all kv positions; with pad != NULL, also the padding
+// blocks' rows described by *pad
+cudaError_t launch_rotate_kr(const Prob &p, const void *kr, const int32_t *anchors, const uint8_t *keep,
+                             const PadRows *pad, const Ws &ws, cudaStream_t st);
 
 // SIMT (CUDA-core) forward / backward, any supported dims, fp32 or bf16
 cudaError_t launch_fwd_simt(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,

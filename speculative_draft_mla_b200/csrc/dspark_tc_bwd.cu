@@ -9,7 +9,8 @@
 // on rotated q and k rope slices; the rope parts of dQ and dK are rotated back,
 // and dK^R, shared by every head (§4), is the sum over heads.
 //
-// Launch sequence (one stream):
+// Launch sequence (one stream; the padding blocks' dq rows and draft-key
+// dK^C / dV are zeroed earlier, by the rope-key rotation launch):
 //   1. k_bwd_prep       per kept block and head group: rotated Q and
 //                       dO copied into anchor-sorted row order, D, LSE*log2(e),
 //                       and the whole backward of the block's own 5 draft keys
@@ -17,8 +18,7 @@
 //                       the group's partial dK^R, and the rows' draft-key dQ
 //                       contribution, stored as the first value of the fp32 dQ
 //                       accumulator (anchor-sorted rows).
-//   2. k_bwd_pad        zeros for padding blocks' rows and draft keys.
-//   3. k_bwd_tc         key-major over the context, one CTA per (b, 64-key
+//   2. k_bwd_tc         key-major over the context, one CTA per (b, 64-key
 //                       tile, head group), one pass over K and V: rows of the
 //                       blocks whose windows meet the tile, in chunks of 64.
 //                       S^T = K Q^T and dP^T = V dO^T in TMEM, P^T and dS^T
@@ -29,9 +29,9 @@
 //                       added into the dQ accumulator with vector reductions.
 //                       dK and dV are written once, by the CTA that owns the
 //                       keys (no atomics).
-//   4. k_bwd_dq_out     rotates the rope part of the accumulated dQ back,
+//   3. k_bwd_dq_out     rotates the rope part of the accumulated dQ back,
 //                       rounds to bf16 and writes dq in the caller's row order.
-//   5. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
+//   4. k_bwd_dkr_reduce sums the per-head-group rope-key partials, rotates
 //                       them back and writes dK^R.
 // The blocks whose windows meet a context tile [t0, t0 + 64) are a contiguous
 // run of the anchor-sorted list (t0 < A <= t0 + 63 + W - 1).
@@ -370,28 +370,6 @@ __global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, in
     if (threadIdx.x == 0 && abort_s) atomicOr(err, kErrTimeout);
 }
 
-// -------------------------------------------------------------- padding
-// Padding blocks (keep = 0 or invalid anchor): dq rows and the block's own
-// draft keys' dkc / dv get zeros (their dkr is zeroed by the reduction).
-__global__ void __launch_bounds__(256) k_bwd_pad(int n_h, int S, int N, int L, const int32_t *anchors,
-                                                 const uint8_t *keep, __nv_bfloat16 *dq, __nv_bfloat16 *dkc,
-                                                 __nv_bfloat16 *dv) {
-    const int n = blockIdx.x, b = blockIdx.y;
-    const int a = anchors[(size_t)b * N + n];
-    if (keep[(size_t)b * N + n] && a >= 0 && a <= S - 2) return;
-    const int R = kBlock * N;
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int h = 0; h < n_h; h++) {
-        const size_t bh = (size_t)b * n_h + h;
-        uint4 *q4 = reinterpret_cast<uint4 *>(dq + (bh * R + kBlock * n) * kDQK);
-        uint4 *k4 = reinterpret_cast<uint4 *>(dkc + (bh * L + S + kBlock * n) * kDC);
-        uint4 *v4 = reinterpret_cast<uint4 *>(dv + (bh * L + S + kBlock * n) * kDV);
-        for (int e = threadIdx.x; e < kBlock * kDQK / 8; e += blockDim.x) q4[e] = z;
-        for (int e = threadIdx.x; e < kBlock * kDC / 8; e += blockDim.x) k4[e] = z;
-        for (int e = threadIdx.x; e < kBlock * kDV / 8; e += blockDim.x) v4[e] = z;
-    }
-}
-
 struct BwdArgs {
     int B, n_h, S, N, W, L, R;
     float scale_log2, scale;
@@ -498,7 +476,6 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     const int cnt = p.cnt[b];
     const int t0 = item * kMK;
     const int32_t *sa = p.sorted_a + (size_t)b * p.N;
-    const int32_t *sn = p.sorted_n + (size_t)b * p.N;
     if (threadIdx.x == 0) {
         // blocks with t0 < A <= t0 + kMK - 1 + W - 1
         int lo = 0, hi = cnt;
@@ -1113,9 +1090,6 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
             (const __nv_bfloat16 *)dout, lse, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs,
             (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, ws.dkr_part,
             (__nv_bfloat16 *)dv, ws.err, p.wait_ns);
-        count_launch();
-        k_bwd_pad<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.L, anchors, keep, (__nv_bfloat16 *)dq,
-                                                   (__nv_bfloat16 *)dkc, (__nv_bfloat16 *)dv);
     }
     CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;

@@ -751,21 +751,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kErrTimeout);
 }
 
-// Rows of blocks that are padding (keep = 0) or have an invalid anchor: O = 0,
-// LSE = -inf for every head (page §3: such a block sees nothing).
-__global__ void __launch_bounds__(256) k_fwd_pad_rows(int n_h, int S, int N, int R, const int32_t *anchors,
-                                                      const uint8_t *keep, __nv_bfloat16 *o, float *lse) {
-    const int n = blockIdx.x, b = blockIdx.y;
-    const int a = anchors[(size_t)b * N + n];
-    if (keep[(size_t)b * N + n] && a >= 0 && a <= S - 2) return;
-    for (int h = 0; h < n_h; h++) {
-        const size_t row0 = ((size_t)b * n_h + h) * R + kBlock * n;
-        uint4 *dst = reinterpret_cast<uint4 *>(o + row0 * kDV);
-        for (int e = threadIdx.x; e < kBlock * kDV / 8; e += blockDim.x) dst[e] = make_uint4(0, 0, 0, 0);
-        if (threadIdx.x < kBlock) lse[row0 + threadIdx.x] = -INFINITY;
-    }
-}
-
 }  // namespace
 
 bool fwd_tc_supported(const Prob &p) {
@@ -776,9 +761,8 @@ bool fwd_tc_supported(const Prob &p) {
 
 cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
                           const uint8_t *keep, void *o, float *lse, const Ws &ws, cudaStream_t st) {
+    // (padding blocks' rows are written by the rope-key rotation launch before this one)
     if (p.B == 0 || p.N == 0) return cudaSuccess;
-    count_launch();
-    k_fwd_pad_rows<<<dim3(p.N, p.B), 256, 0, st>>>(p.n_h, p.S, p.N, p.R, anchors, keep, (__nv_bfloat16 *)o, lse);
     CUtensorMap m_kc3, m_kr, m_v3, m_kc38, m_kr8, m_v38;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, kr_rows = (uint64_t)p.B * p.L;
     if (!make_map3_bf16(&m_kc3, kc, kDC, kv_rows, 64) || !make_map_bf16(&m_kr, ws.kr_rot, kDR, kr_rows, 64) ||

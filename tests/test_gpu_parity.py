@@ -81,6 +81,22 @@ def test_large_scores_page_dims(oracle_mod, qscale):
     compare_full(gpu, oracle_full(oracle_mod, c, 400, 128, bwd=False), torch.bfloat16)
 
 
+@pytest.mark.parametrize("qscale", [1.5, 2.0])
+def test_large_scores_backward_page_dims(oracle_mod, qscale):
+    """Where the backward's bf16 bound is claimed to hold beyond N(0, 1)
+    queries: every output, gradients included, at Q x 1.5 and Q x 2 (score
+    spread 1.5-2x the workloads'). An fp64 emulation of the bf16 roundings
+    alone (rope key rounded after rotation, O rounded before D, outputs
+    rounded) stays inside the bound on dK^C here (worst excess -0.018 at x1.5,
+    -0.009 at x2) and leaves it at x3 (+0.003), which is why the test above
+    compares only the forward at x3 and beyond."""
+    c = synth.random_case(45, 1, 400, 30, 128, 2, 192, 64, 256, "bf16")
+    c["q"] = (c["q"].float() * qscale).to(torch.bfloat16)
+    c["anchors"][0, 0] = 0
+    gpu = run_gpu(c, 400, 128)
+    compare_full(gpu, oracle_full(oracle_mod, c, 400, 128), torch.bfloat16)
+
+
 def test_no_blocks():
     """N = 0: nothing to attend; the backward still writes zero key gradients."""
     c = synth.random_case(50, 2, 40, 0, 8, 2, 16, 8, 16, "bf16")
