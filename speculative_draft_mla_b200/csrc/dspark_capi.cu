@@ -179,6 +179,7 @@ dspark_status dspark_attn_fwd(const dspark_problem *pp, const void *q, const voi
     pad.rows[0] = p.R;
     pad.width[0] = p.d_v;
     pad.lse = lse;
+    pad.clear = w.sched;  // the tensor-core forward takes its work items from this counter
     DSPARK_CUDA(launch_rotate_kr(p, kr, anchors, keep, tc ? &pad : nullptr, w, st));
     if (tc)
         DSPARK_CUDA(launch_fwd_tc(p, q, kc, v, anchors, keep, o, lse, w, st));

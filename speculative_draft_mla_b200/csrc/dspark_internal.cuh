@@ -34,7 +34,7 @@ struct Prob {
 
 // Workspace layout (byte offsets, each 256-aligned).
 struct WsLayout {
-    size_t err;       // uint32 error word (+ pad)
+    size_t err;       // uint32 error word; at +128 the tensor-core forward's int32 work-item counter
     size_t cnt;       // int32 [B]     kept blocks per batch row
     size_t sorted_n;  // int32 [B, N]  block index of the i-th smallest anchor
     size_t sorted_a;  // int32 [B, N]  its anchor
@@ -86,6 +86,7 @@ inline WsLayout ws_layout(const Prob &p) {
 // Typed views of the workspace.
 struct Ws {
     uint32_t *err;
+    int32_t *sched;  // work-item counter of the tensor-core forward (in the error word's section)
     int32_t *cnt, *sorted_n, *sorted_a;
     float2 *rope;
     void *kr_rot;
@@ -101,6 +102,7 @@ inline Ws ws_view(const Prob &p, void *base) {
     char *c = (char *)base;
     Ws w;
     w.err = (uint32_t *)(c + l.err);
+    w.sched = (int32_t *)(c + l.err + 128);
     w.cnt = (int32_t *)(c + l.cnt);
     w.sorted_n = (int32_t *)(c + l.sorted_n);
     w.sorted_a = (int32_t *)(c + l.sorted_a);
@@ -122,6 +124,37 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// ---- programmatic dependent launch ----------------------------------------
+// The kernels of one call (and of consecutive calls) form a chain in the
+// stream. Launched with programmatic stream serialization, a kernel may start
+// (its CTAs be scheduled, its prologue touching only shared and tensor memory
+// run) while the kernel before it finishes; pdl_wait() then blocks until that
+// kernel has completed and its memory operations are visible, so every such
+// kernel calls it before its first access to global memory. pdl_trigger()
+// lets the next kernel start early (it is scheduled once every CTA of this
+// one has triggered or exited); only the short single-wave kernels ahead of a
+// kernel with a real prologue call it early (early dependents parked beside a
+// long multi-wave kernel's last wave slowed it down), the others trigger by
+// exiting. Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // ---- launch accounting -----------------------------------------------------
 // Every kernel launch goes through count_launch() so that the launch counter of
 // the C ABI reports the device work a caller issued.
@@ -142,6 +175,7 @@ struct PadRows {
     int first[3];  // row of block 0's first position (0 for query rows, S for draft keys)
     int width[3];  // elements per row, a multiple of 8
     float *lse;    // [B, n_h, 5N] fp32: -inf for the block's rows (NULL = none)
+    int32_t *clear;  // a word set to 0 (the forward's work-item counter; NULL = none)
 };
 
 // rotated rope keys for all kv positions; with pad != NULL, also the padding

@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, in
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
     const int h0 = hg * kHeads, nhh = min(kHeads, n_h - h0);  // the group's heads
+    pdl_wait();
     if (i >= cnt[b]) {
         for (int hh = w; hh < nhh; hh += kWarps + 1)
             for (int r = 0; r < kBlock; r++) {
@@ -473,6 +474,7 @@ __global__ void __launch_bounds__(bw::kThreads, 1)
     const int region = (int)blockIdx.x / p.n_ctx, item = (int)blockIdx.x % p.n_ctx;
     const int b = region / p.HG, hg = region % p.HG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
     const int cnt = p.cnt[b];
     const int t0 = item * kMK;
     const int32_t *sa = p.sorted_a + (size_t)b * p.N;
@@ -995,6 +997,7 @@ __global__ void __launch_bounds__(160) k_bwd_dq_out(int n_h, int N, const int32_
                                                     const float2 *__restrict__ tab, const float *__restrict__ dqacc,
                                                     __nv_bfloat16 *__restrict__ dq) {
     const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    pdl_wait();
     if (i >= cnt[b]) return;
     const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = kBlock * N;
@@ -1027,32 +1030,37 @@ __global__ void __launch_bounds__(256) k_bwd_dkr_reduce(int B, int S, int N, int
                                                         const int32_t *anchors, const uint8_t *keep,
                                                         const float2 *tab, const float *part,
                                                         __nv_bfloat16 *dkr) {
-    const size_t wid = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (wid >= (size_t)B * L) return;
-    const int b = (int)(wid / L), key = (int)(wid % L);
-    int pos = key;
-    bool live = true;
-    if (key >= S) {
-        const int n = (key - S) / kBlock, i = (key - S) % kBlock;
-        const int a = anchors[(size_t)b * N + n];
-        live = keep[(size_t)b * N + n] && a >= 0 && a <= S - 2;
-        pos = a + i;
-    }
-    float x0 = 0.f, x1 = 0.f;
-    if (live) {
-        const int groups = key < S ? HG : HGd;  // context keys: the tensor-core kernel's groups
-        for (int g = 0; g < groups; g++) {
-            const float2 v = *reinterpret_cast<const float2 *>(part + (((size_t)g * B + b) * L + key) * kDR + 2 * lane);
-            x0 += v.x;
-            x1 += v.y;
+    pdl_wait();
+    for (size_t wid = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wid < (size_t)B * L;
+         wid += (size_t)gridDim.x * (blockDim.x >> 5)) {
+        const int b = (int)(wid / L), key = (int)(wid % L);
+        int pos = key;
+        bool live = true;
+        if (key >= S) {
+            const int n = (key - S) / kBlock, i = (key - S) % kBlock;
+            const int a = anchors[(size_t)b * N + n];
+            live = keep[(size_t)b * N + n] && a >= 0 && a <= S - 2;
+            pos = a + i;
         }
-        const float2 cs = tab[(size_t)pos * (kDR / 2) + lane];
-        const float y0 = x0 * cs.x + x1 * cs.y, y1 = x1 * cs.x - x0 * cs.y;
-        x0 = y0;
-        x1 = y1;
+        float x0 = 0.f, x1 = 0.f;
+        if (live) {
+            const int groups = key < S ? HG : HGd;  // context keys: the tensor-core kernel's groups
+            const float *src = part + ((size_t)b * L + key) * kDR + 2 * lane;
+            const size_t gstride = (size_t)B * L * kDR;
+#pragma unroll 4
+            for (int g = 0; g < groups; g++) {
+                const float2 v = *reinterpret_cast<const float2 *>(src + g * gstride);
+                x0 += v.x;
+                x1 += v.y;
+            }
+            const float2 cs = tab[(size_t)pos * (kDR / 2) + lane];
+            const float y0 = x0 * cs.x + x1 * cs.y, y1 = x1 * cs.x - x0 * cs.y;
+            x0 = y0;
+            x1 = y1;
+        }
+        *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
     }
-    *reinterpret_cast<__nv_bfloat162 *>(dkr + ((size_t)b * L + key) * kDR + 2 * lane) = __floats2bfloat162_rn(x0, x1);
 }
 
 // Row stages of the one-pass kernel.
@@ -1084,12 +1092,14 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
         count_launch();
         cudaError_t ep = cudaFuncSetAttribute(k_bwd_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, pr::kSmem);
         if (ep != cudaSuccess) return ep;
-        k_bwd_prep<<<dim3(p.N, bwd_prep_groups(p), p.B), pr::kThreads, pr::kSmem, st>>>(
-            p.n_h, p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
-            (const __nv_bfloat16 *)ws.kr_rot, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)o,
-            (const __nv_bfloat16 *)dout, lse, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope, (__nv_bfloat16 *)ws.qs,
-            (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, ws.dkr_part,
-            (__nv_bfloat16 *)dv, ws.err, p.wait_ns);
+        ep = launch_pdl(k_bwd_prep, dim3(p.N, bwd_prep_groups(p), p.B), dim3(pr::kThreads), pr::kSmem, st, p.n_h,
+                        p.S, p.N, p.L, p.scale, p.scale_log2, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc,
+                        (const __nv_bfloat16 *)ws.kr_rot, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)o,
+                        (const __nv_bfloat16 *)dout, lse, (const int32_t *)ws.cnt, (const int32_t *)ws.sorted_n,
+                        (const int32_t *)ws.sorted_a, (const float2 *)ws.rope, (__nv_bfloat16 *)ws.qs,
+                        (__nv_bfloat16 *)ws.dos, ws.dvec, ws.lses, ws.dqacc, (__nv_bfloat16 *)dkc, ws.dkr_part,
+                        (__nv_bfloat16 *)dv, ws.err, p.wait_ns);
+        if (ep != cudaSuccess) return ep;
     }
     CUtensorMap m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64;
     const uint64_t kv_rows = (uint64_t)p.B * p.n_h * p.L, q_rows = (uint64_t)p.B * p.n_h * p.R;
@@ -1127,17 +1137,21 @@ cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const vo
     cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<kRS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_tc<kRS><<<grid, bw::kThreads, smem, st>>>(m_kc3_64, m_kr64, m_v3_64, m_qs3_64, m_dos3_64, a);
+    if ((e = launch_pdl(k_bwd_tc<kRS>, dim3(grid), dim3(bw::kThreads), smem, st, m_kc3_64, m_kr64, m_v3_64, m_qs3_64,
+                        m_dos3_64, a)) != cudaSuccess)
+        return e;
     if (p.N > 0) {
         count_launch();
-        k_bwd_dq_out<<<dim3(p.N, p.n_h, p.B), 160, 0, st>>>(p.n_h, p.N, ws.cnt, ws.sorted_n, ws.sorted_a, ws.rope,
-                                                             ws.dqacc, (__nv_bfloat16 *)dq);
+        if ((e = launch_pdl(k_bwd_dq_out, dim3(p.N, p.n_h, p.B), dim3(160), 0, st, p.n_h, p.N,
+                            (const int32_t *)ws.cnt, (const int32_t *)ws.sorted_n, (const int32_t *)ws.sorted_a,
+                            (const float2 *)ws.rope, (const float *)ws.dqacc, (__nv_bfloat16 *)dq)) != cudaSuccess)
+            return e;
     }
     const size_t warps = (size_t)p.B * p.L;
     count_launch();
-    k_bwd_dkr_reduce<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.B, p.S, p.N, p.L, HG, bwd_prep_groups(p), anchors,
-                                                                   keep, ws.rope, ws.dkr_part, (__nv_bfloat16 *)dkr);
-    return cudaGetLastError();
+    return launch_pdl(k_bwd_dkr_reduce, dim3((unsigned)std::min<size_t>((warps + 7) / 8, 148 * 8)), dim3(256), 0, st,
+                      p.B, p.S, p.N, p.L, HG, bwd_prep_groups(p), anchors, keep, (const float2 *)ws.rope,
+                      (const float *)ws.dkr_part, (__nv_bfloat16 *)dkr);
 }
 
 }  // namespace dspark

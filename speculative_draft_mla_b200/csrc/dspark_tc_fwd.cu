@@ -13,8 +13,9 @@
 // are sorted by anchor, neighbouring items read overlapping windows close
 // together in time, so the overlap is served by L2.
 //
-// Persistent: one CTA per SM walks the items blockIdx.x, + gridDim.x, ...
-// K/V tiles, S buffers and pipeline phases are counted over all of a CTA's
+// Persistent: one CTA per SM; each takes its next work item from a global
+// counter (items in the order of item_at), so all CTAs stay busy until the
+// items run out. K/V tiles, S buffers and pipeline phases are counted over all of a CTA's
 // items, so the K/V stream runs on across item boundaries; the next item's
 // raw Q rows are staged (and their rope slice rotated) while the current item
 // runs, moved into TMEM as soon as its last QK has completed, and the finished
@@ -93,12 +94,16 @@ constexpr int kDraftBlocksPerTile = kBN / 8;  // 8 key slots per block
 // 64-column slices 1 KB apart and 8-key groups 4 KB apart.
 constexpr int kDraftKcBlock = 3 * 1024, kDraftKr = 3 * kKChunk, kDraftVBlock = 4 * 1024;
 constexpr int kSmemBytes = oBar + 512 + 1024;  // barriers + alignment slack
-// barrier words: K and V full/empty per stage, 28 more, 6 counters, then one more barrier
-static_assert((2 * (kKS + kVS) + 32) * 8 <= 512, "barrier area too small");
+// barrier words: K and V full/empty per stage, 28 more, 6 counters, one more
+// barrier, the item ring's 2 x kRing barriers and its kRing slots
+constexpr int kRing = 4;
+static_assert((2 * (kKS + kVS) + 32 + 2 * kRing + kRing / 2) * 8 <= 512, "barrier area too small");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 constexpr int kSoftWarps = 8;
 constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10, kWarpQ = 11;
+// roles that read the item ring: K and V producers, the MMA issuer, the softmax warps
+constexpr int kItemReaders = 3 + kSoftWarps;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
@@ -116,8 +121,11 @@ struct FwdArgs {
     __nv_bfloat16 *o;
     float *lse;
     uint32_t *err;
+    int B;
     int n_groups;  // groups of kG blocks per batch row (work items per (b, h))
     int n_items;   // n_groups * n_h * B
+    int n_work;    // counter values that name an item: n_items + n_h * B
+    int *sched;    // work-item counter, 0 at launch
     uint64_t wait_ns;  // limit of the pipeline waits (ns)
 };
 
@@ -139,18 +147,34 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 // this thread's bulk stores are complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Work item w = (group g, head h, batch b), g fastest (neighbouring items read
-// overlapping context windows of one head close together in time).
+// Work items in the order the CTAs take them from the counter: first every
+// full group of kG blocks, w = (group g, head h, batch b) with g fastest
+// (neighbouring groups of one head read overlapping context windows, close
+// together in time, so the overlap is served by L2); then, from w = n_items
+// on, the last, partial group of each (b, h) whose kept count is not a
+// multiple of kG. Small items at the end even out the CTAs' finishing times.
 struct Item {
     int b, gcnt, nrows, ctx_lo, n_ctx, T;
     size_t bh;
     const int32_t *sa, *sn;
 };
 __device__ __forceinline__ bool item_at(const FwdArgs &p, int w, Item &it) {
-    const int g = w % p.n_groups, h = (w / p.n_groups) % p.n_h, b = w / (p.n_groups * p.n_h);
-    const int cnt = p.cnt[b];
+    int g, h, b, cnt;
+    if (w < p.n_items) {
+        g = w % p.n_groups;
+        h = (w / p.n_groups) % p.n_h;
+        b = w / (p.n_groups * p.n_h);
+        cnt = p.cnt[b];
+        if (g * kG + kG > cnt) return false;  // past the row's blocks, or its partial group
+    } else {
+        const int r = w - p.n_items;
+        h = r % p.n_h;
+        b = r / p.n_h;
+        cnt = p.cnt[b];
+        if (cnt % kG == 0) return false;  // no partial group
+        g = cnt / kG;
+    }
     const int i0 = g * kG;
-    if (i0 >= cnt) return false;  // this batch row has fewer groups
     it.b = b;
     it.gcnt = min(kG, cnt - i0);
     it.nrows = kBlock * it.gcnt;
@@ -163,16 +187,13 @@ __device__ __forceinline__ bool item_at(const FwdArgs &p, int w, Item &it) {
     it.bh = (size_t)b * p.n_h + h;
     return true;
 }
-// The next valid item of this CTA at or after w (w advances by gridDim.x).
-__device__ __forceinline__ bool next_item(const FwdArgs &p, int &w, Item &it) {
-    for (; w < p.n_items; w += gridDim.x)
-        if (item_at(p, w, it)) return true;
-    return false;
-}
 
-// Persistent: one CTA per SM walks its work items (blockIdx.x, + gridDim.x,
-// ...). Tiles, S buffers and pipeline phases are counted over all of the
-// CTA's items, so K/V loads run on across item boundaries.
+// Persistent: one CTA per SM. The loader warp takes the CTA's next work item
+// from a global counter (so every CTA stays busy until the items run out) and
+// publishes it in a ring of kRing slots in shared memory, from which the other
+// roles read the same sequence. Tiles, S buffers and pipeline phases are
+// counted over all of the CTA's items, so K/V loads run on across item
+// boundaries.
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tm_kc3, const __grid_constant__ CUtensorMap tm_kr,
              const __grid_constant__ CUtensorMap tm_v3, const __grid_constant__ CUtensorMap tm_kc38,
@@ -198,6 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *counters = reinterpret_cast<int *>(sfull + 28);
     // per item: the staged raw Q rows' rope slice rotated (loader warp)
     uint64_t *qrot = sfull + 31;
+    // item ring: slot published (loader warp), slot read by every reader role
+    uint64_t *ifull = sfull + 32, *ifree = ifull + kRing;
+    volatile int *ring = reinterpret_cast<volatile int *>(ifree + kRing);
     float *xm = reinterpret_cast<float *>(sm + oX);         // [s][half][row]
     float *xl = reinterpret_cast<float *>(sm + oX + 2048);  // [half][row]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -229,6 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(ostaged, kSoftWarps);
         mbar_init(oread, 1);
         mbar_init(drain, 1);
+        for (int s = 0; s < kRing; s++) {
+            mbar_init(&ifull[s], 1);
+            mbar_init(&ifree[s], kItemReaders);
+        }
         for (int i = 0; i < 8; i++) mbar_init(&xbar[i], 2);
         for (int i = 0; i < 4; i++) mbar_init(&lbar[i], 2);
         *abort_flag = 0;
@@ -241,9 +269,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();  // the zeroed stages are read by TMA-fed MMAs
     tc_fence_before();
+    pdl_wait();  // the kernels before this one (rotated rope keys, item counter) have completed
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+
+    // Item k of the CTA's sequence from ring slot k % kRing: 1 = an item, 0 =
+    // past the last one, -1 = the wait gave up. take_w is called by a whole
+    // warp, take_1 by one thread; release: this reader is done with the slot.
+    auto take_w = [&](int k, Item &it) -> int {
+        const int s = k % kRing;
+        if (!warp_all(mbar_wait(&ifull[s], (k / kRing) & 1, abort_flag, wlim))) return -1;
+        const int w = ring[s];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ifree[s]);
+        return w >= 0 && item_at(p, w, it) ? 1 : 0;
+    };
+    auto take_1 = [&](int k, Item &it, bool release) -> int {
+        const int s = k % kRing;
+        if (!mbar_wait(&ifull[s], (k / kRing) & 1, abort_flag, wlim)) return -1;
+        const int w = ring[s];
+        if (release) mbar_arrive(&ifree[s]);
+        return w >= 0 && item_at(p, w, it) ? 1 : 0;
+    };
 
     if (warp == kWarpK || warp == kWarpV) {
         // ------------------------------------------------------ producers
@@ -256,7 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tt = 0;  // tiles over all items
         bool ok = true;
         Item it;
-        for (int w = blockIdx.x; ok && next_item(p, w, it); w += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            const int f = take_w(k, it);
+            if (f < 0) ok = false;
+            if (f <= 0) break;
             // lane l holds the block index of group block l
             const int my_n = lane < it.gcnt ? it.sn[lane] : 0;
             for (int t = 0; t < it.T; ++t, ++tt) {
@@ -358,15 +409,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(qrot);
             return true;
         };
+        // Item k of the CTA's sequence: the next valid item from the global
+        // counter, published in ring slot k % kRing once every reader is done
+        // with the item kRing before it (1 = an item, 0 = none left, published
+        // as -1, -1 = a wait gave up). Called by the whole warp.
+        auto fetch = [&](int k, Item &it) -> int {
+            const int s = k % kRing;
+            if (k >= kRing && !warp_all(mbar_wait(&ifree[s], ((k / kRing) - 1) & 1, abort_flag, wlim))) return -1;
+            int w = -1;
+            if (lane == 0) {
+                Item probe;
+                for (;;) {
+                    const int x = atomicAdd(p.sched, 1);
+                    if (x >= p.n_work) break;
+                    if (item_at(p, x, probe)) {
+                        w = x;
+                        break;
+                    }
+                }
+                ring[s] = w;
+                mbar_arrive(&ifull[s]);
+            }
+            w = __shfl_sync(0xffffffffu, w, 0);
+            return w >= 0 && item_at(p, w, it) ? 1 : 0;
+        };
         Item it, nx;
-        int w = blockIdx.x, ic = 0;
-        bool has = next_item(p, w, it), ok = true;
+        int ic = 0;
+        int f = fetch(0, it);
+        bool ok = f >= 0, has = f > 0, hasn = false;
         if (has) {
             load_q(it, 0);
             ok = rotate_q(it, 0);
         }
-        int wn = w + gridDim.x;
-        bool hasn = has && next_item(p, wn, nx);
+        if (ok && has) {
+            f = fetch(1, nx);
+            ok = f >= 0;
+            hasn = f > 0;
+        }
         if (ok && hasn) {  // item 1's raw Q once item 0's is in TMEM
             ok = warp_all(mbar_wait(stgfree, 0, abort_flag, wlim));
             if (ok) {
@@ -388,18 +467,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(oread);
             // the item after next: its raw Q into the staging area
-            int w2 = wn + gridDim.x;
             Item n2;
-            const bool has2 = hasn && next_item(p, w2, n2);
+            bool has2 = false;
+            if (hasn) {
+                f = fetch(ic + 2, n2);
+                if (f < 0) {
+                    ok = false;
+                    break;
+                }
+                has2 = f > 0;
+            }
             if (has2) {
                 load_q(n2, ic + 2);
                 ok = rotate_q(n2, ic + 2);
             }
             ++ic;
-            w = wn;
             it = nx;
             has = hasn;
-            wn = w2;
             nx = n2;
             hasn = has2;
         }
@@ -461,11 +545,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // item's first tile, the item's Q is in TMEM; P V when its P is in
             // TMEM and its V landed and, at an item's first tile, the previous
             // item's O has been read out.
+            // (the QK cursor reads each item first; the P V cursor releases it)
             Item ik, ip;
-            int wk = blockIdx.x, wp = blockIdx.x;
-            bool hk = next_item(p, wk, ik), hp = next_item(p, wp, ip);
+            int f = take_1(0, ik, false);
+            bool ok = f >= 0, hk = f > 0, hp = false;
+            if (ok) {
+                f = take_1(0, ip, true);
+                ok = f >= 0;
+                hp = f > 0;
+            }
             int nk = 0, np = 0, icK = 0, icP = 0, tK = 0, tP = 0;
-            bool ok = true;
             uint64_t t_idle = 0;
             while (ok && hp) {
                 bool issued = false;
@@ -477,8 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (++tK == ik.T) {
                         tK = 0;
                         ++icK;
-                        wk += gridDim.x;
-                        hk = next_item(p, wk, ik);
+                        const int g = take_1(icK, ik, false);
+                        if (g < 0) ok = false;
+                        hk = g > 0;
                     }
                     issued = true;
                 }
@@ -491,8 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (++tP == ip.T) {
                         tP = 0;
                         ++icP;
-                        wp += gridDim.x;
-                        hp = next_item(p, wp, ip);
+                        const int g = take_1(icP, ip, true);
+                        if (g < 0) ok = false;
+                        hp = g > 0;
                     }
                     issued = true;
                 }
@@ -547,8 +638,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tg = 0;  // tiles over all items
         int ic = 0;
         Item it, nx;
-        int w = blockIdx.x;
-        bool has = next_item(p, w, it);
+        const int f0 = take_w(0, it);
+        ok = f0 >= 0;
+        bool has = f0 > 0;
         if (has) {
             move_q(it, 0);
             __syncwarp();
@@ -665,8 +757,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The next item's Q into TMEM (its raw rows are staged; every QK of
             // this item has completed, as all its S tiles have been read), so
             // that its QK can start while this item's O is written out.
-            int wn = w + gridDim.x;
-            const bool hasn = next_item(p, wn, nx);
+            const int fn = take_w(ic + 1, nx);
+            if (fn < 0) {
+                ok = false;
+                break;
+            }
+            const bool hasn = fn > 0;
             if (hasn) {
                 move_q(nx, ic + 1);
                 if (!ok) break;
@@ -718,13 +814,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (live && hf == 0) p.lse[it.bh * p.R + kBlock * n + j] = (m_used + log2f(ltot)) * kLn2;
             ++ic;
-            w = wn;
             it = nx;
             has = hasn;
         }
     }
 
     // ---------------------------------------------------------- teardown
+    pdl_trigger();
     __syncthreads();
     if (*abort_flag) {
         // Drain what may still be in flight, each wait bounded on its own.
@@ -786,14 +882,17 @@ cudaError_t launch_fwd_tc(const Prob &p, const void *q, const void *kc, const vo
     a.lse = lse;
     a.err = ws.err;
     a.wait_ns = p.wait_ns;
+    a.B = p.B;
+    a.sched = ws.sched;
     a.n_groups = (p.N + kG - 1) / kG;
     a.n_items = a.n_groups * p.n_h * p.B;
+    a.n_work = a.n_items + p.n_h * p.B;
     int dev = 0, nsm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     count_launch();
-    k_fwd_tc<<<std::min(a.n_items, nsm), kThreads, kSmemBytes, st>>>(m_kc3, m_kr, m_v3, m_kc38, m_kr8, m_v38, a);
-    return cudaGetLastError();
+    return launch_pdl(k_fwd_tc, dim3(std::min(a.n_items, nsm)), dim3(kThreads), kSmemBytes, st, m_kc3, m_kr, m_v3,
+                      m_kc38, m_kr8, m_v38, a);
 }
 
 }  // namespace dspark
