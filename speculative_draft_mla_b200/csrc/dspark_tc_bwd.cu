@@ -90,7 +90,7 @@ __device__ __forceinline__ bool compute_warps_or(bool x, int nthreads) {
 }
 constexpr int kWarps = 4;                  // compute warps
 constexpr int kHeads = 16;                 // heads per CTA at most
-constexpr int kStages = 6;                 // staged heads
+constexpr int kStages = 4;                 // staged heads
 constexpr int kRowsB = kBlock * kDQK * 2;  // 5 rows of 256 bf16 (q, O, dO, V)
 constexpr int kKcB = kBlock * kDC * 2;     // 5 rows of K^C
 constexpr int oQ = 0, oO = kRowsB, oDO = 2 * kRowsB, oV = 3 * kRowsB, oKc = 4 * kRowsB;
@@ -102,7 +102,7 @@ constexpr int kSmem = kStages * kStageB + 128;  // dynamic: the stages (+ alignm
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-__global__ void __launch_bounds__(pr::kThreads, 2) k_bwd_prep(int n_h, int S, int N, int L, float scale, float scale_log2,
+__global__ void __launch_bounds__(pr::kThreads, 4) k_bwd_prep(int n_h, int S, int N, int L, float scale, float scale_log2,
                                                   const __nv_bfloat16 *__restrict__ q,
                                                   const __nv_bfloat16 *__restrict__ kc,
                                                   const __nv_bfloat16 *__restrict__ krr,
