@@ -6,13 +6,16 @@ descriptor, forward (O, LSE), backward (dQ, dK^C, dK^R, dV), all through the C
 ABI. Default workload: B=2, S=8192, N=512, W=128, 64 heads, 192+64 / 256, bf16.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID]
-                  [--impl reference] [--no-cpu-baseline] [--no-e2e]
+                  [--impl reference] [--no-cpu-baseline] [--no-e2e] [--desc-timing]
+                  [--part attention|draft-inputs]
 
 Prints one JSON line (rank 0). With N > 1 (torchrun) every rank processes its
 own batch (batch sharding, weak scaling, no collective on the data path); the
 time is the max over ranks and the value the rows of all ranks over that time.
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
-workload instead.
+workload instead. ``--part draft-inputs`` times instead the step before the
+attention: GPU anchor sampling and the draft block's inputs (ids, positions,
+labels, predecessors, eval_mask) for the workload's batch shape, on one GPU.
 """
 import argparse
 import datetime
@@ -272,6 +275,60 @@ def run_reference(args, wl):
     print(json.dumps(out), flush=True)
 
 
+def run_draft_inputs(args, wl, capi, device):
+    """Anchor sampling + draft-block inputs for the workload's (B, S, N): one
+    step = dspark_sample_anchors_gpu + dspark_build_draft_inputs. Algorithmic
+    bytes: the loss_mask, the six input ids a block reads (x_A .. x_{A+5}), the
+    anchors and keep written and the five [B, 5N] outputs."""
+    from oracle import draft_inputs as odi
+    # the workload's loss mask (the first draw of its input generator)
+    lm_h = synth._draw_loss_mask(wl, torch.Generator().manual_seed(1000 + wl.id)).to(torch.uint8)
+    g = torch.Generator().manual_seed(77)
+    ids_h = torch.randint(0, 154880, (wl.B, wl.S), generator=g, dtype=torch.int32)
+    lm, ids = lm_h.to(device), ids_h.to(device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        an, kp = capi.sample_anchors_gpu(lm, wl.N, 1000 + i)
+        return capi.build_draft_inputs(ids, lm, an, kp)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clk:
+        torch.cuda.synchronize()
+        n0 = capi.launch_counter()
+        start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        end.record(stream)
+        torch.cuda.synchronize()
+        n1 = capi.launch_counter()
+    ms = start.elapsed_time(end) / args.steps
+    rows = wl.B * 5 * wl.N
+    nbytes = wl.B * wl.S + wl.B * wl.N * (6 * 4 + 4 + 1) + rows * (4 * 4 + 1)
+    hbm, _, _, src = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    t0 = time.perf_counter()
+    an_o, kp_o = odi.sample_anchors(lm_h.numpy(), wl.N, 1000)
+    odi.build_draft_inputs(ids_h.numpy(), lm_h.numpy(), an_o, kp_o)
+    cpu_s = time.perf_counter() - t0
+    out = {"metric": "draft rows/sec (anchor sampling + draft-block inputs, 1 B200)", "value": rows / (ms * 1e-3),
+           "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+           "config": {"workload": wl.name, "B": wl.B, "S": wl.S, "N": wl.N, "part": "draft-inputs",
+                      "l2": "inputs far smaller than L2 (the step is launch- and latency-bound)"},
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                        "traffic": None, "kernel": "k_sample_anchors + k_build_draft_inputs",
+                        "peak_source": src + " (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
+                        "bytes": nbytes},
+           "cpu_baseline": {"value": rows / cpu_s, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                            "sample": "the whole step once (oracle.draft_inputs, pure Python), %.2f s" % cpu_s},
+           "clocks": clk.summary(), "gpu_launches": n1 - n0}
+    print(json.dumps(out))
+
+
 def config_of(wl):
     return {"workload": wl.name, "B": wl.B, "S": wl.S, "N": wl.N, "W": wl.W, "n_h": wl.n_h, "d_c": wl.d_c,
             "d_r": wl.d_r, "d_v": wl.d_v, "rope_base": wl.rope_base, "rows": wl.rows,
@@ -288,6 +345,7 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--part", default="attention", choices=["attention", "draft-inputs"])
     ap.add_argument("--desc-timing", action="store_true",
                     help="also time the descriptor build alone (an event between it and the forward call)")
     args = ap.parse_args()
@@ -310,6 +368,10 @@ def main():
         dbuild.build()
     barrier(world)
     capi.load()
+    if args.part == "draft-inputs":
+        if rank == 0:
+            run_draft_inputs(args, wl, capi, device)
+        return
 
     host = synth.make_inputs(wl)
     in_bytes = sum(t.numel() * t.element_size() for t in host.values())

@@ -194,6 +194,46 @@ DSPARK_API uint64_t dspark_set_wait_limit_ns(uint64_t ns);
 DSPARK_API int64_t dspark_sample_anchors(const uint8_t *loss_mask, int32_t B, int32_t S, int32_t N, uint64_t seed,
                               int32_t *anchors_out, uint8_t *keep_out);
 
+/* GPU anchor sampler, page §2 "anchor sampling": for each batch row b the
+ * candidates are A in [0, S-2] with loss_mask[A] = loss_mask[A+1] = 1, where
+ * loss_mask[S-1] is read as 0 (§6). Each candidate gets the key k_A = output A
+ * (counted from 0) of SplitMix64 started from state seed + b, and the
+ * min(N, #candidates) candidates with the smallest (k_A, A) are kept (a uniform
+ * draw without replacement), written in ascending order of A; the remaining
+ * entries are padding blocks, anchor 0 and keep 0 (§3). Deterministic for a
+ * given seed. This draw differs from dspark_sample_anchors' (a shuffle, in draw
+ * order); both are uniform.
+ *   loss_mask [B, S] uint8, anchors [B, N] int32 (4-byte aligned),
+ *   keep [B, N] uint8: device pointers, owned by the caller.
+ * Limits: B >= 0, 1 <= S < 2^30, 0 <= N <= 8192. Launches one kernel on the
+ * stream; returns a status from the host checks (nothing is written on error)
+ * or DSPARK_ERR_CUDA if the launch fails. */
+DSPARK_API dspark_status dspark_sample_anchors_gpu(const uint8_t *loss_mask, int32_t B, int32_t S, int32_t N,
+                                                   uint64_t seed, int32_t *anchors, uint8_t *keep, void *stream);
+
+/* Draft-block inputs for anchors / keep [B, N] (page §2 "Draft block", §5
+ * Markov head, §6 "Label" and "eval_mask"). For block n with anchor A and
+ * offset j = 0..4, row 5n + j of each [B, 5N] output holds
+ *   draft_ids    x_A at j = 0, mask_id at j = 1..4 (the page's MASK is 154821)
+ *   position_ids A + j (the block's RoPE positions on the KV axis)
+ *   labels       y_j = x_{A+j+1}
+ *   prev_ids     x_{A+j} (the anchor, then the gold tokens: the Markov head's
+ *                predecessors)
+ *   eval_mask    1 while every step j' <= j has A+j'+1 < S, loss_mask[A+j'+1] = 1
+ *                (loss_mask[S-1] read as 0) and keep = 1 (a prefix product
+ *                along the block), else 0.
+ * Positions outside [0, S) read as mask_id (draft_ids, prev_ids) and -1
+ * (labels); such steps have eval_mask 0.
+ *   input_ids [B, S] int32, loss_mask [B, S] uint8, anchors [B, N] int32,
+ *   keep [B, N] uint8; outputs int32 except eval_mask (uint8). Device pointers
+ *   owned by the caller; int32 arrays 4-byte aligned.
+ * Limits, errors and launches as dspark_sample_anchors_gpu. */
+DSPARK_API dspark_status dspark_build_draft_inputs(const int32_t *input_ids, const uint8_t *loss_mask, int32_t B,
+                                                   int32_t S, int32_t N, const int32_t *anchors, const uint8_t *keep,
+                                                   int32_t mask_id, int32_t *draft_ids, int32_t *position_ids,
+                                                   int32_t *labels, int32_t *prev_ids, uint8_t *eval_mask,
+                                                   void *stream);
+
 #ifdef __cplusplus
 }
 #endif

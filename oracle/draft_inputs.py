@@ -78,6 +78,8 @@ def build_draft_inputs(input_ids, loss_mask, anchors, keep, mask_id=MASK_ID):
       eval_mask  = prefix product over j of [A+j+1 < S and
                    loss_mask[A+j+1] = 1 (loss_mask[S-1] read as 0) and
                    keep = 1]                                           (§6)
+    Positions outside [0, S) (also for an anchor outside the page's range)
+    read as MASK (ids, prev) and -1 (labels), and end the eval_mask prefix.
     Returns a dict of [B, 5N] arrays (int32, eval_mask uint8)."""
     x = np.asarray(input_ids)
     lm = np.array(loss_mask, dtype=np.uint8, copy=True)
@@ -87,17 +89,21 @@ def build_draft_inputs(input_ids, loss_mask, anchors, keep, mask_id=MASK_ID):
     N = anchors.shape[1]
     out = {k: np.zeros((B, BLOCK * N), np.int32) for k in ("draft_ids", "position_ids", "labels", "prev_ids")}
     out["eval_mask"] = np.zeros((B, BLOCK * N), np.uint8)
+
+    def inside(p):
+        return 0 <= p < S
+
     for b in range(B):
         for n in range(N):
             A = int(anchors[b, n])
             on = bool(keep[b, n])
             for j in range(BLOCK):
                 r = BLOCK * n + j
-                out["draft_ids"][b, r] = int(x[b, A]) if j == 0 else mask_id
+                out["draft_ids"][b, r] = int(x[b, A]) if j == 0 and inside(A) else mask_id
                 out["position_ids"][b, r] = A + j
-                out["labels"][b, r] = int(x[b, A + j + 1]) if A + j + 1 < S else -1
-                out["prev_ids"][b, r] = int(x[b, A + j]) if A + j < S else mask_id
-                step = A + j + 1 < S and lm[b, A + j + 1] == 1 and keep[b, n] == 1
+                out["labels"][b, r] = int(x[b, A + j + 1]) if inside(A + j + 1) else -1
+                out["prev_ids"][b, r] = int(x[b, A + j]) if inside(A + j) else mask_id
+                step = inside(A + j + 1) and lm[b, A + j + 1] == 1 and keep[b, n] == 1
                 on = on and step
                 out["eval_mask"][b, r] = 1 if on else 0
     return out

@@ -19,7 +19,8 @@ STATUS = {0: "OK", 1: "ERR_NULL", 2: "ERR_SHAPE", 3: "ERR_DTYPE", 4: "ERR_ANCHOR
           6: "ERR_CUDA", 7: "ERR_DEVICE", 8: "ERR_ALIGN", 9: "ERR_UNSUPPORTED"}
 EXPORTS = ("dspark_workspace_size", "dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd",
            "dspark_get_error", "dspark_status_string", "dspark_sample_anchors", "dspark_launch_counter",
-           "dspark_set_wait_limit_ns")
+           "dspark_set_wait_limit_ns", "dspark_sample_anchors_gpu", "dspark_build_draft_inputs")
+MASK_ID = 154821  # the page's MASK token id
 
 
 class Problem(ctypes.Structure):
@@ -62,6 +63,11 @@ def load():
     lib.dspark_attn_fwd_noalloc.restype = ctypes.c_int
     lib.dspark_launch_counter.argtypes = []
     lib.dspark_launch_counter.restype = ctypes.c_uint64
+    i32 = ctypes.c_int32
+    lib.dspark_sample_anchors_gpu.argtypes = [vp, i32, i32, i32, ctypes.c_uint64, vp, vp, vp]
+    lib.dspark_sample_anchors_gpu.restype = ctypes.c_int
+    lib.dspark_build_draft_inputs.argtypes = [vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp]
+    lib.dspark_build_draft_inputs.restype = ctypes.c_int
     lib.dspark_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.dspark_set_wait_limit_ns.restype = ctypes.c_uint64
     for f in ("dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd", "dspark_get_error"):
@@ -202,6 +208,41 @@ def set_wait_limit_ns(ns):
     """Limit (ns) of the kernels' pipeline waits for later calls; 0 restores
     the default (2 s). Returns the previous limit."""
     return int(load().dspark_set_wait_limit_ns(int(ns)))
+
+
+def sample_anchors_gpu(loss_mask, N, seed, stream=None):
+    """GPU anchor sampler: loss_mask uint8 [B, S] (CUDA) -> (anchors int32 [B, N], keep uint8 [B, N])."""
+    _cuda(loss_mask)
+    if loss_mask.dtype != torch.uint8:
+        raise TypeError("loss_mask must be uint8")
+    B, S = loss_mask.shape
+    anchors = torch.empty(B, N, dtype=torch.int32, device=loss_mask.device)
+    keep = torch.empty(B, N, dtype=torch.uint8, device=loss_mask.device)
+    _check(load().dspark_sample_anchors_gpu(_ptr(loss_mask), B, S, N, ctypes.c_uint64(seed & (2 ** 64 - 1)),
+                                            _ptr(anchors), _ptr(keep), _stream(stream, loss_mask.device)),
+           "dspark_sample_anchors_gpu")
+    return anchors, keep
+
+
+def build_draft_inputs(input_ids, loss_mask, anchors, keep, mask_id=MASK_ID, stream=None):
+    """Draft-block inputs: input_ids int32 [B, S], loss_mask uint8 [B, S], anchors int32 / keep uint8
+    [B, N] (CUDA) -> dict of [B, 5N] tensors: draft_ids, position_ids, labels, prev_ids (int32) and
+    eval_mask (uint8)."""
+    _cuda(input_ids, loss_mask, anchors, keep)
+    if input_ids.dtype != torch.int32 or anchors.dtype != torch.int32 or loss_mask.dtype != torch.uint8 or \
+            keep.dtype != torch.uint8:
+        raise TypeError("input_ids / anchors int32, loss_mask / keep uint8")
+    B, S = input_ids.shape
+    N = anchors.shape[1]
+    dev = input_ids.device
+    out = {k: torch.empty(B, 5 * N, dtype=torch.int32, device=dev)
+           for k in ("draft_ids", "position_ids", "labels", "prev_ids")}
+    out["eval_mask"] = torch.empty(B, 5 * N, dtype=torch.uint8, device=dev)
+    _check(load().dspark_build_draft_inputs(_ptr(input_ids), _ptr(loss_mask), B, S, N, _ptr(anchors), _ptr(keep),
+                                            int(mask_id), _ptr(out["draft_ids"]), _ptr(out["position_ids"]),
+                                            _ptr(out["labels"]), _ptr(out["prev_ids"]), _ptr(out["eval_mask"]),
+                                            _stream(stream, dev)), "dspark_build_draft_inputs")
+    return out
 
 
 def sample_anchors(loss_mask, N, seed):

@@ -250,6 +250,37 @@ dspark_status dspark_get_error(void *workspace, void *stream) {
 
 uint64_t dspark_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
 
+static bool aligned4(const void *x) { return ((uintptr_t)x & 3u) == 0; }
+
+dspark_status dspark_sample_anchors_gpu(const uint8_t *loss_mask, int32_t B, int32_t S, int32_t N, uint64_t seed,
+                                        int32_t *anchors, uint8_t *keep, void *stream) {
+    if (B < 0 || S < 1 || N < 0) return DSPARK_ERR_SHAPE;
+    if (S >= (1 << 30) || N > 8192) return DSPARK_ERR_UNSUPPORTED;
+    if ((int64_t)B * N == 0) return DSPARK_OK;
+    if (!loss_mask || !anchors || !keep) return DSPARK_ERR_NULL;
+    if (!aligned4(anchors)) return DSPARK_ERR_ALIGN;
+    DSPARK_CUDA(launch_sample_anchors(loss_mask, B, S, N, seed, anchors, keep, (cudaStream_t)stream));
+    return DSPARK_OK;
+}
+
+dspark_status dspark_build_draft_inputs(const int32_t *input_ids, const uint8_t *loss_mask, int32_t B, int32_t S,
+                                        int32_t N, const int32_t *anchors, const uint8_t *keep, int32_t mask_id,
+                                        int32_t *draft_ids, int32_t *position_ids, int32_t *labels,
+                                        int32_t *prev_ids, uint8_t *eval_mask, void *stream) {
+    if (B < 0 || S < 1 || N < 0) return DSPARK_ERR_SHAPE;
+    if (S >= (1 << 30) || N > 8192) return DSPARK_ERR_UNSUPPORTED;
+    if ((int64_t)B * N == 0) return DSPARK_OK;
+    if (!input_ids || !loss_mask || !anchors || !keep || !draft_ids || !position_ids || !labels || !prev_ids ||
+        !eval_mask)
+        return DSPARK_ERR_NULL;
+    if (!aligned4(input_ids) || !aligned4(anchors) || !aligned4(draft_ids) || !aligned4(position_ids) ||
+        !aligned4(labels) || !aligned4(prev_ids))
+        return DSPARK_ERR_ALIGN;
+    DSPARK_CUDA(launch_build_draft_inputs(input_ids, loss_mask, B, S, N, anchors, keep, mask_id, draft_ids,
+                                          position_ids, labels, prev_ids, eval_mask, (cudaStream_t)stream));
+    return DSPARK_OK;
+}
+
 uint64_t dspark_set_wait_limit_ns(uint64_t ns) {
     if (ns == 0 || ns > kWaitTimeoutNs) ns = kWaitTimeoutNs;
     return g_wait_ns.exchange(ns, std::memory_order_relaxed);

@@ -190,6 +190,15 @@ cudaError_t launch_bwd_simt(const Prob &p, const void *q, const void *kc, const 
                             const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,
                             void *dkc, void *dkr, void *dv, const Ws &ws, cudaStream_t st);
 
+// draft inputs: GPU anchor sampler and the draft block's ids, positions, labels,
+// Markov predecessors and eval_mask
+cudaError_t launch_sample_anchors(const uint8_t *loss_mask, int B, int S, int N, uint64_t seed, int32_t *anchors,
+                                  uint8_t *keep, cudaStream_t st);
+cudaError_t launch_build_draft_inputs(const int32_t *input_ids, const uint8_t *loss_mask, int B, int S, int N,
+                                      const int32_t *anchors, const uint8_t *keep, int mask_id, int32_t *draft_ids,
+                                      int32_t *position_ids, int32_t *labels, int32_t *prev_ids, uint8_t *eval_mask,
+                                      cudaStream_t st);
+
 // tcgen05 backward for bf16 at the page's head widths
 cudaError_t launch_bwd_tc(const Prob &p, const void *q, const void *kc, const void *v, const int32_t *anchors,
                           const uint8_t *keep, const void *o, const float *lse, const void *dout, void *dq,

@@ -138,3 +138,26 @@ def test_wait_limit_setter(lib):
     assert capi.set_wait_limit_ns(5 * default) == 1000
     assert capi.set_wait_limit_ns(0) == default
     assert capi.set_wait_limit_ns(0) == default
+
+
+def test_draft_input_validation(lib):
+    """Host checks of the GPU sampler and builder return before any device work."""
+    vp = ctypes.c_void_p
+    odd = vp(0x1001)  # never dereferenced: every call below fails its host checks
+    ok = vp(0x1000)
+    S_, N_ = 100, 10
+    assert lib.dspark_sample_anchors_gpu(ok, -1, S_, N_, 1, ok, ok, None) == 2
+    assert lib.dspark_sample_anchors_gpu(ok, 1, 0, N_, 1, ok, ok, None) == 2
+    assert lib.dspark_sample_anchors_gpu(ok, 1, S_, 9000, 1, ok, ok, None) == 9
+    assert lib.dspark_sample_anchors_gpu(None, 1, S_, N_, 1, ok, ok, None) == 1
+    assert lib.dspark_sample_anchors_gpu(ok, 1, S_, N_, 1, odd, ok, None) == 8
+    assert lib.dspark_sample_anchors_gpu(None, 0, S_, N_, 1, None, None, None) == 0  # nothing to do
+    args = [ok, ok, 1, S_, N_, ok, ok, 154821, ok, ok, ok, ok, ok, None]
+    assert lib.dspark_build_draft_inputs(*args[:2], -1, *args[3:]) == 2
+    bad = list(args)
+    bad[8] = None
+    assert lib.dspark_build_draft_inputs(*bad) == 1
+    bad = list(args)
+    bad[10] = odd
+    assert lib.dspark_build_draft_inputs(*bad) == 8
+    assert lib.dspark_build_draft_inputs(*args[:4], 0, *args[5:]) == 0
