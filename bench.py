@@ -7,7 +7,7 @@ ABI. Default workload: B=2, S=8192, N=512, W=128, 64 heads, 192+64 / 256, bf16.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID]
                   [--impl reference] [--no-cpu-baseline] [--no-e2e] [--desc-timing]
-                  [--part attention|draft-inputs]
+                  [--part attention|draft-inputs|loss]
 
 Prints one JSON line (rank 0). With N > 1 (torchrun) every rank processes its
 own batch (batch sharding, weak scaling, no collective on the data path); the
@@ -15,7 +15,9 @@ time is the max over ranks and the value the rows of all ranks over that time.
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workload instead. ``--part draft-inputs`` times instead the step before the
 attention: GPU anchor sampling and the draft block's inputs (ids, positions,
-labels, predecessors, eval_mask) for the workload's batch shape, on one GPU.
+labels, predecessors, eval_mask) for the workload's batch shape, on one GPU;
+``--part loss`` times the training loss over the workload's B * 5N draft steps
+(V = 154880 synthetic bf16 student and teacher logits) with its gradient.
 """
 import argparse
 import datetime
@@ -329,6 +331,71 @@ def run_draft_inputs(args, wl, capi, device):
     print(json.dumps(out))
 
 
+def run_loss(args, wl, capi, device):
+    """The DSpark loss over the workload's B * 5N draft steps, V = 154880: one
+    step = dspark_loss_fwd_bwd (loss means and the gradients with respect to
+    the student logits and the confidence logits). Algorithmic bytes: student
+    and teacher logits read once, the logit gradient written once, the per-step
+    scalars (label, confidence logit, eval_mask, its gradient)."""
+    from oracle import dspark_loss as odl
+    V = 154880
+    R = wl.B * 5 * wl.N
+    g = torch.Generator(device=device).manual_seed(4242)
+    L = (torch.randn(R, V, generator=g, device=device) * 3).to(torch.bfloat16)
+    T = (torch.randn(R, V, generator=g, device=device) * 3).to(torch.bfloat16)
+    y = torch.randint(0, V, (R,), generator=g, device=device, dtype=torch.int32)
+    c = torch.randn(R, generator=g, device=device)
+    m = (torch.rand(R, generator=g, device=device) < 0.9).to(torch.uint8)
+    out, grad, gconf, ws = capi.dspark_loss(L, T, y, c, m)
+    lib = capi.load()
+    st = capi._stream(None, device)
+    ptr = capi._ptr
+
+    def step():
+        capi._check(lib.dspark_loss_fwd_bwd(R, V, ptr(L), ptr(T), ptr(y), ptr(c), ptr(m), 1.0, 0.9, 1.0, ptr(out),
+                                            ptr(grad), ptr(gconf), ptr(ws), ws.numel(), st), "dspark_loss_fwd_bwd")
+
+    for _ in range(args.warmup):
+        step()
+    capi.get_error(ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device) as clk:
+        torch.cuda.synchronize()
+        n0 = capi.launch_counter()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+        n1 = capi.launch_counter()
+    capi.get_error(ws)
+    ms = start.elapsed_time(end) / args.steps
+    nbytes = 3 * R * V * 2 + R * (4 + 4 + 1 + 4 + 16)
+    hbm, _, _, src = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    # the oracle (fp64 NumPy) on a few steps, scaled to steps/s
+    k = 4
+    t0 = time.perf_counter()
+    odl.loss_fwd_bwd(L[:k].double().cpu().numpy(), T[:k].double().cpu().numpy(), y[:k].cpu().numpy(),
+                     c[:k].double().cpu().numpy(), m[:k].cpu().numpy())
+    cpu_s = time.perf_counter() - t0
+    res = {"metric": "draft steps/sec (DSpark loss + gradient, V=154880, bf16, 1 B200)", "value": R / (ms * 1e-3),
+           "unit": "steps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": wl.name, "rows": R, "V": V, "part": "loss",
+                      "l2": "inputs larger than L2 (no flush between steps)"},
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                        "traffic": None, "kernel": "dspark_loss_fwd_bwd call (all its kernels)",
+                        "peak_source": src + " (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
+                        "bytes": nbytes},
+           "cpu_baseline": {"value": k / cpu_s, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                            "sample": "%d of the %d steps (fp64 NumPy, one thread), %.2f s" % (k, R, cpu_s)},
+           "clocks": clk.summary(), "gpu_launches": n1 - n0}
+    print(json.dumps(res))
+
+
 def config_of(wl):
     return {"workload": wl.name, "B": wl.B, "S": wl.S, "N": wl.N, "W": wl.W, "n_h": wl.n_h, "d_c": wl.d_c,
             "d_r": wl.d_r, "d_v": wl.d_v, "rope_base": wl.rope_base, "rows": wl.rows,
@@ -345,7 +412,7 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--part", default="attention", choices=["attention", "draft-inputs"])
+    ap.add_argument("--part", default="attention", choices=["attention", "draft-inputs", "loss"])
     ap.add_argument("--desc-timing", action="store_true",
                     help="also time the descriptor build alone (an event between it and the forward call)")
     args = ap.parse_args()
@@ -368,9 +435,9 @@ def main():
         dbuild.build()
     barrier(world)
     capi.load()
-    if args.part == "draft-inputs":
+    if args.part != "attention":
         if rank == 0:
-            run_draft_inputs(args, wl, capi, device)
+            (run_draft_inputs if args.part == "draft-inputs" else run_loss)(args, wl, capi, device)
         return
 
     host = synth.make_inputs(wl)

@@ -234,6 +234,46 @@ DSPARK_API dspark_status dspark_build_draft_inputs(const int32_t *input_ids, con
                                                    int32_t *labels, int32_t *prev_ids, uint8_t *eval_mask,
                                                    void *stream);
 
+/* Bytes of device workspace dspark_loss_fwd_bwd needs for R rows (256-byte
+ * aligned). */
+DSPARK_API size_t dspark_loss_workspace_size(int32_t R);
+
+/* The DSpark training loss over R draft steps and its gradient (page §6).
+ * Row r holds student logits L_r = student_logits[r] and teacher logits
+ * T_r = teacher_logits[r] over the vocabulary (V entries each), the label
+ * y_r = labels[r], the confidence-head logit c_r = conf_logits[r] and
+ * m_r = eval_mask[r] (0 / 1). With p = softmax(L_r), q = softmax(T_r):
+ *   CE_r  = logsumexp(L_r) - L_r[y_r]
+ *   L1_r  = sum_i |p_i - q_i|
+ *   a_r   = clip(1 - L1_r / 2, 0, 1)            (a target: no gradient)
+ *   BCE_r = max(c_r, 0) - c_r a_r + log(1 + exp(-|c_r|))
+ *   loss  = ce_alpha CE + l1_alpha L1 + conf_alpha BCE, each the sum over the
+ *           counted steps (m_r = 1) divided by their number M (the page's
+ *           coefficients are 1, 0.9 and 1).
+ * Writes loss_out[4] = {loss, CE mean, L1 mean, BCE mean} and, when given,
+ *   grad_logits[r][i] = (m_r / M) (ce_alpha (p_i - [i = y_r])
+ *                                  + l1_alpha p_i (s_i - sum_j s_j p_j)),
+ *       s = sign(p - q) (0 where p = q), rounded to bf16 (every element of
+ *       every row is written, zeros for uncounted rows),
+ *   grad_conf[r] = (m_r / M) conf_alpha (sigmoid(c_r) - a_r).
+ * M = 0 gives a zero loss and zero gradients; a label outside [0, V) adds no
+ * CE term. Teacher logits get no gradient.
+ *   student_logits, teacher_logits, grad_logits: [R, V] bf16, 16-byte aligned;
+ *   labels [R] int32, conf_logits [R] float, eval_mask [R] uint8, grad_conf [R]
+ *   float, loss_out [4] float: device pointers owned by the caller;
+ *   grad_logits and grad_conf may be NULL (loss only).
+ * Limits: R >= 0, V >= 8 and a multiple of 8, V <= 229376. Host checks return
+ * before any launch; a bounded wait that gives up is reported through the
+ * workspace as in dspark_get_error (DSPARK_ERR_DEVICE). Launches four
+ * operations on the stream (a count, the loss kernel in clusters of 8 CTAs, a
+ * fixed-order reduction and a memset). */
+DSPARK_API dspark_status dspark_loss_fwd_bwd(int32_t R, int32_t V, const void *student_logits,
+                                             const void *teacher_logits, const int32_t *labels,
+                                             const float *conf_logits, const uint8_t *eval_mask, float ce_alpha,
+                                             float l1_alpha, float conf_alpha, float *loss_out, void *grad_logits,
+                                             float *grad_conf, void *workspace, size_t workspace_bytes,
+                                             void *stream);
+
 #ifdef __cplusplus
 }
 #endif

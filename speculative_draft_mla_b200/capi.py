@@ -19,7 +19,8 @@ STATUS = {0: "OK", 1: "ERR_NULL", 2: "ERR_SHAPE", 3: "ERR_DTYPE", 4: "ERR_ANCHOR
           6: "ERR_CUDA", 7: "ERR_DEVICE", 8: "ERR_ALIGN", 9: "ERR_UNSUPPORTED"}
 EXPORTS = ("dspark_workspace_size", "dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd",
            "dspark_get_error", "dspark_status_string", "dspark_sample_anchors", "dspark_launch_counter",
-           "dspark_set_wait_limit_ns", "dspark_sample_anchors_gpu", "dspark_build_draft_inputs")
+           "dspark_set_wait_limit_ns", "dspark_sample_anchors_gpu", "dspark_build_draft_inputs",
+           "dspark_loss_workspace_size", "dspark_loss_fwd_bwd")
 MASK_ID = 154821  # the page's MASK token id
 
 
@@ -68,6 +69,11 @@ def load():
     lib.dspark_sample_anchors_gpu.restype = ctypes.c_int
     lib.dspark_build_draft_inputs.argtypes = [vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp]
     lib.dspark_build_draft_inputs.restype = ctypes.c_int
+    lib.dspark_loss_workspace_size.argtypes = [i32]
+    lib.dspark_loss_workspace_size.restype = sz
+    f32 = ctypes.c_float
+    lib.dspark_loss_fwd_bwd.argtypes = [i32, i32, vp, vp, vp, vp, vp, f32, f32, f32, vp, vp, vp, vp, sz, vp]
+    lib.dspark_loss_fwd_bwd.restype = ctypes.c_int
     lib.dspark_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.dspark_set_wait_limit_ns.restype = ctypes.c_uint64
     for f in ("dspark_build_descriptor", "dspark_attn_fwd", "dspark_attn_bwd", "dspark_get_error"):
@@ -243,6 +249,31 @@ def build_draft_inputs(input_ids, loss_mask, anchors, keep, mask_id=MASK_ID, str
                                             _ptr(out["labels"]), _ptr(out["prev_ids"]), _ptr(out["eval_mask"]),
                                             _stream(stream, dev)), "dspark_build_draft_inputs")
     return out
+
+
+CE_ALPHA, L1_ALPHA, CONF_ALPHA = 1.0, 0.9, 1.0  # the page's loss coefficients
+
+
+def dspark_loss(student_logits, teacher_logits, labels, conf_logits, eval_mask, with_grad=True,
+                alphas=(CE_ALPHA, L1_ALPHA, CONF_ALPHA), workspace=None, stream=None):
+    """DSpark loss over R draft steps: bf16 [R, V] logits, int32 labels, float conf logits, uint8
+    eval_mask (CUDA). Returns (loss [4] float: total, CE, L1, BCE means; grad_logits or None;
+    grad_conf or None; workspace)."""
+    _cuda(student_logits, teacher_logits, labels, conf_logits, eval_mask)
+    if student_logits.dtype != torch.bfloat16 or teacher_logits.dtype != torch.bfloat16:
+        raise TypeError("logits must be bf16")
+    R, V = student_logits.shape
+    dev = student_logits.device
+    if workspace is None:
+        workspace = torch.empty(int(load().dspark_loss_workspace_size(R)), dtype=torch.uint8, device=dev)
+    out = torch.empty(4, dtype=torch.float32, device=dev)
+    grad = torch.empty_like(student_logits) if with_grad else None
+    gconf = torch.empty(R, dtype=torch.float32, device=dev) if with_grad else None
+    _check(load().dspark_loss_fwd_bwd(R, V, _ptr(student_logits), _ptr(teacher_logits), _ptr(labels),
+                                      _ptr(conf_logits), _ptr(eval_mask), float(alphas[0]), float(alphas[1]),
+                                      float(alphas[2]), _ptr(out), _ptr(grad), _ptr(gconf), _ptr(workspace),
+                                      workspace.numel(), _stream(stream, dev)), "dspark_loss_fwd_bwd")
+    return out, grad, gconf, workspace
 
 
 def sample_anchors(loss_mask, N, seed):

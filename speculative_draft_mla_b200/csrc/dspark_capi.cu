@@ -281,6 +281,29 @@ dspark_status dspark_build_draft_inputs(const int32_t *input_ids, const uint8_t 
     return DSPARK_OK;
 }
 
+size_t dspark_loss_workspace_size(int32_t R) { return R < 0 ? 0 : loss_workspace_size(R); }
+
+dspark_status dspark_loss_fwd_bwd(int32_t R, int32_t V, const void *student_logits, const void *teacher_logits,
+                                  const int32_t *labels, const float *conf_logits, const uint8_t *eval_mask,
+                                  float ce_alpha, float l1_alpha, float conf_alpha, float *loss_out,
+                                  void *grad_logits, float *grad_conf, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    if (R < 0 || V < 8 || (V % 8) != 0) return DSPARK_ERR_SHAPE;
+    if (V > 229376 || (int64_t)R * V >= (1ll << 40)) return DSPARK_ERR_UNSUPPORTED;  // two row slices per CTA
+    if (!loss_out || !workspace || (R > 0 && (!student_logits || !teacher_logits || !labels || !conf_logits ||
+                                              !eval_mask)))
+        return DSPARK_ERR_NULL;
+    if (workspace_bytes < loss_workspace_size(R) || ((uintptr_t)workspace & 255u)) return DSPARK_ERR_WORKSPACE;
+    if ((R > 0 && (!aligned16(student_logits) || !aligned16(teacher_logits))) ||
+        (grad_logits && !aligned16(grad_logits)) || !aligned4(loss_out) || (labels && !aligned4(labels)) ||
+        (conf_logits && !aligned4(conf_logits)) || (grad_conf && !aligned4(grad_conf)))
+        return DSPARK_ERR_ALIGN;
+    DSPARK_CUDA(launch_loss(R, V, student_logits, teacher_logits, labels, conf_logits, eval_mask, ce_alpha, l1_alpha,
+                            conf_alpha, loss_out, grad_logits, grad_conf, workspace,
+                            g_wait_ns.load(std::memory_order_relaxed), (cudaStream_t)stream));
+    return DSPARK_OK;
+}
+
 uint64_t dspark_set_wait_limit_ns(uint64_t ns) {
     if (ns == 0 || ns > kWaitTimeoutNs) ns = kWaitTimeoutNs;
     return g_wait_ns.exchange(ns, std::memory_order_relaxed);
