@@ -6,7 +6,7 @@
 #include <cstdlib>
 #include <cstring>
 
-#include "dspark_internal.cuh"
+#include "dspark_steps.cuh"
 
 using namespace dspark;
 

@@ -12,7 +12,7 @@
 // per batch row finds the N-th smallest key by a radix select and compacts the
 // chosen anchors in ascending order with a block-wide scan.
 
-#include "dspark_internal.cuh"
+#include "dspark_steps.cuh"
 
 namespace dspark {
 

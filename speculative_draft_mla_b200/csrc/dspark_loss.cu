@@ -20,6 +20,7 @@
 
 #include <algorithm>
 
+#include "dspark_steps.cuh"
 #include "dspark_tc_common.cuh"
 
 namespace cg = cooperative_groups;
