@@ -12,8 +12,9 @@
 // one row at a time, each CTA 1/kCl of L and T in shared memory, loaded by 1-D
 // bulk copies; the CTAs exchange their partial (max, sum) pairs and then their
 // (L1, sum s p) partials through distributed shared memory, so every logit is
-// read from HBM once and every gradient written once. Each CTA has two row
-// buffers: the next row's copies land while the current row is computed.
+// read from HBM once and every gradient written once. Two CTAs share an SM
+// (one row slice each, of two different rows), so one's copies and barrier
+// waits overlap the other's passes.
 // Per element: exp of L and T for the normalisers, p and q for L1, p again for
 // the gradient (sign(p - q) is taken in the log domain).
 #include <cooperative_groups.h>
@@ -30,7 +31,8 @@ namespace dspark {
 namespace {
 
 constexpr int kCl = 8;         // CTAs per row (cluster size)
-constexpr int kThr = 896;      // threads per CTA (28 warps at <= 73 registers: one CTA per SM)
+constexpr int kThr = 448;      // threads per CTA (14 warps at <= 73 registers: two CTAs per SM)
+constexpr int kBufs = 1;       // row buffers per CTA (two CTAs per SM overlap each other's waits)
 constexpr int kWarps = kThr / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -93,7 +95,7 @@ __device__ __forceinline__ void block_reduce(float (&v)[kN], int op, float (*red
     for (int i = 0; i < kN; i++) v[i] = res[i];
 }
 
-__global__ void __launch_bounds__(kThr, 1) k_dspark_loss(const LossArgs p) {
+__global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u);
     __nv_bfloat16 *buf = reinterpret_cast<__nv_bfloat16 *>(sm);  // [2][L | T][seg]
@@ -128,20 +130,30 @@ __global__ void __launch_bounds__(kThr, 1) k_dspark_loss(const LossArgs p) {
         }
     };
     int issued = 0, waited = 0;  // row loads issued / completed (thread 0's count)
-    if (threadIdx.x == 0 && cid < p.R) {
+    if (kBufs == 2 && threadIdx.x == 0 && cid < p.R) {
         issue(cid, 0);
         issued = 1;
     }
     int it = 0;
     for (int r = cid; r < p.R; r += ncl, ++it) {
-        const int b = it & 1;
-        __syncthreads();  // every thread is done with buffer b ^ 1 (the previous row)
-        if (threadIdx.x == 0 && r + ncl < p.R && !*abort_flag) {
-            tc::fence_proxy_async_smem();
-            issue(r + ncl, b ^ 1);
-            issued = it + 2;
+        const int b = kBufs == 2 ? (it & 1) : 0;
+        // every thread is done with the buffer the next copy fills (the
+        // previous row's), then the copies of the row after (two buffers) or
+        // of this row (one buffer)
+        __syncthreads();
+        if (threadIdx.x == 0 && !*abort_flag) {
+            if (kBufs == 2 && r + ncl < p.R) {
+                tc::fence_proxy_async_smem();
+                issue(r + ncl, b ^ 1);
+                issued = it + 2;
+            } else if (kBufs == 1) {
+                tc::fence_proxy_async_smem();
+                issue(r, 0);
+                issued = it + 1;
+            }
         }
-        bool ok = !*abort_flag && tc::warp_all(tc::mbar_wait(&full[b], (it >> 1) & 1, abort_flag, p.wait_ns));
+        const uint32_t ph = kBufs == 2 ? (uint32_t)((it >> 1) & 1) : (uint32_t)(it & 1);
+        bool ok = !*abort_flag && tc::warp_all(tc::mbar_wait(&full[b], ph, abort_flag, p.wait_ns));
         if (threadIdx.x == 0 && ok) waited = it + 1;
         const uint4 *Lv = reinterpret_cast<const uint4 *>(buf + (size_t)(2 * b) * p.seg);
         const uint4 *Tv = reinterpret_cast<const uint4 *>(buf + (size_t)(2 * b + 1) * p.seg);
@@ -306,7 +318,8 @@ __global__ void __launch_bounds__(kThr, 1) k_dspark_loss(const LossArgs p) {
     // peer may still read its shared memory
     if (threadIdx.x == 0 && *abort_flag) {
         volatile int never = 0;
-        for (int t = waited; t < issued; ++t) tc::mbar_wait(&full[t & 1], (t >> 1) & 1, &never);
+        for (int t = waited; t < issued; ++t)
+            tc::mbar_wait(&full[kBufs == 2 ? (t & 1) : 0], kBufs == 2 ? (t >> 1) & 1 : t & 1, &never);
         atomicOr(p.err, kErrTimeout);
     }
     cluster.sync();
@@ -387,7 +400,7 @@ cudaError_t launch_loss(int R, int V, const void *L, const void *T, const int32_
         a.stats = stats;
         a.err = err;
         a.wait_ns = wait_ns;
-        const size_t smem = (size_t)8 * a.seg + 128;
+        const size_t smem = (size_t)4 * kBufs * a.seg + 128;
         if ((e = cudaFuncSetAttribute(k_dspark_loss, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
             cudaSuccess)
             return e;
