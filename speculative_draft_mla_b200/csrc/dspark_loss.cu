@@ -15,8 +15,9 @@
 // read from HBM once and every gradient written once. Two CTAs share an SM
 // (one row slice each, of two different rows), so one's copies and barrier
 // waits overlap the other's passes.
-// Per element: exp of L and T for the normalisers, p and q for L1, p again for
-// the gradient (sign(p - q) is taken in the log domain).
+// Per element: exp of L and T for the normalisers, p and q for L1 (sign(p - q)
+// taken in the log domain); that pass leaves p (bf16) and the sign in place of
+// the logits, from which the gradient pass works without an exponential.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -236,20 +237,31 @@ __global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
         }
         __syncthreads();
         const float lseL2 = res[0], lseT2 = res[1], Ly = res[2];
-        // L1 and sum_i s_i p_i over this CTA's elements
+        // L1 and sum_i s_i p_i over this CTA's elements; p (bf16) and s = sign(p - q)
+        // replace the slices' logits for the gradient pass (L[y] was taken above)
         float acc[2] = {0.f, 0.f};
+        uint4 *Lw = reinterpret_cast<uint4 *>(buf + (size_t)(2 * b) * p.seg);
+        uint4 *Tw = reinterpret_cast<uint4 *>(buf + (size_t)(2 * b + 1) * p.seg);
         for (int v = threadIdx.x; v < nv; v += kThr) {
-            float a[8], c[8];
+            float a[8], c[8], pv[8], sv[8];
             unpack8(Lv[v], a);
             unpack8(Tv[v], c);
 #pragma unroll
             for (int i = 0; i < 8; i++) {
                 const float la = fmaf(a[i], kLog2e, -lseL2), lc = fmaf(c[i], kLog2e, -lseT2);
                 const float pi = tc::ex2(la), qi = tc::ex2(lc);
+                const float si = la > lc ? 1.f : (la < lc ? -1.f : 0.f);
                 acc[0] += fabsf(pi - qi);
-                acc[1] += la > lc ? pi : (la < lc ? -pi : 0.f);
+                acc[1] += si * pi;
+                pv[i] = pi;
+                sv[i] = si;
             }
+            Lw[v] = make_uint4(tc::pack_bf16x2(pv[0], pv[1]), tc::pack_bf16x2(pv[2], pv[3]),
+                               tc::pack_bf16x2(pv[4], pv[5]), tc::pack_bf16x2(pv[6], pv[7]));
+            Tw[v] = make_uint4(tc::pack_bf16x2(sv[0], sv[1]), tc::pack_bf16x2(sv[2], sv[3]),
+                               tc::pack_bf16x2(sv[4], sv[5]), tc::pack_bf16x2(sv[6], sv[7]));
         }
+        tc::fence_proxy_async_smem();  // these writes precede the copy that refills the buffer
         block_reduce<2>(acc, 0, red, res);
         if (threadIdx.x == 0) {
             x2[0] = acc[0];
@@ -284,16 +296,12 @@ __global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
             const float cw = yvalid ? w * p.ce_alpha : 0.f, lw = w * p.l1_alpha;
             uint4 *G = reinterpret_cast<uint4 *>(p.grad + (size_t)r * p.V + e0);
             for (int v = threadIdx.x; v < nv; v += kThr) {
-                float a[8], c[8];
-                unpack8(Lv[v], a);
-                unpack8(Tv[v], c);
+                float pv[8], sv[8];
+                unpack8(Lv[v], pv);  // p and s stored by the L1 pass
+                unpack8(Tv[v], sv);
                 float g[8];
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const float la = fmaf(a[i], kLog2e, -lseL2), lc = fmaf(c[i], kLog2e, -lseT2);
-                    const float s = la > lc ? 1.f : (la < lc ? -1.f : 0.f);
-                    g[i] = tc::ex2(la) * (cw + lw * (s - Sb));
-                }
+                for (int i = 0; i < 8; i++) g[i] = pv[i] * (cw + lw * (sv[i] - Sb));
                 const int ky = y - e0 - 8 * v;  // y's place in this vector, if there
                 if (yvalid && ky >= 0 && ky < 8) {
 #pragma unroll
