@@ -96,6 +96,53 @@ __device__ __forceinline__ void block_reduce(float (&v)[kN], int op, float (*red
     for (int i = 0; i < kN; i++) v[i] = res[i];
 }
 
+// Merge of per-thread (max m, sum z of exp(x - m)) pairs for two quantities
+// over the CTA: each warp takes its maximum and rescales its sums to it, then
+// warp 0 merges the warps' pairs; res[0..3] = (m0, z0, m1, z1) for every thread.
+__device__ __forceinline__ void block_merge_mz(float (&m)[2], float (&z)[2], float (*red)[4], float *res) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        float M = m[k];
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+        float zz = m[k] > -INFINITY ? z[k] * tc::ex2((m[k] - M) * kLog2e) : 0.f;
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, d);
+        m[k] = M;
+        z[k] = zz;
+    }
+    if (lane == 0) {
+        red[warp][0] = m[0];
+        red[warp][1] = z[0];
+        red[warp][2] = m[1];
+        red[warp][3] = z[1];
+    }
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const float wm = lane < kWarps ? red[lane][2 * k] : -INFINITY;
+            const float wz = lane < kWarps ? red[lane][2 * k + 1] : 0.f;
+            float M = wm;
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+            float zz = wm > -INFINITY ? wz * tc::ex2((wm - M) * kLog2e) : 0.f;
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, d);
+            if (lane == 0) {
+                res[2 * k] = M;
+                res[2 * k + 1] = zz;
+            }
+        }
+    }
+    __syncthreads();
+    m[0] = res[0];
+    z[0] = res[1];
+    m[1] = res[2];
+    z[1] = res[3];
+}
+
 __global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u);
@@ -189,11 +236,8 @@ __global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
                 tz[1] += tc::ex2(fmaf(c[i], kLog2e, -mc));
             }
         }
-        float mx[2] = {tm[0], tm[1]};
-        block_reduce<2>(mx, 1, red, res);
-        float zs[2] = {tm[0] > -INFINITY ? tz[0] * tc::ex2((tm[0] - mx[0]) * kLog2e) : 0.f,
-                       tm[1] > -INFINITY ? tz[1] * tc::ex2((tm[1] - mx[1]) * kLog2e) : 0.f};
-        block_reduce<2>(zs, 0, red, res);
+        float mx[2] = {tm[0], tm[1]}, zs[2] = {tz[0], tz[1]};
+        block_merge_mz(mx, zs, red, res);
         if (threadIdx.x == 0) {
             const bool mine = yvalid && y >= e0 && y < e0 + len;
             x1[0] = mx[0];
