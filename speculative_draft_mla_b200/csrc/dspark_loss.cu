@@ -96,6 +96,25 @@ __device__ __forceinline__ void block_reduce(float (&v)[kN], int op, float (*red
     for (int i = 0; i < kN; i++) v[i] = res[i];
 }
 
+// Bounded wait for a row's copies (once per row, so the clock is read at every
+// poll): gives up when the CTA's abort flag is raised or after limit_ns (then
+// raises it). Returns false when it gave up. try_wait may suspend the thread
+// for a while before it reports "not yet", which is what the waiting warps
+// should do while the SM's other CTA computes; a limit below 1 ms is honoured
+// by polling without suspending instead.
+__device__ __forceinline__ bool wait_row(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint64_t limit_ns) {
+    const bool fine = limit_ns < 1000000ull;
+    const uint64_t t0 = tc::globaltimer();
+    for (;;) {
+        if (fine ? tc::mbar_test(bar, parity) : tc::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (tc::globaltimer() - t0 > limit_ns) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // Merge of per-thread (max m, sum z of exp(x - m)) pairs for two quantities
 // over the CTA: each warp takes its maximum and rescales its sums to it, then
 // warp 0 merges the warps' pairs; res[0..3] = (m0, z0, m1, z1) for every thread.
@@ -201,7 +220,7 @@ __global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
             }
         }
         const uint32_t ph = kBufs == 2 ? (uint32_t)((it >> 1) & 1) : (uint32_t)(it & 1);
-        bool ok = !*abort_flag && tc::warp_all(tc::mbar_wait(&full[b], ph, abort_flag, p.wait_ns));
+        bool ok = !*abort_flag && tc::warp_all(wait_row(&full[b], ph, abort_flag, p.wait_ns));
         if (threadIdx.x == 0 && ok) waited = it + 1;
         const uint4 *Lv = reinterpret_cast<const uint4 *>(buf + (size_t)(2 * b) * p.seg);
         const uint4 *Tv = reinterpret_cast<const uint4 *>(buf + (size_t)(2 * b + 1) * p.seg);

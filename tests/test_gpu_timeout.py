@@ -61,3 +61,30 @@ def test_wait_limit_runs_out_and_context_recovers():
     torch.cuda.synchronize()
     after = run_gpu(c, wl.S, wl.W)  # raises if the error word is set
     _same(before, after)
+
+
+def test_wait_limit_loss_cluster_kernel():
+    """The loss kernel's CTAs wait for their row copies with the same bounded
+    waits; one that gives up stops issuing copies but keeps taking part in
+    every cluster barrier (the cluster's CTAs run the same rows), drains its
+    copies and reports the device error; the next call is clean."""
+    g = torch.Generator(device="cuda").manual_seed(3)
+    R, V = 64, 154880
+    L = torch.randn(R, V, generator=g, device="cuda").to(torch.bfloat16)
+    T = torch.randn(R, V, generator=g, device="cuda").to(torch.bfloat16)
+    y = torch.randint(0, V, (R,), generator=g, device="cuda", dtype=torch.int32)
+    c = torch.randn(R, generator=g, device="cuda")
+    m = torch.ones(R, dtype=torch.uint8, device="cuda")
+    out0, g0, gc0, ws = capi.dspark_loss(L, T, y, c, m)
+    capi.get_error(ws)
+    prev = capi.set_wait_limit_ns(1)
+    try:
+        capi.dspark_loss(L, T, y, c, m, workspace=ws)
+        with pytest.raises(capi.DsparkError) as e:
+            capi.get_error(ws)
+        assert e.value.status == ERR_DEVICE
+    finally:
+        assert capi.set_wait_limit_ns(prev) == 1
+    out1, g1, gc1, ws = capi.dspark_loss(L, T, y, c, m, workspace=ws)
+    capi.get_error(ws)
+    assert torch.equal(out0, out1) and torch.equal(g0, g1) and torch.equal(gc0, gc1)
