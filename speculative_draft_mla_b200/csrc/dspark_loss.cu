@@ -165,7 +165,7 @@ __device__ __forceinline__ void block_merge_mz(float (&m)[2], float (&z)[2], flo
 __global__ void __launch_bounds__(kThr, 2) k_dspark_loss(const LossArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u);
-    __nv_bfloat16 *buf = reinterpret_cast<__nv_bfloat16 *>(sm);  // [2][L | T][seg]
+    __nv_bfloat16 *buf = reinterpret_cast<__nv_bfloat16 *>(sm);  // [kBufs][L | T][seg]
     __shared__ float red[kWarps][4];
     __shared__ float res[4];  // block results, then the row's exchanged values
     __shared__ float x1[6];  // this CTA's max L, sum L, max T, sum T, L[y], has y
